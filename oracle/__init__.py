@@ -1,0 +1,273 @@
+"""CPU oracle for the deterministic MoE layer forward (test infrastructure only).
+
+Only the test suite, the package smoke check and the benchmark's CPU-baseline
+leg may import this package. It wraps oracle/moe_oracle.cpp (plain C++,
+OpenMP) through ctypes and orchestrates its steps with plain numpy; it shares
+no code with the CUDA library.
+
+Parity pins: every function here is checked in tests/ against something other
+than itself (brute force, closed forms, library routines, the pages' worked
+numbers). The design notes list them; no function is left unpinned.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+_f32p = ctypes.POINTER(ctypes.c_float)
+_f64p = ctypes.POINTER(ctypes.c_double)
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        L.oracle_route_topk.argtypes = [_f32p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                        _i32p, _f32p, _f64p]
+        L.oracle_route_topk.restype = ctypes.c_int
+        L.oracle_schedule.argtypes = [_i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                      ctypes.c_int32, ctypes.c_int32, ctypes.c_int64, _i32p, _i32p,
+                                      _i32p, _i32p, _i64p]
+        L.oracle_schedule.restype = ctypes.c_int
+        L.oracle_place_closed_form.argtypes = [_i32p] + [ctypes.c_int32] * 5 + [_i32p, _i32p]
+        L.oracle_place_closed_form.restype = ctypes.c_int
+        L.oracle_place_queue_sim.argtypes = [_i32p] + [ctypes.c_int32] * 5 + [ctypes.c_int64, _i32p,
+                                                                               _i32p, _i32p]
+        L.oracle_place_queue_sim.restype = ctypes.c_int
+        L.oracle_wave_floor.argtypes = [ctypes.c_int64] * 3
+        L.oracle_wave_floor.restype = ctypes.c_int64
+        L.oracle_dispatch_rows.argtypes = [_u16p, ctypes.c_int32, ctypes.c_int32, _i32p, _i64p,
+                                           ctypes.c_int64, _u16p]
+        L.oracle_dispatch_rows.restype = None
+        ptr_arr = ctypes.POINTER(ctypes.c_void_p)
+        L.oracle_ffn_rows.argtypes = [_u16p, ctypes.c_int64, _i32p, ctypes.c_int32, ctypes.c_int32,
+                                      ptr_arr, ptr_arr, ptr_arr, _u16p, _f64p]
+        L.oracle_ffn_rows.restype = None
+        L.oracle_combine_f64.argtypes = [_f64p, ctypes.c_int32, _i64p, _f64p, ctypes.c_int64,
+                                         ctypes.c_int32, _f64p, _u16p]
+        L.oracle_combine_f64.restype = None
+        L.oracle_combine_f32.argtypes = [_f32p, ctypes.c_int32, _i64p, _f32p, ctypes.c_int64,
+                                         ctypes.c_int32, _u16p]
+        L.oracle_combine_f32.restype = None
+        L.oracle_round_bf16.argtypes = [ctypes.c_double]
+        L.oracle_round_bf16.restype = ctypes.c_uint16
+        L.oracle_num_threads.restype = ctypes.c_int
+        L.oracle_set_num_threads.argtypes = [ctypes.c_int]
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray, t):
+    assert a.flags["C_CONTIGUOUS"], "oracle inputs must be C-contiguous"
+    return a.ctypes.data_as(t)
+
+
+def _np(x, dtype):
+    """torch tensor or array-like -> contiguous numpy array of dtype (CPU)."""
+    if hasattr(x, "detach"):
+        import torch
+        x = x.detach().cpu().contiguous()
+        if x.dtype == torch.bfloat16:
+            x = x.view(torch.int16)
+        x = x.numpy()
+    a = np.asarray(x)
+    dt = np.dtype(dtype)
+    if a.dtype != dt and a.dtype.kind in "iu" and dt.kind in "iu" and a.dtype.itemsize == dt.itemsize:
+        a = a.view(dt)  # reinterpret bits (bf16 / int16 -> uint16)
+    return np.ascontiguousarray(a, dtype=dt)
+
+
+def num_threads() -> int:
+    return lib().oracle_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    lib().oracle_set_num_threads(int(n))
+
+
+def round_bf16(v: float) -> int:
+    return int(lib().oracle_round_bf16(float(v)))
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def rows_cap(P: int, N: int, k: int, E: int, pad: int) -> int:
+    """Upper bound on padded rows: every route, plus at most pad-1 padding rows per expert."""
+    return P * N * k + E * (pad - 1)
+
+
+def route_topk(logits, k: int):
+    """ids int32 [T,k], gates fp32 [T,k], gates fp64 [T,k] (top-k by logit desc, id asc)."""
+    lg = _np(logits, np.float32)
+    T, E = lg.shape
+    ids = np.zeros((T, k), np.int32)
+    g32 = np.zeros((T, k), np.float32)
+    g64 = np.zeros((T, k), np.float64)
+    rc = lib().oracle_route_topk(_p(lg, _f32p), T, E, k, _p(ids, _i32p), _p(g32, _f32p),
+                                 _p(g64, _f64p))
+    if rc:
+        raise ValueError(f"oracle_route_topk rc={rc}")
+    return ids, g32, g64
+
+
+def schedule(ids, P: int, N: int, k: int, E: int, pad: int = 256):
+    """Counting-sort schedule. Returns dict(phi [rows,2], offsets [E+1], counts [E,P],
+    route_row [P,N,k], reads, counter_words, threads)."""
+    idn = _np(ids, np.int32).reshape(-1)
+    cap = max(rows_cap(P, N, k, E, pad), 1)
+    phi = np.full((cap, 2), -7, np.int32)
+    offsets = np.zeros(E + 1, np.int32)
+    counts = np.zeros((E, P), np.int32)
+    rr = np.zeros((P, N, k), np.int32)
+    stats = np.zeros(3, np.int64)
+    rc = lib().oracle_schedule(_p(idn, _i32p), P, N, k, E, pad, cap, _p(phi, _i32p),
+                               _p(offsets, _i32p), _p(counts, _i32p), _p(rr, _i32p),
+                               _p(stats, _i64p))
+    if rc:
+        raise ValueError(f"oracle_schedule rc={rc}")
+    rows = int(offsets[E])
+    return dict(phi=phi[:rows].copy(), offsets=offsets, counts=counts, route_row=rr,
+                reads=int(stats[0]), counter_words=int(stats[1]), threads=int(stats[2]))
+
+
+def place_closed_form(ids, P: int, N: int, k: int, E: int, pad: int = 256):
+    idn = _np(ids, np.int32).reshape(-1)
+    offsets = np.zeros(E + 1, np.int32)
+    rr = np.zeros((P, N, k), np.int32)
+    rc = lib().oracle_place_closed_form(_p(idn, _i32p), P, N, k, E, pad, _p(offsets, _i32p),
+                                        _p(rr, _i32p))
+    if rc:
+        raise ValueError(f"oracle_place_closed_form rc={rc}")
+    return offsets, rr
+
+
+def place_queue_sim(ids, P: int, N: int, k: int, E: int, pad: int = 256):
+    idn = _np(ids, np.int32).reshape(-1)
+    cap = max(rows_cap(P, N, k, E, pad), 1)
+    offsets = np.zeros(E + 1, np.int32)
+    rr = np.zeros((P, N, k), np.int32)
+    phi = np.full((cap, 2), -7, np.int32)
+    rc = lib().oracle_place_queue_sim(_p(idn, _i32p), P, N, k, E, pad, cap, _p(offsets, _i32p),
+                                      _p(rr, _i32p), _p(phi, _i32p))
+    if rc:
+        raise ValueError(f"oracle_place_queue_sim rc={rc}")
+    return offsets, rr, phi[: int(offsets[E])].copy()
+
+
+def wave_floor(H: int, I: int, C: int) -> int:
+    return int(lib().oracle_wave_floor(H, I, C))
+
+
+def dispatch_rows(x_bits: np.ndarray, N: int, phi: np.ndarray, rows) -> np.ndarray:
+    """Gather rows of Phi from x ([P*N, H] bf16 bits) -> [n, H] bf16 bits."""
+    xb = _np(x_bits, np.uint16)
+    H = xb.shape[1]
+    phn = np.ascontiguousarray(phi, np.int32)
+    rws = np.ascontiguousarray(np.asarray(rows, np.int64))
+    out = np.zeros((len(rws), H), np.uint16)
+    lib().oracle_dispatch_rows(_p(xb, _u16p), N, H, _p(phn, _i32p), _p(rws, _i64p), len(rws),
+                               _p(out, _u16p))
+    return out
+
+
+def ffn_rows(xg_bits: np.ndarray, experts, W1: dict, W3: dict, W2: dict, H: int, I: int):
+    """SwiGLU FFN of rows xg_bits [n,H] (bf16 bits) with per-row experts.
+
+    W1/W3/W2 map expert id -> numpy uint16 arrays [H,I] / [H,I] / [I,H].
+    Returns h bf16 bits [n,I] and y fp64 [n,H].
+    """
+    xb = np.ascontiguousarray(xg_bits, np.uint16)
+    ex = np.ascontiguousarray(np.asarray(experts, np.int32))
+    n = len(ex)
+    E = int(ex.max()) + 1 if n else 1
+    keep = []
+    arrs = []
+    for Wd in (W1, W3, W2):
+        a = (ctypes.c_void_p * E)()
+        for e, w in Wd.items():
+            if e < E:
+                w = np.ascontiguousarray(w, np.uint16)
+                keep.append(w)
+                a[e] = w.ctypes.data
+        arrs.append(a)
+    for e in set(ex.tolist()):
+        if not (arrs[0][e] and arrs[1][e] and arrs[2][e]):
+            raise ValueError(f"weights of expert {e} not given")
+    h = np.zeros((n, I), np.uint16)
+    y = np.zeros((n, H), np.float64)
+    if n:
+        lib().oracle_ffn_rows(_p(xb, _u16p), n, _p(ex, _i32p), H, I,
+                              ctypes.cast(arrs[0], ctypes.POINTER(ctypes.c_void_p)),
+                              ctypes.cast(arrs[1], ctypes.POINTER(ctypes.c_void_p)),
+                              ctypes.cast(arrs[2], ctypes.POINTER(ctypes.c_void_p)),
+                              _p(h, _u16p), _p(y, _f64p))
+    return h, y
+
+
+def combine_f64(y: np.ndarray, sel, g, k: int):
+    """out[a] = sum_j g[a,j] * y[sel[a,j]] (fp64). Returns (out64, out_bf16_bits)."""
+    yy = np.ascontiguousarray(y, np.float64)
+    H = yy.shape[1]
+    s = np.ascontiguousarray(np.asarray(sel, np.int64).reshape(-1))
+    gg = np.ascontiguousarray(np.asarray(g, np.float64).reshape(-1))
+    n = len(s) // k
+    out64 = np.zeros((n, H), np.float64)
+    outb = np.zeros((n, H), np.uint16)
+    lib().oracle_combine_f64(_p(yy, _f64p), H, _p(s, _i64p), _p(gg, _f64p), n, k, _p(out64, _f64p),
+                             _p(outb, _u16p))
+    return out64, outb
+
+
+def combine_f32(y: np.ndarray, sel, g, k: int) -> np.ndarray:
+    """Fixed-order fp32 combine (fmaf, ascending slot) -> bf16 bits [n, H]."""
+    yy = np.ascontiguousarray(y, np.float32)
+    H = yy.shape[1]
+    s = np.ascontiguousarray(np.asarray(sel, np.int64).reshape(-1))
+    gg = np.ascontiguousarray(np.asarray(g, np.float32).reshape(-1))
+    n = len(s) // k
+    outb = np.zeros((n, H), np.uint16)
+    lib().oracle_combine_f32(_p(yy, _f32p), H, _p(s, _i64p), _p(gg, _f32p), n, k, _p(outb, _u16p))
+    return outb
+
+
+def expert_of_rows(offsets: np.ndarray, rows) -> np.ndarray:
+    """Expert l of each row: the segment with offsets[l] <= row < offsets[l+1]."""
+    off = np.asarray(offsets, np.int64)
+    return (np.searchsorted(off, np.asarray(rows, np.int64), side="right") - 1).astype(np.int32)
+
+
+def layer_tokens(logits, x_bits, weights, P: int, N: int, k: int, E: int, H: int, I: int,
+                 tokens, pad: int = 256):
+    """The whole layer for a set of tokens: route all tokens, schedule all routes,
+    then dispatch, FFN and combine only the rows the chosen tokens need.
+
+    weights: (W1, W3, W2) dicts expert -> numpy uint16 arrays (only the experts
+    the chosen tokens use need to be present).
+    Returns dict with ids, gates32, gates64, sched, out64 [n,H], out_bf16 [n,H],
+    y rows per (token, slot) and h rows.
+    """
+    ids, g32, g64 = route_topk(logits, k)
+    sch = schedule(ids.reshape(P, N, k), P, N, k, E, pad)
+    toks = np.asarray(tokens, np.int64)
+    rr = sch["route_row"].reshape(P * N, k)
+    sel_rows = rr[toks].reshape(-1).astype(np.int64)
+    uniq, inv = np.unique(sel_rows, return_inverse=True)
+    xg = dispatch_rows(x_bits, N, sch["phi"], uniq)
+    ex = expert_of_rows(sch["offsets"], uniq)
+    h, y = ffn_rows(xg, ex, *weights, H=H, I=I)
+    out64, outb = combine_f64(y, inv.reshape(len(toks), k), g64[toks], k)
+    return dict(ids=ids, gates32=g32, gates64=g64, sched=sch, out64=out64, out_bf16=outb,
+                rows=uniq, row_index=inv.reshape(len(toks), k), xg=xg, h=h, y=y,
+                experts=ex)
