@@ -1,0 +1,57 @@
+// Internal launchers shared by the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// Kernels launched by this library in this process (moe_launch_count).
+void note_launches(int64_t n);
+
+// Number of SMs of the current device (cached per device).
+int device_sm_count();
+
+// A token slice [t0, t0+Tm) of every peer: the unit the schedule, dispatch,
+// FFN and combine work on (the whole input is t0 = 0, Tm = N).
+struct Slice {
+  int32_t t0, Tm;
+};
+
+// Step 1
+cudaError_t launch_route_topk(const float* logits, int32_t* ids, float* gates, int64_t n_tokens,
+                              int32_t E, int32_t k, cudaStream_t s);
+
+// Step 2
+constexpr int kSchedBlockRoutes = 2048;  // routes per counting block (8 warps x 256)
+size_t schedule_ws_bytes(int32_t P, int32_t N, int32_t k, int32_t E);
+cudaError_t launch_schedule(const int32_t* ids, const moe_shape_t& sh, Slice sl, int32_t* phi,
+                            int32_t* offsets, int32_t* counts, int32_t* route_row, int32_t* ws,
+                            int32_t* dev_status, cudaStream_t s);
+
+// Step 3a
+cudaError_t launch_dispatch(const uint16_t* x, const int32_t* phi, const int32_t* offsets,
+                            uint16_t* xg, const moe_shape_t& sh, int64_t rows_max,
+                            int32_t* dev_status, cudaStream_t s);
+
+// Step 3b (two kernels; ev_mid, if not null, is recorded between them)
+cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint16_t* W3,
+                              const uint16_t* W2, const int32_t* offsets, const int32_t* counts,
+                              uint16_t* h, float* y, const moe_shape_t& sh, int64_t rows_max,
+                              int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_mid);
+
+// Step 4
+cudaError_t launch_combine(const float* y, const int32_t* route_row, const float* gates,
+                           uint16_t* out, const moe_shape_t& sh, Slice sl, int64_t rows_max,
+                           int32_t* dev_status, cudaStream_t s);
+
+// Failure-detection self test (bounded wait on an mbarrier nothing completes).
+cudaError_t launch_selftest_wait(int32_t* dev_status, int64_t timeout_ns, cudaStream_t s);
+
+// Default limit of every bounded device wait.
+constexpr int64_t kWaitTimeoutNs = 1000000000ll;
+
+}  // namespace moe

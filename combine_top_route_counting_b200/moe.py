@@ -1,0 +1,243 @@
+"""Thin Python binding of libmoe_b200.so (the C ABI in include/moe.h).
+
+Argument marshalling only: each function checks dtypes, devices and
+contiguity of torch tensors and passes their device pointers, sizes and the
+current CUDA stream to the C entry point of the same name. Every step of the
+layer runs in the library's CUDA kernels; there is no Python or CPU fallback,
+and loading fails loudly when the shared library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+_lib = None
+
+MOE_OK = 0
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_INVALID_ARG", 2: "MOE_UNSUPPORTED_SHAPE",
+                3: "MOE_WORKSPACE_TOO_SMALL", 4: "MOE_CUDA_ERROR", 5: "MOE_DEVICE_TIMEOUT",
+                6: "MOE_BAD_EXPERT_ID", 7: "MOE_BAD_SCHEDULE"}
+DEV_BAD_EXPERT_ID = 0x1
+DEV_TIMEOUT = 0x2
+DEV_BAD_SCHEDULE = 0x4
+N_STAGE_EVENTS = 7
+STAGES = ("route", "schedule", "dispatch", "ffn_gemm1", "ffn_gemm2", "combine")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("P", ctypes.c_int32), ("N", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("pad", ctypes.c_int32)]
+
+    def __repr__(self):
+        return "Shape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+def shape(P: int, N: int, E: int, k: int, H: int = 0, I: int = 0, pad: int = 256) -> Shape:
+    return Shape(P, N, E, k, H, I, pad)
+
+
+_vp = ctypes.c_void_p
+_SIGS = {
+    "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "moe_status_from_device_flags": ([ctypes.c_int32], ctypes.c_int),
+    "moe_rows_max": ([ctypes.POINTER(Shape)], ctypes.c_int64),
+    "moe_schedule_workspace_bytes": ([ctypes.POINTER(Shape)], ctypes.c_size_t),
+    "moe_layer_workspace_bytes": ([ctypes.POINTER(Shape)], ctypes.c_size_t),
+    "moe_layer_host_workspace_bytes": ([ctypes.POINTER(Shape)], ctypes.c_size_t),
+    "moe_route_topk": ([_vp, _vp, _vp, ctypes.POINTER(Shape), _vp], ctypes.c_int),
+    "moe_schedule": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp, ctypes.POINTER(Shape),
+                      _vp], ctypes.c_int),
+    "moe_dispatch": ([_vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Shape), _vp], ctypes.c_int),
+    "moe_expert_ffn": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Shape), _vp],
+                       ctypes.c_int),
+    "moe_combine": ([_vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Shape), _vp], ctypes.c_int),
+    "moe_layer_forward": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int32, _vp, ctypes.c_size_t, _vp,
+                           ctypes.POINTER(Shape), _vp, ctypes.POINTER(_vp)], ctypes.c_int),
+    "moe_layer_forward_host": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int32, _vp,
+                                ctypes.c_size_t, _vp, ctypes.POINTER(Shape), _vp], ctypes.c_int),
+    "moe_launch_count": ([], ctypes.c_int64),
+    "moe_selftest_bounded_wait": ([_vp, ctypes.c_int64, _vp], ctypes.c_int),
+}
+
+
+def load():
+    """Load the shared library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -c 'import __graft_entry__ as g; g.build()'`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def exported_symbols():
+    return sorted(_SIGS)
+
+
+# ---------------------------------------------------------------- marshalling
+def _ptr(t: torch.Tensor | None, dtype: torch.dtype, name: str, device=True):
+    if t is None:
+        return None
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if device and not t.is_cuda:
+        raise TypeError(f"{name}: expected a CUDA tensor")
+    if not device and t.is_cuda:
+        raise TypeError(f"{name}: expected a host tensor")
+    if not t.is_contiguous():
+        raise TypeError(f"{name}: must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(status: int, where: str):
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+def status_string(status: int) -> str:
+    return load().moe_status_string(status).decode()
+
+
+def status_from_device_flags(flags: int) -> int:
+    return load().moe_status_from_device_flags(int(flags))
+
+
+def rows_max(sh: Shape) -> int:
+    return int(load().moe_rows_max(ctypes.byref(sh)))
+
+
+def schedule_workspace_bytes(sh: Shape) -> int:
+    return int(load().moe_schedule_workspace_bytes(ctypes.byref(sh)))
+
+
+def layer_workspace_bytes(sh: Shape) -> int:
+    return int(load().moe_layer_workspace_bytes(ctypes.byref(sh)))
+
+
+def layer_host_workspace_bytes(sh: Shape) -> int:
+    return int(load().moe_layer_host_workspace_bytes(ctypes.byref(sh)))
+
+
+def launch_count() -> int:
+    return int(load().moe_launch_count())
+
+
+# ---------------------------------------------------------------- entry points
+def moe_route_topk(logits, ids, gates, sh: Shape, stream=None):
+    _check(load().moe_route_topk(_ptr(logits, torch.float32, "logits"),
+                                 _ptr(ids, torch.int32, "ids"), _ptr(gates, torch.float32, "gates"),
+                                 ctypes.byref(sh), _stream(stream)), "moe_route_topk")
+
+
+def moe_schedule(ids, phi, offsets, counts, route_row, ws, dev_status, sh: Shape, stream=None):
+    _check(load().moe_schedule(_ptr(ids, torch.int32, "ids"), _ptr(phi, torch.int32, "phi"),
+                               _ptr(offsets, torch.int32, "offsets"),
+                               _ptr(counts, torch.int32, "counts"),
+                               _ptr(route_row, torch.int32, "route_row"),
+                               _ptr(ws, torch.uint8, "ws"), ws.numel(),
+                               _ptr(dev_status, torch.int32, "dev_status"), ctypes.byref(sh),
+                               _stream(stream)), "moe_schedule")
+
+
+def moe_dispatch(x, phi, offsets, xg, dev_status, sh: Shape, stream=None):
+    _check(load().moe_dispatch(_ptr(x, torch.bfloat16, "x"), _ptr(phi, torch.int32, "phi"),
+                               _ptr(offsets, torch.int32, "offsets"),
+                               _ptr(xg, torch.bfloat16, "xg"),
+                               _ptr(dev_status, torch.int32, "dev_status"), ctypes.byref(sh),
+                               _stream(stream)), "moe_dispatch")
+
+
+def moe_expert_ffn(xg, W1, W3, W2, offsets, counts, h, y, dev_status, sh: Shape, stream=None):
+    _check(load().moe_expert_ffn(_ptr(xg, torch.bfloat16, "xg"), _ptr(W1, torch.bfloat16, "W1"),
+                                 _ptr(W3, torch.bfloat16, "W3"), _ptr(W2, torch.bfloat16, "W2"),
+                                 _ptr(offsets, torch.int32, "offsets"),
+                                 _ptr(counts, torch.int32, "counts"),
+                                 _ptr(h, torch.bfloat16, "h"), _ptr(y, torch.float32, "y"),
+                                 _ptr(dev_status, torch.int32, "dev_status"), ctypes.byref(sh),
+                                 _stream(stream)), "moe_expert_ffn")
+
+
+def moe_combine(y, route_row, gates, out, dev_status, sh: Shape, stream=None):
+    _check(load().moe_combine(_ptr(y, torch.float32, "y"),
+                              _ptr(route_row, torch.int32, "route_row"),
+                              _ptr(gates, torch.float32, "gates"), _ptr(out, torch.bfloat16, "out"),
+                              _ptr(dev_status, torch.int32, "dev_status"), ctypes.byref(sh),
+                              _stream(stream)), "moe_combine")
+
+
+def _events(events):
+    if events is None:
+        return None
+    if len(events) != N_STAGE_EVENTS:
+        raise ValueError(f"need {N_STAGE_EVENTS} events")
+    arr = (ctypes.c_void_p * N_STAGE_EVENTS)()
+    for i, e in enumerate(events):
+        arr[i] = e.cuda_event if hasattr(e, "cuda_event") else int(e)
+    return ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+
+
+def moe_layer_forward(logits, x, W1, W3, W2, out, ws, dev_status, sh: Shape, minibatch_tokens=0,
+                      stream=None, stage_events=None):
+    _check(load().moe_layer_forward(_ptr(logits, torch.float32, "logits"),
+                                    _ptr(x, torch.bfloat16, "x"), _ptr(W1, torch.bfloat16, "W1"),
+                                    _ptr(W3, torch.bfloat16, "W3"), _ptr(W2, torch.bfloat16, "W2"),
+                                    _ptr(out, torch.bfloat16, "out"), int(minibatch_tokens),
+                                    _ptr(ws, torch.uint8, "ws"), ws.numel(),
+                                    _ptr(dev_status, torch.int32, "dev_status"),
+                                    ctypes.byref(sh), _stream(stream), _events(stage_events)),
+           "moe_layer_forward")
+
+
+def moe_layer_forward_host(logits_host, x_host, W1, W3, W2, out_host, ws, dev_status, sh: Shape,
+                           minibatch_tokens=0, stream=None):
+    _check(load().moe_layer_forward_host(
+        _ptr(logits_host, torch.float32, "logits_host", device=False),
+        _ptr(x_host, torch.bfloat16, "x_host", device=False), _ptr(W1, torch.bfloat16, "W1"),
+        _ptr(W3, torch.bfloat16, "W3"), _ptr(W2, torch.bfloat16, "W2"),
+        _ptr(out_host, torch.bfloat16, "out_host", device=False), int(minibatch_tokens),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _ptr(dev_status, torch.int32, "dev_status"),
+        ctypes.byref(sh), _stream(stream)), "moe_layer_forward_host")
+
+
+def moe_selftest_bounded_wait(dev_status, timeout_ns: int, stream=None):
+    _check(load().moe_selftest_bounded_wait(_ptr(dev_status, torch.int32, "dev_status"),
+                                            int(timeout_ns), _stream(stream)),
+           "moe_selftest_bounded_wait")
+
+
+# ---------------------------------------------------------------- buffers
+def alloc_schedule_outputs(sh: Shape, device="cuda"):
+    """Device buffers of moe_schedule: phi, offsets, counts, route_row, ws, dev_status."""
+    rm = rows_max(sh)
+    return dict(
+        phi=torch.empty((max(rm, 1), 2), dtype=torch.int32, device=device),
+        offsets=torch.empty(sh.E + 1, dtype=torch.int32, device=device),
+        counts=torch.empty((sh.E, sh.P), dtype=torch.int32, device=device),
+        route_row=torch.empty((sh.P, sh.N, sh.k), dtype=torch.int32, device=device),
+        ws=torch.empty(max(schedule_workspace_bytes(sh), 16), dtype=torch.uint8, device=device),
+        dev_status=torch.zeros(1, dtype=torch.int32, device=device),
+    )

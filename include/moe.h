@@ -1,0 +1,212 @@
+/*
+ * moe.h -- C ABI of libmoe_b200.so: the forward pass of one deterministic
+ * Mixture-of-Experts layer on one B200 (sm_100a).
+ *
+ * The layer has four steps:
+ *   1. top-k routing from router logits;
+ *   2. the pull-dispatch schedule table Phi, built on the device as a
+ *      single-pass counting sort;
+ *   3. a pull gather of the tokens into contiguous per-expert buffers and a
+ *      grouped SwiGLU expert FFN (bf16 operands, fp32 accumulation);
+ *   4. a gate-weighted combine back to token order in a fixed floating-point
+ *      order, so identical inputs give bitwise-identical outputs.
+ *
+ * Sources (page title, section):
+ *   "Mixture-of-Kittens: A MoE Megakernel for GB300 NVL72" (MoK notes),
+ *     section 2 "Push vs. Pull" (two-column pull table; on-device schedule
+ *     generation with counts T, M, offsets S and the stable cross-rank
+ *     position p), section 3 "The Goldilocks Minibatch Size T",
+ *     section 5 "Megakernel Fusion" (SwiGLU expert GEMMs).
+ *   "Scan once, scatter once", section "The fix is a counting sort" (count,
+ *     prefix, pad to 256 rows, scatter once).
+ *   "Beyond Peak TFLOPs", sections 2.A and 2.B (pull dispatch / push combine,
+ *     no dynamic allocation or host round trips) and its opening (bitwise
+ *     reproducible outputs from a fixed floating-point order).
+ *
+ * Expert-parallel peers are logical partitions of one GPU's memory: peer r
+ * owns tokens r*N .. r*N+N-1 of every [P*N, ...] token array.
+ *
+ * Conventions for every entry point:
+ *   - All pointers are DEVICE pointers unless the name ends in _host.
+ *     bf16 tensors are passed as uint16_t bit patterns. All arrays are dense,
+ *     row-major, and must be 16-byte aligned (256-byte alignment recommended).
+ *   - The caller owns and allocates every buffer; the library never allocates
+ *     device memory and never synchronises with the host. Work is enqueued on
+ *     `stream` (a cudaStream_t; NULL = the legacy default stream) and runs
+ *     asynchronously; results are valid once the stream has been synchronised.
+ *   - Errors found from the arguments alone are returned synchronously as a
+ *     moe_status_t, before anything is enqueued. Errors that depend on data
+ *     (an expert id outside [0,E), an inconsistent schedule, a device wait
+ *     that timed out) are OR-ed as MOE_DEV_* flags into *dev_status, which
+ *     the caller zeroes beforehand and reads after synchronising. Kernels never
+ *     trap: on bad data they skip the offending element and raise the flag.
+ *   - Calls that share buffers must not overlap on the GPU.
+ *   - Shape limits: 1 <= P <= 64; 0 <= N; 1 <= E <= 1024; 1 <= k <= min(E, 16);
+ *     P*N*k and the padded row count below 2^31. The expert FFN and the layer
+ *     additionally need H % 256 == 0, I % 128 == 0, pad % 128 == 0.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Problem shape. P peers x N tokens each, E experts, top-k routing, hidden
+ * size H, expert intermediate size I, expert segment padding `pad` rows
+ * (256 in the pages' scheduler). */
+typedef struct moe_shape {
+  int32_t P, N, E, k, H, I, pad;
+} moe_shape_t;
+
+typedef int moe_status_t;
+enum {
+  MOE_OK = 0,
+  MOE_INVALID_ARG = 1,          /* null pointer, negative size, misaligned buffer */
+  MOE_UNSUPPORTED_SHAPE = 2,    /* shape outside the limits above */
+  MOE_WORKSPACE_TOO_SMALL = 3,
+  MOE_CUDA_ERROR = 4,           /* a CUDA runtime call failed (e.g. no device) */
+  MOE_DEVICE_TIMEOUT = 5,       /* host view of MOE_DEV_TIMEOUT */
+  MOE_BAD_EXPERT_ID = 6,        /* host view of MOE_DEV_BAD_EXPERT_ID */
+  MOE_BAD_SCHEDULE = 7          /* host view of MOE_DEV_BAD_SCHEDULE */
+};
+
+/* Flags OR-ed into *dev_status by kernels. */
+#define MOE_DEV_BAD_EXPERT_ID 0x1  /* an id outside [0,E): that route is dropped */
+#define MOE_DEV_TIMEOUT       0x2  /* a bounded device wait gave up (~1 s) */
+#define MOE_DEV_BAD_SCHEDULE  0x4  /* offsets/Phi/route_row out of range: element skipped */
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(moe_status_t s);
+
+/* Status code for a set of MOE_DEV_* flags (the most severe one; MOE_OK if 0). */
+moe_status_t moe_status_from_device_flags(int32_t flags);
+
+/* Upper bound on the rows of the padded, expert-sorted layout:
+ * P*N*k + E*(pad-1), rounded up to a multiple of pad (and of 256).
+ * Phi, the gathered buffer xg, h and y are sized with it. -1 on a bad shape. */
+int64_t moe_rows_max(const moe_shape_t* shape);
+
+/* Bytes of scratch `ws` that moe_schedule needs for `shape`. */
+size_t moe_schedule_workspace_bytes(const moe_shape_t* shape);
+
+/* Bytes of scratch `ws` that moe_layer_forward needs (ids, gates, Phi,
+ * offsets, counts, route_row, the schedule's scratch, xg, h and y). */
+size_t moe_layer_workspace_bytes(const moe_shape_t* shape);
+
+/* Bytes of scratch for moe_layer_forward_host: the above plus device copies
+ * of the logits, the activations and the output. */
+size_t moe_layer_host_workspace_bytes(const moe_shape_t* shape);
+
+/* Step 1 -- top-k routing ("routing tensor" of MoK notes section 2; gates as
+ * the softmax over the chosen logits).
+ * logits: fp32 [P*N, E]. For each token the k largest logits are chosen in
+ * descending order, ties to the lower expert id; ids: int32 [P*N, k] (slot j
+ * = j-th largest); gates: fp32 [P*N, k], gates[t,j] = exp(l_j - l_0) /
+ * sum_j' exp(l_j' - l_0). Logits must be finite or -inf, with at least one
+ * finite logit per token. */
+moe_status_t moe_route_topk(const float* logits, int32_t* ids, float* gates,
+                            const moe_shape_t* shape, void* stream);
+
+/* Step 2 -- the pull-dispatch schedule Phi ("Scan once, scatter once", the
+ * four stages of "The fix is a counting sort"; placement of MoK notes
+ * section 2).
+ * ids: int32 [P, N, k]; route (r, q), q = i*k + j, is slot j of token i of
+ * peer r. With M[l,r] = routes of peer r to expert l, T[l] = sum_r M[l,r],
+ * Tp[l] = ceil(T[l]/pad)*pad and S the exclusive prefix sum of Tp:
+ *   offsets: int32 [E+1] = S (offsets[E] = rows in use);
+ *   counts:  int32 [E, P] = M;
+ *   phi:     int32 [moe_rows_max, 2]; row S[l]+p holds (src_rank, src_idx) =
+ *            (r, i) of the route whose stable rank within (l, r) is o (routes
+ *            of one peer in ascending q), where
+ *            p = sum_{r'} min(M[l,r'], o) + |{r' < r : M[l,r'] > o}|;
+ *            rows S[l]+T[l] .. S[l+1]-1 hold (-1,-1); rows >= offsets[E] are
+ *            not written;
+ *   route_row: int32 [P, N, k] = the Phi row of each route.
+ * ws: scratch of moe_schedule_workspace_bytes (contents irrelevant on entry).
+ * An id outside [0,E) raises MOE_DEV_BAD_EXPERT_ID, is not placed, and its
+ * route_row is -1. Each route is read twice (count, scatter). */
+moe_status_t moe_schedule(const int32_t* ids, int32_t* phi, int32_t* offsets, int32_t* counts,
+                          int32_t* route_row, void* ws, size_t ws_bytes, int32_t* dev_status,
+                          const moe_shape_t* shape, void* stream);
+
+/* Step 3a -- pull dispatch ("Beyond Peak TFLOPs" 2.A, MoK notes section 2:
+ * tokens land zero-copy in contiguous per-expert buffers).
+ * x: bf16 [P*N, H]; xg: bf16 [moe_rows_max, H]. For row < offsets[E]:
+ * xg[row] = x[src_rank*N + src_idx] with (src_rank, src_idx) = phi[row], and
+ * padding rows (src_rank < 0) are zero. Rows >= offsets[E] are not written.
+ * An out-of-range Phi entry raises MOE_DEV_BAD_SCHEDULE and zeroes the row. */
+moe_status_t moe_dispatch(const uint16_t* x, const int32_t* phi, const int32_t* offsets,
+                          uint16_t* xg, int32_t* dev_status, const moe_shape_t* shape,
+                          void* stream);
+
+/* Step 3b -- grouped SwiGLU expert FFN (MoK notes section 5), a persistent
+ * tcgen05 grouped GEMM pair with bf16 operands and fp32 accumulation.
+ * W1 (gate), W3 (up): bf16 [E, H, I]; W2 (down): bf16 [E, I, H].
+ * For every row in expert l's segment [offsets[l], offsets[l+1]):
+ *   h[row] = bf16_rne( silu(xg[row].W1[l]) * (xg[row].W3[l]) ),  h: bf16 [moe_rows_max, I]
+ *   y[row] = h[row].W2[l] (fp32),                                 y: fp32 [moe_rows_max, H]
+ * counts (int32 [E,P], may be NULL): when given, 128-row tiles that hold only
+ * padding rows are skipped and their h/y rows are left unwritten; rows that
+ * carry routes are always written. Each output element is computed by one
+ * CTA with a fixed K order: the result is bitwise deterministic.
+ * offsets must be non-decreasing multiples of 128 with offsets[E] <=
+ * moe_rows_max (else MOE_DEV_BAD_SCHEDULE, nothing written). */
+moe_status_t moe_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint16_t* W3,
+                            const uint16_t* W2, const int32_t* offsets, const int32_t* counts,
+                            uint16_t* h, float* y, int32_t* dev_status,
+                            const moe_shape_t* shape, void* stream);
+
+/* Step 4 -- push combine in a fixed floating-point order ("Scan once, scatter
+ * once" opening and "Beyond Peak TFLOPs" opening: bitwise-reproducible outputs).
+ * out[t] = bf16_rne(acc) with acc = 0.0f; acc = fmaf(gates[t,j], y[route_row[t,j]], acc)
+ * for j = 0..k-1 in ascending order. out: bf16 [P*N, H]. A route_row outside
+ * [0, moe_rows_max) contributes nothing and raises MOE_DEV_BAD_SCHEDULE. */
+moe_status_t moe_combine(const float* y, const int32_t* route_row, const float* gates,
+                         uint16_t* out, int32_t* dev_status, const moe_shape_t* shape,
+                         void* stream);
+
+/* Steps 1-4 in one call, all enqueued on `stream` with no host round trip.
+ * minibatch_tokens: transfer slice T in tokens per peer (MoK notes section 3);
+ * 0 or >= N = one slice. Slice s covers tokens [s*T, (s+1)*T) of every peer and
+ * runs schedule -> dispatch -> FFN -> combine on them; routing runs once over
+ * all tokens. Every output row is computed with the same arithmetic whatever
+ * the slicing, so out is bitwise identical for every T.
+ * ws: scratch of moe_layer_workspace_bytes. stage_events: NULL, or an array of
+ * 7 cudaEvent_t recorded (single-slice runs only) before routing, schedule,
+ * dispatch, FFN GEMM1, FFN GEMM2, combine, and after combine. */
+moe_status_t moe_layer_forward(const float* logits, const uint16_t* x, const uint16_t* W1,
+                               const uint16_t* W3, const uint16_t* W2, uint16_t* out,
+                               int32_t minibatch_tokens, void* ws, size_t ws_bytes,
+                               int32_t* dev_status, const moe_shape_t* shape, void* stream,
+                               void* const* stage_events);
+
+/* moe_layer_forward with HOST inputs and output: logits_host fp32 [P*N, E],
+ * x_host bf16 [P*N, H] and out_host bf16 [P*N, H] live in host memory (pinned
+ * memory makes the copies asynchronous); the weights, ws (of
+ * moe_layer_host_workspace_bytes) and dev_status are device memory. The
+ * host->device copies, the layer and the device->host copy are all enqueued
+ * on `stream`; out_host is valid after the stream is synchronised. */
+moe_status_t moe_layer_forward_host(const float* logits_host, const uint16_t* x_host,
+                                    const uint16_t* W1, const uint16_t* W3, const uint16_t* W2,
+                                    uint16_t* out_host, int32_t minibatch_tokens, void* ws,
+                                    size_t ws_bytes, int32_t* dev_status,
+                                    const moe_shape_t* shape, void* stream);
+
+/* Number of kernels this library has launched in the calling process. */
+int64_t moe_launch_count(void);
+
+/* Failure-detection self test: launches one kernel that waits, with the same
+ * bounded wait the FFN pipeline uses, on an mbarrier that nothing completes,
+ * giving up after timeout_ns nanoseconds; it then raises MOE_DEV_TIMEOUT in
+ * *dev_status. The context stays usable. */
+moe_status_t moe_selftest_bounded_wait(int32_t* dev_status, int64_t timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

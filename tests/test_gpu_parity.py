@@ -1,0 +1,346 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Bit-exact on ids, Phi, offsets, counts, route_row, the gathered buffer and the
+fixed-order combine; within the stated tolerance on gates, expert outputs and
+the layer output; bitwise run-to-run and across transfer-slice sizes.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from combine_top_route_counting_b200 import inputs
+from tests.helpers import (OUT_TOL, Y_TOL, bf16_to_f64, bits, expert_weights_host, literal_rms_err,
+                           rms_floor_err, sha)
+
+pytestmark = pytest.mark.gpu
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+DEV = "cuda"
+
+
+def _sched_gpu(moe, ids_dev, P, N, k, E, pad=256):
+    sh = moe.shape(P, N, E, k, pad=pad)
+    b = moe.alloc_schedule_outputs(sh)
+    b["phi"].fill_(-7)
+    moe.moe_schedule(ids_dev, b["phi"], b["offsets"], b["counts"], b["route_row"], b["ws"],
+                     b["dev_status"], sh)
+    torch.cuda.synchronize()
+    return {k_: v.cpu().numpy() for k_, v in b.items()}
+
+
+def _assert_sched_equal(g, o):
+    rows = int(o["offsets"][-1])
+    assert (g["offsets"] == o["offsets"]).all()
+    assert (g["counts"] == o["counts"]).all()
+    assert (g["route_row"] == o["route_row"]).all()
+    assert (g["phi"][:rows] == o["phi"]).all()
+    assert int(g["dev_status"][0]) == 0
+
+
+# ---------------------------------------------------------------- schedule
+def test_schedule_handworked(cuda_lib):
+    moe = cuda_lib
+    for c in json.load(open(os.path.join(GOLD, "schedule_handworked.json")))["cases"]:
+        ids = torch.tensor(c["ids"], dtype=torch.int32, device=DEV)
+        g = _sched_gpu(moe, ids, c["P"], c["N"], c["k"], c["E"], c["pad"])
+        rows = c["offsets"][-1]
+        assert g["phi"][:rows].tolist() == c["phi"]
+        assert g["offsets"].tolist() == c["offsets"]
+        assert g["counts"].tolist() == c["counts"]
+        assert g["route_row"].tolist() == c["route_row"]
+
+
+def test_schedule_sweep_945(cuda_lib):
+    moe = cuda_lib
+    n = 0
+    for P, N, E, k, ids in inputs.sweep_cases():
+        g = _sched_gpu(moe, ids.to(DEV), P, N, k, E)
+        o = oracle.schedule(ids.numpy(), P, N, k, E, 256)
+        _assert_sched_equal(g, o)
+        n += 1
+    assert n == 945
+
+
+def test_schedule_full_scheduler_workload(cuda_lib):
+    moe = cuda_lib
+    w = inputs.WORKLOADS["sched"]
+    ids = inputs.make_sched_ids(w)
+    g = _sched_gpu(moe, ids.to(DEV), w.P, w.N, w.k, w.E)
+    o = oracle.schedule(ids.numpy(), w.P, w.N, w.k, w.E, 256)
+    _assert_sched_equal(g, o)
+    assert o["reads"] == 917504
+
+
+@pytest.mark.parametrize("case", ["empty", "one_expert", "k_eq_E", "hot", "many_blocks", "P64"])
+def test_schedule_edge_cases(cuda_lib, case):
+    moe = cuda_lib
+    if case == "empty":
+        P, N, E, k = 3, 0, 5, 2
+        ids = torch.zeros((P, N, k), dtype=torch.int32)
+    elif case == "one_expert":
+        P, N, E, k = 4, 1000, 1, 1
+        ids = torch.zeros((P, N, k), dtype=torch.int32)
+    elif case == "k_eq_E":
+        P, N, E, k = 2, 300, 6, 6
+        ids = inputs.make_ids_uniform(P, N, E, k, seed=11)
+    elif case == "hot":  # every route of peer 0 to expert 3, others uniform
+        P, N, E, k = 5, 900, 40, 4
+        ids = inputs.make_ids_uniform(P, N, E, k, seed=12)
+        ids[0, :, 0] = 3
+        ids[0, :, 1:] = torch.where(ids[0, :, 1:] == 3, torch.full_like(ids[0, :, 1:], 7),
+                                    ids[0, :, 1:])
+    elif case == "many_blocks":  # ragged last block, several blocks per peer
+        P, N, E, k = 3, 5000, 17, 3
+        ids = inputs.make_ids_uniform(P, N, E, k, seed=13)
+    else:
+        P, N, E, k = 64, 200, 256, 16
+        ids = inputs.make_ids_uniform(P, N, E, k, seed=14)
+    g = _sched_gpu(moe, ids.to(DEV), P, N, k, E)
+    o = oracle.schedule(ids.numpy(), P, N, k, E, 256)
+    _assert_sched_equal(g, o)
+
+
+def test_schedule_bad_expert_id_flags_and_drops(cuda_lib):
+    moe = cuda_lib
+    P, N, E, k = 2, 50, 8, 2
+    ids = inputs.make_ids_uniform(P, N, E, k, seed=21)
+    bad = ids.clone()
+    bad[1, 7, 1] = 99
+    g = _sched_gpu(moe, bad.to(DEV), P, N, k, E)
+    assert int(g["dev_status"][0]) & moe.DEV_BAD_EXPERT_ID
+    assert g["route_row"][1, 7, 1] == -1
+    assert moe.status_from_device_flags(int(g["dev_status"][0])) == 6
+    # the other routes still form a valid schedule of their own
+    placed = g["route_row"].reshape(-1)
+    placed = placed[placed >= 0]
+    assert len(np.unique(placed)) == P * N * k - 1
+
+
+# ---------------------------------------------------------------- routing
+@pytest.mark.parametrize("name", ["tiny", "mid", "kimi", "zipf"])
+def test_route_topk(cuda_lib, name):
+    moe = cuda_lib
+    w = inputs.WORKLOADS[name]
+    lg = inputs.make_logits(w)
+    sh = moe.shape(**w.shape())
+    ids = torch.empty((w.n_tokens, w.k), dtype=torch.int32, device=DEV)
+    gates = torch.empty((w.n_tokens, w.k), dtype=torch.float32, device=DEV)
+    moe.moe_route_topk(lg.to(DEV), ids, gates, sh)
+    torch.cuda.synchronize()
+    o_ids, o_g32, o_g64 = oracle.route_topk(lg, w.k)
+    assert (ids.cpu().numpy() == o_ids).all()
+    g = gates.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(g - o_g64) / o_g64) < 1e-6   # a few fp32 ulp (expf + divide)
+    if w.n_empty:
+        assert not np.isin(o_ids, inputs.empty_experts(w)).any()
+
+
+def test_route_topk_ties(cuda_lib):
+    moe = cuda_lib
+    w = json.load(open(os.path.join(GOLD, "worked_numbers.json")))["topk_ties"]
+    row = [float(v) for v in w["logits"]]
+    lg = torch.tensor([row] * 3, dtype=torch.float32)
+    lg[1] = torch.tensor([0.0] * 5)  # all tied: lowest ids first
+    sh = moe.shape(1, 3, 5, w["k"])
+    ids = torch.empty((3, w["k"]), dtype=torch.int32, device=DEV)
+    gates = torch.empty((3, w["k"]), dtype=torch.float32, device=DEV)
+    moe.moe_route_topk(lg.to(DEV), ids, gates, sh)
+    o_ids, _, o_g64 = oracle.route_topk(lg, w["k"])
+    assert ids.cpu().numpy()[0].tolist() == w["ids"]
+    assert (ids.cpu().numpy() == o_ids).all()
+    np.testing.assert_allclose(gates.cpu().numpy(), o_g64, rtol=1e-6)
+
+
+# ---------------------------------------------------------------- stages on small layers
+def _stage_run(moe, w, W1, W3, W2, lg, x):
+    """Run every stage through its own entry point; return device tensors."""
+    sh = moe.shape(**w.shape())
+    T, k = w.n_tokens, w.k
+    ids = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    gates = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    moe.moe_route_topk(lg, ids, gates, sh)
+    b = moe.alloc_schedule_outputs(sh)
+    moe.moe_schedule(ids, b["phi"], b["offsets"], b["counts"], b["route_row"], b["ws"],
+                     b["dev_status"], sh)
+    rm = moe.rows_max(sh)
+    xg = torch.empty((rm, w.H), dtype=torch.bfloat16, device=DEV)
+    moe.moe_dispatch(x, b["phi"], b["offsets"], xg, b["dev_status"], sh)
+    h = torch.empty((rm, w.I), dtype=torch.bfloat16, device=DEV)
+    y = torch.empty((rm, w.H), dtype=torch.float32, device=DEV)
+    moe.moe_expert_ffn(xg, W1, W3, W2, b["offsets"], b["counts"], h, y, b["dev_status"], sh)
+    out = torch.empty((T, w.H), dtype=torch.bfloat16, device=DEV)
+    moe.moe_combine(y, b["route_row"], gates, out, b["dev_status"], sh)
+    torch.cuda.synchronize()
+    return dict(ids=ids, gates=gates, xg=xg, h=h, y=y, out=out, **b)
+
+
+def test_tiny_all_stages_vs_oracle(cuda_lib):
+    moe = cuda_lib
+    w = inputs.WORKLOADS["tiny"]
+    lg, x = inputs.make_logits(w), inputs.make_x(w)
+    W1, W3, W2 = inputs.make_weights(w)
+    r = _stage_run(moe, w, W1.to(DEV), W3.to(DEV), W2.to(DEV), lg.to(DEV), x.to(DEV))
+    assert int(r["dev_status"].item()) == 0
+    o_ids, o_g32, o_g64 = oracle.route_topk(lg, w.k)
+    s = oracle.schedule(o_ids.reshape(w.P, w.N, w.k), w.P, w.N, w.k, w.E, 256)
+    g = {k_: r[k_].cpu().numpy() for k_ in ("phi", "offsets", "counts", "route_row")}
+    g["dev_status"] = r["dev_status"].cpu().numpy()
+    _assert_sched_equal(g, s)
+    rows = int(s["offsets"][-1])
+    # dispatch: bit-exact on every row in use, padding rows zero
+    o_xg = oracle.dispatch_rows(bits(x), w.N, s["phi"], np.arange(rows))
+    assert (bits(r["xg"][:rows]) == o_xg).all()
+    # FFN on every row that carries a route
+    real = np.nonzero(s["phi"][:, 0] >= 0)[0]
+    ex = oracle.expert_of_rows(s["offsets"], real)
+    Wd = expert_weights_host(W1, W3, W2, range(w.E))
+    o_h, o_y = oracle.ffn_rows(o_xg[real], ex, *Wd, H=w.H, I=w.I)
+    gh = bits(r["h"][torch.from_numpy(real).to(DEV)])
+    assert (gh == o_h).mean() > 0.995
+    gy = r["y"][torch.from_numpy(real).to(DEV)].cpu().numpy()
+    assert rms_floor_err(gy, o_y) < Y_TOL
+    # combine: bit-exact against the fixed-order definition on the GPU's own y and gates
+    y_np = r["y"].cpu().numpy()
+    exp = oracle.combine_f32(y_np, g["route_row"].reshape(-1, w.k), r["gates"].cpu().numpy(), w.k)
+    assert (bits(r["out"]) == exp).all()
+    # end to end against the oracle's fp64 layer output
+    res = oracle.layer_tokens(lg, bits(x), Wd, w.P, w.N, w.k, w.E, w.H, w.I, range(w.n_tokens))
+    assert rms_floor_err(bf16_to_f64(bits(r["out"])), res["out64"]) < OUT_TOL
+
+
+def test_ffn_no_counts_computes_padding_rows(cuda_lib):
+    """Without counts the FFN also computes padding tiles: zero rows give zero h and y."""
+    moe = cuda_lib
+    w = inputs.WORKLOADS["tiny"]
+    lg, x = inputs.make_logits(w), inputs.make_x(w)
+    W1, W3, W2 = [t.to(DEV) for t in inputs.make_weights(w)]
+    r = _stage_run(moe, w, W1, W3, W2, lg.to(DEV), x.to(DEV))
+    sh = moe.shape(**w.shape())
+    rows = int(r["offsets"][-1].item())
+    h2 = torch.full_like(r["h"], 7.0)
+    y2 = torch.full_like(r["y"], 7.0)
+    moe.moe_expert_ffn(r["xg"], W1, W3, W2, r["offsets"], None, h2, y2, r["dev_status"], sh)
+    torch.cuda.synchronize()
+    pad = torch.from_numpy(np.nonzero(r["phi"][:rows, 0].cpu().numpy() < 0)[0]).to(DEV)
+    assert (y2[pad] == 0).all() and (h2[pad].float() == 0).all()
+    real = torch.from_numpy(np.nonzero(r["phi"][:rows, 0].cpu().numpy() >= 0)[0]).to(DEV)
+    assert torch.equal(y2[real], r["y"][real]) and torch.equal(h2[real], r["h"][real])
+
+
+def test_mid_stages_sampled(cuda_lib):
+    moe = cuda_lib
+    w = inputs.WORKLOADS["mid"]
+    lg, x = inputs.make_logits(w), inputs.make_x(w)
+    W1, W3, W2 = inputs.make_weights(w)
+    r = _stage_run(moe, w, W1.to(DEV), W3.to(DEV), W2.to(DEV), lg.to(DEV), x.to(DEV))
+    assert int(r["dev_status"].item()) == 0
+    o_ids, _, o_g64 = oracle.route_topk(lg, w.k)
+    assert (r["ids"].cpu().numpy() == o_ids).all()
+    s = oracle.schedule(o_ids.reshape(w.P, w.N, w.k), w.P, w.N, w.k, w.E, 256)
+    g = {k_: r[k_].cpu().numpy() for k_ in ("phi", "offsets", "counts", "route_row", "dev_status")}
+    _assert_sched_equal(g, s)
+    rows = int(s["offsets"][-1])
+    o_xg = oracle.dispatch_rows(bits(x), w.N, s["phi"], np.arange(rows))
+    assert (bits(r["xg"][:rows]) == o_xg).all()
+    # FFN on sampled rows: first/last row of several experts plus random rows
+    rng = np.random.default_rng(5)
+    real = np.nonzero(s["phi"][:, 0] >= 0)[0]
+    pick = np.unique(np.concatenate([real[:3], real[-3:], rng.choice(real, 250, replace=False)]))
+    ex = oracle.expert_of_rows(s["offsets"], pick)
+    Wd = expert_weights_host(W1, W3, W2, ex)
+    o_h, o_y = oracle.ffn_rows(o_xg[pick], ex, *Wd, H=w.H, I=w.I)
+    idx = torch.from_numpy(pick).to(DEV)
+    assert (bits(r["h"][idx]) == o_h).mean() > 0.995
+    assert rms_floor_err(r["y"][idx].cpu().numpy(), o_y) < Y_TOL
+    # combine bit-exact on sampled tokens
+    toks = inputs.sample_tokens(w.n_tokens, 300, seed=2)
+    rr = g["route_row"].reshape(-1, w.k)[toks]
+    yt = r["y"][torch.from_numpy(np.unique(rr)).to(DEV)].cpu().numpy()
+    remap = np.searchsorted(np.unique(rr), rr)
+    exp = oracle.combine_f32(yt, remap, r["gates"].cpu().numpy()[toks], w.k)
+    assert (bits(r["out"])[toks] == exp).all()
+
+
+# ---------------------------------------------------------------- whole layer
+_LAYER_CACHE = {}
+
+
+def _layer_inputs(name):
+    if name not in _LAYER_CACHE:
+        _LAYER_CACHE.clear()
+        torch.cuda.empty_cache()
+        w = inputs.WORKLOADS[name]
+        big = w.H * w.I * w.E > 1e9
+        lg, x = inputs.make_logits(w), inputs.make_x(w)
+        W = inputs.make_weights(w, device=DEV if big else "cpu")
+        _LAYER_CACHE[name] = (w, lg, x, W)
+    return _LAYER_CACHE[name]
+
+
+def _layer_gpu(moe, w, lg_d, x_d, Wd, minibatch=0, ws=None):
+    sh = moe.shape(**w.shape())
+    if ws is None:
+        ws = torch.empty(moe.layer_workspace_bytes(sh), dtype=torch.uint8, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = torch.empty((w.n_tokens, w.H), dtype=torch.bfloat16, device=DEV)
+    moe.moe_layer_forward(lg_d, x_d, *Wd, out, ws, st, sh, minibatch_tokens=minibatch)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    return out, ws
+
+
+@pytest.mark.parametrize("name,n_tok", [("tiny", 512), ("mid", 96), ("kimi", 6), ("zipf", 6)])
+def test_layer_vs_oracle(cuda_lib, name, n_tok):
+    moe = cuda_lib
+    w, lg, x, W = _layer_inputs(name)
+    Wd = [t.to(DEV) for t in W]
+    out, ws = _layer_gpu(moe, w, lg.to(DEV), x.to(DEV), Wd)
+    toks = inputs.sample_tokens(w.n_tokens, n_tok, seed=w.wid)
+    o_ids, _, _ = oracle.route_topk(lg[toks], w.k)
+    Wh = expert_weights_host(*Wd, np.unique(o_ids))
+    res = oracle.layer_tokens(lg, bits(x), Wh, w.P, w.N, w.k, w.E, w.H, w.I, toks)
+    got = bf16_to_f64(bits(out[torch.tensor(toks, device=DEV)]))
+    err = rms_floor_err(got, res["out64"])
+    print(f"{name}: rms-floor err {err:.3e}, literal max|d|/rms {literal_rms_err(got, res['out64']):.3e}")
+    assert err < OUT_TOL
+    if name == "zipf":
+        ids_all = res["ids"]
+        assert not np.isin(ids_all, inputs.empty_experts(w)).any()
+        counts = np.bincount(ids_all.reshape(-1), minlength=w.E)
+        assert counts.max() > 0.10 * ids_all.size, "a hot expert takes >10% of routes"
+        s = res["sched"]
+        assert (np.diff(s["offsets"])[inputs.empty_experts(w)] == 0).all()
+
+
+@pytest.mark.parametrize("name", ["tiny", "mid", "kimi"])
+def test_layer_bitwise_deterministic_and_slice_invariant(cuda_lib, name):
+    moe = cuda_lib
+    w, lg, x, W = _layer_inputs(name)
+    Wd = [t.to(DEV) for t in W]
+    lg_d, x_d = lg.to(DEV), x.to(DEV)
+    out0, ws = _layer_gpu(moe, w, lg_d, x_d, Wd)
+    h0 = sha(out0)
+    for _ in range(2):
+        out1, _ = _layer_gpu(moe, w, lg_d, x_d, Wd, ws=ws)
+        assert sha(out1) == h0
+    for T in ([w.minibatch] if w.minibatch else []) + [max(1, w.N // 3), 97]:
+        outT, _ = _layer_gpu(moe, w, lg_d, x_d, Wd, minibatch=T, ws=ws)
+        assert sha(outT) == h0, f"transfer slice {T} changed the output"
+
+
+def test_layer_host_entry_matches_device_entry(cuda_lib):
+    moe = cuda_lib
+    w, lg, x, W = _layer_inputs("mid")
+    Wd = [t.to(DEV) for t in W]
+    out_d, _ = _layer_gpu(moe, w, lg.to(DEV), x.to(DEV), Wd)
+    sh = moe.shape(**w.shape())
+    ws = torch.empty(moe.layer_host_workspace_bytes(sh), dtype=torch.uint8, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out_h = torch.empty((w.n_tokens, w.H), dtype=torch.bfloat16).pin_memory()
+    moe.moe_layer_forward_host(lg.pin_memory(), x.pin_memory(), *Wd, out_h, ws, st, sh)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert torch.equal(out_h, out_d.cpu())

@@ -1,0 +1,77 @@
+"""Failure detection on the GPU without a fault: bounded device waits and the
+error paths of the C ABI."""
+import ctypes
+
+import pytest
+import torch
+
+from combine_top_route_counting_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def test_bounded_wait_times_out_and_context_survives(cuda_lib):
+    moe = cuda_lib
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    moe.moe_selftest_bounded_wait(st, 20_000_000)  # 20 ms on an mbarrier nothing completes
+    torch.cuda.synchronize()
+    assert int(st.item()) & moe.DEV_TIMEOUT
+    assert moe.status_from_device_flags(int(st.item())) == 5
+    # the context is still usable
+    a = torch.arange(10, device="cuda")
+    assert int(a.sum().item()) == 45
+
+
+def test_host_side_errors(cuda_lib):
+    moe = cuda_lib
+    sh = moe.shape(1, 16, 8, 2, 256, 128)
+    L = moe.load()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    # null pointers
+    assert L.moe_route_topk(None, None, None, ctypes.byref(sh), None) == 1
+    # unsupported shapes
+    bad = moe.shape(1, 16, 8, 9)  # k > E
+    assert moe.rows_max(bad) == -1
+    assert moe.layer_workspace_bytes(moe.shape(1, 16, 8, 2, 200, 128)) == 0  # H % 256 != 0
+    # workspace too small
+    w = inputs.WORKLOADS["tiny"]
+    x = torch.zeros((w.n_tokens, w.H), dtype=torch.bfloat16, device="cuda")
+    lg = torch.zeros((w.n_tokens, w.E), dtype=torch.float32, device="cuda")
+    W1 = torch.zeros((w.E, w.H, w.I), dtype=torch.bfloat16, device="cuda")
+    W2 = torch.zeros((w.E, w.I, w.H), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty_like(x)
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    shw = moe.shape(**w.shape())
+    with pytest.raises(moe.MoeError) as e:
+        moe.moe_layer_forward(lg, x, W1, W1, W2, out, ws, st, shw)
+    assert e.value.status == 3
+    with pytest.raises(TypeError):
+        moe.moe_layer_forward(lg.cpu(), x, W1, W1, W2, out, ws, st, shw)
+
+
+def test_corrupt_schedule_is_flagged_not_faulted(cuda_lib):
+    moe = cuda_lib
+    w = inputs.WORKLOADS["tiny"]
+    sh = moe.shape(**w.shape())
+    rm = moe.rows_max(sh)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    # offsets beyond rows_max: dispatch and FFN refuse and flag
+    offsets = torch.full((w.E + 1,), rm + 256, dtype=torch.int32, device="cuda")
+    offsets[0] = 0
+    phi = torch.full((rm, 2), -1, dtype=torch.int32, device="cuda")
+    x = torch.zeros((w.n_tokens, w.H), dtype=torch.bfloat16, device="cuda")
+    xg = torch.zeros((rm, w.H), dtype=torch.bfloat16, device="cuda")
+    moe.moe_dispatch(x, phi, offsets, xg, st, sh)
+    W1 = torch.zeros((w.E, w.H, w.I), dtype=torch.bfloat16, device="cuda")
+    W2 = torch.zeros((w.E, w.I, w.H), dtype=torch.bfloat16, device="cuda")
+    h = torch.zeros((rm, w.I), dtype=torch.bfloat16, device="cuda")
+    y = torch.zeros((rm, w.H), dtype=torch.float32, device="cuda")
+    moe.moe_expert_ffn(xg, W1, W1, W2, offsets, None, h, y, st, sh)
+    # route_row out of range: combine skips the slot and flags
+    rr = torch.full((w.n_tokens, w.k), rm + 5, dtype=torch.int32, device="cuda")
+    g = torch.ones((w.n_tokens, w.k), dtype=torch.float32, device="cuda")
+    out = torch.empty((w.n_tokens, w.H), dtype=torch.bfloat16, device="cuda")
+    moe.moe_combine(y, rr, g, out, st, sh)
+    torch.cuda.synchronize()
+    assert int(st.item()) & moe.DEV_BAD_SCHEDULE
+    assert (out.float() == 0).all()

@@ -1,0 +1,84 @@
+"""The C-ABI library loads without a GPU and exports every symbol the header
+declares; host-side checks return before any CUDA call (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from combine_top_route_counting_b200 import moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from combine_top_route_counting_b200 import build
+    build.build()
+    return moe.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = header_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in moe.h but not exported"
+    assert sorted(moe.exported_symbols()) == names, "binding covers exactly the header's functions"
+
+
+def test_host_only_queries(lib):
+    sh = moe.shape(8, 7168, 384, 8, 7168, 2048)
+    # rows_max = P*N*k + E*(pad-1) rounded up to 256
+    assert moe.rows_max(sh) == (8 * 7168 * 8 + 384 * 255 + 255) // 256 * 256
+    assert moe.schedule_workspace_bytes(sh) == 8 * 28 * 384 * 4   # [P][blocks of 2048 routes][E]
+    ws = moe.layer_workspace_bytes(sh)
+    rm = moe.rows_max(sh)
+    assert ws >= rm * (7168 * 2 + 2048 * 2 + 7168 * 4)
+    assert moe.layer_host_workspace_bytes(sh) > ws
+    assert moe.status_string(0) == "MOE_OK" and moe.status_string(3) == "MOE_WORKSPACE_TOO_SMALL"
+    assert moe.status_from_device_flags(0) == 0
+    assert moe.status_from_device_flags(moe.DEV_BAD_EXPERT_ID) == 6
+    assert moe.status_from_device_flags(moe.DEV_TIMEOUT | moe.DEV_BAD_EXPERT_ID) == 5
+
+
+@pytest.mark.parametrize("bad", [dict(P=0), dict(P=65), dict(E=0), dict(E=1025), dict(k=0),
+                                 dict(k=17), dict(k=9, E=8), dict(N=-1), dict(pad=0)])
+def test_shape_limits(lib, bad):
+    args = dict(P=2, N=16, E=8, k=2, H=256, I=128, pad=256)
+    args.update(bad)
+    sh = moe.shape(**args)
+    assert moe.rows_max(sh) == -1
+    assert moe.layer_workspace_bytes(sh) == 0
+
+
+@pytest.mark.parametrize("H,I,pad", [(128, 128, 256), (384, 128, 256), (256, 64, 256),
+                                     (256, 128, 64)])
+def test_ffn_shape_limits(lib, H, I, pad):
+    sh = moe.shape(2, 16, 8, 2, H, I, pad)
+    assert moe.layer_workspace_bytes(sh) == 0
+
+
+def test_argument_errors_return_before_cuda(lib):
+    sh = moe.shape(1, 16, 8, 2, 256, 128)
+    L = lib
+    assert L.moe_route_topk(None, None, None, ctypes.byref(sh), None) == 1
+    assert L.moe_route_topk(None, None, None, None, None) == 1
+    assert L.moe_schedule(None, None, None, None, None, None, 0, None, ctypes.byref(sh), None) == 1
+    assert L.moe_expert_ffn(*([None] * 9), ctypes.byref(sh), None) == 1
+    assert L.moe_layer_forward(*([None] * 6), 0, None, 0, None, ctypes.byref(sh), None, None) == 1
+    assert L.moe_selftest_bounded_wait(None, 1000, None) == 1
+    # misaligned pointers are rejected
+    assert L.moe_combine(ctypes.c_void_p(8), ctypes.c_void_p(16), ctypes.c_void_p(16),
+                         ctypes.c_void_p(16), ctypes.c_void_p(16), ctypes.byref(sh), None) == 1
+    # negative minibatch
+    p = ctypes.c_void_p(256)
+    assert L.moe_layer_forward(p, p, p, p, p, p, -1, p, 1 << 40, p, ctypes.byref(sh), None,
+                               None) == 1
+    # workspace too small
+    assert L.moe_layer_forward(p, p, p, p, p, p, 0, p, 16, p, ctypes.byref(sh), None, None) == 3
