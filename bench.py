@@ -1,0 +1,452 @@
+"""Benchmark of the deterministic MoE layer forward on B200.
+
+python bench.py --gpus N --steps K --warmup W [--workload kimi] [--impl ours|reference]
+
+One step = one moe_layer_forward over one batch of the workload (routing,
+schedule Phi, dispatch, grouped SwiGLU FFN, combine), inputs resident in HBM.
+With N > 1 (launched by torchrun) every rank runs an independent replica on
+its own GPU (the layer is not sharded here): value = tokens of all ranks /
+max-over-ranks device time. Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (test infrastructure) on a bounded
+sample of the same workload on the host cores, as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer fwd tokens/s @1 B200; Φ build µs; % of tensor/HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
+
+
+def env_rank():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sus=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=FALLBACK_HBM_GBS, bf16=FALLBACK_BF16_TFLOPS,
+                bf16_sus=FALLBACK_BF16_TFLOPS_SUSTAINED, source="fallback")
+
+
+def workload_desc(w) -> str:
+    return (f"{w.name}: P={w.P} peers x {w.N} tokens, H={w.H}, I={w.I}, E={w.E}, top-{w.k}, "
+            f"pad {w.pad}")
+
+
+# ---------------------------------------------------------------- algorithmic work
+def algorithmic_work(w, rows_used: int, rows_real: int):
+    """Bytes / flops each stage must move or compute (real routes only)."""
+    T, R, H, I, E, k = w.n_tokens, w.n_routes, w.H, w.I, w.E, w.k
+    return {
+        "route": dict(bytes=T * E * 4 + R * 8),
+        "schedule": dict(bytes=2 * R * 4 + rows_used * 8 + R * 4),
+        "dispatch": dict(bytes=R * H * 2 + rows_used * H * 2),
+        "ffn_gemm1": dict(flops=2 * rows_real * H * 2 * I),
+        "ffn_gemm2": dict(flops=2 * rows_real * I * H),
+        "combine": dict(bytes=R * H * 4 + T * H * 2 + R * 8),
+    }
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            self.fh = os.fdopen(fd, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], [], set()
+        for line in open(self.path):
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 10:
+                continue
+            if self.uuid and self.uuid not in f[1].lower().replace("gpu-", ""):
+                continue
+            try:
+                sm.append(float(f[2]))
+                mx.append(float(f[3]))
+            except ValueError:
+                continue
+            for name, col in (("hw_slowdown", 6), ("hw_thermal_slowdown", 7),
+                              ("sw_thermal_slowdown", 8), ("sw_power_cap", 9)):
+                if f[col].lower().startswith("active"):
+                    reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def gpu_uuid(dev) -> str | None:
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid).lower()
+        return u.replace("gpu-", "") or None
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------- ranks
+def reduce_max(values, group_ready: bool, device=None):
+    """Element-wise max over ranks (device time is reported as the slowest rank)."""
+    if not group_ready:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().tolist()
+
+
+def init_dist(world: int, local_rank: int, backend: str = "nccl"):
+    if world <= 1:
+        return False
+    import torch
+    import torch.distributed as dist
+    kw = dict(backend=backend, timeout=datetime.timedelta(seconds=300))
+    if backend == "nccl":
+        kw["device_id"] = torch.device("cuda", local_rank)
+    dist.init_process_group(**kw)
+    return True
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+def oracle_sample(w, lg, x_cpu, W_dev, row_budget_s: float, n_comb: int = 256):
+    """Time the CPU oracle on a bounded sample of the workload and scale it to
+    tokens/s: route + schedule over the whole batch, dispatch + FFN of R rows
+    of one expert (R grown until the budget), combine of n_comb tokens."""
+    import numpy as np
+    import torch
+
+    import oracle
+
+    cores = oracle.num_threads()
+    t0 = time.perf_counter()
+    ids, g32, g64 = oracle.route_topk(lg, w.k)
+    s = oracle.schedule(ids.reshape(w.P, w.N, w.k), w.P, w.N, w.k, w.E, w.pad)
+    t_rs = time.perf_counter() - t0
+    counts = s["counts"].sum(1)
+    e = int(np.argmax(counts))
+    seg = np.arange(s["offsets"][e], s["offsets"][e] + counts[e])
+    to_bits = lambda t: t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+    Wh = tuple({e: to_bits(W[e])} for W in W_dev)
+    xb = to_bits(x_cpu)
+    R, t_ffn = 2, 0.0
+    while True:
+        rows = seg[:R]
+        t1 = time.perf_counter()
+        xg = oracle.dispatch_rows(xb, w.N, s["phi"], rows)
+        _, y = oracle.ffn_rows(xg, np.full(len(rows), e, np.int32), *Wh, H=w.H, I=w.I)
+        t_ffn = time.perf_counter() - t1
+        if t_ffn > row_budget_s / 3 or R >= len(seg):
+            break
+        R = min(len(seg), R * 3)
+    t_row = t_ffn / len(rows)
+    n_comb = min(n_comb, w.n_tokens)
+    sel = np.random.default_rng(0).integers(0, len(rows), size=(n_comb, w.k))
+    t2 = time.perf_counter()
+    oracle.combine_f64(y, sel, g64[:n_comb], w.k)
+    t_comb = (time.perf_counter() - t2) / n_comb
+    per_token = t_rs / w.n_tokens + w.k * t_row + t_comb
+    sample = (f"route+schedule over all {w.n_tokens} tokens ({t_rs:.2f} s); dispatch+FFN of "
+              f"{len(rows)} rows of expert {e} ({t_ffn:.2f} s); combine of {n_comb} tokens; "
+              f"tokens/s = 1/(t_route_sched/{w.n_tokens} + {w.k}*t_row + t_combine)")
+    return dict(value=1.0 / per_token, cores=cores, sample=sample,
+                seconds=t_rs + t_ffn + t_comb * n_comb)
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank, world, _ = env_rank()
+    if rank != 0:
+        return 0
+    import torch
+
+    from combine_top_route_counting_b200 import inputs
+    w = inputs.WORKLOADS[args.workload]
+    lg, x = inputs.make_logits(w), inputs.make_x(w)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    W = inputs.make_weights(w, device=dev)
+    vals, secs = [], []
+    last = None
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample(w, lg, x, W, row_budget_s=args.ref_row_budget, n_comb=64)
+        if i >= args.warmup:
+            vals.append(r["value"])
+            secs.append(r["seconds"])
+        last = r
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * w.n_tokens / value, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(w), "note": "CPU oracle (plain C++/OpenMP, fp64) "
+                   "on a bounded per-step sample scaled to tokens/s"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": last["cores"],
+                         "kind": "oracle", "sample": last["sample"]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+
+    from combine_top_route_counting_b200 import inputs, moe
+
+    rank, world, local_rank = env_rank()
+    if world != args.gpus:
+        print(f"bench: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    ready = init_dist(world, local_rank)
+    moe.load()
+
+    w = inputs.WORKLOADS[args.workload]
+    sh = moe.shape(**w.shape())
+    lg_cpu, x_cpu = inputs.make_logits(w), inputs.make_x(w)
+    W = inputs.make_weights(w, device=dev)
+    lg, x = lg_cpu.to(dev), x_cpu.to(dev)
+    ws = torch.empty(moe.layer_workspace_bytes(sh), dtype=torch.uint8, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = torch.empty((w.n_tokens, w.H), dtype=torch.bfloat16, device=dev)
+    mb = args.minibatch
+
+    def step(events=None):
+        moe.moe_layer_forward(lg, x, *W, out, ws, st, sh, minibatch_tokens=mb, stage_events=events)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.N_STAGE_EVENTS)]
+          for _ in range(args.steps)]
+    for row in ev:
+        for e in row:
+            e.record()  # creates the event
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} during warm-up")
+    if ready:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(gpu_uuid(dev))
+    clocks.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    n0 = moe.launch_count()
+    t_start.record()
+    for i in range(args.steps):
+        step(ev[i] if mb == 0 else None)
+    t_end.record()
+    torch.cuda.synchronize()
+    launches = moe.launch_count() - n0
+    if ready:
+        torch.distributed.barrier()
+    ms = t_start.elapsed_time(t_end)
+
+    stage_ms = {}
+    if mb == 0:
+        for s_i, name in enumerate(moe.STAGES):
+            stage_ms[name] = statistics.mean(ev[i][s_i].elapsed_time(ev[i][s_i + 1])
+                                             for i in range(args.steps))
+
+    # end to end through the host-buffer entry: H2D of logits and x, the layer, D2H of out
+    e2e = None
+    if not args.no_e2e:
+        del ws
+        torch.cuda.empty_cache()
+        wsh = torch.empty(moe.layer_host_workspace_bytes(sh), dtype=torch.uint8, device=dev)
+        lg_h, x_h = lg_cpu.pin_memory(), x_cpu.pin_memory()
+        out_h = torch.empty((w.n_tokens, w.H), dtype=torch.bfloat16).pin_memory()
+        for _ in range(2):
+            moe.moe_layer_forward_host(lg_h, x_h, *W, out_h, wsh, st, sh, minibatch_tokens=mb)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        chk = 0.0
+        e0.record()
+        for _ in range(args.e2e_steps):
+            moe.moe_layer_forward_host(lg_h, x_h, *W, out_h, wsh, st, sh, minibatch_tokens=mb)
+        e1.record()
+        torch.cuda.synchronize()
+        chk += float(out_h[0, :8].float().sum())  # the host reads the result
+        e2e_ms = e0.elapsed_time(e1)
+        e2e = dict(ms=e2e_ms, h2d=lg_cpu.numel() * 4 + x_cpu.numel() * 2,
+                   d2h=out_h.numel() * 2, chk=chk)
+        del wsh
+    clk = clocks.stop()
+
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())}")
+
+    names = list(stage_ms)
+    vec = [ms] + [stage_ms[n] for n in names] + ([e2e["ms"]] if e2e else [])
+    vec = reduce_max(vec, ready, device=dev)
+    ms = vec[0]
+    stage_ms = dict(zip(names, vec[1:1 + len(names)]))
+    if e2e:
+        e2e["ms"] = vec[-1]
+
+    if rank == 0:
+        tokens = w.n_tokens * world * args.steps
+        value = tokens / (ms / 1e3)
+        peaks = load_peaks()
+        rows_used = schedule_rows(moe, w, sh, lg)
+        work = algorithmic_work(w, rows_used, w.n_routes)
+        stages = {}
+        for name, t in stage_ms.items():
+            d = {"ms": t}
+            if "bytes" in work[name]:
+                gbs = work[name]["bytes"] / (t / 1e3) / 1e9
+                d.update(bytes=work[name]["bytes"], gbs=gbs, frac_hbm=gbs / peaks["hbm"])
+            else:
+                tf = work[name]["flops"] / (t / 1e3) / 1e12
+                d.update(flops=work[name]["flops"], tflops=tf, frac_bf16=tf / peaks["bf16_sus"])
+            stages[name] = d
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": workload_desc(w), "tokens_per_step_per_gpu": w.n_tokens,
+                       "minibatch_tokens": mb or w.N, "parallelism": f"replicas x{world}",
+                       "rows_padded": rows_used,
+                       "l2": "inputs larger than L2: 33.8 GB of expert weights and 14 GB of "
+                             "fp32 expert outputs stream through HBM every step",
+                       "weights": "random-init bf16 N(0,0.02)"},
+        }
+        if stage_ms:
+            line["phi_build_us"] = stage_ms["schedule"] * 1e3
+            g1 = stages["ffn_gemm1"]
+            line["roofline"] = {
+                "kernel": "ffn_gemm_kernel<0> (GEMM1 + SwiGLU)", "bound": "tensor",
+                "achieved": g1["tflops"], "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
+                "frac": g1["tflops"] / peaks["bf16_sus"],
+                "peak_note": f"dense bf16, sustained, of {peaks['source']}",
+                "traffic": gemm1_traffic(w.n_routes),
+            }
+            line["stages"] = stages
+        line["gpu_launches"] = launches
+        if e2e:
+            line["e2e"] = {"value": w.n_tokens * world * args.e2e_steps / (e2e["ms"] / 1e3),
+                           "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
+                           "d2h_bytes_per_step": e2e["d2h"],
+                           "api": "moe_layer_forward_host (pinned host logits/x/out)"}
+        line["clocks"] = clk
+        if world == 1 and not args.no_cpu_baseline:
+            r = oracle_sample(w, lg_cpu, x_cpu, W, row_budget_s=args.cpu_budget)
+            line["cpu_baseline"] = {"value": r["value"], "unit": "tokens/s", "cores": r["cores"],
+                                    "kind": "oracle", "sample": r["sample"]}
+        print(json.dumps(line), flush=True)
+    if ready:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def schedule_rows(moe, w, sh, lg) -> int:
+    """Padded rows the schedule uses for this batch (offsets[E]), via the library."""
+    import torch
+    ids = torch.empty((w.n_tokens, w.k), dtype=torch.int32, device=lg.device)
+    gates = torch.empty((w.n_tokens, w.k), dtype=torch.float32, device=lg.device)
+    moe.moe_route_topk(lg, ids, gates, sh)
+    b = moe.alloc_schedule_outputs(sh, device=lg.device)
+    moe.moe_schedule(ids, b["phi"], b["offsets"], b["counts"], b["route_row"], b["ws"],
+                     b["dev_status"], sh)
+    return int(b["offsets"][-1].item())
+
+
+def gemm1_traffic(n_routes: int):
+    """DRAM bytes per GEMM1 launch from the committed ncu summary, scaled to this
+    launch by routes; None when the summary is missing or the kernel changed since."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "ffn_gemm1_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    for ln in open(path):
+        if ":" in ln:
+            a, b = ln.split(":", 1)
+            kv[a.strip()] = b.strip()
+    h = hashlib.sha256()
+    for f in ("expert_ffn.cu", "sm100.cuh"):
+        h.update(open(os.path.join(ROOT, "combine_top_route_counting_b200", "csrc", f), "rb").read())
+    if kv.get("kernel_source_sha256") != h.hexdigest():
+        return None
+    try:
+        return float(kv["dram_bytes_per_route"]) * n_routes
+    except (KeyError, ValueError):
+        return None
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="kimi")
+    ap.add_argument("--minibatch", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--ref-row-budget", type=float, default=3.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -62,6 +62,9 @@ WORKLOADS = {
     "mid": Workload("mid", 2, P=4, N=4096, E=64, k=4, H=2048, I=1024),
     "kimi": Workload("kimi", 3, P=8, N=7168, E=384, k=8, H=7168, I=2048, minibatch=2368),
     "zipf": Workload("zipf", 4, P=8, N=7168, E=384, k=8, H=7168, I=2048, logits="zipf", n_empty=8),
+    # Kimi expert shapes with 16 experts and ~1,200 routes each (as at full size):
+    # a few GB on the device, for profiler captures of the FFN kernels
+    "kimi_e16": Workload("kimi_e16", 5, P=1, N=2400, E=16, k=8, H=7168, I=2048),
 }
 
 
