@@ -9,21 +9,33 @@
 //          h = bf16_rne(silu(acc_W1) * acc_W3)
 //   GEMM2: y = h . W2[l]  (fp32)
 //
-// Design (one persistent CTA per SM, 256 threads, warp-specialised):
-//   warp 0      TMA producer: 4-stage ring of {A 128x64, B 64x256} bf16
-//               tiles, 128-byte swizzle, mbarrier complete_tx
-//   warp 1      TMEM allocator and MMA issuer: tcgen05.mma kind::f16,
-//               M=128 N=256 K=16, A K-major, B MN-major (the weights are
-//               stored [K, N] with N contiguous, so no transpose is needed)
-//   warps 4-7   epilogue: tcgen05.ld of the fp32 accumulator (one TMEM lane
-//               per row), SwiGLU or fp32 store to global memory
+// Design (persistent, one CTA per SM, 384 threads, warp-specialised):
+//   warp 0      TMA producer: ring of {A 128x64, B 64 x (256/CG)} bf16 tiles,
+//               128-byte swizzle, mbarrier complete_tx
+//   warp 1      TMEM allocator and MMA issuer: tcgen05.mma kind::f16, K=16,
+//               A K-major, B MN-major (the weights are stored [K, N] with N
+//               contiguous, so no transpose is needed)
+//   warps 4-11  epilogue: tcgen05.ld of the fp32 accumulator (one TMEM lane per
+//               row, two warps per lane quarter splitting the columns),
+//               SwiGLU or fp32, 32-byte vector stores
 //   TMEM        2 x 256 fp32 columns: the accumulator of tile i+1 fills while
 //               the epilogue drains tile i
-// A 128-row M-tile never straddles two experts because every segment is a
-// multiple of 128 rows; the expert of a tile comes from a binary search over
-// the segment offsets held in shared memory. Tiles holding only padding rows
-// are skipped. Tiles are visited m-major, so the CTAs running at one time
-// share an expert's weights and the A rows of a few M-tiles through L2.
+// Two geometries (CG = CTAs per MMA):
+//   CG = 2 (segments padded to multiples of 256, the pages' padding): a
+//     cluster of two CTAs on two SMs computes a 256x256 tile with
+//     tcgen05.mma.cta_group::2 (M=256, N=256): each CTA loads its 128 rows of
+//     A and 128 of the 256 B columns, so each SM moves half the operand bytes
+//     per flop of a single-SM 128x256 tile. 6-stage ring of 32 KB.
+//   CG = 1 (segments multiples of 128 only): 128x256 tile per CTA with
+//     cta_group::1, 4-stage ring of 48 KB.
+// GEMM1's B tile is [W1 cols | W3 cols] of the same 128 h columns, so one
+// N=256 MMA produces both halves of SwiGLU (with CG = 2, CTA 0 holds the W1
+// half and CTA 1 the W3 half). A tile never straddles two experts because
+// every segment is a multiple of the tile height; the expert of a tile comes
+// from a binary search over the segment offsets held in shared memory. Tiles
+// holding only padding rows are skipped. Tiles are visited m-major, so the
+// CTAs running at one time share an expert's weights and the A rows of a few
+// M-tiles through L2.
 //
 // Every output element is produced by one CTA with a fixed K order (no
 // split-K, no atomics): the result is bitwise deterministic and independent
@@ -44,27 +56,32 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128;
-constexpr int BN = 256;  // accumulator columns per tile
-constexpr int BK = 64;   // K per stage: one 128-byte swizzle row of bf16
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;             // 16 KB
-constexpr int B_ATOM_BYTES = 64 * BK * 2;        // one 64-column x 64-K box: 8 KB
-constexpr int B_BYTES = (BN / 64) * B_ATOM_BYTES;  // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 48 KB
-constexpr int NUM_THREADS = 256;
-constexpr int TMEM_COLS = 512;                   // 2 accumulators x 256 columns
+constexpr int NUM_THREADS = 384;  // 12 warps: TMA, MMA, 2 idle, 8 epilogue
+constexpr int EPI_WARP0 = 4;
+constexpr int NUM_EPI_WARPS = 8;
+constexpr int TMEM_COLS = 512;    // 2 accumulators x 256 fp32 columns
 constexpr int UMMA_K = 16;
-constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*B MN-major*/ 1);
-static_assert(STAGE_BYTES % 1024 == 0 && A_BYTES % 1024 == 0, "swizzle atoms stay 1024-aligned");
 
-// barrier slots
-constexpr int BAR_FULL = 0;
-constexpr int BAR_EMPTY = STAGES;
-constexpr int BAR_TFULL = 2 * STAGES;
-constexpr int BAR_TEMPTY = 2 * STAGES + 2;
-constexpr int BAR_DRAIN = 2 * STAGES + 4;
-constexpr int NUM_BARS = 2 * STAGES + 5;
+// Tile geometry for CG CTAs per MMA (1: one SM, 2: a CTA pair on two SMs).
+template <int CG>
+struct Cfg {
+  static constexpr int BM = 128 * CG;      // rows per tile (each CTA holds 128)
+  static constexpr int BN = 256;           // accumulator columns per tile
+  static constexpr int BK = 64;            // K per stage: one 128-byte swizzle row of bf16
+  static constexpr int B_ATOMS = BN / CG / 64;   // 64-column B boxes held per CTA
+  static constexpr int A_BYTES = 128 * BK * 2;   // 16 KB
+  static constexpr int B_ATOM_BYTES = 64 * BK * 2;  // 8 KB
+  static constexpr int STAGE_BYTES = A_BYTES + B_ATOMS * B_ATOM_BYTES;  // 48 / 32 KB
+  static constexpr int STAGES = CG == 1 ? 4 : 6;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*B MN-major*/ 1);
+  static constexpr int BAR_FULL = 0;
+  static constexpr int BAR_EMPTY = STAGES;
+  static constexpr int BAR_TFULL = 2 * STAGES;
+  static constexpr int BAR_TEMPTY = 2 * STAGES + 2;
+  static constexpr int BAR_DRAIN = 2 * STAGES + 4;
+  static constexpr int NUM_BARS = 2 * STAGES + 5;
+  static_assert(STAGE_BYTES % 1024 == 0 && A_BYTES % 1024 == 0, "swizzle atoms stay 1024-aligned");
+};
 
 struct FfnParams {
   const int32_t* offsets;  // [E+1]
@@ -78,9 +95,11 @@ struct FfnParams {
   int64_t timeout_ns;
 };
 
+template <int CG>
 size_t smem_bytes_for(int E) {
-  return 1024 /*alignment slack*/ + static_cast<size_t>(STAGES) * STAGE_BYTES +
-         NUM_BARS * 8 + 16 + static_cast<size_t>(2 * E + 1) * 4;
+  using C = Cfg<CG>;
+  return 1024 /*alignment slack*/ + static_cast<size_t>(C::STAGES) * C::STAGE_BYTES +
+         C::NUM_BARS * 8 + 16 + static_cast<size_t>(2 * E + 1) * 4;
 }
 
 __device__ __forceinline__ float silu(float a) { return a / (1.0f + expf(-a)); }
@@ -93,15 +112,20 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // MODE 0: GEMM1 + SwiGLU -> bf16 h. MODE 1: GEMM2 -> fp32 y.
-template <int MODE>
+// CG = 1: one CTA per 128x256 tile. CG = 2: a cluster of two CTAs (a tcgen05
+// CTA pair) per 256x256 tile; CTA r loads rows [128r, 128r+128) of A and
+// columns [128r, 128r+128) of B, the leader (r = 0) issues the pair MMAs and
+// each CTA drains its own 128 TMEM lanes.
+template <int MODE, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const FfnParams p) {
+  using C = Cfg<CG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* bad_flag = abort_flag + 1;
   int32_t* s_off = reinterpret_cast<int32_t*>(tmem_slot + 4);  // [E+1] segment starts
@@ -109,17 +133,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int E = p.E;
+  const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
 
   if (tid == 0) {
-    for (int i = 0; i < STAGES; ++i) {
-      mbar_init(smem_u32(&bars[BAR_FULL + i]), 1);
-      mbar_init(smem_u32(&bars[BAR_EMPTY + i]), 1);
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(smem_u32(&bars[C::BAR_FULL + i]), 1);
+      mbar_init(smem_u32(&bars[C::BAR_EMPTY + i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&bars[BAR_TFULL + i]), 1);
-      mbar_init(smem_u32(&bars[BAR_TEMPTY + i]), 128);
+      mbar_init(smem_u32(&bars[C::BAR_TFULL + i]), 1);
+      mbar_init(smem_u32(&bars[C::BAR_TEMPTY + i]), NUM_EPI_WARPS * CG);
     }
-    mbar_init(smem_u32(&bars[BAR_DRAIN]), 1);
+    mbar_init(smem_u32(&bars[C::BAR_DRAIN]), 1);
     *abort_flag = 0;
     *bad_flag = 0;
     fence_mbar_init();
@@ -133,7 +159,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   for (int l = tid; l < E; l += NUM_THREADS) {
     const int a = s_off[l], b = s_off[l + 1];
-    bool bad = a < 0 || b < a || (a & (BM - 1)) || (b & (BM - 1)) || b > p.rows_max;
+    bool bad = a < 0 || b < a || (a % C::BM) || (b % C::BM) || b > p.rows_max;
     int T = b - a;
     if (p.counts) {
       int t = 0;
@@ -145,27 +171,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     s_end[l] = a + T;
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    if (CG == 2) {
+      tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (CG == 2) cluster_sync();  // the peer's barriers exist before anything targets them
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const bool bad_sched = *bad_flag != 0;
   if (bad_sched && tid == 0) atomicOr(p.dev_status, MOE_DEV_BAD_SCHEDULE);
 
   const int rows_used = bad_sched ? 0 : s_off[E];
-  const int tiles_n = (MODE == 0) ? p.Nout / 128 : p.Nout / BN;
-  const int num_tiles = (rows_used / BM) * tiles_n;
-  const int kblocks = p.K / BK;
+  const int tiles_n = (MODE == 0) ? p.Nout / 128 : p.Nout / C::BN;
+  const int num_tiles = (rows_used / C::BM) * tiles_n;
+  const int kblocks = p.K / C::BK;
+  const int first_tile = (CG == 2) ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int tile_step = (CG == 2) ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   const WaitCtx wc{abort_flag, p.dev_status, p.timeout_ns, MOE_DEV_TIMEOUT};
+  const int64_t drain_ns = p.timeout_ns < 100000000ll ? p.timeout_ns : 100000000ll;
 
   // tile -> (first row, n-tile, expert); false if the tile holds only padding
   auto tile_info = [&](int tile, int& row0, int& n, int& l) -> bool {
     const int m = tile / tiles_n;
     n = tile - m * tiles_n;
-    row0 = m * BM;
+    row0 = m * C::BM;
     int lo = 0, hi = E - 1;  // largest l with s_off[l] <= row0
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -179,116 +214,145 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      // the leader's full barriers count the bytes of both CTAs of a pair
+      const uint32_t full0 = smem_u32(&bars[C::BAR_FULL]);
+      const uint32_t full_tgt0 = (CG == 2) ? mapa_shared(full0, 0) : full0;
       int stage = 0;
       uint32_t phase = 0;
       int64_t issued = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
         int row0, n, l;
         if (!tile_info(tile, row0, n, l)) continue;
+        const int arow = row0 + static_cast<int>(rank) * 128;
         const int yb = l * p.K;
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!wait_bounded(smem_u32(&bars[BAR_EMPTY + stage]), phase ^ 1u, wc)) {
+          if (!wait_bounded(smem_u32(&bars[C::BAR_EMPTY + stage]), phase ^ 1u, wc)) {
             ok = false;
             break;
           }
-          const uint32_t full = smem_u32(&bars[BAR_FULL + stage]);
-          const uint32_t sA = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t sB = sA + A_BYTES;
-          mbar_arrive_expect_tx(full, STAGE_BYTES);
-          tma_load_2d(sA, &tmA, kb * BK, row0, full);
-          if (MODE == 0) {
-            tma_load_2d(sB + 0 * B_ATOM_BYTES, &tmB0, n * 128, yb + kb * BK, full);
-            tma_load_2d(sB + 1 * B_ATOM_BYTES, &tmB0, n * 128 + 64, yb + kb * BK, full);
-            tma_load_2d(sB + 2 * B_ATOM_BYTES, &tmB1, n * 128, yb + kb * BK, full);
-            tma_load_2d(sB + 3 * B_ATOM_BYTES, &tmB1, n * 128 + 64, yb + kb * BK, full);
-          } else {
+          const uint32_t full_local = full0 + stage * 8;
+          const uint32_t full_tgt = full_tgt0 + stage * 8;
+          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sB = sA + C::A_BYTES;
+          const int ky = yb + kb * C::BK;
+          if (leader) mbar_arrive_expect_tx(full_local, CG * C::STAGE_BYTES);
+          if (CG == 1) {
+            tma_load_2d(sA, &tmA, kb * C::BK, arow, full_tgt);
+            if (MODE == 0) {
+              tma_load_2d(sB + 0 * C::B_ATOM_BYTES, &tmB0, n * 128, ky, full_tgt);
+              tma_load_2d(sB + 1 * C::B_ATOM_BYTES, &tmB0, n * 128 + 64, ky, full_tgt);
+              tma_load_2d(sB + 2 * C::B_ATOM_BYTES, &tmB1, n * 128, ky, full_tgt);
+              tma_load_2d(sB + 3 * C::B_ATOM_BYTES, &tmB1, n * 128 + 64, ky, full_tgt);
+            } else {
 #pragma unroll
-            for (int b = 0; b < BN / 64; ++b)
-              tma_load_2d(sB + b * B_ATOM_BYTES, &tmB0, n * BN + b * 64, yb + kb * BK, full);
+              for (int b = 0; b < 4; ++b)
+                tma_load_2d(sB + b * C::B_ATOM_BYTES, &tmB0, n * C::BN + b * 64, ky, full_tgt);
+            }
+          } else {
+            tma_load_2d_pair(sA, &tmA, kb * C::BK, arow, full_tgt);
+            // GEMM1: CTA 0 holds W1's columns, CTA 1 W3's (the two SwiGLU halves);
+            // GEMM2: CTA r holds W2 columns [n*256 + 128r, +128).
+            const CUtensorMap* mb = (MODE == 0 && rank == 1) ? &tmB1 : &tmB0;
+            const int x0 = (MODE == 0) ? n * 128 : n * C::BN + static_cast<int>(rank) * 128;
+            tma_load_2d_pair(sB, mb, x0, ky, full_tgt);
+            tma_load_2d_pair(sB + C::B_ATOM_BYTES, mb, x0 + 64, ky, full_tgt);
           }
           ++issued;
-          if (++stage == STAGES) {
+          if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
-      // make sure no load is still landing in shared memory when the CTA exits
-      const int64_t first = issued > STAGES ? issued - STAGES : 0;
-      for (int64_t j = first; j < issued; ++j)
-        wait_drain(smem_u32(&bars[BAR_FULL + (j % STAGES)]), static_cast<uint32_t>((j / STAGES) & 1),
-                   p.timeout_ns);
+      // no load may still be landing in shared memory when the CTA exits: the
+      // leader sees its full barriers complete; a follower sees the stage
+      // released by the leader's MMAs (which waited for the data)
+      const int64_t first = issued > C::STAGES ? issued - C::STAGES : 0;
+      for (int64_t j = first; j < issued; ++j) {
+        const int st = static_cast<int>(j % C::STAGES);
+        const uint32_t par = static_cast<uint32_t>((j / C::STAGES) & 1);
+        wait_drain(smem_u32(&bars[(leader ? C::BAR_FULL : C::BAR_EMPTY) + st]), par, drain_ns);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
         int row0, n, l;
         if (!tile_info(tile, row0, n, l)) continue;
-        if (!wait_bounded(smem_u32(&bars[BAR_TEMPTY + acc]), acc_phase ^ 1u, wc)) {
+        if (!wait_bounded<CG == 2>(smem_u32(&bars[C::BAR_TEMPTY + acc]), acc_phase ^ 1u, wc)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!wait_bounded(smem_u32(&bars[BAR_FULL + stage]), phase, wc)) {
+          if (!wait_bounded(smem_u32(&bars[C::BAR_FULL + stage]), phase, wc)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sA = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t sB = sA + A_BYTES;
+          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sB = sA + C::A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+          for (int kk = 0; kk < C::BK / UMMA_K; ++kk) {
             // A: K-major, advance 16 bf16 = 32 bytes inside the swizzled row.
             // B: MN-major, advance 16 K-rows = two 8-row groups = 2048 bytes.
             const uint64_t a_desc = smem_desc_sw128(sA + kk * 32, 16, 1024);
-            const uint64_t b_desc = smem_desc_sw128(sB + kk * 2048, B_ATOM_BYTES, 1024);
-            tc_mma_f16(d_tmem, a_desc, b_desc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            const uint64_t b_desc = smem_desc_sw128(sB + kk * 2048, C::B_ATOM_BYTES, 1024);
+            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+            if (CG == 2) tc_mma_f16_pair(d_tmem, a_desc, b_desc, C::IDESC, accum);
+            else tc_mma_f16(d_tmem, a_desc, b_desc, C::IDESC, accum);
           }
-          tc_commit(smem_u32(&bars[BAR_EMPTY + stage]));
-          if (++stage == STAGES) {
+          if (CG == 2) tc_commit_pair_mc(smem_u32(&bars[C::BAR_EMPTY + stage]), 0x3);
+          else tc_commit(smem_u32(&bars[C::BAR_EMPTY + stage]));
+          if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(smem_u32(&bars[BAR_TFULL + acc]));
+        if (CG == 2) tc_commit_pair_mc(smem_u32(&bars[C::BAR_TFULL + acc]), 0x3);
+        else tc_commit(smem_u32(&bars[C::BAR_TFULL + acc]));
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1u;
       }
       // all MMAs issued by this thread have completed once this arrives
-      tc_commit(smem_u32(&bars[BAR_DRAIN]));
-      wait_drain(smem_u32(&bars[BAR_DRAIN]), 0, p.timeout_ns);
+      if (CG == 2) tc_commit_pair(smem_u32(&bars[C::BAR_DRAIN]));
+      else tc_commit(smem_u32(&bars[C::BAR_DRAIN]));
+      wait_drain(smem_u32(&bars[C::BAR_DRAIN]), 0, p.timeout_ns);
     }
-  } else if (warp >= 4) {
+  } else if (warp >= EPI_WARP0) {
     // ------------------------------------------------------------ epilogue
-    const int q = warp - 4;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;                  // TMEM lane quarter this warp may access
+    const int half = (warp - EPI_WARP0) >> 2;  // which half of the tile's columns
+    const uint32_t tempty0 = smem_u32(&bars[C::BAR_TEMPTY]);
+    const uint32_t tempty_tgt0 = (CG == 2) ? mapa_shared(tempty0, 0) : tempty0;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int tile = first_tile; tile < num_tiles; tile += tile_step) {
       int row0, n, l;
       if (!tile_info(tile, row0, n, l)) continue;
-      if (!wait_bounded(smem_u32(&bars[BAR_TFULL + acc]), acc_phase, wc)) break;
+      if (!wait_bounded(smem_u32(&bars[C::BAR_TFULL + acc]), acc_phase, wc)) break;
       tc_fence_after();
-      const int64_t row = row0 + q * 32 + lane;
+      const int64_t row = row0 + static_cast<int>(rank) * 128 + q * 32 + lane;
       const uint32_t tbase =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::BN);
       if (MODE == 0) {
-        uint4* hrow = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) +
-                                               row * p.Nout + n * 128);
+        // accumulator columns [0,128) = x.W1, [128,256) = x.W3 for h columns n*128 + j
+        __nv_bfloat16* hrow =
+            reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.Nout + n * 128 + half * 64;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t ra[32], rb[32];
-          tmem_ld_32cols(tbase + c * 32, ra);
-          tmem_ld_32cols(tbase + 128 + c * 32, rb);
+          tmem_ld_32cols(tbase + half * 64 + c * 32, ra);
+          tmem_ld_32cols(tbase + 128 + half * 64 + c * 32, rb);
           tmem_ld_wait();
           uint32_t pk[16];
 #pragma unroll
@@ -297,37 +361,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const float h1 = silu(__uint_as_float(ra[2 * i + 1])) * __uint_as_float(rb[2 * i + 1]);
             pk[i] = pack_bf16x2(h0, h1);
           }
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            hrow[c * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          const uint32_t(&lo)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&pk[0]);
+          const uint32_t(&hi)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&pk[8]);
+          st_global_v8(hrow + c * 32, lo);
+          st_global_v8(hrow + c * 32 + 16, hi);
         }
       } else {
-        float4* yrow = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + row * p.Nout +
-                                                 n * BN);
+        float* yrow = reinterpret_cast<float*>(p.out) + row * p.Nout + n * C::BN + half * 128;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t rv[32];
-          tmem_ld_32cols(tbase + c * 32, rv);
+          tmem_ld_32cols(tbase + half * 128 + c * 32, rv);
           tmem_ld_wait();
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            yrow[c * 8 + v] = make_float4(__uint_as_float(rv[4 * v]), __uint_as_float(rv[4 * v + 1]),
-                                          __uint_as_float(rv[4 * v + 2]),
-                                          __uint_as_float(rv[4 * v + 3]));
+          for (int v = 0; v < 4; ++v)
+            st_global_v8(yrow + c * 32 + v * 8, *reinterpret_cast<const uint32_t(*)[8]>(&rv[8 * v]));
         }
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&bars[BAR_TEMPTY + acc]));
+      __syncwarp();
+      if (lane == 0) {
+        if (CG == 2) mbar_arrive_cluster(tempty_tgt0 + acc * 8);
+        else mbar_arrive(tempty0 + acc * 8);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
   }
 
   __syncthreads();
+  if (CG == 2) cluster_sync();  // the peer no longer reads this CTA's smem or TMEM
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if (CG == 2) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -361,16 +429,32 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE>
+template <int MODE, int CG>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const FfnParams& p, cudaStream_t s) {
-  const size_t smem = smem_bytes_for(p.E);
-  cudaError_t e = cudaFuncSetAttribute(ffn_gemm_kernel<MODE>,
+  const size_t smem = smem_bytes_for<CG>(p.E);
+  cudaError_t e = cudaFuncSetAttribute(ffn_gemm_kernel<MODE, CG>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  ffn_gemm_kernel<MODE><<<device_sm_count(), NUM_THREADS, smem, s>>>(a, b0, b1, p);
+  const int sms = device_sm_count();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(CG == 2 ? (sms / 2) * 2 : sms);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  if (CG == 2) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  e = cudaLaunchKernelEx(&cfg, ffn_gemm_kernel<MODE, CG>, a, b0, b1, p);
   note_launches(1);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -383,19 +467,22 @@ cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint
   const int E = sh.E, H = sh.H, I = sh.I;
   CUtensorMap mA1, mW1, mW3, mA2, mW2;
   const uint64_t EH = static_cast<uint64_t>(E) * H, EI = static_cast<uint64_t>(E) * I;
-  if (!make_map(&mA1, xg, H, rows_max, 64, BM) || !make_map(&mW1, W1, I, EH, 64, 64) ||
-      !make_map(&mW3, W3, I, EH, 64, 64) || !make_map(&mA2, h, I, rows_max, 64, BM) ||
+  if (!make_map(&mA1, xg, H, rows_max, 64, 128) || !make_map(&mW1, W1, I, EH, 64, 64) ||
+      !make_map(&mW3, W3, I, EH, 64, 64) || !make_map(&mA2, h, I, rows_max, 64, 128) ||
       !make_map(&mW2, W2, H, EI, 64, 64))
     return cudaErrorInvalidValue;
+  // Segments that are multiples of 256 rows run on CTA pairs (256x256 tiles);
+  // otherwise (pad a multiple of 128 only) on single CTAs (128x256 tiles).
+  const bool pair = (sh.pad % 256) == 0;
   FfnParams p1{offsets, counts, E, sh.P, H, I, rows_max, h, dev_status, kWaitTimeoutNs};
-  cudaError_t e = launch_mode<0>(mA1, mW1, mW3, p1, s);
+  cudaError_t e = pair ? launch_mode<0, 2>(mA1, mW1, mW3, p1, s) : launch_mode<0, 1>(mA1, mW1, mW3, p1, s);
   if (e != cudaSuccess) return e;
   if (ev_mid) {
     e = cudaEventRecord(ev_mid, s);
     if (e != cudaSuccess) return e;
   }
   FfnParams p2{offsets, counts, E, sh.P, I, H, rows_max, y, dev_status, kWaitTimeoutNs};
-  return launch_mode<1>(mA2, mW2, mW2, p2, s);
+  return pair ? launch_mode<1, 2>(mA2, mW2, mW2, p2, s) : launch_mode<1, 1>(mA2, mW2, mW2, p2, s);
 }
 
 // ---------------------------------------------------------------- self test

@@ -344,3 +344,21 @@ def test_layer_host_entry_matches_device_entry(cuda_lib):
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     assert torch.equal(out_h, out_d.cpu())
+
+
+def test_layer_pad128_single_cta_path(cuda_lib):
+    """Segments padded to 128 rows run the single-CTA (128x256 tile) FFN kernels."""
+    moe = cuda_lib
+    w0 = inputs.WORKLOADS["tiny"]
+    w = inputs.Workload("tiny_pad128", w0.wid, P=2, N=100, E=w0.E, k=w0.k, H=w0.H, I=w0.I, pad=128)
+    lg = torch.randn((w.n_tokens, w.E), generator=torch.Generator().manual_seed(77))
+    x = torch.randn((w.n_tokens, w.H), generator=torch.Generator().manual_seed(78)).to(torch.bfloat16)
+    W1, W3, W2 = inputs.make_weights(w0)
+    Wd = [t.to(DEV) for t in (W1, W3, W2)]
+    out, _ = _layer_gpu(moe, w, lg.to(DEV), x.to(DEV), Wd)
+    Wh = expert_weights_host(W1, W3, W2, range(w.E))
+    res = oracle.layer_tokens(lg, bits(x), Wh, w.P, w.N, w.k, w.E, w.H, w.I, range(w.n_tokens),
+                              pad=128)
+    assert rms_floor_err(bf16_to_f64(bits(out)), res["out64"]) < OUT_TOL
+    assert all(int(v) % 128 == 0 for v in res["sched"]["offsets"])
+    assert any(int(v) % 256 != 0 for v in res["sched"]["offsets"])
