@@ -67,6 +67,8 @@ _SIGS = {
                            ctypes.POINTER(Shape), _vp, ctypes.POINTER(_vp)], ctypes.c_int),
     "moe_layer_forward_host": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int32, _vp,
                                 ctypes.c_size_t, _vp, ctypes.POINTER(Shape), _vp], ctypes.c_int),
+    "moe_schedule_static_ws": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Shape), _vp],
+                               ctypes.c_int),
     "moe_launch_count": ([], ctypes.c_int64),
     "moe_selftest_bounded_wait": ([_vp, ctypes.c_int64, _vp], ctypes.c_int),
 }
@@ -161,6 +163,20 @@ def moe_schedule(ids, phi, offsets, counts, route_row, ws, dev_status, sh: Shape
                                _ptr(ws, torch.uint8, "ws"), ws.numel(),
                                _ptr(dev_status, torch.int32, "dev_status"), ctypes.byref(sh),
                                _stream(stream)), "moe_schedule")
+
+
+def moe_schedule_static_ws(ids, phi, offsets, counts, route_row, dev_status, sh: Shape,
+                           stream=None):
+    """moe_schedule with the library's fixed 4 MiB device scratch instead of a
+    caller-provided workspace (for callers that cannot allocate one)."""
+    _check(load().moe_schedule_static_ws(_ptr(ids, torch.int32, "ids"),
+                                         _ptr(phi, torch.int32, "phi"),
+                                         _ptr(offsets, torch.int32, "offsets"),
+                                         _ptr(counts, torch.int32, "counts"),
+                                         _ptr(route_row, torch.int32, "route_row"),
+                                         _ptr(dev_status, torch.int32, "dev_status"),
+                                         ctypes.byref(sh), _stream(stream)),
+           "moe_schedule_static_ws")
 
 
 def moe_dispatch(x, phi, offsets, xg, dev_status, sh: Shape, stream=None):

@@ -133,6 +133,26 @@ moe_status_t moe_schedule(const int32_t* ids, int32_t* phi, int32_t* offsets, in
                           int32_t* route_row, void* ws, size_t ws_bytes, int32_t* dev_status,
                           const moe_shape_t* shape, void* stream);
 
+/* moe_schedule without a caller-provided scratch buffer. The source pages have
+ * no counterpart: this entry point exists for callers that cannot allocate
+ * device memory for `ws` -- for instance a plugin that a host application
+ * calls with only its input and output buffers, or a serving loop that bans
+ * cudaMalloc on its hot path because an allocation can synchronise the device.
+ * Arguments, outputs and device-status behaviour are those of moe_schedule.
+ * The scratch is a fixed 4 MiB device array inside the library (1,048,576
+ * int32 words; every GPU that loads the library holds it until the process
+ * exits); shapes needing more, i.e. P * ceil(N*k/2048) * E > 1,048,576, are
+ * rejected with MOE_WORKSPACE_TOO_SMALL before anything is enqueued. The
+ * first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. All calls share the one array and it keeps the last call's
+ * contents (the kernels overwrite every word they read), so calls that
+ * overlap on the GPU -- e.g. on two streams at once -- race and must be
+ * serialised by the caller. Allocates no device or host memory. */
+moe_status_t moe_schedule_static_ws(const int32_t* ids, int32_t* phi, int32_t* offsets,
+                                    int32_t* counts, int32_t* route_row, int32_t* dev_status,
+                                    const moe_shape_t* shape, void* stream);
+
 /* Step 3a -- pull dispatch ("Beyond Peak TFLOPs" 2.A, MoK notes section 2:
  * tokens land zero-copy in contiguous per-expert buffers).
  * x: bf16 [P*N, H]; xg: bf16 [moe_rows_max, H]. For row < offsets[E]:
