@@ -108,65 +108,192 @@ int device_sm_count() {
 
 namespace {
 
+struct LayerBufs {
+  int32_t *ids, *route_row, *phi, *offsets, *counts, *sched;
+  float *gates, *y;
+  uint16_t *xg, *h;
+};
+
+LayerBufs layer_bufs(void* ws, const LayerWs& w) {
+  LayerBufs b;
+  b.ids = at<int32_t>(ws, w.ids);
+  b.gates = at<float>(ws, w.gates);
+  b.route_row = at<int32_t>(ws, w.route_row);
+  b.phi = at<int32_t>(ws, w.phi);
+  b.offsets = at<int32_t>(ws, w.offsets);
+  b.counts = at<int32_t>(ws, w.counts);
+  b.sched = at<int32_t>(ws, w.sched);
+  b.xg = at<uint16_t>(ws, w.xg);
+  b.h = at<uint16_t>(ws, w.h);
+  b.y = at<float>(ws, w.y);
+  return b;
+}
+
+// Schedule -> dispatch -> FFN -> combine for one token slice (steps 2-4).
+// ev (7 events, may be null) marks the stage boundaries 1..6.
+cudaError_t run_slice(const LayerBufs& b, const uint16_t* x, const uint16_t* W1, const uint16_t* W3,
+                      const uint16_t* W2, uint16_t* out, Slice sl, const moe_shape_t* sh,
+                      int32_t* dev_status, cudaStream_t s, void* const* ev) {
+  const int64_t rows_max = rows_max_of(sh);
+  auto rec = [&](int i) -> cudaError_t {
+    return (ev && ev[i]) ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) : cudaSuccess;
+  };
+  cudaError_t e;
+  if ((e = rec(1)) != cudaSuccess) return e;
+  if ((e = launch_schedule(b.ids, *sh, sl, b.phi, b.offsets, b.counts, b.route_row, b.sched,
+                           dev_status, s)) != cudaSuccess)
+    return e;
+  // The pull dispatch runs as its own HBM-bound gather: feeding GEMM1 with TMA
+  // row gathers instead (moe_expert_ffn_gather) measured 3x slower on B200, the
+  // gathers delivering far fewer bytes per clock than the MMAs use.
+  if ((e = rec(2)) != cudaSuccess) return e;
+  if ((e = launch_dispatch(x, b.phi, b.offsets, b.xg, *sh, rows_max, dev_status, s)) != cudaSuccess)
+    return e;
+  if ((e = rec(3)) != cudaSuccess) return e;
+  cudaEvent_t mid = (ev && ev[4]) ? static_cast<cudaEvent_t>(ev[4]) : nullptr;
+  if ((e = launch_expert_ffn(b.xg, W1, W3, W2, b.offsets, b.counts, b.h, b.y, *sh, rows_max,
+                             dev_status, s, mid)) != cudaSuccess)
+    return e;
+  if ((e = rec(5)) != cudaSuccess) return e;
+  if ((e = launch_combine(b.y, b.route_row, b.gates, out, *sh, sl, rows_max, dev_status, s)) !=
+      cudaSuccess)
+    return e;
+  return rec(6);
+}
+
 // The layer body on device buffers (shared by both layer entry points).
 moe_status_t layer_body(const float* logits, const uint16_t* x, const uint16_t* W1,
                         const uint16_t* W3, const uint16_t* W2, uint16_t* out,
                         int32_t minibatch_tokens, void* ws, int32_t* dev_status,
                         const moe_shape_t* sh, cudaStream_t s, void* const* ev) {
-  const LayerWs w = layer_ws(sh);
-  const int64_t rows_max = rows_max_of(sh);
-  int32_t* ids = at<int32_t>(ws, w.ids);
-  float* gates = at<float>(ws, w.gates);
-  int32_t* route_row = at<int32_t>(ws, w.route_row);
-  int32_t* phi = at<int32_t>(ws, w.phi);
-  int32_t* offsets = at<int32_t>(ws, w.offsets);
-  int32_t* counts = at<int32_t>(ws, w.counts);
-  int32_t* sched = at<int32_t>(ws, w.sched);
-  uint16_t* xg = at<uint16_t>(ws, w.xg);
-  uint16_t* h = at<uint16_t>(ws, w.h);
-  float* y = at<float>(ws, w.y);
-
+  const LayerBufs b = layer_bufs(ws, layer_ws(sh));
   const int32_t N = sh->N;
   const int32_t T = (minibatch_tokens <= 0 || minibatch_tokens >= N) ? N : minibatch_tokens;
-  const bool single = (T == N);
-  auto rec = [&](int i) -> cudaError_t {
-    if (!ev || !single || !ev[i]) return cudaSuccess;
-    return cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s);
-  };
-
-  cudaError_t e = rec(0);
+  void* const* ev_use = (T == N) ? ev : nullptr;  // stage events: single-slice runs only
+  cudaError_t e = (ev_use && ev_use[0]) ? cudaEventRecord(static_cast<cudaEvent_t>(ev_use[0]), s)
+                                        : cudaSuccess;
   if (e == cudaSuccess)
-    e = launch_route_topk(logits, ids, gates, static_cast<int64_t>(sh->P) * N, sh->E, sh->k, s);
+    e = launch_route_topk(logits, b.ids, b.gates, static_cast<int64_t>(sh->P) * N, sh->E, sh->k, s);
   if (e != cudaSuccess) return from_cuda(e);
   if (N == 0) {
-    rec(1);
-    rec(2);
-    rec(3);
-    rec(4);
-    rec(5);
-    return from_cuda(rec(6));
+    for (int i = 1; i < 7 && ev_use; ++i)
+      if (ev_use[i]) cudaEventRecord(static_cast<cudaEvent_t>(ev_use[i]), s);
+    return MOE_OK;
   }
-  for (int32_t t0 = 0; t0 < N; t0 += T) {
+  for (int32_t t0 = 0; t0 < N && e == cudaSuccess; t0 += T) {
     const Slice sl{t0, (N - t0) < T ? (N - t0) : T};
-    if ((e = rec(1)) != cudaSuccess) break;
-    if ((e = launch_schedule(ids, *sh, sl, phi, offsets, counts, route_row, sched, dev_status, s)) !=
-        cudaSuccess)
-      break;
-    if ((e = rec(2)) != cudaSuccess) break;
-    if ((e = launch_dispatch(x, phi, offsets, xg, *sh, rows_max, dev_status, s)) != cudaSuccess)
-      break;
-    if ((e = rec(3)) != cudaSuccess) break;
-    cudaEvent_t mid = (ev && single) ? static_cast<cudaEvent_t>(ev[4]) : nullptr;
-    if ((e = launch_expert_ffn(xg, W1, W3, W2, offsets, counts, h, y, *sh, rows_max, dev_status, s,
-                               mid)) != cudaSuccess)
-      break;
-    if ((e = rec(5)) != cudaSuccess) break;
-    if ((e = launch_combine(y, route_row, gates, out, *sh, sl, rows_max, dev_status, s)) !=
-        cudaSuccess)
-      break;
-    if ((e = rec(6)) != cudaSuccess) break;
+    e = run_slice(b, x, W1, W3, W2, out, sl, sh, dev_status, s, ev_use);
   }
   return from_cuda(e);
+}
+
+// Per-device copy engines' streams and events of moe_layer_forward_host,
+// created on first use and kept until the process exits.
+constexpr int kRing = 4;
+struct CopyRes {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t entry = nullptr, lg = nullptr, fin = nullptr;
+  cudaEvent_t ex[kRing] = {}, ed[kRing] = {};
+  bool ready = false;
+};
+std::mutex g_copy_mu;
+CopyRes g_copy[64];
+
+cudaError_t copy_res(CopyRes** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  CopyRes& r = g_copy[dev];
+  if (!r.ready) {
+    const unsigned ef = cudaEventDisableTiming;
+    if ((e = cudaStreamCreateWithFlags(&r.h2d, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithFlags(&r.d2h, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&r.entry, ef)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&r.lg, ef)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&r.fin, ef)) != cudaSuccess) return e;
+    for (int i = 0; i < kRing; ++i) {
+      if ((e = cudaEventCreateWithFlags(&r.ex[i], ef)) != cudaSuccess) return e;
+      if ((e = cudaEventCreateWithFlags(&r.ed[i], ef)) != cudaSuccess) return e;
+    }
+    r.ready = true;
+  }
+  *out = &r;
+  return cudaSuccess;
+}
+
+// Host-buffer layer: the rows of slice [t0, t0+Tm) of every peer are copied in
+// on the h2d stream while the previous slice computes on `s`, and copied out
+// on the d2h stream while the next one computes (the transfer minibatch of
+// "Mixture-of-Kittens" notes section 3 and "Beyond Peak TFLOPs" section 1:
+// chunk k transfers while chunk k-1 computes).
+cudaError_t layer_host_pipeline(const float* logits_host, const uint16_t* x_host,
+                                const uint16_t* W1, const uint16_t* W3, const uint16_t* W2,
+                                uint16_t* out_host, int32_t minibatch_tokens, void* ws,
+                                int32_t* dev_status, const moe_shape_t* sh, cudaStream_t s) {
+  std::lock_guard<std::mutex> lock(g_copy_mu);
+  CopyRes* cr = nullptr;
+  cudaError_t e = copy_res(&cr);
+  if (e != cudaSuccess) return e;
+  const LayerWs w = layer_ws(sh);
+  const LayerBufs b = layer_bufs(ws, w);
+  float* logits = at<float>(ws, w.logits);
+  uint16_t* x = at<uint16_t>(ws, w.x);
+  uint16_t* out = at<uint16_t>(ws, w.out);
+  const int32_t P = sh->P, N = sh->N, H = sh->H;
+  const size_t row_bytes = static_cast<size_t>(H) * 2;
+  const int32_t T = (minibatch_tokens <= 0 || minibatch_tokens >= N) ? N : minibatch_tokens;
+  const int32_t S = N == 0 ? 0 : (N + T - 1) / T;
+  auto copy_rows = [&](void* dst, const void* src, int32_t t0, int32_t tm, cudaMemcpyKind kind,
+                       cudaStream_t cs) -> cudaError_t {
+    for (int32_t r = 0; r < P; ++r) {
+      const size_t off = (static_cast<size_t>(r) * N + t0) * row_bytes;
+      cudaError_t ee = cudaMemcpyAsync(static_cast<char*>(dst) + off,
+                                       static_cast<const char*>(src) + off, tm * row_bytes, kind, cs);
+      if (ee != cudaSuccess) return ee;
+    }
+    return cudaSuccess;
+  };
+  // the copies may only start once earlier work on `s` no longer uses ws
+  if ((e = cudaEventRecord(cr->entry, s)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(cr->h2d, cr->entry, 0)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(cr->d2h, cr->entry, 0)) != cudaSuccess) return e;
+  const size_t tokens = static_cast<size_t>(P) * N;
+  if ((e = cudaMemcpyAsync(logits, logits_host, tokens * sh->E * 4, cudaMemcpyHostToDevice,
+                           cr->h2d)) != cudaSuccess)
+    return e;
+  if ((e = cudaEventRecord(cr->lg, cr->h2d)) != cudaSuccess) return e;
+  if (S > 0) {
+    if ((e = copy_rows(x, x_host, 0, T < N ? T : N, cudaMemcpyHostToDevice, cr->h2d)) != cudaSuccess)
+      return e;
+    if ((e = cudaEventRecord(cr->ex[0], cr->h2d)) != cudaSuccess) return e;
+  }
+  if ((e = cudaStreamWaitEvent(s, cr->lg, 0)) != cudaSuccess) return e;
+  if ((e = launch_route_topk(logits, b.ids, b.gates, static_cast<int64_t>(tokens), sh->E, sh->k,
+                             s)) != cudaSuccess)
+    return e;
+  for (int32_t i = 0; i < S; ++i) {
+    const int32_t t0 = i * T, tm = (N - t0) < T ? (N - t0) : T;
+    if (i + 1 < S) {  // prefetch the next slice's rows
+      const int32_t t1 = t0 + T, tm1 = (N - t1) < T ? (N - t1) : T;
+      if ((e = copy_rows(x, x_host, t1, tm1, cudaMemcpyHostToDevice, cr->h2d)) != cudaSuccess)
+        return e;
+      if ((e = cudaEventRecord(cr->ex[(i + 1) % kRing], cr->h2d)) != cudaSuccess) return e;
+    }
+    if ((e = cudaStreamWaitEvent(s, cr->ex[i % kRing], 0)) != cudaSuccess) return e;
+    if ((e = run_slice(b, x, W1, W3, W2, out, Slice{t0, tm}, sh, dev_status, s, nullptr)) !=
+        cudaSuccess)
+      return e;
+    if ((e = cudaEventRecord(cr->ed[i % kRing], s)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(cr->d2h, cr->ed[i % kRing], 0)) != cudaSuccess) return e;
+    if ((e = copy_rows(out_host, out, t0, tm, cudaMemcpyDeviceToHost, cr->d2h)) != cudaSuccess)
+      return e;
+  }
+  // `s` completes only after the last copy out (and every copy in)
+  if ((e = cudaEventRecord(cr->fin, cr->d2h)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(s, cr->fin, 0)) != cudaSuccess) return e;
+  if ((e = cudaEventRecord(cr->fin, cr->h2d)) != cudaSuccess) return e;
+  return cudaStreamWaitEvent(s, cr->fin, 0);
 }
 
 }  // namespace
@@ -271,6 +398,23 @@ moe_status_t moe_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint16
                                      static_cast<cudaStream_t>(stream), nullptr));
 }
 
+moe_status_t moe_expert_ffn_gather(const uint16_t* x, const int32_t* phi, const uint16_t* W1,
+                                   const uint16_t* W3, const uint16_t* W2, const int32_t* offsets,
+                                   const int32_t* counts, uint16_t* h, float* y,
+                                   int32_t* dev_status, const moe_shape_t* shape, void* stream) {
+  moe_status_t st = check_ffn_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!phi || !W1 || !W3 || !W2 || !offsets || !h || !y || !dev_status ||
+      (shape->N > 0 && !x))
+    return MOE_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(phi) || !aligned16(W1) || !aligned16(W3) || !aligned16(W2) ||
+      !aligned16(h) || !aligned16(y))
+    return MOE_INVALID_ARG;
+  return from_cuda(launch_expert_ffn_gather(x, phi, W1, W3, W2, offsets, counts, h, y, *shape,
+                                            rows_max_of(shape), dev_status,
+                                            static_cast<cudaStream_t>(stream), nullptr));
+}
+
 moe_status_t moe_combine(const float* y, const int32_t* route_row, const float* gates,
                          uint16_t* out, int32_t* dev_status, const moe_shape_t* shape,
                          void* stream) {
@@ -318,20 +462,8 @@ moe_status_t moe_layer_forward_host(const float* logits_host, const uint16_t* x_
   if (minibatch_tokens < 0) return MOE_INVALID_ARG;
   const LayerWs w = layer_ws(shape);
   if (ws_bytes < w.total_host) return MOE_WORKSPACE_TOO_SMALL;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t tokens = static_cast<size_t>(shape->P) * shape->N;
-  float* logits = at<float>(ws, w.logits);
-  uint16_t* x = at<uint16_t>(ws, w.x);
-  uint16_t* out = at<uint16_t>(ws, w.out);
-  cudaError_t e = cudaMemcpyAsync(logits, logits_host, tokens * shape->E * 4,
-                                  cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(x, x_host, tokens * shape->H * 2, cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) return MOE_CUDA_ERROR;
-  st = layer_body(logits, x, W1, W3, W2, out, minibatch_tokens, ws, dev_status, shape, s, nullptr);
-  if (st != MOE_OK) return st;
-  e = cudaMemcpyAsync(out_host, out, tokens * shape->H * 2, cudaMemcpyDeviceToHost, s);
-  return from_cuda(e);
+  return from_cuda(layer_host_pipeline(logits_host, x_host, W1, W3, W2, out_host, minibatch_tokens,
+                                       ws, dev_status, shape, static_cast<cudaStream_t>(stream)));
 }
 
 int64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

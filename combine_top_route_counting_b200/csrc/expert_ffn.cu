@@ -84,6 +84,9 @@ struct Cfg {
 };
 
 struct FfnParams {
+  const int2* phi;         // [rows_max] (src_rank, src_idx): GATHER only
+  int32_t n_per_peer;      // N (GATHER: token row = src_rank * N + src_idx)
+  int32_t oob_row;         // P*N: a row index outside x, which reads as zeros
   const int32_t* offsets;  // [E+1]
   const int32_t* counts;   // [E, P] or null
   int32_t E, P;
@@ -112,11 +115,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // MODE 0: GEMM1 + SwiGLU -> bf16 h. MODE 1: GEMM2 -> fp32 y.
+// GATHER (MODE 0 only): the A operand is pulled straight from the token
+// activations x by the schedule Phi ("zero-copy, direct landing"): every lane
+// of the producer warp gathers 4 of the CTA's 128 rows per K step with a TMA
+// tile::gather4 load, so no gathered copy of the tokens is materialised.
 // CG = 1: one CTA per 128x256 tile. CG = 2: a cluster of two CTAs (a tcgen05
 // CTA pair) per 256x256 tile; CTA r loads rows [128r, 128r+128) of A and
 // columns [128r, 128r+128) of B, the leader (r = 0) issues the pair MMAs and
 // each CTA drains its own 128 TMEM lanes.
-template <int MODE, int CG>
+template <int MODE, int CG, bool GATHER>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const FfnParams p) {
@@ -211,7 +218,80 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     return row0 < s_end[l];
   };
 
-  if (warp == 0) {
+  if (warp == 0 && GATHER) {
+    // ------------------------------------------------------------ TMA producer (row gather)
+    const uint32_t full0 = smem_u32(&bars[C::BAR_FULL]);
+    const uint32_t full_tgt0 = (CG == 2) ? mapa_shared(full0, 0) : full0;
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t issued = 0;
+    bool ok = true;
+    int bad = 0;
+    for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
+      int row0, n, l;
+      if (!tile_info(tile, row0, n, l)) continue;
+      const int arow = row0 + static_cast<int>(rank) * 128;
+      // rows arow + 4*lane .. +3 of the tile: their token rows in x
+      int tok[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int2 e = __ldg(p.phi + arow + 4 * lane + i);
+        const bool v = e.x >= 0 && e.x < p.P && e.y >= 0 && e.y < p.n_per_peer;
+        if (!v && (e.x >= 0 || e.y != -1)) bad = 1;  // (-1,-1) is padding
+        tok[i] = v ? e.x * p.n_per_peer + e.y : p.oob_row;
+      }
+      const int ky0 = l * p.K;
+      for (int kb = 0; kb < kblocks; ++kb) {
+        uint32_t w_ok = 1;
+        if (lane == 0) w_ok = wait_bounded(smem_u32(&bars[C::BAR_EMPTY + stage]), phase ^ 1u, wc) ? 1u : 0u;
+        w_ok = __shfl_sync(0xFFFFFFFFu, w_ok, 0);
+        if (!w_ok) {
+          ok = false;
+          break;
+        }
+        const uint32_t full_local = full0 + stage * 8;
+        const uint32_t full_tgt = full_tgt0 + stage * 8;
+        const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
+        const uint32_t sB = sA + C::A_BYTES;
+        const int ky = ky0 + kb * C::BK;
+        if (lane == 0 && leader) mbar_arrive_expect_tx(full_local, CG * C::STAGE_BYTES);
+        __syncwarp();
+        // 4 rows x 128 bytes land at sA + 512*lane: the same 128-byte-swizzled
+        // layout a 128-row box load produces
+        if (CG == 2)
+          tma_gather4_pair(sA + lane * 512, &tmA, kb * C::BK, tok[0], tok[1], tok[2], tok[3], full_tgt);
+        else
+          tma_gather4(sA + lane * 512, &tmA, kb * C::BK, tok[0], tok[1], tok[2], tok[3], full_tgt);
+        if (lane == 0) {
+          if (CG == 1) {
+            tma_load_2d(sB + 0 * C::B_ATOM_BYTES, &tmB0, n * 128, ky, full_tgt);
+            tma_load_2d(sB + 1 * C::B_ATOM_BYTES, &tmB0, n * 128 + 64, ky, full_tgt);
+            tma_load_2d(sB + 2 * C::B_ATOM_BYTES, &tmB1, n * 128, ky, full_tgt);
+            tma_load_2d(sB + 3 * C::B_ATOM_BYTES, &tmB1, n * 128 + 64, ky, full_tgt);
+          } else {
+            const CUtensorMap* mb = (rank == 1) ? &tmB1 : &tmB0;
+            tma_load_2d_pair(sB, mb, n * 128, ky, full_tgt);
+            tma_load_2d_pair(sB + C::B_ATOM_BYTES, mb, n * 128 + 64, ky, full_tgt);
+          }
+        }
+        ++issued;
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (bad) atomicOr(p.dev_status, MOE_DEV_BAD_SCHEDULE);
+    __syncwarp();
+    if (lane == 0) {
+      const int64_t first = issued > C::STAGES ? issued - C::STAGES : 0;
+      for (int64_t j = first; j < issued; ++j) {
+        const int st = static_cast<int>(j % C::STAGES);
+        const uint32_t par = static_cast<uint32_t>((j / C::STAGES) & 1);
+        wait_drain(smem_u32(&bars[(leader ? C::BAR_FULL : C::BAR_EMPTY) + st]), par, drain_ns);
+      }
+    }
+  } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       // the leader's full barriers count the bytes of both CTAs of a pair
@@ -344,45 +424,57 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int64_t row = row0 + static_cast<int>(rank) * 128 + q * 32 + lane;
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::BN);
+      // TMEM reads are double-buffered: chunk c+1 is in flight while chunk c
+      // is converted and stored.
       if (MODE == 0) {
         // accumulator columns [0,128) = x.W1, [128,256) = x.W3 for h columns n*128 + j
         __nv_bfloat16* hrow =
             reinterpret_cast<__nv_bfloat16*>(p.out) + row * p.Nout + n * 128 + half * 64;
-#pragma unroll 1
+        uint32_t ra[2][32], rb[2][32];
+        tmem_ld_32cols(tbase + half * 64, ra[0]);
+        tmem_ld_32cols(tbase + 128 + half * 64, rb[0]);
+        tmem_ld_wait();
+#pragma unroll
         for (int c = 0; c < 2; ++c) {
-          uint32_t ra[32], rb[32];
-          tmem_ld_32cols(tbase + half * 64 + c * 32, ra);
-          tmem_ld_32cols(tbase + 128 + half * 64 + c * 32, rb);
-          tmem_ld_wait();
+          if (c + 1 < 2) {
+            tmem_ld_32cols(tbase + half * 64 + (c + 1) * 32, ra[(c + 1) & 1]);
+            tmem_ld_32cols(tbase + 128 + half * 64 + (c + 1) * 32, rb[(c + 1) & 1]);
+          }
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float h0 = silu(__uint_as_float(ra[2 * i])) * __uint_as_float(rb[2 * i]);
-            const float h1 = silu(__uint_as_float(ra[2 * i + 1])) * __uint_as_float(rb[2 * i + 1]);
+            const float h0 = silu(__uint_as_float(ra[c & 1][2 * i])) * __uint_as_float(rb[c & 1][2 * i]);
+            const float h1 =
+                silu(__uint_as_float(ra[c & 1][2 * i + 1])) * __uint_as_float(rb[c & 1][2 * i + 1]);
             pk[i] = pack_bf16x2(h0, h1);
           }
-          const uint32_t(&lo)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&pk[0]);
-          const uint32_t(&hi)[8] = *reinterpret_cast<const uint32_t(*)[8]>(&pk[8]);
-          st_global_v8(hrow + c * 32, lo);
-          st_global_v8(hrow + c * 32 + 16, hi);
+          st_global_v8(hrow + c * 32, *reinterpret_cast<const uint32_t(*)[8]>(&pk[0]));
+          st_global_v8(hrow + c * 32 + 16, *reinterpret_cast<const uint32_t(*)[8]>(&pk[8]));
+          if (c + 1 < 2) tmem_ld_wait();
         }
       } else {
         float* yrow = reinterpret_cast<float*>(p.out) + row * p.Nout + n * C::BN + half * 128;
-#pragma unroll 1
+        uint32_t rv[2][32];
+        tmem_ld_32cols(tbase + half * 128, rv[0]);
+        tmem_ld_wait();
+#pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t rv[32];
-          tmem_ld_32cols(tbase + half * 128 + c * 32, rv);
-          tmem_ld_wait();
+          if (c + 1 < 4) tmem_ld_32cols(tbase + half * 128 + (c + 1) * 32, rv[(c + 1) & 1]);
 #pragma unroll
           for (int v = 0; v < 4; ++v)
-            st_global_v8(yrow + c * 32 + v * 8, *reinterpret_cast<const uint32_t(*)[8]>(&rv[8 * v]));
+            st_global_v8(yrow + c * 32 + v * 8,
+                         *reinterpret_cast<const uint32_t(*)[8]>(&rv[c & 1][8 * v]));
+          if (c + 1 < 4) tmem_ld_wait();
         }
       }
+      // The accumulator may be overwritten once every lane's tcgen05.ld has
+      // completed (tcgen05.wait::ld above); the global stores need no ordering
+      // against the next MMAs, so the arrive is relaxed (no memory fence).
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if (CG == 2) mbar_arrive_cluster(tempty_tgt0 + acc * 8);
-        else mbar_arrive(tempty0 + acc * 8);
+        if (CG == 2) mbar_arrive_relaxed_cluster(tempty_tgt0 + acc * 8);
+        else mbar_arrive_relaxed(tempty0 + acc * 8);
       }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
@@ -429,11 +521,11 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE, int CG>
+template <int MODE, int CG, bool GATHER = false>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const FfnParams& p, cudaStream_t s) {
   const size_t smem = smem_bytes_for<CG>(p.E);
-  cudaError_t e = cudaFuncSetAttribute(ffn_gemm_kernel<MODE, CG>,
+  cudaError_t e = cudaFuncSetAttribute(ffn_gemm_kernel<MODE, CG, GATHER>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -452,7 +544,7 @@ cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUten
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  e = cudaLaunchKernelEx(&cfg, ffn_gemm_kernel<MODE, CG>, a, b0, b1, p);
+  e = cudaLaunchKernelEx(&cfg, ffn_gemm_kernel<MODE, CG, GATHER>, a, b0, b1, p);
   note_launches(1);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -474,14 +566,42 @@ cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint
   // Segments that are multiples of 256 rows run on CTA pairs (256x256 tiles);
   // otherwise (pad a multiple of 128 only) on single CTAs (128x256 tiles).
   const bool pair = (sh.pad % 256) == 0;
-  FfnParams p1{offsets, counts, E, sh.P, H, I, rows_max, h, dev_status, kWaitTimeoutNs};
+  FfnParams p1{nullptr, 0, 0, offsets, counts, E, sh.P, H, I, rows_max, h, dev_status, kWaitTimeoutNs};
   cudaError_t e = pair ? launch_mode<0, 2>(mA1, mW1, mW3, p1, s) : launch_mode<0, 1>(mA1, mW1, mW3, p1, s);
   if (e != cudaSuccess) return e;
   if (ev_mid) {
     e = cudaEventRecord(ev_mid, s);
     if (e != cudaSuccess) return e;
   }
-  FfnParams p2{offsets, counts, E, sh.P, I, H, rows_max, y, dev_status, kWaitTimeoutNs};
+  FfnParams p2{nullptr, 0, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status, kWaitTimeoutNs};
+  return pair ? launch_mode<1, 2>(mA2, mW2, mW2, p2, s) : launch_mode<1, 1>(mA2, mW2, mW2, p2, s);
+}
+
+cudaError_t launch_expert_ffn_gather(const uint16_t* x, const int32_t* phi, const uint16_t* W1,
+                                     const uint16_t* W3, const uint16_t* W2,
+                                     const int32_t* offsets, const int32_t* counts, uint16_t* h,
+                                     float* y, const moe_shape_t& sh, int64_t rows_max,
+                                     int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_mid) {
+  const int E = sh.E, H = sh.H, I = sh.I;
+  const int64_t tokens = static_cast<int64_t>(sh.P) * sh.N;
+  CUtensorMap mX, mW1, mW3, mA2, mW2;
+  const uint64_t EH = static_cast<uint64_t>(E) * H, EI = static_cast<uint64_t>(E) * I;
+  // x viewed as [P*N, H] with a one-row box: the gather4 form
+  if (!make_map(&mX, x, H, static_cast<uint64_t>(tokens > 0 ? tokens : 1), 64, 1) ||
+      !make_map(&mW1, W1, I, EH, 64, 64) || !make_map(&mW3, W3, I, EH, 64, 64) ||
+      !make_map(&mA2, h, I, rows_max, 64, 128) || !make_map(&mW2, W2, H, EI, 64, 64))
+    return cudaErrorInvalidValue;
+  const bool pair = (sh.pad % 256) == 0;
+  FfnParams p1{reinterpret_cast<const int2*>(phi), sh.N, static_cast<int32_t>(tokens), offsets,
+               counts, E, sh.P, H, I, rows_max, h, dev_status, kWaitTimeoutNs};
+  cudaError_t e = pair ? launch_mode<0, 2, true>(mX, mW1, mW3, p1, s)
+                       : launch_mode<0, 1, true>(mX, mW1, mW3, p1, s);
+  if (e != cudaSuccess) return e;
+  if (ev_mid) {
+    e = cudaEventRecord(ev_mid, s);
+    if (e != cudaSuccess) return e;
+  }
+  FfnParams p2{nullptr, 0, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status, kWaitTimeoutNs};
   return pair ? launch_mode<1, 2>(mA2, mW2, mW2, p2, s) : launch_mode<1, 1>(mA2, mW2, mW2, p2, s);
 }
 

@@ -43,6 +43,13 @@ cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint
                               uint16_t* h, float* y, const moe_shape_t& sh, int64_t rows_max,
                               int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_mid);
 
+// Steps 3a+3b fused: GEMM1 pulls its A rows from x by Phi (no xg buffer)
+cudaError_t launch_expert_ffn_gather(const uint16_t* x, const int32_t* phi, const uint16_t* W1,
+                                     const uint16_t* W3, const uint16_t* W2,
+                                     const int32_t* offsets, const int32_t* counts, uint16_t* h,
+                                     float* y, const moe_shape_t& sh, int64_t rows_max,
+                                     int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_mid);
+
 // Step 4
 cudaError_t launch_combine(const float* y, const int32_t* route_row, const float* gates,
                            uint16_t* out, const moe_shape_t& sh, Slice sl, int64_t rows_max,

@@ -5,11 +5,19 @@
 // every token the k largest logits are taken in descending order, ties to the
 // lower expert id; the gates are the softmax over those k logits.
 //
-// One warp per token. Lane `lane` holds logits lane, lane+32, ... (each
-// register column is one coalesced 128-byte load). Each of the k rounds is a
-// lane-local best followed by a butterfly argmax over the warp under the
-// total order (value descending, id ascending); the owner lane marks the
-// winner as taken. HBM-bound: the logits are read once.
+// One warp per token; lane `lane` holds logits lane, lane+32, ... (each
+// register column is one coalesced 128-byte load). Selection avoids k rounds
+// of warp-wide argmax:
+//   1. tau = the k-th largest of the 32 lane maxima (a warp bitonic sort).
+//      These are k actual logits of the token, so tau is at most its k-th
+//      largest logit: every chosen expert has a logit >= tau.
+//   2. The few logits >= tau (usually a little more than k) are compacted
+//      into shared memory; each candidate's rank under the total order
+//      (value descending, id ascending) is counted against the others, and
+//      ranks 0..k-1 are the slots. Exact: ranks of a total order are unique.
+//   3. If more than 32 logits reach tau (heavy ties, -inf logits), the warp
+//      falls back to k rounds of butterfly argmax over all its logits.
+// HBM-bound: the logits are read once.
 #include <cfloat>
 #include <climits>
 #include <cmath>
@@ -20,6 +28,7 @@ namespace moe {
 namespace {
 
 constexpr int kMaxK = 16;
+constexpr int kCand = 32;  // candidate buffer per warp
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 __device__ __forceinline__ bool better(float v, int id, float bv, int bid) {
@@ -31,31 +40,79 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
                                                          int32_t* __restrict__ ids,
                                                          float* __restrict__ gates,
                                                          int64_t n_tokens, int E, int k) {
-  const int lane = threadIdx.x & 31;
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  __shared__ float s_cv[8][kCand];
+  __shared__ int s_ci[8][kCand];
+  __shared__ float s_sv[8][kMaxK];
+  __shared__ int s_si[8][kMaxK];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + w;
   if (t >= n_tokens) return;  // whole warp leaves together
   const float* row = logits + t * E;
 
   float v[VPL];
-  uint32_t taken = 0;
+  float m = -INFINITY;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int e = i * 32 + lane;
-    if (e < E) {
-      v[i] = __ldg(row + e);
-    } else {
-      v[i] = -INFINITY;
-      taken |= 1u << i;  // not an expert
-    }
+    v[i] = (e < E) ? __ldg(row + e) : -INFINITY;
+    m = fmaxf(m, v[i]);
   }
 
-  float sel_v[kMaxK];
-  int sel_id[kMaxK];
+  // 1. tau: k-th largest lane maximum (bitonic sort, descending across lanes)
+  float x = m;
 #pragma unroll
-  for (int j = 0; j < kMaxK; ++j) {
-    sel_v[j] = -INFINITY;
-    sel_id[j] = 0;
-    if (j < k) {
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const float o = __shfl_xor_sync(kFull, x, stride);
+      const bool asc = (lane & size) != 0;  // final stage (size 32): descending
+      const bool lower = (lane & stride) == 0;
+      x = (lower != asc) ? fmaxf(x, o) : fminf(x, o);
+    }
+  }
+  const float tau = __shfl_sync(kFull, x, k - 1);
+
+  // 2. compact the logits >= tau
+  int c = 0;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) c += (i * 32 + lane < E && v[i] >= tau) ? 1 : 0;
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int total = __shfl_sync(kFull, incl, 31);
+
+  if (total <= kCand) {
+    int pos = incl - c;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = i * 32 + lane;
+      if (e < E && v[i] >= tau) {
+        s_cv[w][pos] = v[i];
+        s_ci[w][pos] = e;
+        ++pos;
+      }
+    }
+    __syncwarp();
+    if (lane < total) {
+      const float cv = s_cv[w][lane];
+      const int ci = s_ci[w][lane];
+      int rank = 0;
+      for (int j = 0; j < total; ++j) rank += better(s_cv[w][j], s_ci[w][j], cv, ci) ? 1 : 0;
+      if (rank < k) {
+        s_sv[w][rank] = cv;
+        s_si[w][rank] = ci;
+      }
+    }
+  } else {
+    // 3. fallback: k rounds of warp argmax over every logit of the token
+    uint32_t taken = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i)
+      if (i * 32 + lane >= E) taken |= 1u << i;
+    for (int j = 0; j < k; ++j) {
       float bv = -INFINITY;
       int bid = INT_MAX;
 #pragma unroll
@@ -76,29 +133,21 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
         }
       }
       if (bid != INT_MAX && (bid & 31) == lane) taken |= 1u << (bid >> 5);
-      sel_v[j] = bv;
-      sel_id[j] = bid;
+      if (lane == 0) {
+        s_sv[w][j] = bv;
+        s_si[w][j] = bid;
+      }
     }
   }
+  __syncwarp();
 
   // gates: softmax over the chosen logits, summed in slot order
-  const float l0 = sel_v[0];
-  float ex[kMaxK];
-  float den = 0.0f;
-#pragma unroll
-  for (int j = 0; j < kMaxK; ++j) {
-    ex[j] = 0.0f;
-    if (j < k) {
-      ex[j] = expf(sel_v[j] - l0);
-      den += ex[j];
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < kMaxK; ++j) {
-    if (j < k && lane == j) {
-      ids[t * k + j] = sel_id[j];
-      gates[t * k + j] = ex[j] / den;
-    }
+  if (lane < k) {
+    const float l0 = s_sv[w][0];
+    float den = 0.0f;
+    for (int j = 0; j < k; ++j) den += expf(s_sv[w][j] - l0);
+    ids[t * k + lane] = s_si[w][lane];
+    gates[t * k + lane] = expf(s_sv[w][lane] - l0) / den;
   }
 }
 

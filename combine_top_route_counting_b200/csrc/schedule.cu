@@ -37,6 +37,15 @@ constexpr int kInvalid = 0x40000000;  // match key of lanes without a valid rout
 constexpr unsigned kFull = 0xFFFFFFFFu;
 static_assert(kWarps * kWarpRoutes == kSchedBlockRoutes, "block covers 2048 routes");
 
+// Programmatic dependent launch: a kernel of the chain lets the next one be
+// scheduled early (launch_dependents) and waits for its predecessor's results
+// before touching them (wait). Every block executes the wait unconditionally,
+// so each kernel completes after its predecessor.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 struct SchedParams {
   const int32_t* ids;
   int32_t P, N, k, E, pad;
@@ -56,6 +65,7 @@ __device__ __forceinline__ int64_t route_index(const SchedParams& p, int r, int 
 
 __global__ void __launch_bounds__(kThreads) sched_count_kernel(SchedParams p) {
   extern __shared__ int32_t hist[];
+  pdl_launch_dependents();
   const int c = blockIdx.x, r = blockIdx.y;
   const int R = p.Tm * p.k;
   for (int l = threadIdx.x; l < p.E; l += kThreads) hist[l] = 0;
@@ -79,14 +89,28 @@ __global__ void __launch_bounds__(kThreads) sched_count_kernel(SchedParams p) {
 }
 
 __global__ void __launch_bounds__(kThreads) sched_scan_kernel(SchedParams p) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int idx = blockIdx.x * kThreads + threadIdx.x;
   if (idx >= p.P * p.E) return;
   const int r = idx / p.E, l = idx - r * p.E;
   int32_t* col = p.ws + static_cast<int64_t>(r) * p.C * p.E + l;
+  const int64_t stride = p.E;
   int run = 0;
-  for (int c = 0; c < p.C; ++c) {
-    const int v = col[static_cast<int64_t>(c) * p.E];
-    col[static_cast<int64_t>(c) * p.E] = run;
+  int c = 0;
+  for (; c + 8 <= p.C; c += 8) {  // eight independent loads in flight
+    int v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = col[(c + u) * stride];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      col[(c + u) * stride] = run;
+      run += v[u];
+    }
+  }
+  for (; c < p.C; ++c) {
+    const int v = col[c * stride];
+    col[c * stride] = run;
     run += v;
   }
   p.counts[l * p.P + r] = run;
@@ -95,6 +119,8 @@ __global__ void __launch_bounds__(kThreads) sched_scan_kernel(SchedParams p) {
 // One block of 1024 threads (E <= 1024): one expert per thread.
 __global__ void __launch_bounds__(1024) sched_offsets_kernel(SchedParams p) {
   __shared__ int32_t warp_tot[32];
+  pdl_launch_dependents();
+  pdl_wait();
   const int l = threadIdx.x, lane = l & 31, w = l >> 5;
   int tp = 0;
   if (l < p.E) {
@@ -125,8 +151,14 @@ __global__ void __launch_bounds__(1024) sched_offsets_kernel(SchedParams p) {
   if (l == 1023) p.offsets[p.E] = incl;  // tp = 0 beyond E: total
 }
 
+// STAGE: counts [E][P] and offsets [E+1] are copied to shared memory (when
+// they fit), so the O(P) placement loop reads them from there.
+template <bool STAGE>
 __global__ void __launch_bounds__(kThreads) sched_scatter_kernel(SchedParams p) {
-  extern __shared__ int32_t wbase[];  // [kWarps][E]
+  extern __shared__ int32_t smem[];
+  int32_t* wbase = smem;                      // [kWarps][E]
+  int32_t* s_cnt = smem + kWarps * p.E;       // [E][P]   (STAGE)
+  int32_t* s_off = s_cnt + p.E * p.P;         // [E+1]    (STAGE)
   const int c = blockIdx.x, r = blockIdx.y;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int R = p.Tm * p.k;
@@ -134,7 +166,8 @@ __global__ void __launch_bounds__(kThreads) sched_scatter_kernel(SchedParams p) 
   for (int l = lane; l < p.E; l += 32) wh[l] = 0;
   __syncwarp();
 
-  // pass 1: this warp's per-expert counts over its 256 routes
+  // pass 1: this warp's per-expert counts over its 256 routes (ids were
+  // written before this chain started)
   const int q0 = c * kSchedBlockRoutes + w * kWarpRoutes;
   int key[kSteps];
 #pragma unroll
@@ -148,6 +181,15 @@ __global__ void __launch_bounds__(kThreads) sched_scatter_kernel(SchedParams p) 
     const unsigned m = __match_any_sync(kFull, key[s]);
     if (key[s] != kInvalid && lane == __ffs(m) - 1) wh[key[s]] += __popc(m);
     __syncwarp();
+  }
+  pdl_wait();  // block bases, counts and offsets come from the previous kernels
+  const int32_t* cnt = p.counts;
+  const int32_t* off = p.offsets;
+  if (STAGE) {
+    for (int i = threadIdx.x; i < p.E * p.P; i += kThreads) s_cnt[i] = p.counts[i];
+    for (int i = threadIdx.x; i <= p.E; i += kThreads) s_off[i] = p.offsets[i];
+    cnt = s_cnt;
+    off = s_off;
   }
   __syncthreads();
 
@@ -180,14 +222,14 @@ __global__ void __launch_bounds__(kThreads) sched_scatter_kernel(SchedParams p) 
     if (q < R) {
       const int64_t g = route_index(p, r, q);
       if (valid) {
-        const int32_t* Ml = p.counts + id * p.P;
+        const int32_t* Ml = cnt + id * p.P;
         int pos = 0;
         for (int r2 = 0; r2 < p.P; ++r2) {
-          const int mm = __ldg(Ml + r2);
+          const int mm = Ml[r2];
           pos += min(mm, o);
           pos += (r2 < r && mm > o) ? 1 : 0;
         }
-        const int row = __ldg(p.offsets + id) + pos;
+        const int row = off[id] + pos;
         reinterpret_cast<int2*>(p.phi)[row] = make_int2(r, p.t0 + q / p.k);
         p.route_row[g] = row;
       } else {
@@ -201,8 +243,8 @@ __global__ void __launch_bounds__(kThreads) sched_scatter_kernel(SchedParams p) 
   const int b = blockIdx.y * gridDim.x + blockIdx.x;
   for (int l = b; l < p.E; l += nb) {
     int T = 0;
-    for (int r2 = 0; r2 < p.P; ++r2) T += __ldg(p.counts + l * p.P + r2);
-    const int start = __ldg(p.offsets + l) + T, end = __ldg(p.offsets + l + 1);
+    for (int r2 = 0; r2 < p.P; ++r2) T += cnt[l * p.P + r2];
+    const int start = off[l] + T, end = off[l + 1];
     for (int row = start + threadIdx.x; row < end; row += kThreads)
       reinterpret_cast<int2*>(p.phi)[row] = make_int2(-1, -1);
   }
@@ -241,19 +283,49 @@ cudaError_t launch_schedule(const int32_t* ids, const moe_shape_t& sh, Slice sl,
   p.ws = ws;
   p.dev_status = dev_status;
   int launched = 0;
+  cudaError_t e = cudaSuccess;
+  // count runs in plain stream order (after whatever wrote ids); scan, offsets
+  // and scatter are launched as programmatic dependents of their predecessor.
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  auto cfg = [&](dim3 grid, dim3 block, size_t smem, bool dependent) {
+    cudaLaunchConfig_t c = {};
+    c.gridDim = grid;
+    c.blockDim = block;
+    c.dynamicSmemBytes = smem;
+    c.stream = s;
+    c.attrs = dependent ? pdl : nullptr;
+    c.numAttrs = dependent ? 1 : 0;
+    return c;
+  };
   if (p.C > 0) {
-    sched_count_kernel<<<dim3(p.C, p.P), kThreads, p.E * sizeof(int32_t), s>>>(p);
+    const cudaLaunchConfig_t c = cfg(dim3(p.C, p.P), dim3(kThreads), p.E * sizeof(int32_t), false);
+    e = cudaLaunchKernelEx(&c, sched_count_kernel, p);
     ++launched;
   }
-  const int scan_blocks = (p.P * p.E + kThreads - 1) / kThreads;
-  sched_scan_kernel<<<scan_blocks, kThreads, 0, s>>>(p);
-  sched_offsets_kernel<<<1, 1024, 0, s>>>(p);
-  launched += 2;
-  if (p.C > 0) {
-    sched_scatter_kernel<<<dim3(p.C, p.P), kThreads, kWarps * p.E * sizeof(int32_t), s>>>(p);
+  if (e == cudaSuccess) {
+    const int scan_blocks = (p.P * p.E + kThreads - 1) / kThreads;
+    const cudaLaunchConfig_t c = cfg(dim3(scan_blocks), dim3(kThreads), 0, p.C > 0);
+    e = cudaLaunchKernelEx(&c, sched_scan_kernel, p);
+    ++launched;
+  }
+  if (e == cudaSuccess) {
+    const cudaLaunchConfig_t c = cfg(dim3(1), dim3(1024), 0, true);
+    e = cudaLaunchKernelEx(&c, sched_offsets_kernel, p);
+    ++launched;
+  }
+  if (e == cudaSuccess && p.C > 0) {
+    const size_t stage_words = static_cast<size_t>(p.E) * p.P + p.E + 1;
+    const bool stage = stage_words <= 8192;
+    const size_t smem = (kWarps * static_cast<size_t>(p.E) + (stage ? stage_words : 0)) * 4;
+    const cudaLaunchConfig_t c = cfg(dim3(p.C, p.P), dim3(kThreads), smem, true);
+    e = stage ? cudaLaunchKernelEx(&c, sched_scatter_kernel<true>, p)
+              : cudaLaunchKernelEx(&c, sched_scatter_kernel<false>, p);
     ++launched;
   }
   note_launches(launched);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -62,6 +62,7 @@ _SIGS = {
     "moe_dispatch": ([_vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Shape), _vp], ctypes.c_int),
     "moe_expert_ffn": ([_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Shape), _vp],
                        ctypes.c_int),
+    "moe_expert_ffn_gather": ([_vp] * 10 + [ctypes.POINTER(Shape), _vp], ctypes.c_int),
     "moe_combine": ([_vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Shape), _vp], ctypes.c_int),
     "moe_layer_forward": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int32, _vp, ctypes.c_size_t, _vp,
                            ctypes.POINTER(Shape), _vp, ctypes.POINTER(_vp)], ctypes.c_int),
@@ -195,6 +196,19 @@ def moe_expert_ffn(xg, W1, W3, W2, offsets, counts, h, y, dev_status, sh: Shape,
                                  _ptr(h, torch.bfloat16, "h"), _ptr(y, torch.float32, "y"),
                                  _ptr(dev_status, torch.int32, "dev_status"), ctypes.byref(sh),
                                  _stream(stream)), "moe_expert_ffn")
+
+
+def moe_expert_ffn_gather(x, phi, W1, W3, W2, offsets, counts, h, y, dev_status, sh: Shape,
+                          stream=None):
+    _check(load().moe_expert_ffn_gather(_ptr(x, torch.bfloat16, "x"), _ptr(phi, torch.int32, "phi"),
+                                        _ptr(W1, torch.bfloat16, "W1"),
+                                        _ptr(W3, torch.bfloat16, "W3"),
+                                        _ptr(W2, torch.bfloat16, "W2"),
+                                        _ptr(offsets, torch.int32, "offsets"),
+                                        _ptr(counts, torch.int32, "counts"),
+                                        _ptr(h, torch.bfloat16, "h"), _ptr(y, torch.float32, "y"),
+                                        _ptr(dev_status, torch.int32, "dev_status"),
+                                        ctypes.byref(sh), _stream(stream)), "moe_expert_ffn_gather")
 
 
 def moe_combine(y, route_row, gates, out, dev_status, sh: Shape, stream=None):

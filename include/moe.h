@@ -180,6 +180,23 @@ moe_status_t moe_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint16
                             uint16_t* h, float* y, int32_t* dev_status,
                             const moe_shape_t* shape, void* stream);
 
+/* Steps 3a + 3b fused -- the pull dispatch lands the tokens directly in the
+ * FFN's operand tiles ("Mixture-of-Kittens" notes section 2, zero-copy direct
+ * landing; "Beyond Peak TFLOPs" 2.A): GEMM1 reads row `row` of its A operand
+ * as x[src_rank*N + src_idx] with (src_rank, src_idx) = phi[row] (zeros for
+ * padding rows) through TMA row gathers, so no gathered buffer exists.
+ * x: bf16 [P*N, H]; phi: int32 [moe_rows_max, 2] as written by moe_schedule;
+ * everything else as moe_expert_ffn, whose h and y it reproduces bit for bit.
+ * An out-of-range Phi entry raises MOE_DEV_BAD_SCHEDULE and reads as zeros.
+ * It needs no [moe_rows_max, H] gathered buffer, but on B200 it runs about 3x
+ * slower than moe_dispatch + moe_expert_ffn (the row gathers deliver fewer
+ * bytes per clock than the tensor cores consume), so moe_layer_forward uses
+ * the latter. */
+moe_status_t moe_expert_ffn_gather(const uint16_t* x, const int32_t* phi, const uint16_t* W1,
+                                   const uint16_t* W3, const uint16_t* W2, const int32_t* offsets,
+                                   const int32_t* counts, uint16_t* h, float* y,
+                                   int32_t* dev_status, const moe_shape_t* shape, void* stream);
+
 /* Step 4 -- push combine in a fixed floating-point order ("Scan once, scatter
  * once" opening and "Beyond Peak TFLOPs" opening: bitwise-reproducible outputs).
  * out[t] = bf16_rne(acc) with acc = 0.0f; acc = fmaf(gates[t,j], y[route_row[t,j]], acc)
@@ -207,9 +224,16 @@ moe_status_t moe_layer_forward(const float* logits, const uint16_t* x, const uin
 /* moe_layer_forward with HOST inputs and output: logits_host fp32 [P*N, E],
  * x_host bf16 [P*N, H] and out_host bf16 [P*N, H] live in host memory (pinned
  * memory makes the copies asynchronous); the weights, ws (of
- * moe_layer_host_workspace_bytes) and dev_status are device memory. The
- * host->device copies, the layer and the device->host copy are all enqueued
- * on `stream`; out_host is valid after the stream is synchronised. */
+ * moe_layer_host_workspace_bytes) and dev_status are device memory.
+ * Transfers overlap compute at the granularity of the transfer slice
+ * `minibatch_tokens` (MoK notes section 3; "Beyond Peak TFLOPs" section 1:
+ * chunk k moves while chunk k-1 computes): the logits and slice 0 are copied
+ * in, then slice s+1's rows are copied in and slice s-1's outputs copied out
+ * while slice s computes on `stream`. 0 = one slice (no overlap). The copies
+ * run on two internal streams per device (host-to-device, device-to-host)
+ * with a few events, created on the first call on that device and kept until
+ * exit; `stream` is made to wait for them, so out_host is valid once `stream`
+ * has been synchronised. Calls from several host threads are serialised. */
 moe_status_t moe_layer_forward_host(const float* logits_host, const uint16_t* x_host,
                                     const uint16_t* W1, const uint16_t* W3, const uint16_t* W2,
                                     uint16_t* out_host, int32_t minibatch_tokens, void* ws,

@@ -154,6 +154,31 @@ def test_route_topk_ties(cuda_lib):
     np.testing.assert_allclose(gates.cpu().numpy(), o_g64, rtol=1e-6)
 
 
+@pytest.mark.parametrize("E,k", [(64, 4), (384, 8), (1024, 16), (7, 7)])
+def test_route_topk_heavy_ties_and_neg_inf(cuda_lib, E, k):
+    """Rows with many equal logits (more than 32 reach the threshold: the
+    fallback path) and rows with -inf logits, mixed with ordinary rows."""
+    moe = cuda_lib
+    g = torch.Generator().manual_seed(E + k)
+    T = 300
+    lg = torch.randn((T, E), generator=g)
+    lg[0::5] = 0.0                                    # all tied
+    lg[1::5, : E // 2] = float("-inf")                # half the experts unreachable
+    lg[2::5] = torch.randint(0, 3, (len(range(2, T, 5)), E), generator=g).float()  # coarse ties
+    lg[3::5, 1:] = float("-inf")                      # one finite logit, the rest -inf
+    sh = moe.shape(1, T, E, k)
+    ids = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    gates = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    moe.moe_route_topk(lg.to(DEV), ids, gates, sh)
+    torch.cuda.synchronize()
+    o_ids, _, o_g64 = oracle.route_topk(lg, k)
+    assert (ids.cpu().numpy() == o_ids).all()
+    g_ = gates.cpu().numpy().astype(np.float64)
+    ok = o_g64 > 0
+    assert np.all(np.abs(g_[ok] - o_g64[ok]) / o_g64[ok] < 1e-6)
+    assert np.all(g_[~ok] == 0)
+
+
 # ---------------------------------------------------------------- stages on small layers
 def _stage_run(moe, w, W1, W3, W2, lg, x):
     """Run every stage through its own entry point; return device tensors."""
@@ -228,6 +253,51 @@ def test_ffn_no_counts_computes_padding_rows(cuda_lib):
     assert (y2[pad] == 0).all() and (h2[pad].float() == 0).all()
     real = torch.from_numpy(np.nonzero(r["phi"][:rows, 0].cpu().numpy() >= 0)[0]).to(DEV)
     assert torch.equal(y2[real], r["y"][real]) and torch.equal(h2[real], r["h"][real])
+
+
+@pytest.mark.parametrize("name,pad", [("tiny", 256), ("mid", 256), ("tiny", 128)])
+def test_ffn_gather_equals_dispatch_then_ffn(cuda_lib, name, pad):
+    """The FFN that pulls its rows from x by Phi reproduces dispatch + FFN bit for bit."""
+    moe = cuda_lib
+    w0 = inputs.WORKLOADS[name]
+    w = inputs.Workload(w0.name, w0.wid, P=w0.P, N=w0.N, E=w0.E, k=w0.k, H=w0.H, I=w0.I, pad=pad)
+    lg, x = inputs.make_logits(w0), inputs.make_x(w0)
+    W1, W3, W2 = [t.to(DEV) for t in inputs.make_weights(w0)]
+    r = _stage_run(moe, w, W1, W3, W2, lg.to(DEV), x.to(DEV))
+    sh = moe.shape(**w.shape())
+    h2 = torch.full_like(r["h"], 3.0)
+    y2 = torch.full_like(r["y"], 3.0)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    moe.moe_expert_ffn_gather(x.to(DEV), r["phi"], W1, W3, W2, r["offsets"], r["counts"], h2, y2,
+                              st, sh)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rows = int(r["offsets"][-1].item())
+    real = torch.from_numpy(np.nonzero(r["phi"][:rows, 0].cpu().numpy() >= 0)[0]).to(DEV)
+    assert torch.equal(h2[real], r["h"][real]) and torch.equal(y2[real], r["y"][real])
+
+
+def test_ffn_gather_flags_corrupt_phi(cuda_lib):
+    """A Phi entry outside [0,P)x[0,N) is reported and its row reads as zeros."""
+    moe = cuda_lib
+    w = inputs.WORKLOADS["tiny"]
+    lg, x = inputs.make_logits(w), inputs.make_x(w)
+    W1, W3, W2 = [t.to(DEV) for t in inputs.make_weights(w)]
+    r = _stage_run(moe, w, W1, W3, W2, lg.to(DEV), x.to(DEV))
+    sh = moe.shape(**w.shape())
+    phi = r["phi"].clone()
+    real = np.nonzero(phi[:, 0].cpu().numpy() >= 0)[0]
+    victim = int(real[5])
+    phi[victim, 1] = w.N + 3  # token index out of range
+    h2 = torch.zeros_like(r["h"])
+    y2 = torch.zeros_like(r["y"])
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    moe.moe_expert_ffn_gather(x.to(DEV), phi, W1, W3, W2, r["offsets"], r["counts"], h2, y2, st, sh)
+    torch.cuda.synchronize()
+    assert int(st.item()) & moe.DEV_BAD_SCHEDULE
+    assert (y2[victim] == 0).all()
+    other = int(real[6])
+    assert torch.equal(y2[other], r["y"][other])
 
 
 def test_mid_stages_sampled(cuda_lib):
@@ -331,7 +401,10 @@ def test_layer_bitwise_deterministic_and_slice_invariant(cuda_lib, name):
         assert sha(outT) == h0, f"transfer slice {T} changed the output"
 
 
-def test_layer_host_entry_matches_device_entry(cuda_lib):
+@pytest.mark.parametrize("minibatch", [0, 1000, 4096, 2368])
+def test_layer_host_entry_matches_device_entry(cuda_lib, minibatch):
+    """Host buffers in and out, transfers overlapped with compute slice by slice
+    (ragged last slice included): identical to the device-buffer entry."""
     moe = cuda_lib
     w, lg, x, W = _layer_inputs("mid")
     Wd = [t.to(DEV) for t in W]
@@ -339,11 +412,13 @@ def test_layer_host_entry_matches_device_entry(cuda_lib):
     sh = moe.shape(**w.shape())
     ws = torch.empty(moe.layer_host_workspace_bytes(sh), dtype=torch.uint8, device=DEV)
     st = torch.zeros(1, dtype=torch.int32, device=DEV)
-    out_h = torch.empty((w.n_tokens, w.H), dtype=torch.bfloat16).pin_memory()
-    moe.moe_layer_forward_host(lg.pin_memory(), x.pin_memory(), *Wd, out_h, ws, st, sh)
-    torch.cuda.synchronize()
-    assert int(st.item()) == 0
-    assert torch.equal(out_h, out_d.cpu())
+    lg_h, x_h = lg.pin_memory(), x.pin_memory()
+    for _ in range(2):  # a second call reuses the workspace and the internal streams
+        out_h = torch.full((w.n_tokens, w.H), 7.0, dtype=torch.bfloat16).pin_memory()
+        moe.moe_layer_forward_host(lg_h, x_h, *Wd, out_h, ws, st, sh, minibatch_tokens=minibatch)
+        torch.cuda.current_stream().synchronize()
+        assert int(st.item()) == 0
+        assert torch.equal(out_h, out_d.cpu())
 
 
 def test_layer_pad128_single_cta_path(cuda_lib):

@@ -39,7 +39,7 @@ def test_host_only_queries(lib):
     assert moe.schedule_workspace_bytes(sh) == 8 * 28 * 384 * 4   # [P][blocks of 2048 routes][E]
     ws = moe.layer_workspace_bytes(sh)
     rm = moe.rows_max(sh)
-    assert ws >= rm * (7168 * 2 + 2048 * 2 + 7168 * 4)
+    assert ws >= rm * (7168 * 2 + 2048 * 2 + 7168 * 4)  # xg, h and y
     assert moe.layer_host_workspace_bytes(sh) > ws
     assert moe.status_string(0) == "MOE_OK" and moe.status_string(3) == "MOE_WORKSPACE_TOO_SMALL"
     assert moe.status_from_device_flags(0) == 0
