@@ -299,8 +299,23 @@ def run_ours(args):
             stage_ms[name] = statistics.mean(ev[i][s_i].elapsed_time(ev[i][s_i + 1])
                                              for i in range(args.steps))
 
-    # end to end through the host-buffer entry: H2D of logits and x, the layer, D2H of out
+    # the same layer sliced at the workload's transfer minibatch (device-resident)
+    mb_row = None
+    if w.minibatch and not args.no_minibatch_row and mb == 0:
+        t0e, t1e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(2):
+            moe.moe_layer_forward(lg, x, *W, out, ws, st, sh, minibatch_tokens=w.minibatch)
+        t0e.record()
+        for _ in range(args.steps):
+            moe.moe_layer_forward(lg, x, *W, out, ws, st, sh, minibatch_tokens=w.minibatch)
+        t1e.record()
+        torch.cuda.synchronize()
+        mb_row = t0e.elapsed_time(t1e)
+
+    # end to end through the host-buffer entry: H2D of logits and x, the layer,
+    # D2H of out, overlapped slice by slice at the transfer minibatch
     e2e = None
+    e2e_mb = args.e2e_minibatch if args.e2e_minibatch >= 0 else w.minibatch
     if not args.no_e2e:
         del ws
         torch.cuda.empty_cache()
@@ -308,13 +323,13 @@ def run_ours(args):
         lg_h, x_h = lg_cpu.pin_memory(), x_cpu.pin_memory()
         out_h = torch.empty((w.n_tokens, w.H), dtype=torch.bfloat16).pin_memory()
         for _ in range(2):
-            moe.moe_layer_forward_host(lg_h, x_h, *W, out_h, wsh, st, sh, minibatch_tokens=mb)
+            moe.moe_layer_forward_host(lg_h, x_h, *W, out_h, wsh, st, sh, minibatch_tokens=e2e_mb)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         chk = 0.0
         e0.record()
         for _ in range(args.e2e_steps):
-            moe.moe_layer_forward_host(lg_h, x_h, *W, out_h, wsh, st, sh, minibatch_tokens=mb)
+            moe.moe_layer_forward_host(lg_h, x_h, *W, out_h, wsh, st, sh, minibatch_tokens=e2e_mb)
         e1.record()
         torch.cuda.synchronize()
         chk += float(out_h[0, :8].float().sum())  # the host reads the result
@@ -328,10 +343,13 @@ def run_ours(args):
         raise RuntimeError(f"device status {int(st.item())}")
 
     names = list(stage_ms)
-    vec = [ms] + [stage_ms[n] for n in names] + ([e2e["ms"]] if e2e else [])
+    vec = ([ms] + [stage_ms[n] for n in names] + ([e2e["ms"]] if e2e else []) +
+           ([mb_row] if mb_row is not None else []))
     vec = reduce_max(vec, ready, device=dev)
     ms = vec[0]
     stage_ms = dict(zip(names, vec[1:1 + len(names)]))
+    if mb_row is not None:
+        mb_row = vec.pop()
     if e2e:
         e2e["ms"] = vec[-1]
 
@@ -379,7 +397,14 @@ def run_ours(args):
             line["e2e"] = {"value": w.n_tokens * world * args.e2e_steps / (e2e["ms"] / 1e3),
                            "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
                            "d2h_bytes_per_step": e2e["d2h"],
-                           "api": "moe_layer_forward_host (pinned host logits/x/out)"}
+                           "api": "moe_layer_forward_host (pinned host logits/x/out)",
+                           "transfer_minibatch_tokens": e2e_mb or w.N,
+                           "ms_per_step": e2e["ms"] / args.e2e_steps}
+        if mb_row is not None:
+            line["minibatch_row"] = {"minibatch_tokens": w.minibatch,
+                                     "ms_per_step": mb_row / args.steps,
+                                     "value": w.n_tokens * world * args.steps / (mb_row / 1e3),
+                                     "unit": "tokens/s"}
         line["clocks"] = clk
         if world == 1 and not args.no_cpu_baseline:
             r = oracle_sample(w, lg_cpu, x_cpu, W, row_budget_s=args.cpu_budget)
@@ -436,6 +461,9 @@ def main(argv=None):
     ap.add_argument("--workload", default="kimi")
     ap.add_argument("--minibatch", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-minibatch", type=int, default=-1,
+                    help="transfer slice of the host-buffer leg (-1: the workload's)")
+    ap.add_argument("--no-minibatch-row", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)

@@ -63,8 +63,13 @@ constexpr int TMEM_COLS = 512;    // 2 accumulators x 256 fp32 columns
 constexpr int UMMA_K = 16;
 
 // Tile geometry for CG CTAs per MMA (1: one SM, 2: a CTA pair on two SMs).
-template <int CG>
+// TMA_STORE (GEMM2 on CTA pairs): the fp32 epilogue stages each warp's 32x32
+// block in 128-byte-swizzled shared memory and writes it with one TMA store,
+// keeping the load/store unit free; it costs one pipeline stage.
+template <int CG, int MODE>
 struct Cfg {
+  static constexpr bool TMA_STORE = (CG == 2 && MODE == 1);
+  static constexpr int STAGING_BYTES = TMA_STORE ? 8 * 4096 : 0;  // 8 warps x 32x32 fp32
   static constexpr int BM = 128 * CG;      // rows per tile (each CTA holds 128)
   static constexpr int BN = 256;           // accumulator columns per tile
   static constexpr int BK = 64;            // K per stage: one 128-byte swizzle row of bf16
@@ -72,7 +77,7 @@ struct Cfg {
   static constexpr int A_BYTES = 128 * BK * 2;   // 16 KB
   static constexpr int B_ATOM_BYTES = 64 * BK * 2;  // 8 KB
   static constexpr int STAGE_BYTES = A_BYTES + B_ATOMS * B_ATOM_BYTES;  // 48 / 32 KB
-  static constexpr int STAGES = CG == 1 ? 4 : 6;
+  static constexpr int STAGES = CG == 1 ? 4 : (TMA_STORE ? 5 : 6);
   static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*B MN-major*/ 1);
   static constexpr int BAR_FULL = 0;
   static constexpr int BAR_EMPTY = STAGES;
@@ -98,11 +103,11 @@ struct FfnParams {
   int64_t timeout_ns;
 };
 
-template <int CG>
+template <int CG, int MODE>
 size_t smem_bytes_for(int E) {
-  using C = Cfg<CG>;
+  using C = Cfg<CG, MODE>;
   return 1024 /*alignment slack*/ + static_cast<size_t>(C::STAGES) * C::STAGE_BYTES +
-         C::NUM_BARS * 8 + 16 + static_cast<size_t>(2 * E + 1) * 4;
+         C::STAGING_BYTES + C::NUM_BARS * 8 + 16 + static_cast<size_t>(2 * E + 1) * 4;
 }
 
 __device__ __forceinline__ float silu(float a) { return a / (1.0f + expf(-a)); }
@@ -126,12 +131,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 template <int MODE, int CG, bool GATHER>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
-                    const __grid_constant__ CUtensorMap tmB1, const FfnParams p) {
-  using C = Cfg<CG>;
+                    const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmY,
+                    const FfnParams p) {
+  using C = Cfg<CG, MODE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;  // TMA_STORE only
+  uint64_t* bars = reinterpret_cast<uint64_t*>(staging + C::STAGING_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* bad_flag = abort_flag + 1;
@@ -161,6 +168,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB0);
     tma_prefetch_desc(&tmB1);
+    if (C::TMA_STORE) tma_prefetch_desc(&tmY);
   }
   for (int l = tid; l <= E; l += NUM_THREADS) s_off[l] = __ldg(p.offsets + l);
   __syncthreads();
@@ -452,6 +460,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           st_global_v8(hrow + c * 32 + 16, *reinterpret_cast<const uint32_t(*)[8]>(&pk[8]));
           if (c + 1 < 2) tmem_ld_wait();
         }
+      } else if (C::TMA_STORE) {
+        // row `lane` of this warp's 32x32 block goes to the staging slot with
+        // 16-byte chunk j at position j ^ (lane & 7): the 128-byte swizzle the
+        // tensor map expects, and no bank conflicts for the 16-byte writes.
+        const uint32_t stg = smem_u32(staging) + (warp - EPI_WARP0) * 4096;
+        const int ycol = n * C::BN + half * 128;
+        const int yrow0 = row0 + static_cast<int>(rank) * 128 + q * 32;
+        uint32_t rv[2][32];
+        tmem_ld_32cols(tbase + half * 128, rv[0]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (c + 1 < 4) tmem_ld_32cols(tbase + half * 128 + (c + 1) * 32, rv[(c + 1) & 1]);
+          if (lane == 0) bulk_wait_read_all();  // the previous store has read the slot
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(stg + lane * 128 + ((j ^ (lane & 7)) << 4), rv[c & 1][4 * j],
+                         rv[c & 1][4 * j + 1], rv[c & 1][4 * j + 2], rv[c & 1][4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmY, stg, ycol + c * 32, yrow0);
+            bulk_commit_group();
+          }
+          if (c + 1 < 4) tmem_ld_wait();
+        }
       } else {
         float* yrow = reinterpret_cast<float*>(p.out) + row * p.Nout + n * C::BN + half * 128;
         uint32_t rv[2][32];
@@ -479,6 +514,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    if (C::TMA_STORE && lane == 0) bulk_wait_all();  // stores complete before the CTA exits
   }
 
   __syncthreads();
@@ -506,25 +542,26 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2D bf16 tensor [outer, inner] (inner contiguous), box [box_outer, box_inner],
-// 128-byte swizzle.
+// 2D tensor [outer, inner] (inner contiguous) of bf16 (or fp32), box
+// [box_outer, box_inner], 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-              uint32_t box_outer) {
+              uint32_t box_outer, bool fp32 = false) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {inner * 2};
+  const cuuint64_t strides[1] = {inner * (fp32 ? 4 : 2)};
   const cuuint32_t box[2] = {box_inner, box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+  return fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int MODE, int CG, bool GATHER = false>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const FfnParams& p, cudaStream_t s) {
-  const size_t smem = smem_bytes_for<CG>(p.E);
+                        const CUtensorMap& yo, const FfnParams& p, cudaStream_t s) {
+  const size_t smem = smem_bytes_for<CG, MODE>(p.E);
   cudaError_t e = cudaFuncSetAttribute(ffn_gemm_kernel<MODE, CG, GATHER>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -544,7 +581,7 @@ cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUten
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  e = cudaLaunchKernelEx(&cfg, ffn_gemm_kernel<MODE, CG, GATHER>, a, b0, b1, p);
+  e = cudaLaunchKernelEx(&cfg, ffn_gemm_kernel<MODE, CG, GATHER>, a, b0, b1, yo, p);
   note_launches(1);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -557,24 +594,26 @@ cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint
                               uint16_t* h, float* y, const moe_shape_t& sh, int64_t rows_max,
                               int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_mid) {
   const int E = sh.E, H = sh.H, I = sh.I;
-  CUtensorMap mA1, mW1, mW3, mA2, mW2;
+  CUtensorMap mA1, mW1, mW3, mA2, mW2, mY;
   const uint64_t EH = static_cast<uint64_t>(E) * H, EI = static_cast<uint64_t>(E) * I;
   if (!make_map(&mA1, xg, H, rows_max, 64, 128) || !make_map(&mW1, W1, I, EH, 64, 64) ||
       !make_map(&mW3, W3, I, EH, 64, 64) || !make_map(&mA2, h, I, rows_max, 64, 128) ||
-      !make_map(&mW2, W2, H, EI, 64, 64))
+      !make_map(&mW2, W2, H, EI, 64, 64) || !make_map(&mY, y, H, rows_max, 32, 32, true))
     return cudaErrorInvalidValue;
   // Segments that are multiples of 256 rows run on CTA pairs (256x256 tiles);
   // otherwise (pad a multiple of 128 only) on single CTAs (128x256 tiles).
   const bool pair = (sh.pad % 256) == 0;
   FfnParams p1{nullptr, 0, 0, offsets, counts, E, sh.P, H, I, rows_max, h, dev_status, kWaitTimeoutNs};
-  cudaError_t e = pair ? launch_mode<0, 2>(mA1, mW1, mW3, p1, s) : launch_mode<0, 1>(mA1, mW1, mW3, p1, s);
+  cudaError_t e = pair ? launch_mode<0, 2>(mA1, mW1, mW3, mA1, p1, s)
+                       : launch_mode<0, 1>(mA1, mW1, mW3, mA1, p1, s);
   if (e != cudaSuccess) return e;
   if (ev_mid) {
     e = cudaEventRecord(ev_mid, s);
     if (e != cudaSuccess) return e;
   }
   FfnParams p2{nullptr, 0, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status, kWaitTimeoutNs};
-  return pair ? launch_mode<1, 2>(mA2, mW2, mW2, p2, s) : launch_mode<1, 1>(mA2, mW2, mW2, p2, s);
+  return pair ? launch_mode<1, 2>(mA2, mW2, mW2, mY, p2, s)
+              : launch_mode<1, 1>(mA2, mW2, mW2, mY, p2, s);
 }
 
 cudaError_t launch_expert_ffn_gather(const uint16_t* x, const int32_t* phi, const uint16_t* W1,
@@ -584,25 +623,27 @@ cudaError_t launch_expert_ffn_gather(const uint16_t* x, const int32_t* phi, cons
                                      int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_mid) {
   const int E = sh.E, H = sh.H, I = sh.I;
   const int64_t tokens = static_cast<int64_t>(sh.P) * sh.N;
-  CUtensorMap mX, mW1, mW3, mA2, mW2;
+  CUtensorMap mX, mW1, mW3, mA2, mW2, mY;
   const uint64_t EH = static_cast<uint64_t>(E) * H, EI = static_cast<uint64_t>(E) * I;
   // x viewed as [P*N, H] with a one-row box: the gather4 form
   if (!make_map(&mX, x, H, static_cast<uint64_t>(tokens > 0 ? tokens : 1), 64, 1) ||
       !make_map(&mW1, W1, I, EH, 64, 64) || !make_map(&mW3, W3, I, EH, 64, 64) ||
-      !make_map(&mA2, h, I, rows_max, 64, 128) || !make_map(&mW2, W2, H, EI, 64, 64))
+      !make_map(&mA2, h, I, rows_max, 64, 128) || !make_map(&mW2, W2, H, EI, 64, 64) ||
+      !make_map(&mY, y, H, rows_max, 32, 32, true))
     return cudaErrorInvalidValue;
   const bool pair = (sh.pad % 256) == 0;
   FfnParams p1{reinterpret_cast<const int2*>(phi), sh.N, static_cast<int32_t>(tokens), offsets,
                counts, E, sh.P, H, I, rows_max, h, dev_status, kWaitTimeoutNs};
-  cudaError_t e = pair ? launch_mode<0, 2, true>(mX, mW1, mW3, p1, s)
-                       : launch_mode<0, 1, true>(mX, mW1, mW3, p1, s);
+  cudaError_t e = pair ? launch_mode<0, 2, true>(mX, mW1, mW3, mX, p1, s)
+                       : launch_mode<0, 1, true>(mX, mW1, mW3, mX, p1, s);
   if (e != cudaSuccess) return e;
   if (ev_mid) {
     e = cudaEventRecord(ev_mid, s);
     if (e != cudaSuccess) return e;
   }
   FfnParams p2{nullptr, 0, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status, kWaitTimeoutNs};
-  return pair ? launch_mode<1, 2>(mA2, mW2, mW2, p2, s) : launch_mode<1, 1>(mA2, mW2, mW2, p2, s);
+  return pair ? launch_mode<1, 2>(mA2, mW2, mW2, mY, p2, s)
+              : launch_mode<1, 1>(mA2, mW2, mW2, mY, p2, s);
 }
 
 // ---------------------------------------------------------------- self test
