@@ -211,18 +211,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const WaitCtx wc{abort_flag, p.dev_status, p.timeout_ns, MOE_DEV_TIMEOUT};
   const int64_t drain_ns = p.timeout_ns < 100000000ll ? p.timeout_ns : 100000000ll;
 
-  // tile -> (first row, n-tile, expert); false if the tile holds only padding
+  // tile -> (first row, n-tile, expert); false if the tile holds only padding.
+  // Tiles are numbered expert by expert (expert e owns tiles
+  // [S[e]/BM * tiles_n, S[e+1]/BM * tiles_n)) and, inside an expert, in a
+  // grouped raster so that tiles sharing operands run close together in time
+  // and find them in L2: chunks of up to RM M-tiles; inside a chunk, groups
+  // of RN N-blocks; inside a group, N fastest. GEMM2 (RN = 1): each W2 column
+  // block's M-tiles are consecutive and the chunk's h rows (8 MB at most)
+  // stay in L2: its DRAM reads equal W2 + h. GEMM1 (RN = all): each gathered
+  // M-tile feeds its 16 N-blocks back to back; measured, this reads less
+  // DRAM than grouping the weight blocks (the gathered M-tile is reused 16x,
+  // a weight block only by the expert's ~5 M-tiles).
+  constexpr int RM = 8;
+  constexpr int RN = (MODE == 0) ? (1 << 20) : 1;
   auto tile_info = [&](int tile, int& row0, int& n, int& l) -> bool {
-    const int m = tile / tiles_n;
-    n = tile - m * tiles_n;
-    row0 = m * C::BM;
-    int lo = 0, hi = E - 1;  // largest l with s_off[l] <= row0
+    const int u = tile / tiles_n;  // the tile's position in M-tile units
+    int lo = 0, hi = E - 1;        // expert: largest l with S[l]/BM <= u
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (s_off[mid] <= row0) lo = mid;
+      if (s_off[mid] / C::BM <= u) lo = mid;
       else hi = mid - 1;
     }
     l = lo;
+    const int m0 = s_off[l] / C::BM;
+    const int mcount = s_off[l + 1] / C::BM - m0;  // >= 1 for the expert owning u
+    const int j = tile - m0 * tiles_n;               // index inside the expert
+    const int mc = j / (RM * tiles_n);               // M chunk
+    const int rows = min(RM, mcount - mc * RM);      // M-tiles in this chunk
+    const int jj = j - mc * RM * tiles_n;
+    const int ng = jj / (rows * RN);                 // N group
+    const int gsize = min(RN, tiles_n - ng * RN);    // N-blocks in this group
+    const int rr = jj - ng * rows * RN;
+    const int m = rr / gsize;
+    n = ng * RN + (rr - m * gsize);
+    row0 = (m0 + mc * RM + m) * C::BM;
     return row0 < s_end[l];
   };
 
@@ -465,6 +487,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // 16-byte chunk j at position j ^ (lane & 7): the 128-byte swizzle the
         // tensor map expects, and no bank conflicts for the 16-byte writes.
         const uint32_t stg = smem_u32(staging) + (warp - EPI_WARP0) * 4096;
+        const uint64_t pol_y = l2_policy_evict_first();
         const int ycol = n * C::BN + half * 128;
         const int yrow0 = row0 + static_cast<int>(rank) * 128 + q * 32;
         uint32_t rv[2][32];
@@ -481,8 +504,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                          rv[c & 1][4 * j + 1], rv[c & 1][4 * j + 2], rv[c & 1][4 * j + 3]);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmY, stg, ycol + c * 32, yrow0);
+          if (lane == 0) {  // y is streamed out and read once, by the combine
+            tma_store_2d_hint(&tmY, stg, ycol + c * 32, yrow0, pol_y);
             bulk_commit_group();
           }
           if (c + 1 < 4) tmem_ld_wait();
