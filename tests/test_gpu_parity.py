@@ -437,3 +437,43 @@ def test_layer_pad128_single_cta_path(cuda_lib):
     assert rms_floor_err(bf16_to_f64(bits(out)), res["out64"]) < OUT_TOL
     assert all(int(v) % 128 == 0 for v in res["sched"]["offsets"])
     assert any(int(v) % 256 != 0 for v in res["sched"]["offsets"])
+
+
+@pytest.mark.parametrize("P,N,E,k,H,I", [
+    (64, 3, 1024, 16, 256, 128),    # most peers, experts and routes per token
+    (1, 1, 8, 2, 256, 128),          # a single token
+    (3, 131, 5, 5, 512, 256),        # k = E, ragged token count
+    (2, 700, 1, 1, 256, 384),        # one expert takes everything
+])
+def test_layer_edge_shapes(cuda_lib, P, N, E, k, H, I):
+    moe = cuda_lib
+    w = inputs.Workload("edge", 7, P=P, N=N, E=E, k=k, H=H, I=I)
+    g = torch.Generator().manual_seed(P * 1000 + N)
+    lg = torch.randn((w.n_tokens, E), generator=g)
+    x = torch.randn((w.n_tokens, H), generator=g).to(torch.bfloat16)
+    W1 = (torch.randn((E, H, I), generator=g) * 0.02).to(torch.bfloat16)
+    W3 = (torch.randn((E, H, I), generator=g) * 0.02).to(torch.bfloat16)
+    W2 = (torch.randn((E, I, H), generator=g) * 0.02).to(torch.bfloat16)
+    Wd = [t.to(DEV) for t in (W1, W3, W2)]
+    out, _ = _layer_gpu(moe, w, lg.to(DEV), x.to(DEV), Wd)
+    toks = inputs.sample_tokens(w.n_tokens, 64, seed=3)
+    o_ids, _, _ = oracle.route_topk(lg[toks], k)
+    Wh = expert_weights_host(W1, W3, W2, np.unique(o_ids))
+    res = oracle.layer_tokens(lg, bits(x), Wh, P, N, k, E, H, I, toks)
+    got = bf16_to_f64(bits(out[torch.tensor(toks, device=DEV)]))
+    assert rms_floor_err(got, res["out64"]) < OUT_TOL
+
+
+def test_layer_no_tokens(cuda_lib):
+    """N = 0: nothing to route; the call succeeds and touches no output."""
+    moe = cuda_lib
+    sh = moe.shape(2, 0, 8, 2, 256, 128)
+    ws = torch.empty(moe.layer_workspace_bytes(sh), dtype=torch.uint8, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    e = torch.empty((0,), device=DEV)
+    W = torch.zeros((8, 256, 128), dtype=torch.bfloat16, device=DEV)
+    W2 = torch.zeros((8, 128, 256), dtype=torch.bfloat16, device=DEV)
+    moe.moe_layer_forward(e.float().reshape(0, 8), e.to(torch.bfloat16).reshape(0, 256), W, W, W2,
+                          e.to(torch.bfloat16).reshape(0, 256), ws, st, sh)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
