@@ -61,6 +61,7 @@ constexpr int EPI_WARP0 = 4;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int TMEM_COLS = 512;    // 2 accumulators x 256 fp32 columns
 constexpr int UMMA_K = 16;
+constexpr int kRing = 4;  // tile ids in flight between the scheduler and the roles
 
 // Tile geometry for CG CTAs per MMA (1: one SM, 2: a CTA pair on two SMs).
 // TMA_STORE (GEMM2 on CTA pairs): the fp32 epilogue stages each warp's 32x32
@@ -84,11 +85,17 @@ struct Cfg {
   static constexpr int BAR_TFULL = 2 * STAGES;
   static constexpr int BAR_TEMPTY = 2 * STAGES + 2;
   static constexpr int BAR_DRAIN = 2 * STAGES + 4;
-  static constexpr int NUM_BARS = 2 * STAGES + 5;
+  static constexpr int BAR_TID_FULL = 2 * STAGES + 5;   // [kRing] tile id posted
+  static constexpr int BAR_TID_EMPTY = 2 * STAGES + 9;  // [kRing] tile id consumed
+  static constexpr int NUM_BARS = 2 * STAGES + 13;
+  // consumers of each tile id: producer, MMA issuer and 8 epilogue warps of
+  // the leader; producer and 8 epilogue warps of the follower
+  static constexpr int TID_CONSUMERS = CG == 2 ? 19 : 10;
   static_assert(STAGE_BYTES % 1024 == 0 && A_BYTES % 1024 == 0, "swizzle atoms stay 1024-aligned");
 };
 
 struct FfnParams {
+  int* tile_counter;       // next tile to hand out (zeroed before each launch)
   const int2* phi;         // [rows_max] (src_rank, src_idx): GATHER only
   int32_t n_per_peer;      // N (GATHER: token row = src_rank * N + src_idx)
   int32_t oob_row;         // P*N: a row index outside x, which reads as zeros
@@ -107,7 +114,7 @@ template <int CG, int MODE>
 size_t smem_bytes_for(int E) {
   using C = Cfg<CG, MODE>;
   return 1024 /*alignment slack*/ + static_cast<size_t>(C::STAGES) * C::STAGE_BYTES +
-         C::STAGING_BYTES + C::NUM_BARS * 8 + 16 + static_cast<size_t>(2 * E + 1) * 4;
+         C::STAGING_BYTES + C::NUM_BARS * 8 + 16 + kRing * 4 + static_cast<size_t>(2 * E + 1) * 4;
 }
 
 __device__ __forceinline__ float silu(float a) { return a / (1.0f + expf(-a)); }
@@ -142,7 +149,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   int* bad_flag = abort_flag + 1;
-  int32_t* s_off = reinterpret_cast<int32_t*>(tmem_slot + 4);  // [E+1] segment starts
+  int* tile_ring = reinterpret_cast<int*>(tmem_slot + 4);       // [kRing] tile ids
+  int32_t* s_off = reinterpret_cast<int32_t*>(tile_ring + kRing);  // [E+1] segment starts
   int32_t* s_end = s_off + (p.E + 1);                            // [E] end of real rows
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -160,6 +168,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&bars[C::BAR_TEMPTY + i]), NUM_EPI_WARPS * CG);
     }
     mbar_init(smem_u32(&bars[C::BAR_DRAIN]), 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(smem_u32(&bars[C::BAR_TID_FULL + i]), 1);
+      mbar_init(smem_u32(&bars[C::BAR_TID_EMPTY + i]), C::TID_CONSUMERS);
+    }
     *abort_flag = 0;
     *bad_flag = 0;
     fence_mbar_init();
@@ -206,9 +218,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int tiles_n = (MODE == 0) ? p.Nout / 128 : p.Nout / C::BN;
   const int num_tiles = (rows_used / C::BM) * tiles_n;
   const int kblocks = p.K / C::BK;
-  const int first_tile = (CG == 2) ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-  const int tile_step = (CG == 2) ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   const WaitCtx wc{abort_flag, p.dev_status, p.timeout_ns, MOE_DEV_TIMEOUT};
+
+  // Dynamic tile order: the leader's scheduler thread takes tile ids from a
+  // device-wide counter and posts them, in order, to a ring that every role
+  // of both CTAs reads. CTAs that run ahead simply take more tiles, so the
+  // tiles in flight stay a narrow window of consecutive ids and the operands
+  // they share are still in L2. (A static round-robin let slow pairs fall
+  // whole experts behind, and GEMM1 read its weights 2.5-4x from DRAM.)
+  // next_tile(): the next id of this role's sequence, -1 at the end, -2 if a
+  // wait gave up. One thread per consuming warp calls it.
+  const uint32_t tid_empty_tgt0 =
+      (CG == 2) ? mapa_shared(smem_u32(&bars[C::BAR_TID_EMPTY]), 0) : smem_u32(&bars[C::BAR_TID_EMPTY]);
+  auto next_tile = [&](int& pos, uint32_t& ph) -> int {
+    const int j = pos % kRing;
+    if (!wait_bounded<CG == 2>(smem_u32(&bars[C::BAR_TID_FULL + j]), ph, wc)) return -2;
+    const int t = reinterpret_cast<volatile int*>(tile_ring)[j];
+    if (CG == 2) mbar_arrive_cluster(tid_empty_tgt0 + j * 8);
+    else mbar_arrive(tid_empty_tgt0 + j * 8);
+    if (++pos % kRing == 0) ph ^= 1u;
+    return t;
+  };
   const int64_t drain_ns = p.timeout_ns < 100000000ll ? p.timeout_ns : 100000000ll;
 
   // tile -> (first row, n-tile, expert); false if the tile holds only padding.
@@ -257,7 +287,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int64_t issued = 0;
     bool ok = true;
     int bad = 0;
-    for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
+    int tpos = 0;
+    uint32_t tph = 0;
+    while (ok) {
+      int tile = 0;
+      if (lane == 0) tile = next_tile(tpos, tph);
+      tile = __shfl_sync(0xFFFFFFFFu, tile, 0);
+      if (tile < 0) break;
       int row0, n, l;
       if (!tile_info(tile, row0, n, l)) continue;
       const int arow = row0 + static_cast<int>(rank) * 128;
@@ -331,7 +367,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       int64_t issued = 0;
       bool ok = true;
-      for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
+      int tpos = 0;
+      uint32_t tph = 0;
+      while (ok) {
+        const int tile = next_tile(tpos, tph);
+        if (tile < 0) break;
         int row0, n, l;
         if (!tile_info(tile, row0, n, l)) continue;
         const int arow = row0 + static_cast<int>(rank) * 128;
@@ -393,7 +433,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = first_tile; ok && tile < num_tiles; tile += tile_step) {
+      int tpos = 0;
+      uint32_t tph = 0;
+      while (ok) {
+        const int tile = next_tile(tpos, tph);
+        if (tile < 0) break;
         int row0, n, l;
         if (!tile_info(tile, row0, n, l)) continue;
         if (!wait_bounded<CG == 2>(smem_u32(&bars[C::BAR_TEMPTY + acc]), acc_phase ^ 1u, wc)) {
@@ -438,6 +482,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       else tc_commit(smem_u32(&bars[C::BAR_DRAIN]));
       wait_drain(smem_u32(&bars[C::BAR_DRAIN]), 0, p.timeout_ns);
     }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ tile scheduler
+    if (lane == 0 && leader) {
+      const uint32_t ring_peer = (CG == 2) ? mapa_shared(smem_u32(tile_ring), 1) : 0u;
+      const uint32_t tfull_peer =
+          (CG == 2) ? mapa_shared(smem_u32(&bars[C::BAR_TID_FULL]), 1) : 0u;
+      uint32_t eph = 0;
+      for (int i = 0;; ++i) {
+        const int j = i % kRing;
+        if (!wait_bounded<CG == 2>(smem_u32(&bars[C::BAR_TID_EMPTY + j]), eph ^ 1u, wc)) break;
+        int t = atomicAdd(p.tile_counter, 1);
+        if (t >= num_tiles) t = -1;
+        reinterpret_cast<volatile int*>(tile_ring)[j] = t;
+        mbar_arrive(smem_u32(&bars[C::BAR_TID_FULL + j]));
+        if (CG == 2) {
+          st_shared_cluster_u32(ring_peer + j * 4, static_cast<uint32_t>(t));
+          mbar_arrive_cluster(tfull_peer + j * 8);
+        }
+        if (j == kRing - 1) eph ^= 1u;
+        if (t < 0) break;
+      }
+    }
   } else if (warp >= EPI_WARP0) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
@@ -446,7 +512,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tempty_tgt0 = (CG == 2) ? mapa_shared(tempty0, 0) : tempty0;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = first_tile; tile < num_tiles; tile += tile_step) {
+    int tpos = 0;
+    uint32_t tph = 0;
+    for (;;) {
+      int tile = 0;
+      if (lane == 0) tile = next_tile(tpos, tph);
+      tile = __shfl_sync(0xFFFFFFFFu, tile, 0);
+      if (tile < 0) break;
       int row0, n, l;
       if (!tile_info(tile, row0, n, l)) continue;
       if (!wait_bounded(smem_u32(&bars[C::BAR_TFULL + acc]), acc_phase, wc)) break;
@@ -550,6 +622,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// Per-device counter the scheduler threads take tile ids from; zeroed on the
+// stream before every launch.
+__device__ int g_tile_counter[1];
+
 // ---------------------------------------------------------------- host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -581,10 +657,31 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Device address of g_tile_counter on the current device (looked up once per device).
+cudaError_t tile_counter_for_current_device(int** out) {
+  static std::mutex mu;
+  static int* ptrs[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* ptr = nullptr;
+    if ((e = cudaGetSymbolAddress(&ptr, g_tile_counter)) != cudaSuccess) return e;
+    ptrs[dev] = static_cast<int*>(ptr);
+  }
+  *out = ptrs[dev];
+  return cudaSuccess;
+}
+
 template <int MODE, int CG, bool GATHER = false>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
-                        const CUtensorMap& yo, const FfnParams& p, cudaStream_t s) {
+                        const CUtensorMap& yo, FfnParams p, cudaStream_t s) {
   const size_t smem = smem_bytes_for<CG, MODE>(p.E);
+  cudaError_t ce = tile_counter_for_current_device(&p.tile_counter);
+  if (ce != cudaSuccess) return ce;
+  if ((ce = cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s)) != cudaSuccess) return ce;
   cudaError_t e = cudaFuncSetAttribute(ffn_gemm_kernel<MODE, CG, GATHER>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -626,7 +723,7 @@ cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint
   // Segments that are multiples of 256 rows run on CTA pairs (256x256 tiles);
   // otherwise (pad a multiple of 128 only) on single CTAs (128x256 tiles).
   const bool pair = (sh.pad % 256) == 0;
-  FfnParams p1{nullptr, 0, 0, offsets, counts, E, sh.P, H, I, rows_max, h, dev_status, kWaitTimeoutNs};
+  FfnParams p1{nullptr, nullptr, 0, 0, offsets, counts, E, sh.P, H, I, rows_max, h, dev_status, kWaitTimeoutNs};
   cudaError_t e = pair ? launch_mode<0, 2>(mA1, mW1, mW3, mA1, p1, s)
                        : launch_mode<0, 1>(mA1, mW1, mW3, mA1, p1, s);
   if (e != cudaSuccess) return e;
@@ -634,7 +731,7 @@ cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint
     e = cudaEventRecord(ev_mid, s);
     if (e != cudaSuccess) return e;
   }
-  FfnParams p2{nullptr, 0, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status, kWaitTimeoutNs};
+  FfnParams p2{nullptr, nullptr, 0, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status, kWaitTimeoutNs};
   return pair ? launch_mode<1, 2>(mA2, mW2, mW2, mY, p2, s)
               : launch_mode<1, 1>(mA2, mW2, mW2, mY, p2, s);
 }
@@ -655,7 +752,7 @@ cudaError_t launch_expert_ffn_gather(const uint16_t* x, const int32_t* phi, cons
       !make_map(&mY, y, H, rows_max, 32, 32, true))
     return cudaErrorInvalidValue;
   const bool pair = (sh.pad % 256) == 0;
-  FfnParams p1{reinterpret_cast<const int2*>(phi), sh.N, static_cast<int32_t>(tokens), offsets,
+  FfnParams p1{nullptr, reinterpret_cast<const int2*>(phi), sh.N, static_cast<int32_t>(tokens), offsets,
                counts, E, sh.P, H, I, rows_max, h, dev_status, kWaitTimeoutNs};
   cudaError_t e = pair ? launch_mode<0, 2, true>(mX, mW1, mW3, mX, p1, s)
                        : launch_mode<0, 1, true>(mX, mW1, mW3, mX, p1, s);
@@ -664,7 +761,7 @@ cudaError_t launch_expert_ffn_gather(const uint16_t* x, const int32_t* phi, cons
     e = cudaEventRecord(ev_mid, s);
     if (e != cudaSuccess) return e;
   }
-  FfnParams p2{nullptr, 0, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status, kWaitTimeoutNs};
+  FfnParams p2{nullptr, nullptr, 0, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status, kWaitTimeoutNs};
   return pair ? launch_mode<1, 2>(mA2, mW2, mW2, mY, p2, s)
               : launch_mode<1, 1>(mA2, mW2, mW2, mY, p2, s);
 }
