@@ -313,7 +313,7 @@ def run_ours(args):
         mb_row = t0e.elapsed_time(t1e)
 
     # end to end through the host-buffer entry: H2D of logits and x, the layer,
-    # D2H of out, overlapped slice by slice at the transfer minibatch
+    # D2H of out; each call's input copy overlaps the previous call's compute
     e2e = None
     e2e_mb = args.e2e_minibatch if args.e2e_minibatch >= 0 else w.minibatch
     if not args.no_e2e:
@@ -461,8 +461,9 @@ def main(argv=None):
     ap.add_argument("--workload", default="kimi")
     ap.add_argument("--minibatch", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--e2e-minibatch", type=int, default=-1,
-                    help="transfer slice of the host-buffer leg (-1: the workload's)")
+    ap.add_argument("--e2e-minibatch", type=int, default=0,
+                    help="transfer slice of the host-buffer leg (0: whole batch; "
+                         "-1: the workload's transfer minibatch)")
     ap.add_argument("--no-minibatch-row", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

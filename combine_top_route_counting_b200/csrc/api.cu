@@ -52,7 +52,7 @@ int64_t rows_max_of(const moe_shape_t* s) {
 // Layout of the layer workspace (offsets in bytes, each kAlign-aligned).
 struct LayerWs {
   size_t ids, gates, route_row, phi, offsets, counts, sched, xg, h, y, total;
-  size_t logits, x, out, total_host;  // moe_layer_forward_host additions
+  size_t logits[2], x[2], out, total_host;  // moe_layer_forward_host additions
 };
 
 LayerWs layer_ws(const moe_shape_t* s) {
@@ -77,8 +77,10 @@ LayerWs layer_ws(const moe_shape_t* s) {
   w.h = take(rows * s->I * 2);
   w.y = take(rows * s->H * 4);
   w.total = o;
-  w.logits = take(tokens * s->E * 4);
-  w.x = take(tokens * s->H * 2);
+  for (int b = 0; b < 2; ++b) {  // consecutive host-buffer calls alternate
+    w.logits[b] = take(tokens * s->E * 4);
+    w.x[b] = take(tokens * s->H * 2);
+  }
   w.out = take(tokens * s->H * 2);
   w.total_host = o;
   return w;
@@ -192,8 +194,10 @@ moe_status_t layer_body(const float* logits, const uint16_t* x, const uint16_t* 
 constexpr int kRing = 4;
 struct CopyRes {
   cudaStream_t h2d = nullptr, d2h = nullptr;
-  cudaEvent_t entry = nullptr, lg = nullptr, fin = nullptr;
+  cudaEvent_t lg = nullptr, fin = nullptr;
   cudaEvent_t ex[kRing] = {}, ed[kRing] = {};
+  cudaEvent_t in_free[2] = {};  // input buffers of parity b no longer read
+  uint64_t calls = 0;
   bool ready = false;
 };
 std::mutex g_copy_mu;
@@ -209,7 +213,8 @@ cudaError_t copy_res(CopyRes** out) {
     const unsigned ef = cudaEventDisableTiming;
     if ((e = cudaStreamCreateWithFlags(&r.h2d, cudaStreamNonBlocking)) != cudaSuccess) return e;
     if ((e = cudaStreamCreateWithFlags(&r.d2h, cudaStreamNonBlocking)) != cudaSuccess) return e;
-    if ((e = cudaEventCreateWithFlags(&r.entry, ef)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&r.in_free[0], ef)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&r.in_free[1], ef)) != cudaSuccess) return e;
     if ((e = cudaEventCreateWithFlags(&r.lg, ef)) != cudaSuccess) return e;
     if ((e = cudaEventCreateWithFlags(&r.fin, ef)) != cudaSuccess) return e;
     for (int i = 0; i < kRing; ++i) {
@@ -222,11 +227,15 @@ cudaError_t copy_res(CopyRes** out) {
   return cudaSuccess;
 }
 
-// Host-buffer layer: the rows of slice [t0, t0+Tm) of every peer are copied in
-// on the h2d stream while the previous slice computes on `s`, and copied out
-// on the d2h stream while the next one computes (the transfer minibatch of
-// "Mixture-of-Kittens" notes section 3 and "Beyond Peak TFLOPs" section 1:
-// chunk k transfers while chunk k-1 computes).
+// Host-buffer layer. Consecutive calls alternate between two device copies of
+// the inputs (parity b), so the host-to-device copy of call i+1 runs while
+// call i still computes: it only waits until call i-1, the last user of the
+// same copies, has finished reading them. Within a call, the rows of slice
+// [t0, t0+Tm) of every peer are copied in on the h2d stream while the
+// previous slice computes on `s`, and copied out on the d2h stream while the
+// next one computes (the transfer minibatch of "Mixture-of-Kittens" notes
+// section 3 and "Beyond Peak TFLOPs" section 1: chunk k transfers while chunk
+// k-1 computes). `s` waits for every copy of the call before the call ends.
 cudaError_t layer_host_pipeline(const float* logits_host, const uint16_t* x_host,
                                 const uint16_t* W1, const uint16_t* W3, const uint16_t* W2,
                                 uint16_t* out_host, int32_t minibatch_tokens, void* ws,
@@ -235,10 +244,11 @@ cudaError_t layer_host_pipeline(const float* logits_host, const uint16_t* x_host
   CopyRes* cr = nullptr;
   cudaError_t e = copy_res(&cr);
   if (e != cudaSuccess) return e;
+  const int b = static_cast<int>(cr->calls++ & 1);
   const LayerWs w = layer_ws(sh);
-  const LayerBufs b = layer_bufs(ws, w);
-  float* logits = at<float>(ws, w.logits);
-  uint16_t* x = at<uint16_t>(ws, w.x);
+  const LayerBufs bufs = layer_bufs(ws, w);
+  float* logits = at<float>(ws, w.logits[b]);
+  uint16_t* x = at<uint16_t>(ws, w.x[b]);
   uint16_t* out = at<uint16_t>(ws, w.out);
   const int32_t P = sh->P, N = sh->N, H = sh->H;
   const size_t row_bytes = static_cast<size_t>(H) * 2;
@@ -254,10 +264,8 @@ cudaError_t layer_host_pipeline(const float* logits_host, const uint16_t* x_host
     }
     return cudaSuccess;
   };
-  // the copies may only start once earlier work on `s` no longer uses ws
-  if ((e = cudaEventRecord(cr->entry, s)) != cudaSuccess) return e;
-  if ((e = cudaStreamWaitEvent(cr->h2d, cr->entry, 0)) != cudaSuccess) return e;
-  if ((e = cudaStreamWaitEvent(cr->d2h, cr->entry, 0)) != cudaSuccess) return e;
+  // the input copies of parity b are free once call i-2 has read them
+  if ((e = cudaStreamWaitEvent(cr->h2d, cr->in_free[b], 0)) != cudaSuccess) return e;
   const size_t tokens = static_cast<size_t>(P) * N;
   if ((e = cudaMemcpyAsync(logits, logits_host, tokens * sh->E * 4, cudaMemcpyHostToDevice,
                            cr->h2d)) != cudaSuccess)
@@ -269,8 +277,8 @@ cudaError_t layer_host_pipeline(const float* logits_host, const uint16_t* x_host
     if ((e = cudaEventRecord(cr->ex[0], cr->h2d)) != cudaSuccess) return e;
   }
   if ((e = cudaStreamWaitEvent(s, cr->lg, 0)) != cudaSuccess) return e;
-  if ((e = launch_route_topk(logits, b.ids, b.gates, static_cast<int64_t>(tokens), sh->E, sh->k,
-                             s)) != cudaSuccess)
+  if ((e = launch_route_topk(logits, bufs.ids, bufs.gates, static_cast<int64_t>(tokens), sh->E,
+                             sh->k, s)) != cudaSuccess)
     return e;
   for (int32_t i = 0; i < S; ++i) {
     const int32_t t0 = i * T, tm = (N - t0) < T ? (N - t0) : T;
@@ -281,7 +289,7 @@ cudaError_t layer_host_pipeline(const float* logits_host, const uint16_t* x_host
       if ((e = cudaEventRecord(cr->ex[(i + 1) % kRing], cr->h2d)) != cudaSuccess) return e;
     }
     if ((e = cudaStreamWaitEvent(s, cr->ex[i % kRing], 0)) != cudaSuccess) return e;
-    if ((e = run_slice(b, x, W1, W3, W2, out, Slice{t0, tm}, sh, dev_status, s, nullptr)) !=
+    if ((e = run_slice(bufs, x, W1, W3, W2, out, Slice{t0, tm}, sh, dev_status, s, nullptr)) !=
         cudaSuccess)
       return e;
     if ((e = cudaEventRecord(cr->ed[i % kRing], s)) != cudaSuccess) return e;
@@ -289,6 +297,8 @@ cudaError_t layer_host_pipeline(const float* logits_host, const uint16_t* x_host
     if ((e = copy_rows(out_host, out, t0, tm, cudaMemcpyDeviceToHost, cr->d2h)) != cudaSuccess)
       return e;
   }
+  // routing and every slice's dispatch have read this call's input copies
+  if ((e = cudaEventRecord(cr->in_free[b], s)) != cudaSuccess) return e;
   // `s` completes only after the last copy out (and every copy in)
   if ((e = cudaEventRecord(cr->fin, cr->d2h)) != cudaSuccess) return e;
   if ((e = cudaStreamWaitEvent(s, cr->fin, 0)) != cudaSuccess) return e;

@@ -169,10 +169,14 @@ moe_status_t moe_dispatch(const uint16_t* x, const int32_t* phi, const int32_t* 
  * For every row in expert l's segment [offsets[l], offsets[l+1]):
  *   h[row] = bf16_rne( silu(xg[row].W1[l]) * (xg[row].W3[l]) ),  h: bf16 [moe_rows_max, I]
  *   y[row] = h[row].W2[l] (fp32),                                 y: fp32 [moe_rows_max, H]
- * counts (int32 [E,P], may be NULL): when given, 128-row tiles that hold only
+ * counts (int32 [E,P], may be NULL): when given, tiles that hold only
  * padding rows are skipped and their h/y rows are left unwritten; rows that
  * carry routes are always written. Each output element is computed by one
- * CTA with a fixed K order: the result is bitwise deterministic.
+ * CTA (pair) with a fixed K order: the result is bitwise deterministic.
+ * The GEMM kernels take their tiles from a tile counter inside the library
+ * (one per device, zeroed on `stream` before each GEMM): FFN calls
+ * (moe_expert_ffn, moe_expert_ffn_gather, the layer entries) must not
+ * overlap on the GPU -- serialise calls made on different streams.
  * offsets must be non-decreasing multiples of 128 with offsets[E] <=
  * moe_rows_max (else MOE_DEV_BAD_SCHEDULE, nothing written). */
 moe_status_t moe_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint16_t* W3,
@@ -225,15 +229,22 @@ moe_status_t moe_layer_forward(const float* logits, const uint16_t* x, const uin
  * x_host bf16 [P*N, H] and out_host bf16 [P*N, H] live in host memory (pinned
  * memory makes the copies asynchronous); the weights, ws (of
  * moe_layer_host_workspace_bytes) and dev_status are device memory.
- * Transfers overlap compute at the granularity of the transfer slice
- * `minibatch_tokens` (MoK notes section 3; "Beyond Peak TFLOPs" section 1:
- * chunk k moves while chunk k-1 computes): the logits and slice 0 are copied
- * in, then slice s+1's rows are copied in and slice s-1's outputs copied out
- * while slice s computes on `stream`. 0 = one slice (no overlap). The copies
- * run on two internal streams per device (host-to-device, device-to-host)
- * with a few events, created on the first call on that device and kept until
- * exit; `stream` is made to wait for them, so out_host is valid once `stream`
- * has been synchronised. Calls from several host threads are serialised. */
+ * Copies overlap compute in two ways:
+ *   - across calls: consecutive calls alternate between two device copies of
+ *     the inputs inside ws, so the host-to-device copy of a call starts as
+ *     soon as the call is made and runs while the previous call computes
+ *     (it waits only for the call before that to finish reading the same
+ *     copies). The host inputs must therefore hold their values when the
+ *     call is made, not only when earlier work on `stream` has finished.
+ *   - within a call, at the transfer slice `minibatch_tokens` (MoK notes
+ *     section 3; "Beyond Peak TFLOPs" section 1: chunk k moves while chunk
+ *     k-1 computes): slice s+1's rows are copied in and slice s-1's outputs
+ *     copied out while slice s computes. 0 = one slice.
+ * The copies run on two internal streams per device (host-to-device,
+ * device-to-host) with a few events, created on the first call on that
+ * device and kept until exit; `stream` waits for every copy of the call, so
+ * out_host is valid once `stream` has been synchronised. Calls from several
+ * host threads are serialised. */
 moe_status_t moe_layer_forward_host(const float* logits_host, const uint16_t* x_host,
                                     const uint16_t* W1, const uint16_t* W3, const uint16_t* W2,
                                     uint16_t* out_host, int32_t minibatch_tokens, void* ws,

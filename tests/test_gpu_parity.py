@@ -404,21 +404,27 @@ def test_layer_bitwise_deterministic_and_slice_invariant(cuda_lib, name):
 @pytest.mark.parametrize("minibatch", [0, 1000, 4096, 2368])
 def test_layer_host_entry_matches_device_entry(cuda_lib, minibatch):
     """Host buffers in and out, transfers overlapped with compute slice by slice
-    (ragged last slice included): identical to the device-buffer entry."""
+    (ragged last slice included) and across calls (two input batches
+    alternated, so both internal input copies and their reuse are exercised):
+    identical to the device-buffer entry."""
     moe = cuda_lib
     w, lg, x, W = _layer_inputs("mid")
     Wd = [t.to(DEV) for t in W]
-    out_d, _ = _layer_gpu(moe, w, lg.to(DEV), x.to(DEV), Wd)
+    perm = torch.randperm(w.n_tokens, generator=torch.Generator().manual_seed(9))
+    batches = [(lg, x), (lg[perm].contiguous(), x[perm].contiguous())]
+    refs = [_layer_gpu(moe, w, a.to(DEV), b.to(DEV), Wd)[0].cpu() for a, b in batches]
     sh = moe.shape(**w.shape())
     ws = torch.empty(moe.layer_host_workspace_bytes(sh), dtype=torch.uint8, device=DEV)
     st = torch.zeros(1, dtype=torch.int32, device=DEV)
-    lg_h, x_h = lg.pin_memory(), x.pin_memory()
-    for _ in range(2):  # a second call reuses the workspace and the internal streams
-        out_h = torch.full((w.n_tokens, w.H), 7.0, dtype=torch.bfloat16).pin_memory()
-        moe.moe_layer_forward_host(lg_h, x_h, *Wd, out_h, ws, st, sh, minibatch_tokens=minibatch)
-        torch.cuda.current_stream().synchronize()
-        assert int(st.item()) == 0
-        assert torch.equal(out_h, out_d.cpu())
+    pinned = [(a.pin_memory(), b.pin_memory()) for a, b in batches]
+    outs = [torch.full((w.n_tokens, w.H), 7.0, dtype=torch.bfloat16).pin_memory() for _ in range(5)]
+    for c in range(5):  # calls issued back to back, synchronised once at the end
+        lg_h, x_h = pinned[c % 2]
+        moe.moe_layer_forward_host(lg_h, x_h, *Wd, outs[c], ws, st, sh, minibatch_tokens=minibatch)
+    torch.cuda.current_stream().synchronize()
+    assert int(st.item()) == 0
+    for c in range(5):
+        assert torch.equal(outs[c], refs[c % 2]), f"call {c}"
 
 
 def test_layer_pad128_single_cta_path(cuda_lib):
