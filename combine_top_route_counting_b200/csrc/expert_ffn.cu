@@ -228,14 +228,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // whole experts behind, and GEMM1 read its weights 2.5-4x from DRAM.)
   // next_tile(): the next id of this role's sequence, -1 at the end, -2 if a
   // wait gave up. One thread per consuming warp calls it.
-  const uint32_t tid_empty_tgt0 =
-      (CG == 2) ? mapa_shared(smem_u32(&bars[C::BAR_TID_EMPTY]), 0) : smem_u32(&bars[C::BAR_TID_EMPTY]);
+  // The slot is released with a release-ordered arrive (the read of the id
+  // must not move after it): CTA scope for the leader's own roles, cluster
+  // scope only for the follower's, whose arrive is remote.
+  const uint32_t tid_empty_local = smem_u32(&bars[C::BAR_TID_EMPTY]);
+  const uint32_t tid_empty_tgt0 = (CG == 2) ? mapa_shared(tid_empty_local, 0) : tid_empty_local;
   auto next_tile = [&](int& pos, uint32_t& ph) -> int {
     const int j = pos % kRing;
     if (!wait_bounded<CG == 2>(smem_u32(&bars[C::BAR_TID_FULL + j]), ph, wc)) return -2;
     const int t = reinterpret_cast<volatile int*>(tile_ring)[j];
-    if (CG == 2) mbar_arrive_cluster(tid_empty_tgt0 + j * 8);
-    else mbar_arrive(tid_empty_tgt0 + j * 8);
+    if (CG == 2 && !leader) mbar_arrive_cluster(tid_empty_tgt0 + j * 8);
+    else mbar_arrive(tid_empty_local + j * 8);
     if (++pos % kRing == 0) ph ^= 1u;
     return t;
   };
