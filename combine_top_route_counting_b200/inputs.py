@@ -73,7 +73,7 @@ def seed_for(wid: int, stream_id: int) -> int:
 
 
 # stream ids
-_S_LOGITS, _S_X, _S_W1, _S_W3, _S_W2, _S_PERM, _S_EMPTY, _S_IDS = range(8)
+_S_LOGITS, _S_X, _S_W1, _S_W3, _S_W2, _S_PERM, _S_EMPTY, _S_IDS, _S_Y, _S_DOUT = range(10)
 
 
 def _gen(seed: int, device="cpu") -> torch.Generator:
@@ -134,6 +134,21 @@ def make_x(w: Workload, device="cpu") -> torch.Tensor:
     return torch.randn((w.n_tokens, w.H), generator=g, dtype=torch.bfloat16, device=device)
 
 
+def make_expert_outputs(w: Workload, rows: int, device="cpu") -> torch.Tensor:
+    """Stand-in expert output rows fp32 [rows, H] ~ N(0, 0.05^2) (about the spread
+    of real expert outputs at these weight scales), for checking the combine
+    stage on inputs that neither side computed."""
+    g = _gen(seed_for(w.wid, _S_Y), device)
+    t = torch.randn((rows, w.H), generator=g, dtype=torch.float32, device=device)
+    return t.mul_(0.05)
+
+
+def make_dout(w: Workload, device="cpu") -> torch.Tensor:
+    """Upstream gradient of the layer output, bf16 [P*N, H] ~ N(0,1)."""
+    g = _gen(seed_for(w.wid, _S_DOUT), device)
+    return torch.randn((w.n_tokens, w.H), generator=g, dtype=torch.bfloat16, device=device)
+
+
 def make_weights(w: Workload, device="cpu"):
     """SwiGLU expert weights (W1 gate, W3 up [E,H,I]; W2 down [E,I,H]), bf16 N(0, 0.02).
 
@@ -190,5 +205,6 @@ def sample_tokens(n_tokens: int, n: int, seed: int) -> list[int]:
 
 __all__ = [
     "Workload", "WORKLOADS", "seed_for", "make_logits", "make_ids_uniform", "make_sched_ids",
-    "make_x", "make_weights", "sweep_cases", "sample_tokens", "empty_experts",
+    "make_x", "make_weights", "make_expert_outputs", "make_dout", "sweep_cases",
+    "sample_tokens", "empty_experts",
 ]

@@ -202,6 +202,26 @@ def _stage_run(moe, w, W1, W3, W2, lg, x):
     return dict(ids=ids, gates=gates, xg=xg, h=h, y=y, out=out, **b)
 
 
+def _check_combine_stage(moe, w, s, o_g32, toks):
+    """moe_combine on seeded stand-in expert outputs y [rows, H] with the oracle's
+    route_row and gates, against the oracle's fixed-order fp32 combine: bit-exact."""
+    sh = moe.shape(**w.shape())
+    rows = int(s["offsets"][-1])
+    y = inputs.make_expert_outputs(w, max(rows, 1))
+    rr = torch.from_numpy(np.ascontiguousarray(s["route_row"].reshape(-1, w.k))).to(DEV)
+    gt = torch.from_numpy(np.ascontiguousarray(o_g32.reshape(-1, w.k))).to(DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = torch.empty((w.n_tokens, w.H), dtype=torch.bfloat16, device=DEV)
+    moe.moe_combine(y.to(DEV), rr, gt, out, st, sh)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    toks = np.asarray(list(toks))
+    rrt = s["route_row"].reshape(-1, w.k)[toks]
+    used = np.unique(rrt)
+    exp = oracle.combine_f32(y.numpy()[used], np.searchsorted(used, rrt), o_g32.reshape(-1, w.k)[toks], w.k)
+    assert (bits(out)[toks] == exp).all()
+
+
 def test_tiny_all_stages_vs_oracle(cuda_lib):
     moe = cuda_lib
     w = inputs.WORKLOADS["tiny"]
@@ -227,10 +247,9 @@ def test_tiny_all_stages_vs_oracle(cuda_lib):
     assert (gh == o_h).mean() > 0.995
     gy = r["y"][torch.from_numpy(real).to(DEV)].cpu().numpy()
     assert rms_floor_err(gy, o_y) < Y_TOL
-    # combine: bit-exact against the fixed-order definition on the GPU's own y and gates
-    y_np = r["y"].cpu().numpy()
-    exp = oracle.combine_f32(y_np, g["route_row"].reshape(-1, w.k), r["gates"].cpu().numpy(), w.k)
-    assert (bits(r["out"]) == exp).all()
+    # combine: bit-exact against the fixed-order definition, both sides fed the
+    # same seeded stand-in expert outputs and the oracle's own gates and route_row
+    _check_combine_stage(moe, w, s, o_g32, range(w.n_tokens))
     # end to end against the oracle's fp64 layer output
     res = oracle.layer_tokens(lg, bits(x), Wd, w.P, w.N, w.k, w.E, w.H, w.I, range(w.n_tokens))
     assert rms_floor_err(bf16_to_f64(bits(r["out"])), res["out64"]) < OUT_TOL
@@ -325,13 +344,9 @@ def test_mid_stages_sampled(cuda_lib):
     idx = torch.from_numpy(pick).to(DEV)
     assert (bits(r["h"][idx]) == o_h).mean() > 0.995
     assert rms_floor_err(r["y"][idx].cpu().numpy(), o_y) < Y_TOL
-    # combine bit-exact on sampled tokens
-    toks = inputs.sample_tokens(w.n_tokens, 300, seed=2)
-    rr = g["route_row"].reshape(-1, w.k)[toks]
-    yt = r["y"][torch.from_numpy(np.unique(rr)).to(DEV)].cpu().numpy()
-    remap = np.searchsorted(np.unique(rr), rr)
-    exp = oracle.combine_f32(yt, remap, r["gates"].cpu().numpy()[toks], w.k)
-    assert (bits(r["out"])[toks] == exp).all()
+    # combine bit-exact on sampled tokens (seeded stand-in expert outputs)
+    _, o_g32, _ = oracle.route_topk(lg, w.k)
+    _check_combine_stage(moe, w, s, o_g32, inputs.sample_tokens(w.n_tokens, 300, seed=2))
 
 
 # ---------------------------------------------------------------- whole layer
