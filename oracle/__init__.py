@@ -1,4 +1,4 @@
-"""CPU oracle for the deterministic MoE layer forward (test infrastructure only).
+"""CPU oracle for the deterministic MoE layer, forward and backward (test infrastructure only).
 
 Only the test suite, the package smoke check and the benchmark's CPU-baseline
 leg may import this package. It wraps oracle/moe_oracle.cpp (plain C++,
@@ -58,6 +58,17 @@ def lib():
         L.oracle_combine_f64.restype = None
         L.oracle_combine_f32.argtypes = [_f32p, ctypes.c_int32, _i64p, _f32p, ctypes.c_int64,
                                          ctypes.c_int32, _u16p]
+        L.oracle_ffn_bwd_rows.argtypes = [_u16p, _u16p, _f64p, ctypes.c_int64, _i32p, ctypes.c_int32,
+                                          ctypes.c_int32, ptr_arr, ptr_arr, ptr_arr, ctypes.c_int,
+                                          _f64p, _f64p, _u16p, _u16p, _u16p]
+        L.oracle_ffn_bwd_rows.restype = None
+        L.oracle_wgrad_expert.argtypes = [_u16p, _u16p, _f64p, ctypes.c_int64, ctypes.c_int32,
+                                          ctypes.c_int32, _u16p, _u16p, _u16p, _i32p, ctypes.c_int32,
+                                          _i32p, ctypes.c_int32, ctypes.c_int, _f64p, _f64p, _f64p]
+        L.oracle_wgrad_expert.restype = None
+        L.oracle_router_bwd.argtypes = [_f64p, _f64p, _i32p, ctypes.c_int64, ctypes.c_int32,
+                                        ctypes.c_int32, _f64p]
+        L.oracle_router_bwd.restype = None
         L.oracle_combine_f32.restype = None
         L.oracle_round_bf16.argtypes = [ctypes.c_double]
         L.oracle_round_bf16.restype = ctypes.c_uint16
@@ -271,3 +282,131 @@ def layer_tokens(logits, x_bits, weights, P: int, N: int, k: int, E: int, H: int
     return dict(ids=ids, gates32=g32, gates64=g64, sched=sch, out64=out64, out_bf16=outb,
                 rows=uniq, row_index=inv.reshape(len(toks), k), xg=xg, h=h, y=y,
                 experts=ex)
+
+
+# ---------------------------------------------------------------- backward
+def _weight_ptr_arrays(experts, W1: dict, W3: dict, W2: dict):
+    ex = np.asarray(experts, np.int32)
+    E = int(ex.max()) + 1 if len(ex) else 1
+    keep, arrs = [], []
+    for Wd in (W1, W3, W2):
+        a = (ctypes.c_void_p * E)()
+        for e, w in Wd.items():
+            if e < E:
+                w = np.ascontiguousarray(w, np.uint16)
+                keep.append(w)
+                a[e] = w.ctypes.data
+        arrs.append(a)
+    for e in set(ex.tolist()):
+        if not (arrs[0][e] and arrs[1][e] and arrs[2][e]):
+            raise ValueError(f"weights of expert {e} not given")
+    return keep, [ctypes.cast(a, ctypes.POINTER(ctypes.c_void_p)) for a in arrs]
+
+
+def ffn_bwd_rows(xg_bits, dys_bits, g, experts, W1: dict, W3: dict, W2: dict, H: int, I: int,
+                 exact: bool = False):
+    """Backward through the SwiGLU expert FFN, one route row at a time.
+
+    xg_bits/dys_bits [n,H] bf16 bits (the row's token activations and upstream
+    gradient), g [n] gates, experts [n]. Returns dict dgate [n] (fp64),
+    dxg [n,H] (fp64) and, unless exact, da/db/hg [n,I] bf16 bits.
+    """
+    xb = np.ascontiguousarray(xg_bits, np.uint16)
+    db_ = np.ascontiguousarray(dys_bits, np.uint16)
+    gg = np.ascontiguousarray(np.asarray(g, np.float64).reshape(-1))
+    ex = np.ascontiguousarray(np.asarray(experts, np.int32))
+    n = len(ex)
+    out = dict(dgate=np.zeros(n, np.float64), dxg=np.zeros((n, H), np.float64),
+               da=np.zeros((n, I), np.uint16), db=np.zeros((n, I), np.uint16),
+               hg=np.zeros((n, I), np.uint16))
+    if n:
+        keep, arrs = _weight_ptr_arrays(ex, W1, W3, W2)
+        lib().oracle_ffn_bwd_rows(_p(xb, _u16p), _p(db_, _u16p), _p(gg, _f64p), n, _p(ex, _i32p),
+                                  H, I, *arrs, int(bool(exact)), _p(out["dgate"], _f64p),
+                                  _p(out["dxg"], _f64p), _p(out["da"], _u16p),
+                                  _p(out["db"], _u16p), _p(out["hg"], _u16p))
+    if exact:
+        for key in ("da", "db", "hg"):
+            del out[key]
+    return out
+
+
+def wgrad_expert(xg_bits, dys_bits, g, W1e, W3e, W2e, hs, is_, exact: bool = False):
+    """Weight gradients of one expert from all R rows it received, at the chosen
+    columns: dW1[hs][:, is_], dW3[hs][:, is_] ([n_h, n_i]) and dW2[is_][:, hs]
+    ([n_i, n_h]), fp64."""
+    xb = np.ascontiguousarray(xg_bits, np.uint16)
+    db_ = np.ascontiguousarray(dys_bits, np.uint16)
+    gg = np.ascontiguousarray(np.asarray(g, np.float64).reshape(-1))
+    R, H = xb.shape if xb.size else (0, np.asarray(W2e).shape[1])
+    I = np.asarray(W1e).shape[1]
+    hh = np.ascontiguousarray(np.asarray(hs, np.int32))
+    ii = np.ascontiguousarray(np.asarray(is_, np.int32))
+    w1, w3, w2 = (np.ascontiguousarray(w, np.uint16) for w in (W1e, W3e, W2e))
+    dW1 = np.zeros((len(hh), len(ii)), np.float64)
+    dW3 = np.zeros((len(hh), len(ii)), np.float64)
+    dW2 = np.zeros((len(ii), len(hh)), np.float64)
+    lib().oracle_wgrad_expert(_p(xb, _u16p) if R else _p(np.zeros(1, np.uint16), _u16p),
+                              _p(db_, _u16p) if R else _p(np.zeros(1, np.uint16), _u16p),
+                              _p(gg, _f64p) if R else _p(np.zeros(1), _f64p), R, H, I,
+                              _p(w1, _u16p), _p(w3, _u16p), _p(w2, _u16p), _p(hh, _i32p), len(hh),
+                              _p(ii, _i32p), len(ii), int(bool(exact)), _p(dW1, _f64p),
+                              _p(dW3, _f64p), _p(dW2, _f64p))
+    return dW1, dW3, dW2
+
+
+def router_bwd(dgate, g, ids, E: int) -> np.ndarray:
+    """dlogits [n,E]: g_j (dgate_j - sum_j' g_j' dgate_j') at the chosen experts, 0 elsewhere."""
+    dg = np.ascontiguousarray(np.asarray(dgate, np.float64))
+    gg = np.ascontiguousarray(np.asarray(g, np.float64))
+    ii = np.ascontiguousarray(np.asarray(ids, np.int32))
+    n, k = ii.shape
+    out = np.zeros((n, E), np.float64)
+    if n:
+        lib().oracle_router_bwd(_p(dg, _f64p), _p(gg, _f64p), _p(ii, _i32p), n, k, E, _p(out, _f64p))
+    return out
+
+
+def layer_backward_tokens(logits, x_bits, dout_bits, weights, k: int, E: int, H: int, I: int,
+                          tokens, exact: bool = False):
+    """Gradients of the layer for a set of tokens: dx [n,H] (fp64, before the
+    bf16 cast), dlogits [n,E] and the gate gradients dgate [n,k].
+
+    Each route (t, j) is one expert row: its token's activations x[t] and
+    upstream gradient dout[t], gate g[t,j] (the fp64 softmax over the chosen
+    logits) and expert ids[t,j]. The push-reverse-dispatch sums a token's k
+    row gradients in ascending slot order.
+    """
+    ids, g32, g64 = route_topk(logits, k)
+    toks = np.asarray(list(tokens), np.int64)
+    n = len(toks)
+    xb = np.asarray(x_bits, np.uint16)[toks]
+    db_ = np.asarray(dout_bits, np.uint16)[toks]
+    rx = np.repeat(xb, k, axis=0)
+    rd = np.repeat(db_, k, axis=0)
+    ex = ids[toks].reshape(-1)
+    r = ffn_bwd_rows(rx, rd, g64[toks].reshape(-1), ex, *weights, H=H, I=I, exact=exact)
+    dxg = r["dxg"].reshape(n, k, H)
+    dx = np.zeros((n, H), np.float64)
+    for j in range(k):
+        dx += dxg[:, j, :]
+    dgate = r["dgate"].reshape(n, k)
+    dlogits = router_bwd(dgate, g64[toks], ids[toks], E)
+    return dict(ids=ids, gates32=g32, gates64=g64, dx64=dx, dgate=dgate, dlogits=dlogits,
+                rows=r)
+
+
+def wgrad_sample(logits, x_bits, dout_bits, weights, k: int, E: int, experts, hs, is_,
+                 exact: bool = False):
+    """dW1/dW3 [n_h, n_i] and dW2 [n_i, n_h] at the chosen columns for each chosen
+    expert: {e: (dW1s, dW3s, dW2s)}. An expert's rows are every route that chose
+    it (token activations, upstream gradient and gate of the route)."""
+    ids, _, g64 = route_topk(logits, k)
+    xb = np.asarray(x_bits, np.uint16)
+    db_ = np.asarray(dout_bits, np.uint16)
+    W1, W3, W2 = weights
+    out = {}
+    for e in experts:
+        t, j = np.nonzero(ids == e)
+        out[e] = wgrad_expert(xb[t], db_[t], g64[t, j], W1[e], W3[e], W2[e], hs, is_, exact)
+    return out

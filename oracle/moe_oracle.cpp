@@ -1,4 +1,4 @@
-// Plain CPU oracle for the deterministic MoE layer forward.
+// Plain CPU oracle for the deterministic MoE layer, forward and backward.
 //
 // TEST INFRASTRUCTURE ONLY. Nothing on the product path may call, link or load
 // this file: only the test suite, the package's smoke check and the benchmark's
@@ -37,6 +37,13 @@
 //  R8 SwiGLU: h = bf16_rne(silu(x.W1) * (x.W3)), y = h.W2;
 //  R9 combine: out = bf16_rne(sum_j g_j * y_j) accumulated from 0 in
 //     ascending slot order (the fp32 fixed-order form uses fmaf).
+//  B1 backward ("Mixture-of-Kittens", MoK overview: one table serves the
+//     forward and backward phases; pull-reverse-combine, push-reverse-
+//     dispatch; section 5: router gradients from the inner product of the
+//     SwiGLU activations and the down-projection dgrads): the exact gradient
+//     of the layer above, with bf16 rounding at every GEMM operand that is
+//     not an input: the saved pre-activations a, b, the SwiGLU output h, the
+//     SwiGLU input gradients da, db and the gate-scaled activations g*h.
 #include <algorithm>
 #include <cfenv>
 #include <cmath>
@@ -429,6 +436,167 @@ void oracle_combine_f32(const float* y, int32_t H, const int64_t* sel, const flo
       }
       out_bf16[a * H + c] = double_to_bf16(static_cast<double>(acc));
     }
+  }
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward (B1). For one route row with token activations x (the gathered
+// row), upstream gradient d (the token's dout row), gate g and expert e:
+//   a = x.W1[e], b = x.W3[e]                 (fp64)
+//   h = silu(a) * b                          (rounded to bf16: the forward's h)
+//   as, bs = a, b                            (rounded to bf16: saved activations)
+//   dhu = d . W2[e]^T                        dhu[i] = sum_c d[c] W2[e][i][c]
+//   dgate = sum_i h[i] dhu[i]                (the gate's gradient, SonicMoE form)
+//   dh = g * dhu
+//   s = 1 / (1 + exp(-as))
+//   da = dh * bs * s * (1 + as * (1 - s))    (d silu(a)/da = s (1 + a (1 - s)))
+//   db = dh * as * s                         (rounded to bf16: GEMM operands)
+//   hg = g * h                               (rounded to bf16: the dW2 operand)
+//   dx_row = da . W1[e]^T + db . W3[e]^T     dx_row[c] = sum_i da[i] W1[e][c][i] + db[i] W3[e][c][i]
+// exact != 0 drops every bf16 rounding: the plain real-number gradient.
+// ---------------------------------------------------------------------------
+namespace {
+
+double rnd(double v, int exact) { return exact ? v : bf16_to_double(double_to_bf16(v)); }
+
+// The element-wise part for one (row, column i): from a, b (unrounded), dhu
+// and g, the values the two backward GEMMs and the gate gradient consume.
+struct BwdElem {
+  double h, da, db, hg;
+};
+
+BwdElem swiglu_bwd_elem(double a, double b, double dhu, double g, int exact) {
+  BwdElem r;
+  r.h = rnd(a / (1.0 + std::exp(-a)) * b, exact);
+  const double as = rnd(a, exact), bs = rnd(b, exact);
+  const double dh = g * dhu;
+  const double s = 1.0 / (1.0 + std::exp(-as));
+  r.da = rnd(dh * bs * s * (1.0 + as * (1.0 - s)), exact);
+  r.db = rnd(dh * as * s, exact);
+  r.hg = rnd(g * r.h, exact);
+  return r;
+}
+
+}  // namespace
+
+extern "C" {
+
+// Per-row backward through the expert FFN (B1).
+// xg, dys: [n, H] bf16 bits (the row's token activations and its token's
+// upstream gradient); g: [n] gate of the row's route; expert: [n].
+// Outputs (each may be null): dgate [n] fp64; dxg [n, H] fp64;
+// da, db, hg [n, I] (exact == 0: bf16 bits of the rounded values; ignored
+// when exact != 0).
+void oracle_ffn_bwd_rows(const uint16_t* xg, const uint16_t* dys, const double* g, int64_t n,
+                         const int32_t* expert, int32_t H, int32_t I,
+                         const uint16_t* const* W1, const uint16_t* const* W3,
+                         const uint16_t* const* W2, int exact, double* dgate, double* dxg,
+                         uint16_t* da_out, uint16_t* db_out, uint16_t* hg_out) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < n; ++r) {
+    const int32_t e = expert[r];
+    const uint16_t* xr = xg + r * H;
+    const uint16_t* dr = dys + r * H;
+    const uint16_t* w1 = W1[e];
+    const uint16_t* w3 = W3[e];
+    const uint16_t* w2 = W2[e];
+    std::vector<double> a(I, 0.0), b(I, 0.0), dhu(I, 0.0), da(I), db(I);
+    for (int32_t c = 0; c < H; ++c) {
+      const double xv = bf16_to_double(xr[c]);
+      for (int32_t i = 0; i < I; ++i) {
+        a[i] += xv * bf16_to_double(w1[static_cast<int64_t>(c) * I + i]);
+        b[i] += xv * bf16_to_double(w3[static_cast<int64_t>(c) * I + i]);
+      }
+    }
+    for (int32_t i = 0; i < I; ++i) {
+      double acc = 0.0;
+      for (int32_t c = 0; c < H; ++c)
+        acc += bf16_to_double(dr[c]) * bf16_to_double(w2[static_cast<int64_t>(i) * H + c]);
+      dhu[i] = acc;
+    }
+    double dg = 0.0;
+    for (int32_t i = 0; i < I; ++i) {
+      const BwdElem v = swiglu_bwd_elem(a[i], b[i], dhu[i], g[r], exact);
+      dg += v.h * dhu[i];
+      da[i] = v.da;
+      db[i] = v.db;
+      if (!exact) {
+        if (da_out) da_out[r * I + i] = double_to_bf16(v.da);
+        if (db_out) db_out[r * I + i] = double_to_bf16(v.db);
+        if (hg_out) hg_out[r * I + i] = double_to_bf16(v.hg);
+      }
+    }
+    if (dgate) dgate[r] = dg;
+    if (dxg) {
+      for (int32_t c = 0; c < H; ++c) {
+        double acc = 0.0;
+        for (int32_t i = 0; i < I; ++i)
+          acc += da[i] * bf16_to_double(w1[static_cast<int64_t>(c) * I + i]) +
+                 db[i] * bf16_to_double(w3[static_cast<int64_t>(c) * I + i]);
+        dxg[r * H + c] = acc;
+      }
+    }
+  }
+}
+
+// Weight gradients of one expert (B1), accumulated over all R rows the
+// expert received ("in one pass over the token dimension"):
+//   dW1[c][i] = sum_rows x[c] da[i],  dW3[c][i] = sum_rows x[c] db[i],
+//   dW2[i][c] = sum_rows hg[i] d[c].
+// Only the entries at the chosen columns are formed: hs (n_h values of c)
+// and is (n_i values of i); outputs dW1s, dW3s [n_h, n_i], dW2s [n_i, n_h].
+// xg, dys: [R, H] bf16 bits; g: [R].
+void oracle_wgrad_expert(const uint16_t* xg, const uint16_t* dys, const double* g, int64_t R,
+                         int32_t H, int32_t I, const uint16_t* W1e, const uint16_t* W3e,
+                         const uint16_t* W2e, const int32_t* hs, int32_t n_h, const int32_t* is,
+                         int32_t n_i, int exact, double* dW1s, double* dW3s, double* dW2s) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int32_t q = 0; q < n_i; ++q) {
+    const int32_t i = is[q];
+    std::vector<double> da(R), db(R), hg(R);
+    for (int64_t r = 0; r < R; ++r) {
+      double a = 0.0, b = 0.0, dhu = 0.0;
+      for (int32_t c = 0; c < H; ++c) {
+        const double xv = bf16_to_double(xg[r * H + c]);
+        a += xv * bf16_to_double(W1e[static_cast<int64_t>(c) * I + i]);
+        b += xv * bf16_to_double(W3e[static_cast<int64_t>(c) * I + i]);
+        dhu += bf16_to_double(dys[r * H + c]) * bf16_to_double(W2e[static_cast<int64_t>(i) * H + c]);
+      }
+      const BwdElem v = swiglu_bwd_elem(a, b, dhu, g[r], exact);
+      da[r] = v.da;
+      db[r] = v.db;
+      hg[r] = v.hg;
+    }
+    for (int32_t p = 0; p < n_h; ++p) {
+      const int32_t c = hs[p];
+      double s1 = 0.0, s3 = 0.0, s2 = 0.0;
+      for (int64_t r = 0; r < R; ++r) {
+        const double xv = bf16_to_double(xg[r * H + c]);
+        s1 += xv * da[r];
+        s3 += xv * db[r];
+        s2 += hg[r] * bf16_to_double(dys[r * H + c]);
+      }
+      dW1s[static_cast<int64_t>(p) * n_i + q] = s1;
+      dW3s[static_cast<int64_t>(p) * n_i + q] = s3;
+      dW2s[static_cast<int64_t>(q) * n_h + p] = s2;
+    }
+  }
+}
+
+// Router backward (B1): gates g_j = softmax over the chosen logits l_j, so
+// dL/dl_j = g_j (dgate_j - sum_j' g_j' dgate_j'); logits that were not
+// chosen get 0. dgate, g, ids: [n, k]; dlogits: [n, E] (fp64).
+void oracle_router_bwd(const double* dgate, const double* g, const int32_t* ids, int64_t n,
+                       int32_t k, int32_t E, double* dlogits) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < n; ++t) {
+    double* out = dlogits + t * E;
+    for (int32_t e = 0; e < E; ++e) out[e] = 0.0;
+    double s = 0.0;
+    for (int32_t j = 0; j < k; ++j) s += g[t * k + j] * dgate[t * k + j];
+    for (int32_t j = 0; j < k; ++j) out[ids[t * k + j]] = g[t * k + j] * (dgate[t * k + j] - s);
   }
 }
 
