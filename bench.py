@@ -10,6 +10,11 @@ max-over-ranks device time. Rank 0 prints one JSON line.
 
 --impl reference times the CPU oracle (test infrastructure) on a bounded
 sample of the same workload on the host cores, as the reference arm.
+
+The line also carries a "backward" object: the training step of the same
+layer (moe_layer_forward_train, which keeps the activations, and
+moe_layer_backward: reverse combine, dgrad GEMMs, reverse dispatch, router
+gradient, wgrad GEMMs) timed on the same batch, with per-stage rooflines.
 """
 from __future__ import annotations
 
@@ -66,6 +71,34 @@ def algorithmic_work(w, rows_used: int, rows_real: int):
         "ffn_gemm2": dict(flops=2 * rows_real * I * H),
         "combine": dict(bytes=R * H * 4 + T * H * 2 + R * 8),
     }
+
+
+def backward_work(w, rows_used: int):
+    """Bytes / flops of each backward stage (real routes only)."""
+    T, R, H, I, E = w.n_tokens, w.n_routes, w.H, w.I, w.E
+    return {
+        "reverse_combine": dict(bytes=R * H * 2 + rows_used * H * 2),
+        "dgrad_h": dict(flops=2 * R * H * I),
+        "dgrad_x": dict(flops=2 * R * 2 * I * H),
+        "reverse_dispatch": dict(bytes=R * H * 4 + T * H * 2 + R * 4),
+        "router_bwd": dict(bytes=R * (I // 128) * 4 + R * 12 + T * E * 4),
+        "wgrad_w2": dict(flops=2 * R * I * H),
+        "wgrad_w13": dict(flops=2 * R * H * 2 * I),
+    }
+
+
+def stage_rooflines(stage_ms: dict, work: dict, peaks: dict) -> dict:
+    out = {}
+    for name, t in stage_ms.items():
+        d = {"ms": t}
+        if "bytes" in work[name]:
+            gbs = work[name]["bytes"] / (t / 1e3) / 1e9
+            d.update(bytes=work[name]["bytes"], gbs=gbs, frac_hbm=gbs / peaks["hbm"])
+        else:
+            tf = work[name]["flops"] / (t / 1e3) / 1e12
+            d.update(flops=work[name]["flops"], tflops=tf, frac_bf16=tf / peaks["bf16_sus"])
+        out[name] = d
+    return out
 
 
 # ---------------------------------------------------------------- clocks
@@ -337,15 +370,65 @@ def run_ours(args):
         e2e = dict(ms=e2e_ms, h2d=lg_cpu.numel() * 4 + x_cpu.numel() * 2,
                    d2h=out_h.numel() * 2, chk=chk)
         del wsh
+    else:
+        del ws
+    torch.cuda.empty_cache()
+
+    # the training step: forward keeping the activations, then the backward
+    bwd = None
+    if not args.no_backward and moe.train_workspace_bytes(sh) > 0:
+        wst = torch.empty(moe.train_workspace_bytes(sh), dtype=torch.uint8, device=dev)
+        dout = inputs.make_dout(w, device=dev)
+        dx = torch.empty((w.n_tokens, w.H), dtype=torch.bfloat16, device=dev)
+        dlg = torch.empty((w.n_tokens, w.E), dtype=torch.float32, device=dev)
+        dW1 = torch.empty((w.E, w.H, w.I), dtype=torch.float32, device=dev)
+        dW3 = torch.empty_like(dW1)
+        dW2 = torch.empty((w.E, w.I, w.H), dtype=torch.float32, device=dev)
+        bev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.N_BWD_EVENTS)]
+               for _ in range(args.bwd_steps)]
+        for row in bev:
+            for e in row:
+                e.record()
+
+        def train_step(events=None):
+            moe.moe_layer_forward_train(lg, x, *W, out, wst, st, sh)
+            moe.moe_layer_backward(dout, *W, dx, dlg, dW1, dW3, dW2, wst, st, sh,
+                                   stage_events=events)
+
+        for _ in range(args.warmup):
+            train_step()
+        torch.cuda.synchronize()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nb0 = moe.launch_count()
+        b0.record()
+        for i in range(args.bwd_steps):
+            train_step(bev[i])
+        b1.record()
+        torch.cuda.synchronize()
+        bwd = dict(train_ms=b0.elapsed_time(b1), launches=moe.launch_count() - nb0,
+                   bwd_ms=statistics.mean(bev[i][0].elapsed_time(bev[i][-1])
+                                          for i in range(args.bwd_steps)),
+                   stages={name: statistics.mean(bev[i][j].elapsed_time(bev[i][j + 1])
+                                                 for i in range(args.bwd_steps))
+                           for j, name in enumerate(moe.BWD_STAGES)})
+        del wst, dW1, dW3, dW2
+        torch.cuda.empty_cache()
     clk = clocks.stop()
 
     if int(st.item()) != 0:
         raise RuntimeError(f"device status {int(st.item())}")
 
     names = list(stage_ms)
+    bnames = list(bwd["stages"]) if bwd else []
     vec = ([ms] + [stage_ms[n] for n in names] + ([e2e["ms"]] if e2e else []) +
-           ([mb_row] if mb_row is not None else []))
+           ([mb_row] if mb_row is not None else []) +
+           ([bwd["train_ms"], bwd["bwd_ms"]] + [bwd["stages"][n] for n in bnames] if bwd else []))
     vec = reduce_max(vec, ready, device=dev)
+    if bwd:
+        nb = 2 + len(bnames)
+        bvec, vec = vec[-nb:], vec[:-nb]
+        bwd["train_ms"], bwd["bwd_ms"] = bvec[0], bvec[1]
+        bwd["stages"] = dict(zip(bnames, bvec[2:]))
     ms = vec[0]
     stage_ms = dict(zip(names, vec[1:1 + len(names)]))
     if mb_row is not None:
@@ -359,16 +442,7 @@ def run_ours(args):
         peaks = load_peaks()
         rows_used = schedule_rows(moe, w, sh, lg)
         work = algorithmic_work(w, rows_used, w.n_routes)
-        stages = {}
-        for name, t in stage_ms.items():
-            d = {"ms": t}
-            if "bytes" in work[name]:
-                gbs = work[name]["bytes"] / (t / 1e3) / 1e9
-                d.update(bytes=work[name]["bytes"], gbs=gbs, frac_hbm=gbs / peaks["hbm"])
-            else:
-                tf = work[name]["flops"] / (t / 1e3) / 1e12
-                d.update(flops=work[name]["flops"], tflops=tf, frac_bf16=tf / peaks["bf16_sus"])
-            stages[name] = d
+        stages = stage_rooflines(stage_ms, work, peaks)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
@@ -405,6 +479,27 @@ def run_ours(args):
                                      "ms_per_step": mb_row / args.steps,
                                      "value": w.n_tokens * world * args.steps / (mb_row / 1e3),
                                      "unit": "tokens/s"}
+        if bwd:
+            bst = stage_rooflines(bwd["stages"], backward_work(w, rows_used), peaks)
+            top = max(bst, key=lambda n: bst[n]["ms"])
+            tokens_b = w.n_tokens * world * args.bwd_steps
+            line["backward"] = {
+                "value": w.n_tokens * world / (bwd["bwd_ms"] / 1e3), "unit": "tokens/s",
+                "ms_per_step": bwd["bwd_ms"],
+                "train_step": {"value": tokens_b / (bwd["train_ms"] / 1e3), "unit": "tokens/s",
+                               "ms_per_step": bwd["train_ms"] / args.bwd_steps,
+                               "what": "moe_layer_forward_train + moe_layer_backward",
+                               "gpu_launches": bwd["launches"] // args.bwd_steps},
+                "steps": args.bwd_steps, "warmup": args.warmup,
+                "stages": bst,
+                "roofline": {"kernel": top, "bound": "tensor" if "tflops" in bst[top] else "hbm",
+                             "achieved": bst[top].get("tflops", bst[top].get("gbs")),
+                             "peak": peaks["bf16_sus"] if "tflops" in bst[top] else peaks["hbm"],
+                             "unit": "TFLOP/s" if "tflops" in bst[top] else "GB/s",
+                             "frac": bst[top].get("frac_bf16", bst[top].get("frac_hbm")),
+                             "traffic": None},
+                "dout": "bf16 N(0,1), seeded",
+            }
         line["clocks"] = clk
         if world == 1 and not args.no_cpu_baseline:
             r = oracle_sample(w, lg_cpu, x_cpu, W, row_budget_s=args.cpu_budget)
@@ -467,6 +562,8 @@ def main(argv=None):
     ap.add_argument("--no-minibatch-row", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--bwd-steps", type=int, default=10)
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-row-budget", type=float, default=3.0)
     args = ap.parse_args(argv)

@@ -15,6 +15,8 @@ constexpr size_t kAlign = 1024;
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// Buffers written with 32-byte vector stores.
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 moe_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_CUDA_ERROR; }
 
@@ -49,10 +51,24 @@ int64_t rows_max_of(const moe_shape_t* s) {
   return (raw + 255) / 256 * 256;
 }
 
+// Extra limits of the backward pass (CTA-pair tiles of 256 rows x 256 columns
+// in every GEMM: segments padded to multiples of 256, I a multiple of 256).
+moe_status_t check_bwd_shape(const moe_shape_t* s) {
+  moe_status_t st = check_ffn_shape(s);
+  if (st != MOE_OK) return st;
+  if (s->I % 256 != 0 || s->pad % 256 != 0) return MOE_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
 // Layout of the layer workspace (offsets in bytes, each kAlign-aligned).
+// The training layout keeps what the backward reads (ids, gates, route_row,
+// Phi, offsets, counts, xg, h and the pre-activations ab) and adds the
+// backward's buffers; dxg [rows, H] fp32 reuses y, which is dead once the
+// forward's combine has run.
 struct LayerWs {
   size_t ids, gates, route_row, phi, offsets, counts, sched, xg, h, y, total;
   size_t logits[2], x[2], out, total_host;  // moe_layer_forward_host additions
+  size_t ab, dys, dab, hg, gate_row, part, total_train;  // training additions
 };
 
 LayerWs layer_ws(const moe_shape_t* s) {
@@ -61,28 +77,37 @@ LayerWs layer_ws(const moe_shape_t* s) {
   const size_t rows = static_cast<size_t>(rows_max_of(s));
   const size_t tokens = static_cast<size_t>(s->P) * s->N;
   size_t o = 0;
-  auto take = [&](size_t bytes) {
-    const size_t at = o;
-    o = align_up(o + (bytes ? bytes : 1), kAlign);
+  auto take = [](size_t& cur, size_t bytes) {
+    const size_t at = cur;
+    cur = align_up(cur + (bytes ? bytes : 1), kAlign);
     return at;
   };
-  w.ids = take(routes * 4);
-  w.gates = take(routes * 4);
-  w.route_row = take(routes * 4);
-  w.phi = take(rows * 8);
-  w.offsets = take((s->E + 1) * 4);
-  w.counts = take(static_cast<size_t>(s->E) * s->P * 4);
-  w.sched = take(schedule_ws_bytes(s->P, s->N, s->k, s->E));
-  w.xg = take(rows * s->H * 2);
-  w.h = take(rows * s->I * 2);
-  w.y = take(rows * s->H * 4);
+  w.ids = take(o, routes * 4);
+  w.gates = take(o, routes * 4);
+  w.route_row = take(o, routes * 4);
+  w.phi = take(o, rows * 8);
+  w.offsets = take(o, (s->E + 1) * 4);
+  w.counts = take(o, static_cast<size_t>(s->E) * s->P * 4);
+  w.sched = take(o, schedule_ws_bytes(s->P, s->N, s->k, s->E));
+  w.xg = take(o, rows * s->H * 2);
+  w.h = take(o, rows * s->I * 2);
+  w.y = take(o, rows * s->H * 4);
   w.total = o;
+  size_t oh = o;
   for (int b = 0; b < 2; ++b) {  // consecutive host-buffer calls alternate
-    w.logits[b] = take(tokens * s->E * 4);
-    w.x[b] = take(tokens * s->H * 2);
+    w.logits[b] = take(oh, tokens * s->E * 4);
+    w.x[b] = take(oh, tokens * s->H * 2);
   }
-  w.out = take(tokens * s->H * 2);
-  w.total_host = o;
+  w.out = take(oh, tokens * s->H * 2);
+  w.total_host = oh;
+  size_t ot = o;
+  w.ab = take(ot, rows * s->I * 4);
+  w.dys = take(ot, rows * s->H * 2);
+  w.dab = take(ot, rows * s->I * 4);
+  w.hg = take(ot, rows * s->I * 2);
+  w.gate_row = take(ot, rows * 4);
+  w.part = take(ot, rows * (s->I / 128) * 4);
+  w.total_train = ot;
   return w;
 }
 
@@ -133,9 +158,11 @@ LayerBufs layer_bufs(void* ws, const LayerWs& w) {
 
 // Schedule -> dispatch -> FFN -> combine for one token slice (steps 2-4).
 // ev (7 events, may be null) marks the stage boundaries 1..6.
+// ab (training, whole batch only): GEMM1 also keeps the pre-activations.
 cudaError_t run_slice(const LayerBufs& b, const uint16_t* x, const uint16_t* W1, const uint16_t* W3,
                       const uint16_t* W2, uint16_t* out, Slice sl, const moe_shape_t* sh,
-                      int32_t* dev_status, cudaStream_t s, void* const* ev) {
+                      int32_t* dev_status, cudaStream_t s, void* const* ev,
+                      uint16_t* ab = nullptr) {
   const int64_t rows_max = rows_max_of(sh);
   auto rec = [&](int i) -> cudaError_t {
     return (ev && ev[i]) ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) : cudaSuccess;
@@ -154,7 +181,7 @@ cudaError_t run_slice(const LayerBufs& b, const uint16_t* x, const uint16_t* W1,
   if ((e = rec(3)) != cudaSuccess) return e;
   cudaEvent_t mid = (ev && ev[4]) ? static_cast<cudaEvent_t>(ev[4]) : nullptr;
   if ((e = launch_expert_ffn(b.xg, W1, W3, W2, b.offsets, b.counts, b.h, b.y, *sh, rows_max,
-                             dev_status, s, mid)) != cudaSuccess)
+                             dev_status, s, mid, ab)) != cudaSuccess)
     return e;
   if ((e = rec(5)) != cudaSuccess) return e;
   if ((e = launch_combine(b.y, b.route_row, b.gates, out, *sh, sl, rows_max, dev_status, s)) !=
@@ -167,8 +194,12 @@ cudaError_t run_slice(const LayerBufs& b, const uint16_t* x, const uint16_t* W1,
 moe_status_t layer_body(const float* logits, const uint16_t* x, const uint16_t* W1,
                         const uint16_t* W3, const uint16_t* W2, uint16_t* out,
                         int32_t minibatch_tokens, void* ws, int32_t* dev_status,
-                        const moe_shape_t* sh, cudaStream_t s, void* const* ev) {
-  const LayerBufs b = layer_bufs(ws, layer_ws(sh));
+                        const moe_shape_t* sh, cudaStream_t s, void* const* ev,
+                        bool train = false) {
+  const LayerWs lw = layer_ws(sh);
+  const LayerBufs b = layer_bufs(ws, lw);
+  uint16_t* ab = train ? at<uint16_t>(ws, lw.ab) : nullptr;
+  if (train) minibatch_tokens = 0;  // one schedule over the whole batch, kept for the backward
   const int32_t N = sh->N;
   const int32_t T = (minibatch_tokens <= 0 || minibatch_tokens >= N) ? N : minibatch_tokens;
   void* const* ev_use = (T == N) ? ev : nullptr;  // stage events: single-slice runs only
@@ -184,9 +215,66 @@ moe_status_t layer_body(const float* logits, const uint16_t* x, const uint16_t* 
   }
   for (int32_t t0 = 0; t0 < N && e == cudaSuccess; t0 += T) {
     const Slice sl{t0, (N - t0) < T ? (N - t0) : T};
-    e = run_slice(b, x, W1, W3, W2, out, sl, sh, dev_status, s, ev_use);
+    e = run_slice(b, x, W1, W3, W2, out, sl, sh, dev_status, s, ev_use, ab);
   }
   return from_cuda(e);
+}
+
+// The backward pass on the state a training forward left in `ws`.
+// ev (8 events, may be null): start, then after the reverse combine, the
+// dh GEMM, the dx GEMM, the reverse dispatch, the router gradient, dW2 and
+// dW1 | dW3.
+cudaError_t backward_body(const uint16_t* dout, const uint16_t* W1, const uint16_t* W3,
+                          const uint16_t* W2, uint16_t* dx, float* dlogits, float* dW1, float* dW3,
+                          float* dW2, void* ws, int32_t* dev_status, const moe_shape_t* sh,
+                          cudaStream_t s, void* const* ev) {
+  const LayerWs w = layer_ws(sh);
+  const LayerBufs b = layer_bufs(ws, w);
+  const int64_t rows_max = rows_max_of(sh);
+  uint16_t* ab = at<uint16_t>(ws, w.ab);
+  uint16_t* dys = at<uint16_t>(ws, w.dys);
+  uint16_t* dab = at<uint16_t>(ws, w.dab);
+  uint16_t* hg = at<uint16_t>(ws, w.hg);
+  float* gate_row = at<float>(ws, w.gate_row);
+  float* part = at<float>(ws, w.part);
+  float* dxg = b.y;
+  auto rec = [&](int i) -> cudaError_t {
+    return (ev && ev[i]) ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) : cudaSuccess;
+  };
+  auto evt = [&](int i) -> cudaEvent_t { return ev ? static_cast<cudaEvent_t>(ev[i]) : nullptr; };
+  cudaError_t e;
+  if ((e = rec(0)) != cudaSuccess) return e;
+  if (sh->N == 0) {  // no routes: every weight gradient is zero
+    const size_t wbytes = static_cast<size_t>(sh->E) * sh->H * sh->I * 4;
+    if ((e = cudaMemsetAsync(dW1, 0, wbytes, s)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dW3, 0, wbytes, s)) != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(dW2, 0, wbytes, s)) != cudaSuccess) return e;
+    for (int i = 1; i < 8; ++i)
+      if ((e = rec(i)) != cudaSuccess) return e;
+    return cudaSuccess;
+  }
+  if ((e = launch_reverse_combine(dout, b.phi, b.offsets, b.route_row, b.gates, dys, gate_row, *sh,
+                                  rows_max, dev_status, s)) != cudaSuccess)
+    return e;
+  if ((e = rec(1)) != cudaSuccess) return e;
+  if ((e = launch_expert_ffn_dgrad(dys, gate_row, ab, b.h, W1, W3, W2, b.offsets, b.counts, dab, hg,
+                                   part, dxg, *sh, rows_max, dev_status, s, evt(2))) != cudaSuccess)
+    return e;
+  if ((e = rec(3)) != cudaSuccess) return e;
+  if ((e = launch_reverse_dispatch(dxg, b.route_row, dx, *sh, rows_max, dev_status, s)) !=
+      cudaSuccess)
+    return e;
+  if ((e = rec(4)) != cudaSuccess) return e;
+  if ((e = launch_router_backward(part, sh->I / 128, b.route_row, b.ids, b.gates, dlogits,
+                                  static_cast<int64_t>(sh->P) * sh->N, sh->E, sh->k, rows_max,
+                                  dev_status, s)) != cudaSuccess)
+    return e;
+  if ((e = rec(5)) != cudaSuccess) return e;
+  // weight gradients last: deferred until every activation gradient is done
+  if ((e = launch_expert_ffn_wgrad(b.xg, dys, dab, hg, b.offsets, b.counts, dW1, dW3, dW2, *sh,
+                                   rows_max, dev_status, s, evt(6))) != cudaSuccess)
+    return e;
+  return rec(7);
 }
 
 // Per-device copy engines' streams and events of moe_layer_forward_host,
@@ -372,7 +460,7 @@ moe_status_t moe_schedule(const int32_t* ids, int32_t* phi, int32_t* offsets, in
   if (st != MOE_OK) return st;
   if (!phi || !offsets || !counts || !dev_status || !ws) return MOE_INVALID_ARG;
   if (shape->N > 0 && (!ids || !route_row)) return MOE_INVALID_ARG;
-  if (!aligned16(ids) || !aligned16(phi) || !aligned16(route_row) || !aligned16(ws))
+  if (!aligned16(ids) || !aligned16(phi) || !aligned16(route_row) || !aligned32(ws))
     return MOE_INVALID_ARG;
   if (ws_bytes < schedule_ws_bytes(shape->P, shape->N, shape->k, shape->E))
     return MOE_WORKSPACE_TOO_SMALL;
@@ -400,8 +488,8 @@ moe_status_t moe_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint16
   moe_status_t st = check_ffn_shape(shape);
   if (st != MOE_OK) return st;
   if (!xg || !W1 || !W3 || !W2 || !offsets || !h || !y || !dev_status) return MOE_INVALID_ARG;
-  if (!aligned16(xg) || !aligned16(W1) || !aligned16(W3) || !aligned16(W2) || !aligned16(h) ||
-      !aligned16(y))
+  if (!aligned16(xg) || !aligned16(W1) || !aligned16(W3) || !aligned16(W2) || !aligned32(h) ||
+      !aligned32(y))
     return MOE_INVALID_ARG;
   return from_cuda(launch_expert_ffn(xg, W1, W3, W2, offsets, counts, h, y, *shape,
                                      rows_max_of(shape), dev_status,
@@ -418,7 +506,7 @@ moe_status_t moe_expert_ffn_gather(const uint16_t* x, const int32_t* phi, const 
       (shape->N > 0 && !x))
     return MOE_INVALID_ARG;
   if (!aligned16(x) || !aligned16(phi) || !aligned16(W1) || !aligned16(W3) || !aligned16(W2) ||
-      !aligned16(h) || !aligned16(y))
+      !aligned32(h) || !aligned32(y))
     return MOE_INVALID_ARG;
   return from_cuda(launch_expert_ffn_gather(x, phi, W1, W3, W2, offsets, counts, h, y, *shape,
                                             rows_max_of(shape), dev_status,
@@ -449,12 +537,144 @@ moe_status_t moe_layer_forward(const float* logits, const uint16_t* x, const uin
   if (!W1 || !W3 || !W2 || !ws || !dev_status || (shape->N > 0 && (!logits || !x || !out)))
     return MOE_INVALID_ARG;
   if (!aligned16(logits) || !aligned16(x) || !aligned16(W1) || !aligned16(W3) || !aligned16(W2) ||
-      !aligned16(out) || !aligned16(ws))
+      !aligned16(out) || !aligned32(ws))
     return MOE_INVALID_ARG;
   if (minibatch_tokens < 0) return MOE_INVALID_ARG;
   if (ws_bytes < layer_ws(shape).total) return MOE_WORKSPACE_TOO_SMALL;
   return layer_body(logits, x, W1, W3, W2, out, minibatch_tokens, ws, dev_status, shape,
                     static_cast<cudaStream_t>(stream), stage_events);
+}
+
+size_t moe_train_workspace_bytes(const moe_shape_t* shape) {
+  if (check_bwd_shape(shape) != MOE_OK) return 0;
+  return layer_ws(shape).total_train;
+}
+
+moe_status_t moe_expert_ffn_train(const uint16_t* xg, const uint16_t* W1, const uint16_t* W3,
+                                  const uint16_t* W2, const int32_t* offsets,
+                                  const int32_t* counts, uint16_t* h, uint16_t* ab, float* y,
+                                  int32_t* dev_status, const moe_shape_t* shape, void* stream) {
+  moe_status_t st = check_bwd_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!xg || !W1 || !W3 || !W2 || !offsets || !h || !ab || !y || !dev_status)
+    return MOE_INVALID_ARG;
+  if (!aligned16(xg) || !aligned16(W1) || !aligned16(W3) || !aligned16(W2) || !aligned32(h) ||
+      !aligned32(ab) || !aligned32(y))
+    return MOE_INVALID_ARG;
+  return from_cuda(launch_expert_ffn(xg, W1, W3, W2, offsets, counts, h, y, *shape,
+                                     rows_max_of(shape), dev_status,
+                                     static_cast<cudaStream_t>(stream), nullptr, ab));
+}
+
+moe_status_t moe_layer_forward_train(const float* logits, const uint16_t* x, const uint16_t* W1,
+                                     const uint16_t* W3, const uint16_t* W2, uint16_t* out,
+                                     void* ws, size_t ws_bytes, int32_t* dev_status,
+                                     const moe_shape_t* shape, void* stream,
+                                     void* const* stage_events) {
+  moe_status_t st = check_bwd_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!W1 || !W3 || !W2 || !ws || !dev_status || (shape->N > 0 && (!logits || !x || !out)))
+    return MOE_INVALID_ARG;
+  if (!aligned16(logits) || !aligned16(x) || !aligned16(W1) || !aligned16(W3) || !aligned16(W2) ||
+      !aligned16(out) || !aligned32(ws))
+    return MOE_INVALID_ARG;
+  if (ws_bytes < layer_ws(shape).total_train) return MOE_WORKSPACE_TOO_SMALL;
+  return layer_body(logits, x, W1, W3, W2, out, 0, ws, dev_status, shape,
+                    static_cast<cudaStream_t>(stream), stage_events, true);
+}
+
+moe_status_t moe_reverse_combine(const uint16_t* dout, const int32_t* phi, const int32_t* offsets,
+                                 const int32_t* route_row, const float* gates, uint16_t* dys,
+                                 float* gate_row, int32_t* dev_status, const moe_shape_t* shape,
+                                 void* stream) {
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->H < 8 || shape->H % 8 != 0) return MOE_UNSUPPORTED_SHAPE;
+  if (!phi || !offsets || !dys || !gate_row || !dev_status ||
+      (shape->N > 0 && (!dout || !route_row || !gates)))
+    return MOE_INVALID_ARG;
+  if (!aligned16(dout) || !aligned16(phi) || !aligned16(dys)) return MOE_INVALID_ARG;
+  return from_cuda(launch_reverse_combine(dout, phi, offsets, route_row, gates, dys, gate_row,
+                                          *shape, rows_max_of(shape), dev_status,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_expert_ffn_dgrad(const uint16_t* dys, const float* gate_row, const uint16_t* ab,
+                                  const uint16_t* h, const uint16_t* W1, const uint16_t* W3,
+                                  const uint16_t* W2, const int32_t* offsets,
+                                  const int32_t* counts, uint16_t* dab, uint16_t* hg,
+                                  float* dgate_part, float* dxg, int32_t* dev_status,
+                                  const moe_shape_t* shape, void* stream) {
+  moe_status_t st = check_bwd_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!dys || !gate_row || !ab || !h || !W1 || !W3 || !W2 || !offsets || !dab || !hg ||
+      !dgate_part || !dxg || !dev_status)
+    return MOE_INVALID_ARG;
+  if (!aligned16(dys) || !aligned16(ab) || !aligned16(h) || !aligned16(W1) || !aligned16(W3) ||
+      !aligned16(W2) || !aligned16(dab) || !aligned16(hg) || !aligned16(dxg))
+    return MOE_INVALID_ARG;
+  return from_cuda(launch_expert_ffn_dgrad(dys, gate_row, ab, h, W1, W3, W2, offsets, counts, dab,
+                                           hg, dgate_part, dxg, *shape, rows_max_of(shape),
+                                           dev_status, static_cast<cudaStream_t>(stream), nullptr));
+}
+
+moe_status_t moe_reverse_dispatch(const float* dxg, const int32_t* route_row, uint16_t* dx,
+                                  int32_t* dev_status, const moe_shape_t* shape, void* stream) {
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->H < 4 || shape->H % 4 != 0) return MOE_UNSUPPORTED_SHAPE;
+  if (!dev_status || (shape->N > 0 && (!dxg || !route_row || !dx))) return MOE_INVALID_ARG;
+  if (!aligned16(dxg) || !aligned16(dx)) return MOE_INVALID_ARG;
+  return from_cuda(launch_reverse_dispatch(dxg, route_row, dx, *shape, rows_max_of(shape),
+                                           dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_router_backward(const float* dgate_part, const int32_t* route_row,
+                                 const int32_t* ids, const float* gates, float* dlogits,
+                                 int32_t* dev_status, const moe_shape_t* shape, void* stream) {
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->I < 128 || shape->I % 128 != 0) return MOE_UNSUPPORTED_SHAPE;
+  if (!dev_status || (shape->N > 0 && (!dgate_part || !route_row || !ids || !gates || !dlogits)))
+    return MOE_INVALID_ARG;
+  return from_cuda(launch_router_backward(dgate_part, shape->I / 128, route_row, ids, gates, dlogits,
+                                          static_cast<int64_t>(shape->P) * shape->N, shape->E,
+                                          shape->k, rows_max_of(shape), dev_status,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_expert_ffn_wgrad(const uint16_t* xg, const uint16_t* dys, const uint16_t* dab,
+                                  const uint16_t* hg, const int32_t* offsets,
+                                  const int32_t* counts, float* dW1, float* dW3, float* dW2,
+                                  int32_t* dev_status, const moe_shape_t* shape, void* stream) {
+  moe_status_t st = check_bwd_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!xg || !dys || !dab || !hg || !offsets || !dW1 || !dW3 || !dW2 || !dev_status)
+    return MOE_INVALID_ARG;
+  if (!aligned16(xg) || !aligned16(dys) || !aligned16(dab) || !aligned16(hg) || !aligned32(dW1) ||
+      !aligned32(dW3) || !aligned32(dW2))
+    return MOE_INVALID_ARG;
+  return from_cuda(launch_expert_ffn_wgrad(xg, dys, dab, hg, offsets, counts, dW1, dW3, dW2, *shape,
+                                           rows_max_of(shape), dev_status,
+                                           static_cast<cudaStream_t>(stream), nullptr));
+}
+
+moe_status_t moe_layer_backward(const uint16_t* dout, const uint16_t* W1, const uint16_t* W3,
+                                const uint16_t* W2, uint16_t* dx, float* dlogits, float* dW1,
+                                float* dW3, float* dW2, void* ws, size_t ws_bytes,
+                                int32_t* dev_status, const moe_shape_t* shape, void* stream,
+                                void* const* stage_events) {
+  moe_status_t st = check_bwd_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!W1 || !W3 || !W2 || !dW1 || !dW3 || !dW2 || !ws || !dev_status ||
+      (shape->N > 0 && (!dout || !dx || !dlogits)))
+    return MOE_INVALID_ARG;
+  if (!aligned16(dout) || !aligned16(W1) || !aligned16(W3) || !aligned16(W2) || !aligned16(dx) ||
+      !aligned32(dW1) || !aligned32(dW3) || !aligned32(dW2) || !aligned32(ws))
+    return MOE_INVALID_ARG;
+  if (ws_bytes < layer_ws(shape).total_train) return MOE_WORKSPACE_TOO_SMALL;
+  return from_cuda(backward_body(dout, W1, W3, W2, dx, dlogits, dW1, dW3, dW2, ws, dev_status,
+                                 shape, static_cast<cudaStream_t>(stream), stage_events));
 }
 
 moe_status_t moe_layer_forward_host(const float* logits_host, const uint16_t* x_host,
@@ -467,7 +687,7 @@ moe_status_t moe_layer_forward_host(const float* logits_host, const uint16_t* x_
   if (!W1 || !W3 || !W2 || !ws || !dev_status ||
       (shape->N > 0 && (!logits_host || !x_host || !out_host)))
     return MOE_INVALID_ARG;
-  if (!aligned16(W1) || !aligned16(W3) || !aligned16(W2) || !aligned16(ws))
+  if (!aligned16(W1) || !aligned16(W3) || !aligned16(W2) || !aligned32(ws))
     return MOE_INVALID_ARG;
   if (minibatch_tokens < 0) return MOE_INVALID_ARG;
   const LayerWs w = layer_ws(shape);

@@ -1,4 +1,8 @@
-// Steps 3a and 4: pull dispatch and fixed-order push combine.
+// Steps 3a and 4: pull dispatch and fixed-order push combine, and their
+// backward twins, which read the same table: pull-reverse-combine and
+// push-reverse-dispatch ("Mixture-of-Kittens: A MoE Megakernel for GB300
+// NVL72", section 2: forward = pull-dispatch / push-combine, backward =
+// pull-reverse-combine / push-reverse-dispatch, one Phi for all four).
 //
 // Dispatch ("Beyond Peak TFLOPs", section 2.A; "Mixture-of-Kittens: A MoE
 // Megakernel for GB300 NVL72", section 2): the destination reads each row's
@@ -6,6 +10,14 @@
 // in a contiguous per-expert buffer. On one GPU this is an HBM-to-HBM row
 // gather: one warp per row, 16-byte vector loads and stores, four in flight
 // per lane; padding rows are written as zeros.
+//
+// Reverse combine: the dispatch gather applied to the upstream gradient,
+// dys[row] = dout[src_rank * N + src_idx], plus the gate of the row's route,
+// gate_row[row] = gates[t, j] for the slot j with route_row[t, j] == row (a
+// warp ballot over the token's k slots); padding rows get zeros.
+//
+// Reverse dispatch: dx[t] = bf16_rne(sum_j dxg[route_row[t, j]]) in ascending
+// slot order from 0, the combine below with unit weights.
 //
 // Combine ("Scan once, scatter once", opening: the floating-point order is
 // fixed so identical inputs give bitwise-identical outputs): out[t] =
@@ -23,12 +35,17 @@ namespace {
 
 constexpr int kMaxK = 16;
 
+// GATE (reverse combine): also gate_row[row] from route_row and gates.
+template <bool GATE>
 __global__ void __launch_bounds__(256) dispatch_kernel(const uint4* __restrict__ x,
                                                        const int2* __restrict__ phi,
                                                        const int32_t* __restrict__ offsets,
                                                        uint4* __restrict__ xg, int P, int N, int E,
                                                        int H, int64_t rows_max,
-                                                       int32_t* dev_status) {
+                                                       int32_t* dev_status,
+                                                       const int32_t* __restrict__ route_row,
+                                                       const float* __restrict__ gates,
+                                                       float* __restrict__ gate_row, int k) {
   const int rows = __ldg(offsets + E);
   if (rows < 0 || rows > rows_max) {
     if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(dev_status, MOE_DEV_BAD_SCHEDULE);
@@ -47,9 +64,17 @@ __global__ void __launch_bounds__(256) dispatch_kernel(const uint4* __restrict__
       if (src.x >= 0 || src.y != -1) bad = 1;  // (-1,-1) is padding; anything else is corrupt
       const uint4 z = make_uint4(0, 0, 0, 0);
       for (int v = lane; v < nv; v += 32) dst[v] = z;
+      if (GATE && lane == 0) gate_row[row] = 0.0f;
       continue;
     }
-    const uint4* s = x + (static_cast<int64_t>(src.x) * N + src.y) * nv;
+    const int64_t tok = static_cast<int64_t>(src.x) * N + src.y;
+    if (GATE) {
+      const int rr = lane < k ? __ldg(route_row + tok * k + lane) : -1;
+      const unsigned hit = __ballot_sync(0xFFFFFFFFu, rr == row);
+      if (hit == 0u) bad = 1;  // Phi and route_row disagree
+      if (lane == 0) gate_row[row] = hit ? __ldg(gates + tok * k + (__ffs(hit) - 1)) : 0.0f;
+    }
+    const uint4* s = x + tok * nv;
     int v = lane;
     for (; v + 96 < nv; v += 128) {
       const uint4 a = __ldg(s + v), b = __ldg(s + v + 32), c = __ldg(s + v + 64),
@@ -71,7 +96,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
          (static_cast<uint32_t>(__bfloat16_as_ushort(b)) << 16);
 }
 
-// K > 0: compile-time k; K == 0: runtime k (<= kMaxK).
+// K > 0: compile-time k; K == 0: runtime k (<= kMaxK). gates == null: unit
+// weights (fmaf(1, v, acc) is the rounded sum acc + v).
 template <int K>
 __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ y,
                                                       const int32_t* __restrict__ route_row,
@@ -94,7 +120,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
     g[j] = 0.0f;
     if (j < kk) {
       const int rr = __ldg(route_row + t * k + j);
-      g[j] = __ldg(gates + t * k + j);
+      g[j] = gates ? __ldg(gates + t * k + j) : 1.0f;
       if (rr >= 0 && rr < rows_max)
         rows[j] = rr;
       else
@@ -130,10 +156,29 @@ cudaError_t launch_dispatch(const uint16_t* x, const int32_t* phi, const int32_t
   const int64_t want = (rows_max + 7) / 8;
   const int64_t cap = static_cast<int64_t>(device_sm_count()) * 8;
   const int blocks = static_cast<int>(want < cap ? want : cap);
-  dispatch_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(x),
-                                         reinterpret_cast<const int2*>(phi), offsets,
-                                         reinterpret_cast<uint4*>(xg), sh.P, sh.N, sh.E, sh.H,
-                                         rows_max, dev_status);
+  dispatch_kernel<false><<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(x),
+                                                reinterpret_cast<const int2*>(phi), offsets,
+                                                reinterpret_cast<uint4*>(xg), sh.P, sh.N, sh.E,
+                                                sh.H, rows_max, dev_status, nullptr, nullptr,
+                                                nullptr, sh.k);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reverse_combine(const uint16_t* dout, const int32_t* phi,
+                                   const int32_t* offsets, const int32_t* route_row,
+                                   const float* gates, uint16_t* dys, float* gate_row,
+                                   const moe_shape_t& sh, int64_t rows_max, int32_t* dev_status,
+                                   cudaStream_t s) {
+  if (rows_max <= 0) return cudaSuccess;
+  const int64_t want = (rows_max + 7) / 8;
+  const int64_t cap = static_cast<int64_t>(device_sm_count()) * 8;
+  const int blocks = static_cast<int>(want < cap ? want : cap);
+  dispatch_kernel<true><<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4*>(dout),
+                                               reinterpret_cast<const int2*>(phi), offsets,
+                                               reinterpret_cast<uint4*>(dys), sh.P, sh.N, sh.E,
+                                               sh.H, rows_max, dev_status, route_row, gates,
+                                               gate_row, sh.k);
   note_launches(1);
   return cudaGetLastError();
 }
@@ -159,6 +204,12 @@ cudaError_t launch_combine(const float* y, const int32_t* route_row, const float
 #undef MOE_COMBINE
   note_launches(1);
   return cudaGetLastError();
+}
+
+cudaError_t launch_reverse_dispatch(const float* dxg, const int32_t* route_row, uint16_t* dx,
+                                    const moe_shape_t& sh, int64_t rows_max, int32_t* dev_status,
+                                    cudaStream_t s) {
+  return launch_combine(dxg, route_row, nullptr, dx, sh, Slice{0, sh.N}, rows_max, dev_status, s);
 }
 
 }  // namespace moe

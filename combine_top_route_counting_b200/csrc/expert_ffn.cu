@@ -108,6 +108,7 @@ struct FfnParams {
   void* out;               // bf16 h [rows_max, I] or fp32 y [rows_max, H]
   int32_t* dev_status;
   int64_t timeout_ns;
+  uint16_t* ab;            // SAVE_AB: bf16 pre-activations [rows_max, 2I], a | b
 };
 
 template <int CG, int MODE>
@@ -127,6 +128,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // MODE 0: GEMM1 + SwiGLU -> bf16 h. MODE 1: GEMM2 -> fp32 y.
+// SAVE_AB (MODE 0, training): the epilogue also keeps the pre-activations
+// a = x.W1 and b = x.W3, rounded to bf16, as ab[row] = [a | b] for the
+// backward pass (which then never recomputes GEMM1).
 // GATHER (MODE 0 only): the A operand is pulled straight from the token
 // activations x by the schedule Phi ("zero-copy, direct landing"): every lane
 // of the producer warp gathers 4 of the CTA's 128 rows per K step with a TMA
@@ -135,7 +139,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // CTA pair) per 256x256 tile; CTA r loads rows [128r, 128r+128) of A and
 // columns [128r, 128r+128) of B, the leader (r = 0) issues the pair MMAs and
 // each CTA drains its own 128 TMEM lanes.
-template <int MODE, int CG, bool GATHER>
+template <int MODE, int CG, bool GATHER, bool SAVE_AB>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmY,
@@ -555,6 +559,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           st_global_v8(hrow + c * 32, *reinterpret_cast<const uint32_t(*)[8]>(&pk[0]));
           st_global_v8(hrow + c * 32 + 16, *reinterpret_cast<const uint32_t(*)[8]>(&pk[8]));
+          if (SAVE_AB) {
+            __nv_bfloat16* arow = reinterpret_cast<__nv_bfloat16*>(p.ab) + row * (2 * p.Nout) +
+                                  n * 128 + half * 64 + c * 32;
+            __nv_bfloat16* brow = arow + p.Nout;
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+              uint32_t qa[8], qb[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                qa[i] = pack_bf16x2(__uint_as_float(ra[c & 1][16 * v + 2 * i]),
+                                    __uint_as_float(ra[c & 1][16 * v + 2 * i + 1]));
+                qb[i] = pack_bf16x2(__uint_as_float(rb[c & 1][16 * v + 2 * i]),
+                                    __uint_as_float(rb[c & 1][16 * v + 2 * i + 1]));
+              }
+              st_global_v8(arow + 16 * v, qa);
+              st_global_v8(brow + 16 * v, qb);
+            }
+          }
           if (c + 1 < 2) tmem_ld_wait();
         }
       } else if (C::TMA_STORE) {
@@ -625,11 +647,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-// Per-device counter the scheduler threads take tile ids from; zeroed on the
-// stream before every launch.
+}  // namespace
+
+// Per-device counter the scheduler threads of the persistent GEMMs take tile
+// ids from; zeroed on the stream before every launch.
 __device__ int g_tile_counter[1];
 
 // ---------------------------------------------------------------- host side
+namespace {
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -644,10 +669,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2D tensor [outer, inner] (inner contiguous) of bf16 (or fp32), box
-// [box_outer, box_inner], 128-byte swizzle.
+}  // namespace
+
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-              uint32_t box_outer, bool fp32 = false) {
+              uint32_t box_outer, bool fp32) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {inner, outer};
@@ -660,7 +685,6 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Device address of g_tile_counter on the current device (looked up once per device).
 cudaError_t tile_counter_for_current_device(int** out) {
   static std::mutex mu;
   static int* ptrs[64] = {nullptr};
@@ -678,14 +702,16 @@ cudaError_t tile_counter_for_current_device(int** out) {
   return cudaSuccess;
 }
 
-template <int MODE, int CG, bool GATHER = false>
+namespace {
+
+template <int MODE, int CG, bool GATHER = false, bool SAVE_AB = false>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const CUtensorMap& yo, FfnParams p, cudaStream_t s) {
   const size_t smem = smem_bytes_for<CG, MODE>(p.E);
   cudaError_t ce = tile_counter_for_current_device(&p.tile_counter);
   if (ce != cudaSuccess) return ce;
   if ((ce = cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s)) != cudaSuccess) return ce;
-  cudaError_t e = cudaFuncSetAttribute(ffn_gemm_kernel<MODE, CG, GATHER>,
+  cudaError_t e = cudaFuncSetAttribute(ffn_gemm_kernel<MODE, CG, GATHER, SAVE_AB>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -704,7 +730,7 @@ cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUten
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  e = cudaLaunchKernelEx(&cfg, ffn_gemm_kernel<MODE, CG, GATHER>, a, b0, b1, yo, p);
+  e = cudaLaunchKernelEx(&cfg, ffn_gemm_kernel<MODE, CG, GATHER, SAVE_AB>, a, b0, b1, yo, p);
   note_launches(1);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -715,7 +741,8 @@ cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUten
 cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint16_t* W3,
                               const uint16_t* W2, const int32_t* offsets, const int32_t* counts,
                               uint16_t* h, float* y, const moe_shape_t& sh, int64_t rows_max,
-                              int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_mid) {
+                              int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_mid,
+                              uint16_t* ab) {
   const int E = sh.E, H = sh.H, I = sh.I;
   CUtensorMap mA1, mW1, mW3, mA2, mW2, mY;
   const uint64_t EH = static_cast<uint64_t>(E) * H, EI = static_cast<uint64_t>(E) * I;
@@ -726,15 +753,20 @@ cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint
   // Segments that are multiples of 256 rows run on CTA pairs (256x256 tiles);
   // otherwise (pad a multiple of 128 only) on single CTAs (128x256 tiles).
   const bool pair = (sh.pad % 256) == 0;
-  FfnParams p1{nullptr, nullptr, 0, 0, offsets, counts, E, sh.P, H, I, rows_max, h, dev_status, kWaitTimeoutNs};
-  cudaError_t e = pair ? launch_mode<0, 2>(mA1, mW1, mW3, mA1, p1, s)
-                       : launch_mode<0, 1>(mA1, mW1, mW3, mA1, p1, s);
+  FfnParams p1{nullptr, nullptr, 0, 0, offsets, counts, E, sh.P, H, I, rows_max, h, dev_status,
+               kWaitTimeoutNs, ab};
+  cudaError_t e;
+  if (ab)  // training: keep the pre-activations (pair tiles only)
+    e = pair ? launch_mode<0, 2, false, true>(mA1, mW1, mW3, mA1, p1, s) : cudaErrorInvalidValue;
+  else
+    e = pair ? launch_mode<0, 2>(mA1, mW1, mW3, mA1, p1, s) : launch_mode<0, 1>(mA1, mW1, mW3, mA1, p1, s);
   if (e != cudaSuccess) return e;
   if (ev_mid) {
     e = cudaEventRecord(ev_mid, s);
     if (e != cudaSuccess) return e;
   }
-  FfnParams p2{nullptr, nullptr, 0, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status, kWaitTimeoutNs};
+  FfnParams p2{nullptr, nullptr, 0, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status,
+               kWaitTimeoutNs, nullptr};
   return pair ? launch_mode<1, 2>(mA2, mW2, mW2, mY, p2, s)
               : launch_mode<1, 1>(mA2, mW2, mW2, mY, p2, s);
 }
@@ -756,7 +788,7 @@ cudaError_t launch_expert_ffn_gather(const uint16_t* x, const int32_t* phi, cons
     return cudaErrorInvalidValue;
   const bool pair = (sh.pad % 256) == 0;
   FfnParams p1{nullptr, reinterpret_cast<const int2*>(phi), sh.N, static_cast<int32_t>(tokens), offsets,
-               counts, E, sh.P, H, I, rows_max, h, dev_status, kWaitTimeoutNs};
+               counts, E, sh.P, H, I, rows_max, h, dev_status, kWaitTimeoutNs, nullptr};
   cudaError_t e = pair ? launch_mode<0, 2, true>(mX, mW1, mW3, mX, p1, s)
                        : launch_mode<0, 1, true>(mX, mW1, mW3, mX, p1, s);
   if (e != cudaSuccess) return e;
@@ -764,7 +796,8 @@ cudaError_t launch_expert_ffn_gather(const uint16_t* x, const int32_t* phi, cons
     e = cudaEventRecord(ev_mid, s);
     if (e != cudaSuccess) return e;
   }
-  FfnParams p2{nullptr, nullptr, 0, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status, kWaitTimeoutNs};
+  FfnParams p2{nullptr, nullptr, 0, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status,
+               kWaitTimeoutNs, nullptr};
   return pair ? launch_mode<1, 2>(mA2, mW2, mW2, mY, p2, s)
               : launch_mode<1, 1>(mA2, mW2, mW2, mY, p2, s);
 }

@@ -1,6 +1,7 @@
 // Internal launchers shared by the C-ABI layer (api.cu) and the kernel files.
 #pragma once
 
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -37,11 +38,13 @@ cudaError_t launch_dispatch(const uint16_t* x, const int32_t* phi, const int32_t
                             uint16_t* xg, const moe_shape_t& sh, int64_t rows_max,
                             int32_t* dev_status, cudaStream_t s);
 
-// Step 3b (two kernels; ev_mid, if not null, is recorded between them)
+// Step 3b (two kernels; ev_mid, if not null, is recorded between them).
+// ab (training, pair tiles only): also keep the bf16 pre-activations [a | b].
 cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint16_t* W3,
                               const uint16_t* W2, const int32_t* offsets, const int32_t* counts,
                               uint16_t* h, float* y, const moe_shape_t& sh, int64_t rows_max,
-                              int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_mid);
+                              int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_mid,
+                              uint16_t* ab = nullptr);
 
 // Steps 3a+3b fused: GEMM1 pulls its A rows from x by Phi (no xg buffer)
 cudaError_t launch_expert_ffn_gather(const uint16_t* x, const int32_t* phi, const uint16_t* W1,
@@ -54,6 +57,53 @@ cudaError_t launch_expert_ffn_gather(const uint16_t* x, const int32_t* phi, cons
 cudaError_t launch_combine(const float* y, const int32_t* route_row, const float* gates,
                            uint16_t* out, const moe_shape_t& sh, Slice sl, int64_t rows_max,
                            int32_t* dev_status, cudaStream_t s);
+
+// 2D tensor map over [outer, inner] (inner contiguous) bf16 (or fp32)
+// elements with box [box_outer, box_inner] and 128-byte swizzle; false if the
+// driver entry point is missing or rejects the arguments.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+              uint32_t box_outer, bool fp32 = false);
+
+// Device address of the tile counter of the persistent GEMMs on the current
+// device (looked up once per device). One counter per device: the FFN
+// launches of one device must not run concurrently.
+cudaError_t tile_counter_for_current_device(int** out);
+
+// ---------------------------------------------------------------- backward
+// Pull-reverse-combine: dys[row] = dout[Phi[row]], gate_row[row] = the gate of
+// the row's route (padding rows: zeros).
+cudaError_t launch_reverse_combine(const uint16_t* dout, const int32_t* phi,
+                                   const int32_t* offsets, const int32_t* route_row,
+                                   const float* gates, uint16_t* dys, float* gate_row,
+                                   const moe_shape_t& sh, int64_t rows_max, int32_t* dev_status,
+                                   cudaStream_t s);
+
+// Expert FFN activation gradients (two kernels; ev_mid recorded between them).
+cudaError_t launch_expert_ffn_dgrad(const uint16_t* dys, const float* gate_row, const uint16_t* ab,
+                                    const uint16_t* h, const uint16_t* W1, const uint16_t* W3,
+                                    const uint16_t* W2, const int32_t* offsets,
+                                    const int32_t* counts, uint16_t* dab, uint16_t* hg,
+                                    float* part, float* dxg, const moe_shape_t& sh,
+                                    int64_t rows_max, int32_t* dev_status, cudaStream_t s,
+                                    cudaEvent_t ev_mid);
+
+// Push-reverse-dispatch: dx[t] = bf16(sum_j dxg[route_row[t, j]]), ascending j.
+cudaError_t launch_reverse_dispatch(const float* dxg, const int32_t* route_row, uint16_t* dx,
+                                    const moe_shape_t& sh, int64_t rows_max, int32_t* dev_status,
+                                    cudaStream_t s);
+
+// Router gradient from the gate-gradient partial sums [rows, npart].
+cudaError_t launch_router_backward(const float* part, int32_t npart, const int32_t* route_row,
+                                   const int32_t* ids, const float* gates, float* dlogits,
+                                   int64_t n_tokens, int32_t E, int32_t k, int64_t rows_max,
+                                   int32_t* dev_status, cudaStream_t s);
+
+// Expert weight gradients (two kernels: dW2, then dW1 | dW3).
+cudaError_t launch_expert_ffn_wgrad(const uint16_t* xg, const uint16_t* dys, const uint16_t* dab,
+                                    const uint16_t* hg, const int32_t* offsets,
+                                    const int32_t* counts, float* dW1, float* dW3, float* dW2,
+                                    const moe_shape_t& sh, int64_t rows_max, int32_t* dev_status,
+                                    cudaStream_t s, cudaEvent_t ev_mid);
 
 // Failure-detection self test (bounded wait on an mbarrier nothing completes).
 cudaError_t launch_selftest_wait(int32_t* dev_status, int64_t timeout_ns, cudaStream_t s);

@@ -174,4 +174,61 @@ cudaError_t launch_route_topk(const float* logits, int32_t* ids, float* gates, i
   return launch_vpl<32>(logits, ids, gates, n_tokens, E, k, s);
 }
 
+// ---------------------------------------------------------------- backward
+// Router gradient ("Mixture-of-Kittens", section 5, SonicMoE gradients: from
+// the inner product of the SwiGLU activations and the down-projection
+// dgrads). dgate[t, j] = sum over the npart partial sums of the route's row,
+// in ascending order; with the gates g = softmax of the chosen logits,
+// dlogits[t, ids[t, j]] = g_j (dgate_j - S), S = sum_j g_j dgate_j (fmaf in
+// ascending slot order); every other logit's gradient is 0. One warp per
+// token, lane j holding slot j.
+namespace {
+__global__ void __launch_bounds__(256) router_bwd_kernel(const float* __restrict__ part, int npart,
+                                                         const int32_t* __restrict__ route_row,
+                                                         const int32_t* __restrict__ ids,
+                                                         const float* __restrict__ gates,
+                                                         float* __restrict__ dlogits,
+                                                         int64_t n_tokens, int E, int k,
+                                                         int64_t rows_max, int32_t* dev_status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (t >= n_tokens) return;
+  float dg = 0.0f, g = 0.0f;
+  int id = -1, bad = 0;
+  if (lane < k) {
+    const int64_t rr = __ldg(route_row + t * k + lane);
+    g = __ldg(gates + t * k + lane);
+    id = __ldg(ids + t * k + lane);
+    if (rr < 0 || rr >= rows_max || id < 0 || id >= E) {
+      bad = 1;
+    } else {
+      const float* pr = part + rr * npart;
+      for (int c = 0; c < npart; ++c) dg += __ldg(pr + c);
+    }
+  }
+  float S = 0.0f;
+  for (int j = 0; j < k; ++j)
+    S = __fmaf_rn(__shfl_sync(0xFFFFFFFFu, g, j), __shfl_sync(0xFFFFFFFFu, dg, j), S);
+  const float dl = g * (dg - S);
+  float* out = dlogits + t * E;
+  for (int e = lane; e < E; e += 32) out[e] = 0.0f;
+  __syncwarp();  // orders the zeros before the k values written below
+  if (lane < k && !bad) out[id] = dl;
+  if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(dev_status, MOE_DEV_BAD_SCHEDULE);
+}
+}  // namespace
+
+cudaError_t launch_router_backward(const float* part, int32_t npart, const int32_t* route_row,
+                                   const int32_t* ids, const float* gates, float* dlogits,
+                                   int64_t n_tokens, int32_t E, int32_t k, int64_t rows_max,
+                                   int32_t* dev_status, cudaStream_t s) {
+  if (n_tokens == 0) return cudaSuccess;
+  const int64_t blocks = (n_tokens + 7) / 8;
+  router_bwd_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(part, npart, route_row, ids, gates,
+                                                                 dlogits, n_tokens, E, k, rows_max,
+                                                                 dev_status);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
 }  // namespace moe

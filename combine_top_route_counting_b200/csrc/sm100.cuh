@@ -340,13 +340,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
          (2ull << 61);                                                           // 128B swizzle
 }
 
-// Instruction descriptor, kind::f16: D fp32, A and B bf16, A K-major,
-// B K-major (b_mn_major = 0) or MN-major (1), shape M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, uint32_t b_mn_major) {
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, each operand
+// K-major (0) or MN-major (1), shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, uint32_t b_mn_major,
+                                                      uint32_t a_mn_major = 0) {
   return (1u << 4)            // D format: f32
          | (1u << 7)          // A format: bf16
          | (1u << 10)         // B format: bf16
-         | (0u << 15)         // A K-major
+         | (a_mn_major << 15) // A major
          | (b_mn_major << 16) // B major
          | ((N >> 3) << 17)   // N / 8
          | ((M >> 4) << 24);  // M / 16

@@ -16,6 +16,7 @@ including where it loses"):
   kimi   P=8 x 7168 tokens, H=7168, I=2048, E=384, top-8 (transfer slice 2368)
   zipf   kimi shapes, expert choice ~ Zipf(1.2) over a seeded expert
          permutation, plus 8 experts that are never chosen
+  tiny_bwd  P=2 x 256 tokens, H=256, I=256, E=8, top-2 (small backward case)
 
 Distributions: router logits fp32 N(0,1); activations bf16 N(0,1); SwiGLU
 weights W1, W3 [E,H,I] and W2 [E,I,H] bf16 N(0, 0.02). Seeds are
@@ -65,6 +66,8 @@ WORKLOADS = {
     # Kimi expert shapes with 16 experts and ~1,200 routes each (as at full size):
     # a few GB on the device, for profiler captures of the FFN kernels
     "kimi_e16": Workload("kimi_e16", 5, P=1, N=2400, E=16, k=8, H=7168, I=2048),
+    # smallest backward case: the backward's GEMMs need I % 256 == 0
+    "tiny_bwd": Workload("tiny_bwd", 6, P=2, N=256, E=8, k=2, H=256, I=256),
 }
 
 

@@ -27,6 +27,9 @@ DEV_TIMEOUT = 0x2
 DEV_BAD_SCHEDULE = 0x4
 N_STAGE_EVENTS = 7
 STAGES = ("route", "schedule", "dispatch", "ffn_gemm1", "ffn_gemm2", "combine")
+N_BWD_EVENTS = 8
+BWD_STAGES = ("reverse_combine", "dgrad_h", "dgrad_x", "reverse_dispatch", "router_bwd",
+              "wgrad_w2", "wgrad_w13")
 
 
 class MoeError(RuntimeError):
@@ -70,6 +73,17 @@ _SIGS = {
                                 ctypes.c_size_t, _vp, ctypes.POINTER(Shape), _vp], ctypes.c_int),
     "moe_schedule_static_ws": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Shape), _vp],
                                ctypes.c_int),
+    "moe_train_workspace_bytes": ([ctypes.POINTER(Shape)], ctypes.c_size_t),
+    "moe_expert_ffn_train": ([_vp] * 10 + [ctypes.POINTER(Shape), _vp], ctypes.c_int),
+    "moe_layer_forward_train": ([_vp] * 7 + [ctypes.c_size_t, _vp, ctypes.POINTER(Shape), _vp,
+                                              ctypes.POINTER(_vp)], ctypes.c_int),
+    "moe_reverse_combine": ([_vp] * 8 + [ctypes.POINTER(Shape), _vp], ctypes.c_int),
+    "moe_expert_ffn_dgrad": ([_vp] * 14 + [ctypes.POINTER(Shape), _vp], ctypes.c_int),
+    "moe_reverse_dispatch": ([_vp] * 4 + [ctypes.POINTER(Shape), _vp], ctypes.c_int),
+    "moe_router_backward": ([_vp] * 6 + [ctypes.POINTER(Shape), _vp], ctypes.c_int),
+    "moe_expert_ffn_wgrad": ([_vp] * 10 + [ctypes.POINTER(Shape), _vp], ctypes.c_int),
+    "moe_layer_backward": ([_vp] * 10 + [ctypes.c_size_t, _vp, ctypes.POINTER(Shape), _vp,
+                                         ctypes.POINTER(_vp)], ctypes.c_int),
     "moe_launch_count": ([], ctypes.c_int64),
     "moe_selftest_bounded_wait": ([_vp, ctypes.c_int64, _vp], ctypes.c_int),
 }
@@ -143,6 +157,10 @@ def layer_workspace_bytes(sh: Shape) -> int:
 
 def layer_host_workspace_bytes(sh: Shape) -> int:
     return int(load().moe_layer_host_workspace_bytes(ctypes.byref(sh)))
+
+
+def train_workspace_bytes(sh: Shape) -> int:
+    return int(load().moe_train_workspace_bytes(ctypes.byref(sh)))
 
 
 def launch_count() -> int:
@@ -219,12 +237,12 @@ def moe_combine(y, route_row, gates, out, dev_status, sh: Shape, stream=None):
                               _stream(stream)), "moe_combine")
 
 
-def _events(events):
+def _events(events, n=N_STAGE_EVENTS):
     if events is None:
         return None
-    if len(events) != N_STAGE_EVENTS:
-        raise ValueError(f"need {N_STAGE_EVENTS} events")
-    arr = (ctypes.c_void_p * N_STAGE_EVENTS)()
+    if len(events) != n:
+        raise ValueError(f"need {n} events")
+    arr = (ctypes.c_void_p * n)()
     for i, e in enumerate(events):
         arr[i] = e.cuda_event if hasattr(e, "cuda_event") else int(e)
     return ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
@@ -251,6 +269,112 @@ def moe_layer_forward_host(logits_host, x_host, W1, W3, W2, out_host, ws, dev_st
         _ptr(out_host, torch.bfloat16, "out_host", device=False), int(minibatch_tokens),
         _ptr(ws, torch.uint8, "ws"), ws.numel(), _ptr(dev_status, torch.int32, "dev_status"),
         ctypes.byref(sh), _stream(stream)), "moe_layer_forward_host")
+
+
+# ---------------------------------------------------------------- backward
+def moe_expert_ffn_train(xg, W1, W3, W2, offsets, counts, h, ab, y, dev_status, sh: Shape,
+                         stream=None):
+    _check(load().moe_expert_ffn_train(_ptr(xg, torch.bfloat16, "xg"), _ptr(W1, torch.bfloat16, "W1"),
+                                       _ptr(W3, torch.bfloat16, "W3"), _ptr(W2, torch.bfloat16, "W2"),
+                                       _ptr(offsets, torch.int32, "offsets"),
+                                       _ptr(counts, torch.int32, "counts"),
+                                       _ptr(h, torch.bfloat16, "h"), _ptr(ab, torch.bfloat16, "ab"),
+                                       _ptr(y, torch.float32, "y"),
+                                       _ptr(dev_status, torch.int32, "dev_status"),
+                                       ctypes.byref(sh), _stream(stream)), "moe_expert_ffn_train")
+
+
+def moe_layer_forward_train(logits, x, W1, W3, W2, out, ws, dev_status, sh: Shape, stream=None,
+                            stage_events=None):
+    _check(load().moe_layer_forward_train(_ptr(logits, torch.float32, "logits"),
+                                          _ptr(x, torch.bfloat16, "x"),
+                                          _ptr(W1, torch.bfloat16, "W1"),
+                                          _ptr(W3, torch.bfloat16, "W3"),
+                                          _ptr(W2, torch.bfloat16, "W2"),
+                                          _ptr(out, torch.bfloat16, "out"),
+                                          _ptr(ws, torch.uint8, "ws"), ws.numel(),
+                                          _ptr(dev_status, torch.int32, "dev_status"),
+                                          ctypes.byref(sh), _stream(stream),
+                                          _events(stage_events)), "moe_layer_forward_train")
+
+
+def moe_reverse_combine(dout, phi, offsets, route_row, gates, dys, gate_row, dev_status, sh: Shape,
+                        stream=None):
+    _check(load().moe_reverse_combine(_ptr(dout, torch.bfloat16, "dout"),
+                                      _ptr(phi, torch.int32, "phi"),
+                                      _ptr(offsets, torch.int32, "offsets"),
+                                      _ptr(route_row, torch.int32, "route_row"),
+                                      _ptr(gates, torch.float32, "gates"),
+                                      _ptr(dys, torch.bfloat16, "dys"),
+                                      _ptr(gate_row, torch.float32, "gate_row"),
+                                      _ptr(dev_status, torch.int32, "dev_status"),
+                                      ctypes.byref(sh), _stream(stream)), "moe_reverse_combine")
+
+
+def moe_expert_ffn_dgrad(dys, gate_row, ab, h, W1, W3, W2, offsets, counts, dab, hg, dgate_part,
+                         dxg, dev_status, sh: Shape, stream=None):
+    _check(load().moe_expert_ffn_dgrad(_ptr(dys, torch.bfloat16, "dys"),
+                                       _ptr(gate_row, torch.float32, "gate_row"),
+                                       _ptr(ab, torch.bfloat16, "ab"), _ptr(h, torch.bfloat16, "h"),
+                                       _ptr(W1, torch.bfloat16, "W1"), _ptr(W3, torch.bfloat16, "W3"),
+                                       _ptr(W2, torch.bfloat16, "W2"),
+                                       _ptr(offsets, torch.int32, "offsets"),
+                                       _ptr(counts, torch.int32, "counts"),
+                                       _ptr(dab, torch.bfloat16, "dab"),
+                                       _ptr(hg, torch.bfloat16, "hg"),
+                                       _ptr(dgate_part, torch.float32, "dgate_part"),
+                                       _ptr(dxg, torch.float32, "dxg"),
+                                       _ptr(dev_status, torch.int32, "dev_status"),
+                                       ctypes.byref(sh), _stream(stream)), "moe_expert_ffn_dgrad")
+
+
+def moe_reverse_dispatch(dxg, route_row, dx, dev_status, sh: Shape, stream=None):
+    _check(load().moe_reverse_dispatch(_ptr(dxg, torch.float32, "dxg"),
+                                       _ptr(route_row, torch.int32, "route_row"),
+                                       _ptr(dx, torch.bfloat16, "dx"),
+                                       _ptr(dev_status, torch.int32, "dev_status"),
+                                       ctypes.byref(sh), _stream(stream)), "moe_reverse_dispatch")
+
+
+def moe_router_backward(dgate_part, route_row, ids, gates, dlogits, dev_status, sh: Shape,
+                        stream=None):
+    _check(load().moe_router_backward(_ptr(dgate_part, torch.float32, "dgate_part"),
+                                      _ptr(route_row, torch.int32, "route_row"),
+                                      _ptr(ids, torch.int32, "ids"),
+                                      _ptr(gates, torch.float32, "gates"),
+                                      _ptr(dlogits, torch.float32, "dlogits"),
+                                      _ptr(dev_status, torch.int32, "dev_status"),
+                                      ctypes.byref(sh), _stream(stream)), "moe_router_backward")
+
+
+def moe_expert_ffn_wgrad(xg, dys, dab, hg, offsets, counts, dW1, dW3, dW2, dev_status, sh: Shape,
+                         stream=None):
+    _check(load().moe_expert_ffn_wgrad(_ptr(xg, torch.bfloat16, "xg"),
+                                       _ptr(dys, torch.bfloat16, "dys"),
+                                       _ptr(dab, torch.bfloat16, "dab"),
+                                       _ptr(hg, torch.bfloat16, "hg"),
+                                       _ptr(offsets, torch.int32, "offsets"),
+                                       _ptr(counts, torch.int32, "counts"),
+                                       _ptr(dW1, torch.float32, "dW1"),
+                                       _ptr(dW3, torch.float32, "dW3"),
+                                       _ptr(dW2, torch.float32, "dW2"),
+                                       _ptr(dev_status, torch.int32, "dev_status"),
+                                       ctypes.byref(sh), _stream(stream)), "moe_expert_ffn_wgrad")
+
+
+def moe_layer_backward(dout, W1, W3, W2, dx, dlogits, dW1, dW3, dW2, ws, dev_status, sh: Shape,
+                       stream=None, stage_events=None):
+    _check(load().moe_layer_backward(_ptr(dout, torch.bfloat16, "dout"),
+                                     _ptr(W1, torch.bfloat16, "W1"), _ptr(W3, torch.bfloat16, "W3"),
+                                     _ptr(W2, torch.bfloat16, "W2"), _ptr(dx, torch.bfloat16, "dx"),
+                                     _ptr(dlogits, torch.float32, "dlogits"),
+                                     _ptr(dW1, torch.float32, "dW1"),
+                                     _ptr(dW3, torch.float32, "dW3"),
+                                     _ptr(dW2, torch.float32, "dW2"),
+                                     _ptr(ws, torch.uint8, "ws"), ws.numel(),
+                                     _ptr(dev_status, torch.int32, "dev_status"),
+                                     ctypes.byref(sh), _stream(stream),
+                                     _events(stage_events, N_BWD_EVENTS)), "moe_layer_backward")
 
 
 def moe_selftest_bounded_wait(dev_status, timeout_ns: int, stream=None):

@@ -1,6 +1,6 @@
 /*
- * moe.h -- C ABI of libmoe_b200.so: the forward pass of one deterministic
- * Mixture-of-Experts layer on one B200 (sm_100a).
+ * moe.h -- C ABI of libmoe_b200.so: the forward and backward passes of one
+ * deterministic Mixture-of-Experts layer on one B200 (sm_100a).
  *
  * The layer has four steps:
  *   1. top-k routing from router logits;
@@ -10,6 +10,8 @@
  *      grouped SwiGLU expert FFN (bf16 operands, fp32 accumulation);
  *   4. a gate-weighted combine back to token order in a fixed floating-point
  *      order, so identical inputs give bitwise-identical outputs.
+ * The backward pass (training) reuses the forward's Phi for both of its
+ * exchanges (see the "Backward" section at the end of this header).
  *
  * Sources (page title, section):
  *   "Mixture-of-Kittens: A MoE Megakernel for GB300 NVL72" (MoK notes),
@@ -29,7 +31,9 @@
  * Conventions for every entry point:
  *   - All pointers are DEVICE pointers unless the name ends in _host.
  *     bf16 tensors are passed as uint16_t bit patterns. All arrays are dense,
- *     row-major, and must be 16-byte aligned (256-byte alignment recommended).
+ *     row-major, and must be 16-byte aligned (256-byte alignment recommended);
+ *     the FFN outputs h, ab and y, the weight gradients and every workspace
+ *     must be 32-byte aligned.
  *   - The caller owns and allocates every buffer; the library never allocates
  *     device memory and never synchronises with the host. Work is enqueued on
  *     `stream` (a cudaStream_t; NULL = the legacy default stream) and runs
@@ -250,6 +254,124 @@ moe_status_t moe_layer_forward_host(const float* logits_host, const uint16_t* x_
                                     uint16_t* out_host, int32_t minibatch_tokens, void* ws,
                                     size_t ws_bytes, int32_t* dev_status,
                                     const moe_shape_t* shape, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Backward (training).
+ *
+ * "Mixture-of-Kittens: A MoE Megakernel for GB300 NVL72": one schedule table
+ * serves all four forward and backward phases (overview), the backward being
+ * pull-reverse-combine and push-reverse-dispatch (section 2); weight
+ * gradients are deferred until every activation gradient is done and
+ * accumulated over the token dimension in one pass for bitwise
+ * reproducibility (overview, backward execution step); the router gradient
+ * is the inner product of the SwiGLU activations and the down-projection
+ * dgrads, so the down projection's output is never kept (section 5,
+ * SonicMoE gradients); forward activations are kept, not recomputed.
+ *
+ * For route (t, j) with expert e, gate g = gates[t,j] and row = route_row[t,j]
+ * (the forward saved a = xg.W1[e], b = xg.W3[e] as bf16 and h as bf16):
+ *   dhu   = dout[t] . W2[e]^T                             (fp32)
+ *   dgate = sum_i h[i] * dhu[i]
+ *   dh    = g * dhu;  s = 1 / (1 + exp(-a))
+ *   da    = bf16(dh * b * s * (1 + a (1 - s))),  db = bf16(dh * a * s),
+ *   hg    = bf16(g * h)
+ *   dxg   = da . W1[e]^T + db . W3[e]^T                   (fp32)
+ *   dx[t] = bf16(sum_j dxg[route_row[t,j]])               (ascending j, from 0)
+ *   dlogits[t, ids[t,j]] = g_j (dgate_j - sum_j' g_j' dgate_j'), 0 elsewhere
+ *   dW1[e] = sum over e's rows of xg^T da, dW3[e] = xg^T db, dW2[e] = hg^T dout
+ *                                                         (fp32, one pass)
+ * Every output element is produced by one thread or one CTA pair in a fixed
+ * order (no atomics, no split-K): the gradients are bitwise reproducible.
+ * Shape limits in addition to the FFN's: I % 256 == 0 and pad % 256 == 0
+ * (every GEMM runs 256 x 256 tiles on CTA pairs). Weight gradients are
+ * written whole: an expert that received no route gets zeros.
+ * ------------------------------------------------------------------------ */
+
+/* Bytes of the workspace of moe_layer_forward_train / moe_layer_backward
+ * (0 if the shape is unsupported): the forward's buffers plus the saved
+ * pre-activations and the backward's buffers (about rows * (9H + 12I) bytes). */
+size_t moe_train_workspace_bytes(const moe_shape_t* shape);
+
+/* moe_expert_ffn that also keeps the pre-activations for the backward:
+ * ab: bf16 [moe_rows_max, 2I], ab[row] = [bf16(a) | bf16(b)] with a, b the
+ * fp32 accumulators of GEMM1 (written for the rows moe_expert_ffn writes h). */
+moe_status_t moe_expert_ffn_train(const uint16_t* xg, const uint16_t* W1, const uint16_t* W3,
+                                  const uint16_t* W2, const int32_t* offsets,
+                                  const int32_t* counts, uint16_t* h, uint16_t* ab, float* y,
+                                  int32_t* dev_status, const moe_shape_t* shape, void* stream);
+
+/* moe_layer_forward over the whole batch (one slice) that leaves in ws (of
+ * moe_train_workspace_bytes) everything moe_layer_backward reads: ids, gates,
+ * Phi, offsets, counts, route_row, the gathered tokens, h and the
+ * pre-activations. out as moe_layer_forward (bitwise the same values).
+ * stage_events: NULL or 7 events as in moe_layer_forward. */
+moe_status_t moe_layer_forward_train(const float* logits, const uint16_t* x, const uint16_t* W1,
+                                     const uint16_t* W3, const uint16_t* W2, uint16_t* out,
+                                     void* ws, size_t ws_bytes, int32_t* dev_status,
+                                     const moe_shape_t* shape, void* stream,
+                                     void* const* stage_events);
+
+/* Pull-reverse-combine: the expert rows pull their upstream gradient through
+ * the forward's Phi. dys[row] = dout[src_rank*N + src_idx] (bf16 [moe_rows_max, H],
+ * padding rows 0) and gate_row[row] = gates[t, j] for the slot with
+ * route_row[t, j] == row (fp32 [moe_rows_max], padding rows 0). A Phi entry
+ * that route_row does not point back to raises MOE_DEV_BAD_SCHEDULE. */
+moe_status_t moe_reverse_combine(const uint16_t* dout, const int32_t* phi, const int32_t* offsets,
+                                 const int32_t* route_row, const float* gates, uint16_t* dys,
+                                 float* gate_row, int32_t* dev_status, const moe_shape_t* shape,
+                                 void* stream);
+
+/* Activation gradients of the expert FFN (two grouped GEMMs):
+ *   dhu = dys . W2[e]^T with the SwiGLU backward fused in its epilogue:
+ *     dab: bf16 [moe_rows_max, 2I] = [da | db], hg: bf16 [moe_rows_max, I],
+ *     dgate_part: fp32 [moe_rows_max, I/128], the gate gradient of each row
+ *     as I/128 partial sums over consecutive 128-column blocks (summed in
+ *     order by moe_router_backward);
+ *   dxg = [da | db] . [W1[e] | W3[e]]^T: fp32 [moe_rows_max, H].
+ * ab and h as left by moe_expert_ffn_train; offsets/counts as for the FFN. */
+moe_status_t moe_expert_ffn_dgrad(const uint16_t* dys, const float* gate_row, const uint16_t* ab,
+                                  const uint16_t* h, const uint16_t* W1, const uint16_t* W3,
+                                  const uint16_t* W2, const int32_t* offsets,
+                                  const int32_t* counts, uint16_t* dab, uint16_t* hg,
+                                  float* dgate_part, float* dxg, int32_t* dev_status,
+                                  const moe_shape_t* shape, void* stream);
+
+/* Push-reverse-dispatch: dx[t] = bf16_rne(acc), acc = 0.0f, acc += dxg[route_row[t,j]]
+ * for j = 0..k-1 in ascending order. dx: bf16 [P*N, H]. */
+moe_status_t moe_reverse_dispatch(const float* dxg, const int32_t* route_row, uint16_t* dx,
+                                  int32_t* dev_status, const moe_shape_t* shape, void* stream);
+
+/* Router gradient: dgate[t,j] = sum of dgate_part[route_row[t,j], 0..I/128-1] in
+ * ascending order; S = sum_j gates[t,j] dgate[t,j] (fmaf, ascending j);
+ * dlogits[t, ids[t,j]] = gates[t,j] * (dgate[t,j] - S); all other entries 0.
+ * dlogits: fp32 [P*N, E]. */
+moe_status_t moe_router_backward(const float* dgate_part, const int32_t* route_row,
+                                 const int32_t* ids, const float* gates, float* dlogits,
+                                 int32_t* dev_status, const moe_shape_t* shape, void* stream);
+
+/* Weight gradients, accumulated per expert over the rows it received in one
+ * pass (K = the expert's real rows, rounded up to 64 with zero padding rows):
+ *   dW2[e] = hg^T . dys  (fp32 [E, I, H]),
+ *   dW1[e] = xg^T . da, dW3[e] = xg^T . db  (fp32 [E, H, I]).
+ * Every entry of the three arrays is written. */
+moe_status_t moe_expert_ffn_wgrad(const uint16_t* xg, const uint16_t* dys, const uint16_t* dab,
+                                  const uint16_t* hg, const int32_t* offsets,
+                                  const int32_t* counts, float* dW1, float* dW3, float* dW2,
+                                  int32_t* dev_status, const moe_shape_t* shape, void* stream);
+
+/* The whole backward on the state moe_layer_forward_train left in ws (same
+ * shape, nothing else written to ws in between): reverse combine, the two
+ * activation-gradient GEMMs, reverse dispatch, router gradient, then the
+ * weight-gradient GEMMs, all on `stream`. dout: bf16 [P*N, H] upstream
+ * gradient; outputs dx bf16 [P*N, H], dlogits fp32 [P*N, E], dW1/dW3 fp32
+ * [E, H, I], dW2 fp32 [E, I, H]. stage_events: NULL or 8 events recorded at
+ * the start and after each of: reverse combine, dh GEMM, dx GEMM, reverse
+ * dispatch, router gradient, dW2 GEMM, dW1|dW3 GEMM. */
+moe_status_t moe_layer_backward(const uint16_t* dout, const uint16_t* W1, const uint16_t* W3,
+                                const uint16_t* W2, uint16_t* dx, float* dlogits, float* dW1,
+                                float* dW3, float* dW2, void* ws, size_t ws_bytes,
+                                int32_t* dev_status, const moe_shape_t* shape, void* stream,
+                                void* const* stage_events);
 
 /* Number of kernels this library has launched in the calling process. */
 int64_t moe_launch_count(void);

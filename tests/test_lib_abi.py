@@ -82,3 +82,38 @@ def test_argument_errors_return_before_cuda(lib):
                                None) == 1
     # workspace too small
     assert L.moe_layer_forward(p, p, p, p, p, p, 0, p, 16, p, ctypes.byref(sh), None, None) == 3
+
+
+def test_backward_shape_limits_and_workspace(lib):
+    kimi = moe.shape(8, 7168, 384, 8, 7168, 2048)
+    rm = moe.rows_max(kimi)
+    tw = moe.train_workspace_bytes(kimi)
+    # forward buffers + ab, dys, dab, hg (dxg reuses y)
+    assert tw >= moe.layer_workspace_bytes(kimi) + rm * (2048 * 4 + 7168 * 2 + 2048 * 4 + 2048 * 2)
+    # the backward runs 256x256 pair tiles only: I % 256 and pad % 256
+    assert moe.train_workspace_bytes(moe.shape(1, 512, 8, 2, 256, 128)) == 0
+    assert moe.train_workspace_bytes(moe.shape(1, 512, 8, 2, 256, 256, pad=128)) == 0
+    assert moe.train_workspace_bytes(moe.shape(1, 512, 8, 2, 256, 256)) > 0
+
+
+def test_backward_argument_errors_return_before_cuda(lib):
+    L = lib
+    sh = moe.shape(1, 16, 8, 2, 256, 256)
+    S = ctypes.byref(sh)
+    assert L.moe_layer_forward_train(*([None] * 7), 0, None, S, None, None) == 1
+    assert L.moe_expert_ffn_train(*([None] * 10), S, None) == 1
+    assert L.moe_reverse_combine(*([None] * 8), S, None) == 1
+    assert L.moe_expert_ffn_dgrad(*([None] * 14), S, None) == 1
+    assert L.moe_reverse_dispatch(*([None] * 4), S, None) == 1
+    assert L.moe_router_backward(*([None] * 6), S, None) == 1
+    assert L.moe_expert_ffn_wgrad(*([None] * 10), S, None) == 1
+    assert L.moe_layer_backward(*([None] * 10), 0, None, S, None, None) == 1
+    p = ctypes.c_void_p(256)
+    # I = 128: unsupported by the backward
+    sh128 = moe.shape(1, 16, 8, 2, 256, 128)
+    assert L.moe_layer_backward(*([p] * 10), 1 << 40, p, ctypes.byref(sh128), None, None) == 2
+    assert L.moe_expert_ffn_wgrad(*([p] * 10), ctypes.byref(sh128), None) == 2
+    # workspace too small; misaligned (16- but not 32-byte) workspace
+    assert L.moe_layer_backward(*([p] * 10), 16, p, S, None, None) == 3
+    assert L.moe_layer_forward_train(*([p] * 6), ctypes.c_void_p(272), 1 << 40, p, S, None,
+                                     None) == 1
