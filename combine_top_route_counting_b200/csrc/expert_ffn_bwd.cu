@@ -639,7 +639,7 @@ cudaError_t launch_expert_ffn_wgrad(const uint16_t* xg, const uint16_t* dys, con
                                     const int32_t* counts, float* dW1, float* dW3, float* dW2,
                                     const moe_shape_t& sh, int64_t rows_max, int32_t* dev_status,
                                     cudaStream_t s, cudaEvent_t ev_mid) {
-  const int E = sh.E, H = sh.H, I = sh.I;
+  const int H = sh.H, I = sh.I;
   CUtensorMap mHg, mDys, mXg, mDab;
   // MN-major operands: 64 columns x 64 rows per box
   if (!make_map(&mHg, hg, I, rows_max, 64, 64) || !make_map(&mDys, dys, H, rows_max, 64, 64) ||
