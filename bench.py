@@ -347,6 +347,7 @@ def run_ours(args):
 
     # end to end through the host-buffer entry: H2D of logits and x, the layer,
     # D2H of out; each call's input copy overlaps the previous call's compute
+    # and its output copy the next call's compute (the async-output entry)
     e2e = None
     e2e_mb = args.e2e_minibatch if args.e2e_minibatch >= 0 else w.minibatch
     if not args.no_e2e:
@@ -355,14 +356,24 @@ def run_ours(args):
         wsh = torch.empty(moe.layer_host_workspace_bytes(sh), dtype=torch.uint8, device=dev)
         lg_h, x_h = lg_cpu.pin_memory(), x_cpu.pin_memory()
         out_h = torch.empty((w.n_tokens, w.H), dtype=torch.bfloat16).pin_memory()
-        for _ in range(2):
-            moe.moe_layer_forward_host(lg_h, x_h, *W, out_h, wsh, st, sh, minibatch_tokens=e2e_mb)
+        out_ready = [torch.cuda.Event() for _ in range(2)]
+        for r in out_ready:
+            r.record()  # creates the event
+
+        def host_step(i):
+            moe.moe_layer_forward_host_async(lg_h, x_h, *W, out_h, wsh, st, sh, out_ready[i % 2],
+                                             minibatch_tokens=e2e_mb)
+
+        for i in range(2):
+            host_step(i)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         chk = 0.0
         e0.record()
-        for _ in range(args.e2e_steps):
-            moe.moe_layer_forward_host(lg_h, x_h, *W, out_h, wsh, st, sh, minibatch_tokens=e2e_mb)
+        for i in range(args.e2e_steps):
+            host_step(i)
+        # the timed region ends when the last step's output is in host memory
+        torch.cuda.current_stream().wait_event(out_ready[(args.e2e_steps - 1) % 2])
         e1.record()
         torch.cuda.synchronize()
         chk += float(out_h[0, :8].float().sum())  # the host reads the result
@@ -471,7 +482,9 @@ def run_ours(args):
             line["e2e"] = {"value": w.n_tokens * world * args.e2e_steps / (e2e["ms"] / 1e3),
                            "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
                            "d2h_bytes_per_step": e2e["d2h"],
-                           "api": "moe_layer_forward_host (pinned host logits/x/out)",
+                           "api": "moe_layer_forward_host_async (pinned host logits/x/out; "
+                                  "the output copy completes on an event, off the compute "
+                                  "stream)",
                            "transfer_minibatch_tokens": e2e_mb or w.N,
                            "ms_per_step": e2e["ms"] / args.e2e_steps}
         if mb_row is not None:

@@ -67,7 +67,7 @@ moe_status_t check_bwd_shape(const moe_shape_t* s) {
 // forward's combine has run.
 struct LayerWs {
   size_t ids, gates, route_row, phi, offsets, counts, sched, xg, h, y, total;
-  size_t logits[2], x[2], out, total_host;  // moe_layer_forward_host additions
+  size_t logits[2], x[2], out[2], total_host;  // moe_layer_forward_host additions
   size_t ab, dys, dab, hg, gate_row, part, total_train;  // training additions
 };
 
@@ -97,8 +97,8 @@ LayerWs layer_ws(const moe_shape_t* s) {
   for (int b = 0; b < 2; ++b) {  // consecutive host-buffer calls alternate
     w.logits[b] = take(oh, tokens * s->E * 4);
     w.x[b] = take(oh, tokens * s->H * 2);
+    w.out[b] = take(oh, tokens * s->H * 2);
   }
-  w.out = take(oh, tokens * s->H * 2);
   w.total_host = oh;
   size_t ot = o;
   w.ab = take(ot, rows * s->I * 4);
@@ -284,7 +284,8 @@ struct CopyRes {
   cudaStream_t h2d = nullptr, d2h = nullptr;
   cudaEvent_t lg = nullptr, fin = nullptr;
   cudaEvent_t ex[kRing] = {}, ed[kRing] = {};
-  cudaEvent_t in_free[2] = {};  // input buffers of parity b no longer read
+  cudaEvent_t in_free[2] = {};   // input buffers of parity b no longer read
+  cudaEvent_t out_free[2] = {};  // output buffer of parity b copied out
   uint64_t calls = 0;
   bool ready = false;
 };
@@ -303,6 +304,8 @@ cudaError_t copy_res(CopyRes** out) {
     if ((e = cudaStreamCreateWithFlags(&r.d2h, cudaStreamNonBlocking)) != cudaSuccess) return e;
     if ((e = cudaEventCreateWithFlags(&r.in_free[0], ef)) != cudaSuccess) return e;
     if ((e = cudaEventCreateWithFlags(&r.in_free[1], ef)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&r.out_free[0], ef)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&r.out_free[1], ef)) != cudaSuccess) return e;
     if ((e = cudaEventCreateWithFlags(&r.lg, ef)) != cudaSuccess) return e;
     if ((e = cudaEventCreateWithFlags(&r.fin, ef)) != cudaSuccess) return e;
     for (int i = 0; i < kRing; ++i) {
@@ -316,18 +319,23 @@ cudaError_t copy_res(CopyRes** out) {
 }
 
 // Host-buffer layer. Consecutive calls alternate between two device copies of
-// the inputs (parity b), so the host-to-device copy of call i+1 runs while
-// call i still computes: it only waits until call i-1, the last user of the
-// same copies, has finished reading them. Within a call, the rows of slice
-// [t0, t0+Tm) of every peer are copied in on the h2d stream while the
+// the inputs and of the output (parity b), so the host-to-device copy of call
+// i+1 runs while call i still computes: it only waits until call i-1, the last
+// user of the same copies, has finished reading them. Within a call, the rows
+// of slice [t0, t0+Tm) of every peer are copied in on the h2d stream while the
 // previous slice computes on `s`, and copied out on the d2h stream while the
 // next one computes (the transfer minibatch of "Mixture-of-Kittens" notes
 // section 3 and "Beyond Peak TFLOPs" section 1: chunk k transfers while chunk
-// k-1 computes). `s` waits for every copy of the call before the call ends.
+// k-1 computes). Without out_ready, `s` waits for every copy of the call
+// before the call ends. With out_ready, `s` does not wait for the copy out
+// (the event marks its end), so call i+1 computes while call i's output
+// travels; call i+2 writes the same device output copy only after it has
+// been copied out.
 cudaError_t layer_host_pipeline(const float* logits_host, const uint16_t* x_host,
                                 const uint16_t* W1, const uint16_t* W3, const uint16_t* W2,
                                 uint16_t* out_host, int32_t minibatch_tokens, void* ws,
-                                int32_t* dev_status, const moe_shape_t* sh, cudaStream_t s) {
+                                int32_t* dev_status, const moe_shape_t* sh, cudaStream_t s,
+                                cudaEvent_t out_ready) {
   std::lock_guard<std::mutex> lock(g_copy_mu);
   CopyRes* cr = nullptr;
   cudaError_t e = copy_res(&cr);
@@ -337,7 +345,7 @@ cudaError_t layer_host_pipeline(const float* logits_host, const uint16_t* x_host
   const LayerBufs bufs = layer_bufs(ws, w);
   float* logits = at<float>(ws, w.logits[b]);
   uint16_t* x = at<uint16_t>(ws, w.x[b]);
-  uint16_t* out = at<uint16_t>(ws, w.out);
+  uint16_t* out = at<uint16_t>(ws, w.out[b]);
   const int32_t P = sh->P, N = sh->N, H = sh->H;
   const size_t row_bytes = static_cast<size_t>(H) * 2;
   const int32_t T = (minibatch_tokens <= 0 || minibatch_tokens >= N) ? N : minibatch_tokens;
@@ -365,6 +373,8 @@ cudaError_t layer_host_pipeline(const float* logits_host, const uint16_t* x_host
     if ((e = cudaEventRecord(cr->ex[0], cr->h2d)) != cudaSuccess) return e;
   }
   if ((e = cudaStreamWaitEvent(s, cr->lg, 0)) != cudaSuccess) return e;
+  // the device output copy of parity b has been copied out by call i-2
+  if ((e = cudaStreamWaitEvent(s, cr->out_free[b], 0)) != cudaSuccess) return e;
   if ((e = launch_route_topk(logits, bufs.ids, bufs.gates, static_cast<int64_t>(tokens), sh->E,
                              sh->k, s)) != cudaSuccess)
     return e;
@@ -387,9 +397,16 @@ cudaError_t layer_host_pipeline(const float* logits_host, const uint16_t* x_host
   }
   // routing and every slice's dispatch have read this call's input copies
   if ((e = cudaEventRecord(cr->in_free[b], s)) != cudaSuccess) return e;
-  // `s` completes only after the last copy out (and every copy in)
-  if ((e = cudaEventRecord(cr->fin, cr->d2h)) != cudaSuccess) return e;
-  if ((e = cudaStreamWaitEvent(s, cr->fin, 0)) != cudaSuccess) return e;
+  if ((e = cudaEventRecord(cr->out_free[b], cr->d2h)) != cudaSuccess) return e;
+  if (out_ready) {
+    // the caller waits on out_ready for out_host; `s` goes on computing
+    if ((e = cudaEventRecord(out_ready, cr->d2h)) != cudaSuccess) return e;
+  } else {
+    // `s` completes only after the last copy out
+    if ((e = cudaEventRecord(cr->fin, cr->d2h)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(s, cr->fin, 0)) != cudaSuccess) return e;
+  }
+  // ... and after every copy in
   if ((e = cudaEventRecord(cr->fin, cr->h2d)) != cudaSuccess) return e;
   return cudaStreamWaitEvent(s, cr->fin, 0);
 }
@@ -693,7 +710,28 @@ moe_status_t moe_layer_forward_host(const float* logits_host, const uint16_t* x_
   const LayerWs w = layer_ws(shape);
   if (ws_bytes < w.total_host) return MOE_WORKSPACE_TOO_SMALL;
   return from_cuda(layer_host_pipeline(logits_host, x_host, W1, W3, W2, out_host, minibatch_tokens,
-                                       ws, dev_status, shape, static_cast<cudaStream_t>(stream)));
+                                       ws, dev_status, shape, static_cast<cudaStream_t>(stream),
+                                       nullptr));
+}
+
+moe_status_t moe_layer_forward_host_async(const float* logits_host, const uint16_t* x_host,
+                                          const uint16_t* W1, const uint16_t* W3,
+                                          const uint16_t* W2, uint16_t* out_host,
+                                          int32_t minibatch_tokens, void* ws, size_t ws_bytes,
+                                          int32_t* dev_status, const moe_shape_t* shape,
+                                          void* stream, void* out_ready) {
+  moe_status_t st = check_ffn_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!out_ready || !W1 || !W3 || !W2 || !ws || !dev_status ||
+      (shape->N > 0 && (!logits_host || !x_host || !out_host)))
+    return MOE_INVALID_ARG;
+  if (!aligned16(W1) || !aligned16(W3) || !aligned16(W2) || !aligned32(ws))
+    return MOE_INVALID_ARG;
+  if (minibatch_tokens < 0) return MOE_INVALID_ARG;
+  if (ws_bytes < layer_ws(shape).total_host) return MOE_WORKSPACE_TOO_SMALL;
+  return from_cuda(layer_host_pipeline(logits_host, x_host, W1, W3, W2, out_host, minibatch_tokens,
+                                       ws, dev_status, shape, static_cast<cudaStream_t>(stream),
+                                       static_cast<cudaEvent_t>(out_ready)));
 }
 
 int64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

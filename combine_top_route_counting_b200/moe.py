@@ -71,6 +71,8 @@ _SIGS = {
                            ctypes.POINTER(Shape), _vp, ctypes.POINTER(_vp)], ctypes.c_int),
     "moe_layer_forward_host": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_int32, _vp,
                                 ctypes.c_size_t, _vp, ctypes.POINTER(Shape), _vp], ctypes.c_int),
+    "moe_layer_forward_host_async": ([_vp] * 6 + [ctypes.c_int32, _vp, ctypes.c_size_t, _vp,
+                                      ctypes.POINTER(Shape), _vp, _vp], ctypes.c_int),
     "moe_schedule_static_ws": ([_vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Shape), _vp],
                                ctypes.c_int),
     "moe_train_workspace_bytes": ([ctypes.POINTER(Shape)], ctypes.c_size_t),
@@ -375,6 +377,22 @@ def moe_layer_backward(dout, W1, W3, W2, dx, dlogits, dW1, dW3, dW2, ws, dev_sta
                                      _ptr(dev_status, torch.int32, "dev_status"),
                                      ctypes.byref(sh), _stream(stream),
                                      _events(stage_events, N_BWD_EVENTS)), "moe_layer_backward")
+
+
+def moe_layer_forward_host_async(logits_host, x_host, W1, W3, W2, out_host, ws, dev_status,
+                                 sh: Shape, out_ready, minibatch_tokens=0, stream=None):
+    """out_ready: a torch.cuda.Event (recorded once before first use, so that it
+    exists) or a raw cudaEvent_t; it completes when out_host holds the output."""
+    ev = out_ready.cuda_event if hasattr(out_ready, "cuda_event") else int(out_ready)
+    if not ev:
+        raise ValueError("out_ready: the event has not been created (record it once first)")
+    _check(load().moe_layer_forward_host_async(
+        _ptr(logits_host, torch.float32, "logits_host", device=False),
+        _ptr(x_host, torch.bfloat16, "x_host", device=False), _ptr(W1, torch.bfloat16, "W1"),
+        _ptr(W3, torch.bfloat16, "W3"), _ptr(W2, torch.bfloat16, "W2"),
+        _ptr(out_host, torch.bfloat16, "out_host", device=False), int(minibatch_tokens),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _ptr(dev_status, torch.int32, "dev_status"),
+        ctypes.byref(sh), _stream(stream), ctypes.c_void_p(ev)), "moe_layer_forward_host_async")
 
 
 def moe_selftest_bounded_wait(dev_status, timeout_ns: int, stream=None):

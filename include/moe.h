@@ -255,6 +255,24 @@ moe_status_t moe_layer_forward_host(const float* logits_host, const uint16_t* x_
                                     size_t ws_bytes, int32_t* dev_status,
                                     const moe_shape_t* shape, void* stream);
 
+/* moe_layer_forward_host whose copy of the output to the host runs off
+ * `stream`: `stream` orders the input copies and the compute, and the copy of
+ * out_host completes when out_ready (a cudaEvent_t the caller created, ideally
+ * with cudaEventDisableTiming) completes; `stream` does not wait for it. So
+ * consecutive calls compute back to back while each call's output travels to
+ * the host (the device keeps two output copies in ws and call i+2 reuses call
+ * i's only after it has been copied out). out_host holds the output once
+ * out_ready has completed; the copies out of all host-buffer calls on a
+ * device run in call order on one internal stream, so a later call may be
+ * handed the same out_host. Everything else as moe_layer_forward_host (same
+ * workspace size). */
+moe_status_t moe_layer_forward_host_async(const float* logits_host, const uint16_t* x_host,
+                                          const uint16_t* W1, const uint16_t* W3,
+                                          const uint16_t* W2, uint16_t* out_host,
+                                          int32_t minibatch_tokens, void* ws, size_t ws_bytes,
+                                          int32_t* dev_status, const moe_shape_t* shape,
+                                          void* stream, void* out_ready);
+
 /* ------------------------------------------------------------------------
  * Backward (training).
  *

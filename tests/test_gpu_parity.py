@@ -442,6 +442,44 @@ def test_layer_host_entry_matches_device_entry(cuda_lib, minibatch):
         assert torch.equal(outs[c], refs[c % 2]), f"call {c}"
 
 
+@pytest.mark.parametrize("minibatch", [0, 2368])
+def test_layer_host_async_entry_matches_device_entry(cuda_lib, minibatch):
+    """The async-output host entry: six calls back to back (two input batches
+    alternated, so both device input copies and both device output copies are
+    reused), one synchronous call in between; each call's host output, read
+    after its own event, equals the device-buffer entry's."""
+    moe = cuda_lib
+    w, lg, x, W = _layer_inputs("mid")
+    Wd = [t.to(DEV) for t in W]
+    perm = torch.randperm(w.n_tokens, generator=torch.Generator().manual_seed(9))
+    batches = [(lg, x), (lg[perm].contiguous(), x[perm].contiguous())]
+    refs = [_layer_gpu(moe, w, a.to(DEV), b.to(DEV), Wd)[0].cpu() for a, b in batches]
+    sh = moe.shape(**w.shape())
+    ws = torch.empty(moe.layer_host_workspace_bytes(sh), dtype=torch.uint8, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pinned = [(a.pin_memory(), b.pin_memory()) for a, b in batches]
+    n = 7
+    outs = [torch.full((w.n_tokens, w.H), 7.0, dtype=torch.bfloat16).pin_memory() for _ in range(n)]
+    evs = [torch.cuda.Event() for _ in range(n)]
+    for e in evs:
+        e.record()  # creates the event
+    torch.cuda.synchronize()
+    for c in range(n):
+        lg_h, x_h = pinned[c % 2]
+        if c == 3:
+            moe.moe_layer_forward_host(lg_h, x_h, *Wd, outs[c], ws, st, sh,
+                                       minibatch_tokens=minibatch)
+            evs[c].record()
+        else:
+            moe.moe_layer_forward_host_async(lg_h, x_h, *Wd, outs[c], ws, st, sh, evs[c],
+                                             minibatch_tokens=minibatch)
+    for c in range(n):
+        evs[c].synchronize()
+        assert torch.equal(outs[c], refs[c % 2]), f"call {c}"
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+
+
 def test_layer_pad128_single_cta_path(cuda_lib):
     """Segments padded to 128 rows run the single-CTA (128x256 tile) FFN kernels."""
     moe = cuda_lib

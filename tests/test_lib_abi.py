@@ -117,3 +117,11 @@ def test_backward_argument_errors_return_before_cuda(lib):
     assert L.moe_layer_backward(*([p] * 10), 16, p, S, None, None) == 3
     assert L.moe_layer_forward_train(*([p] * 6), ctypes.c_void_p(272), 1 << 40, p, S, None,
                                      None) == 1
+
+
+def test_host_async_entry_needs_an_event(lib):
+    sh = moe.shape(1, 16, 8, 2, 256, 128)
+    p = ctypes.c_void_p(256)
+    args = [p] * 6 + [0, p, 1 << 40, p, ctypes.byref(sh), None]
+    assert lib.moe_layer_forward_host_async(*args, None) == 1
+    assert lib.moe_layer_forward_host_async(*args[:8], 16, p, ctypes.byref(sh), None, p) == 3
