@@ -172,9 +172,9 @@ cudaError_t run_slice(const LayerBufs& b, const uint16_t* x, const uint16_t* W1,
   if ((e = launch_schedule(b.ids, *sh, sl, b.phi, b.offsets, b.counts, b.route_row, b.sched,
                            dev_status, s)) != cudaSuccess)
     return e;
-  // The pull dispatch runs as its own HBM-bound gather: feeding GEMM1 with TMA
-  // row gathers instead (moe_expert_ffn_gather) measured 3x slower on B200, the
-  // gathers delivering far fewer bytes per clock than the MMAs use.
+  // The pull dispatch runs as its own HBM-bound gather: feeding GEMM1 with row
+  // gathers instead (moe_expert_ffn_gather) measured 2.6-3x slower on B200,
+  // the gathers delivering far fewer bytes per clock than the MMAs use.
   if ((e = rec(2)) != cudaSuccess) return e;
   if ((e = launch_dispatch(x, b.phi, b.offsets, b.xg, *sh, rows_max, dev_status, s)) != cudaSuccess)
     return e;

@@ -98,7 +98,6 @@ struct FfnParams {
   int* tile_counter;       // next tile to hand out (zeroed before each launch)
   const int2* phi;         // [rows_max] (src_rank, src_idx): GATHER only
   int32_t n_per_peer;      // N (GATHER: token row = src_rank * N + src_idx)
-  int32_t oob_row;         // P*N: a row index outside x, which reads as zeros
   const int32_t* offsets;  // [E+1]
   const int32_t* counts;   // [E, P] or null
   int32_t E, P;
@@ -109,6 +108,7 @@ struct FfnParams {
   int32_t* dev_status;
   int64_t timeout_ns;
   uint16_t* ab;            // SAVE_AB: bf16 pre-activations [rows_max, 2I], a | b
+  const void* x;           // GATHER: token activations bf16 [P*N, H]
 };
 
 template <int CG, int MODE>
@@ -132,9 +132,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // a = x.W1 and b = x.W3, rounded to bf16, as ab[row] = [a | b] for the
 // backward pass (which then never recomputes GEMM1).
 // GATHER (MODE 0 only): the A operand is pulled straight from the token
-// activations x by the schedule Phi ("zero-copy, direct landing"): every lane
-// of the producer warp gathers 4 of the CTA's 128 rows per K step with a TMA
-// tile::gather4 load, so no gathered copy of the tokens is materialised.
+// activations x by the schedule Phi ("zero-copy, direct landing"), so no
+// gathered copy of the tokens is materialised. Warps 0 and 3 (64 threads)
+// copy the CTA's 128 A rows per K step with 16-byte cp.async: thread t owns
+// the 16-byte chunk t % 8 of rows t / 8 + 8i (i < 16), written where the
+// 128-byte swizzle puts it (chunk c of row r at c ^ (r % 8)); padding rows
+// are zero-filled. A thread signals a stage once its copies into it have
+// completed (cp.async groups, three stages behind) and it has fenced them to
+// the async proxy that tcgen05.mma reads through; then one arrive per warp
+// on the leader's full barrier. B still comes by TMA (warp 0, lane 0).
 // CG = 1: one CTA per 128x256 tile. CG = 2: a cluster of two CTAs (a tcgen05
 // CTA pair) per 256x256 tile; CTA r loads rows [128r, 128r+128) of A and
 // columns [128r, 128r+128) of B, the leader (r = 0) issues the pair MMAs and
@@ -164,7 +170,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (tid == 0) {
     for (int i = 0; i < C::STAGES; ++i) {
-      mbar_init(smem_u32(&bars[C::BAR_FULL + i]), 1);
+      // GATHER: + one arrive per A-producer warp of each CTA of the pair
+      mbar_init(smem_u32(&bars[C::BAR_FULL + i]), GATHER ? 1 + 2 * CG : 1);
       mbar_init(smem_u32(&bars[C::BAR_EMPTY + i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -174,7 +181,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(smem_u32(&bars[C::BAR_DRAIN]), 1);
     for (int i = 0; i < kRing; ++i) {
       mbar_init(smem_u32(&bars[C::BAR_TID_FULL + i]), 1);
-      mbar_init(smem_u32(&bars[C::BAR_TID_EMPTY + i]), C::TID_CONSUMERS);
+      // GATHER: warp 3 of each CTA reads the tile ids too
+      mbar_init(smem_u32(&bars[C::BAR_TID_EMPTY + i]), C::TID_CONSUMERS + (GATHER ? CG : 0));
     }
     *abort_flag = 0;
     *bad_flag = 0;
@@ -285,17 +293,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     return row0 < s_end[l];
   };
 
-  if (warp == 0 && GATHER) {
-    // ------------------------------------------------------------ TMA producer (row gather)
+  if ((warp == 0 || warp == 3) && GATHER) {
+    // ------------------------------------------------------------ producers (row gather)
+    constexpr int kLag = 3;  // cp.async groups in flight per thread before a stage is signalled
+    static_assert(kLag < C::STAGES, "a stage is signalled before its slot is needed again");
+    const int pt = (warp == 0 ? 0 : 32) + lane;  // producer thread 0..63
+    const int cchunk = pt & 7;                   // 16-byte chunk of the 128-byte row
+    const int r0 = pt >> 3;                      // rows r0 + 8i of the CTA's 128
+    const uint32_t swz = static_cast<uint32_t>((cchunk ^ (r0 & 7)) << 4);
     const uint32_t full0 = smem_u32(&bars[C::BAR_FULL]);
     const uint32_t full_tgt0 = (CG == 2) ? mapa_shared(full0, 0) : full0;
+    const uint16_t* xsrc = reinterpret_cast<const uint16_t*>(p.x);
     int stage = 0;
     uint32_t phase = 0;
-    int64_t issued = 0;
+    int64_t issued = 0, signalled = 0;
     bool ok = true;
     int bad = 0;
     int tpos = 0;
     uint32_t tph = 0;
+    // make the copies of the oldest unsignalled stage visible to the async
+    // proxy and arrive on its full barrier (once per warp)
+    auto signal_oldest = [&](int keep) {
+      if (keep == 0) asm volatile("cp.async.wait_group 0;" ::: "memory");
+      else asm volatile("cp.async.wait_group %0;" ::"n"(kLag) : "memory");
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        const int st = static_cast<int>(signalled % C::STAGES);
+        if (CG == 2 && !leader) mbar_arrive_cluster(full_tgt0 + st * 8);
+        else mbar_arrive(full0 + st * 8);
+      }
+      ++signalled;
+    };
     while (ok) {
       int tile = 0;
       if (lane == 0) tile = next_tile(tpos, tph);
@@ -304,14 +333,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int row0, n, l;
       if (!tile_info(tile, row0, n, l)) continue;
       const int arow = row0 + static_cast<int>(rank) * 128;
-      // rows arow + 4*lane .. +3 of the tile: their token rows in x
-      int tok[4];
+      // token rows of this thread's 16 A rows (padding and invalid entries: zero-fill)
+      const uint16_t* src[16];
+      uint32_t valid = 0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int2 e = __ldg(p.phi + arow + 4 * lane + i);
+      for (int i = 0; i < 16; ++i) {
+        const int2 e = __ldg(p.phi + arow + r0 + 8 * i);
         const bool v = e.x >= 0 && e.x < p.P && e.y >= 0 && e.y < p.n_per_peer;
         if (!v && (e.x >= 0 || e.y != -1)) bad = 1;  // (-1,-1) is padding
-        tok[i] = v ? e.x * p.n_per_peer + e.y : p.oob_row;
+        src[i] = xsrc + (v ? (static_cast<int64_t>(e.x) * p.n_per_peer + e.y) * p.K : 0) + cchunk * 8;
+        valid |= (v ? 1u : 0u) << i;
       }
       const int ky0 = l * p.K;
       for (int kb = 0; kb < kblocks; ++kb) {
@@ -322,20 +353,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ok = false;
           break;
         }
-        const uint32_t full_local = full0 + stage * 8;
-        const uint32_t full_tgt = full_tgt0 + stage * 8;
         const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
         const uint32_t sB = sA + C::A_BYTES;
-        const int ky = ky0 + kb * C::BK;
-        if (lane == 0 && leader) mbar_arrive_expect_tx(full_local, CG * C::STAGE_BYTES);
-        __syncwarp();
-        // 4 rows x 128 bytes land at sA + 512*lane: the same 128-byte-swizzled
-        // layout a 128-row box load produces
-        if (CG == 2)
-          tma_gather4_pair(sA + lane * 512, &tmA, kb * C::BK, tok[0], tok[1], tok[2], tok[3], full_tgt);
-        else
-          tma_gather4(sA + lane * 512, &tmA, kb * C::BK, tok[0], tok[1], tok[2], tok[3], full_tgt);
-        if (lane == 0) {
+        if (warp == 0 && lane == 0) {
+          const uint32_t full_tgt = full_tgt0 + stage * 8;
+          const int ky = ky0 + kb * C::BK;
+          if (leader) mbar_arrive_expect_tx(full0 + stage * 8, CG * (C::STAGE_BYTES - C::A_BYTES));
           if (CG == 1) {
             tma_load_2d(sB + 0 * C::B_ATOM_BYTES, &tmB0, n * 128, ky, full_tgt);
             tma_load_2d(sB + 1 * C::B_ATOM_BYTES, &tmB0, n * 128 + 64, ky, full_tgt);
@@ -347,16 +370,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             tma_load_2d_pair(sB + C::B_ATOM_BYTES, mb, n * 128 + 64, ky, full_tgt);
           }
         }
+        const int koff = kb * C::BK;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t dst = sA + static_cast<uint32_t>((r0 + 8 * i) * 128) + swz;
+          const uint32_t nbytes = ((valid >> i) & 1u) ? 16u : 0u;  // 0: zero-fill
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst),
+                       "l"(src[i] + koff), "r"(nbytes)
+                       : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
         ++issued;
         if (++stage == C::STAGES) {
           stage = 0;
           phase ^= 1u;
         }
+        if (issued - signalled > kLag) signal_oldest(kLag);
       }
+    }
+    if (ok) {
+      while (signalled < issued) signal_oldest(0);
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");  // no copy may land after exit
     }
     if (bad) atomicOr(p.dev_status, MOE_DEV_BAD_SCHEDULE);
     __syncwarp();
-    if (lane == 0) {
+    if (warp == 0 && lane == 0) {
+      // no TMA load may still be landing in shared memory when the CTA exits
       const int64_t first = issued > C::STAGES ? issued - C::STAGES : 0;
       for (int64_t j = first; j < issued; ++j) {
         const int st = static_cast<int>(j % C::STAGES);
@@ -454,7 +494,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
         for (int kb = 0; kb < kblocks; ++kb) {
-          if (!wait_bounded(smem_u32(&bars[C::BAR_FULL + stage]), phase, wc)) {
+          // GATHER with CTA pairs: the follower's producers release its A rows
+          // at cluster scope, so the wait acquires at cluster scope
+          if (!wait_bounded<GATHER && CG == 2>(smem_u32(&bars[C::BAR_FULL + stage]), phase, wc)) {
             ok = false;
             break;
           }
@@ -753,7 +795,7 @@ cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint
   // Segments that are multiples of 256 rows run on CTA pairs (256x256 tiles);
   // otherwise (pad a multiple of 128 only) on single CTAs (128x256 tiles).
   const bool pair = (sh.pad % 256) == 0;
-  FfnParams p1{nullptr, nullptr, 0, 0, offsets, counts, E, sh.P, H, I, rows_max, h, dev_status,
+  FfnParams p1{nullptr, nullptr, 0, offsets, counts, E, sh.P, H, I, rows_max, h, dev_status,
                kWaitTimeoutNs, ab};
   cudaError_t e;
   if (ab)  // training: keep the pre-activations (pair tiles only)
@@ -765,7 +807,7 @@ cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint
     e = cudaEventRecord(ev_mid, s);
     if (e != cudaSuccess) return e;
   }
-  FfnParams p2{nullptr, nullptr, 0, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status,
+  FfnParams p2{nullptr, nullptr, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status,
                kWaitTimeoutNs, nullptr};
   return pair ? launch_mode<1, 2>(mA2, mW2, mW2, mY, p2, s)
               : launch_mode<1, 1>(mA2, mW2, mW2, mY, p2, s);
@@ -777,27 +819,25 @@ cudaError_t launch_expert_ffn_gather(const uint16_t* x, const int32_t* phi, cons
                                      float* y, const moe_shape_t& sh, int64_t rows_max,
                                      int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_mid) {
   const int E = sh.E, H = sh.H, I = sh.I;
-  const int64_t tokens = static_cast<int64_t>(sh.P) * sh.N;
-  CUtensorMap mX, mW1, mW3, mA2, mW2, mY;
+  CUtensorMap mW1, mW3, mA2, mW2, mY;
   const uint64_t EH = static_cast<uint64_t>(E) * H, EI = static_cast<uint64_t>(E) * I;
-  // x viewed as [P*N, H] with a one-row box: the gather4 form
-  if (!make_map(&mX, x, H, static_cast<uint64_t>(tokens > 0 ? tokens : 1), 64, 1) ||
-      !make_map(&mW1, W1, I, EH, 64, 64) || !make_map(&mW3, W3, I, EH, 64, 64) ||
+  if (!make_map(&mW1, W1, I, EH, 64, 64) || !make_map(&mW3, W3, I, EH, 64, 64) ||
       !make_map(&mA2, h, I, rows_max, 64, 128) || !make_map(&mW2, W2, H, EI, 64, 64) ||
       !make_map(&mY, y, H, rows_max, 32, 32, true))
     return cudaErrorInvalidValue;
   const bool pair = (sh.pad % 256) == 0;
-  FfnParams p1{nullptr, reinterpret_cast<const int2*>(phi), sh.N, static_cast<int32_t>(tokens), offsets,
-               counts, E, sh.P, H, I, rows_max, h, dev_status, kWaitTimeoutNs, nullptr};
-  cudaError_t e = pair ? launch_mode<0, 2, true>(mX, mW1, mW3, mX, p1, s)
-                       : launch_mode<0, 1, true>(mX, mW1, mW3, mX, p1, s);
+  // GEMM1's A rows come from x by Phi (cp.async); its A tensor map is unused
+  FfnParams p1{nullptr, reinterpret_cast<const int2*>(phi), sh.N, offsets, counts, E, sh.P, H,
+               I, rows_max, h, dev_status, kWaitTimeoutNs, nullptr, x};
+  cudaError_t e = pair ? launch_mode<0, 2, true>(mW1, mW1, mW3, mW1, p1, s)
+                       : launch_mode<0, 1, true>(mW1, mW1, mW3, mW1, p1, s);
   if (e != cudaSuccess) return e;
   if (ev_mid) {
     e = cudaEventRecord(ev_mid, s);
     if (e != cudaSuccess) return e;
   }
-  FfnParams p2{nullptr, nullptr, 0, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status,
-               kWaitTimeoutNs, nullptr};
+  FfnParams p2{nullptr, nullptr, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status,
+               kWaitTimeoutNs, nullptr, nullptr};
   return pair ? launch_mode<1, 2>(mA2, mW2, mW2, mY, p2, s)
               : launch_mode<1, 1>(mA2, mW2, mW2, mY, p2, s);
 }

@@ -192,12 +192,14 @@ moe_status_t moe_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint16
  * FFN's operand tiles ("Mixture-of-Kittens" notes section 2, zero-copy direct
  * landing; "Beyond Peak TFLOPs" 2.A): GEMM1 reads row `row` of its A operand
  * as x[src_rank*N + src_idx] with (src_rank, src_idx) = phi[row] (zeros for
- * padding rows) through TMA row gathers, so no gathered buffer exists.
+ * padding rows) with 16-byte asynchronous copies, so no gathered buffer
+ * exists.
  * x: bf16 [P*N, H]; phi: int32 [moe_rows_max, 2] as written by moe_schedule;
  * everything else as moe_expert_ffn, whose h and y it reproduces bit for bit.
  * An out-of-range Phi entry raises MOE_DEV_BAD_SCHEDULE and reads as zeros.
- * It needs no [moe_rows_max, H] gathered buffer, but on B200 it runs about 3x
- * slower than moe_dispatch + moe_expert_ffn (the row gathers deliver fewer
+ * It needs no [moe_rows_max, H] gathered buffer, but on B200 its GEMM1 runs
+ * about 2.6x slower than moe_dispatch + moe_expert_ffn (each gathered A tile
+ * is re-read for every output column block, and row gathers deliver fewer
  * bytes per clock than the tensor cores consume), so moe_layer_forward uses
  * the latter. */
 moe_status_t moe_expert_ffn_gather(const uint16_t* x, const int32_t* phi, const uint16_t* W1,
