@@ -485,7 +485,7 @@ def run_ours(args):
                            "api": "moe_layer_forward_host_async (pinned host logits/x/out; "
                                   "the output copy completes on an event, off the compute "
                                   "stream)",
-                           "transfer_minibatch_tokens": e2e_mb or w.N,
+                           "transfer_minibatch_tokens": e2e_mb or w.N, "steps": args.e2e_steps,
                            "ms_per_step": e2e["ms"] / args.e2e_steps}
         if mb_row is not None:
             line["minibatch_row"] = {"minibatch_tokens": w.minibatch,
@@ -568,7 +568,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="kimi")
     ap.add_argument("--minibatch", type=int, default=0)
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=0,
+                    help="steps of the host-buffer leg (0: the same as --steps)")
     ap.add_argument("--e2e-minibatch", type=int, default=0,
                     help="transfer slice of the host-buffer leg (0: whole batch; "
                          "-1: the workload's transfer minibatch)")
@@ -580,6 +581,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-row-budget", type=float, default=3.0)
     args = ap.parse_args(argv)
+    if args.e2e_steps <= 0:
+        args.e2e_steps = args.steps
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -341,6 +341,73 @@ def test_layer_backward_edge_shapes(cuda_lib, P, N, E, k, H, I):
     assert int((r["dW1"].abs().sum((1, 2)) > 0).sum().item()) == len(used)
 
 
+def test_layer_backward_pad512_skipped_tiles(cuda_lib):
+    """Segments padded to 512 rows: tiles holding only padding rows are skipped
+    by every GEMM (their rows stay unwritten), and the weight gradients run
+    over each expert's real rows only: still within the bound of the oracle."""
+    moe = cuda_lib
+    w = inputs.Workload("pad512", 9, P=2, N=300, E=6, k=2, H=256, I=256, pad=512)
+    c = dict(w=w, lg=inputs.make_logits(w), x=inputs.make_x(w), dout=inputs.make_dout(w),
+             W=[t.to(DEV) for t in inputs.make_weights(w)])
+    sh = moe.shape(**w.shape())
+    ws = torch.full((moe.train_workspace_bytes(sh),), 0xFF, dtype=torch.uint8, device=DEV)  # NaN-filled
+    r = _train_step(moe, c, ws=ws)
+    ids_all, _, _ = oracle.route_topk(c["lg"], w.k)
+    s = oracle.schedule(ids_all.reshape(w.P, w.N, w.k), w.P, w.N, w.k, w.E, 512)
+    assert (np.diff(s["offsets"]) - np.bincount(ids_all.reshape(-1), minlength=w.E) >= 256).any(), \
+        "the case has at least one padding-only tile"
+    _check_dx_dlogits(w, c, r, list(range(w.n_tokens)), c["W"])
+    _check_wgrad(w, c, r, list(range(w.E)), list(range(w.H)), list(range(w.I)))
+
+
+def test_backward_stages_without_counts_equal_with_counts(cuda_lib):
+    """counts = NULL: the GEMMs take whole segments (padding rows included) and
+    give bit-identical activation and weight gradients (padding rows add exact
+    zeros to every sum)."""
+    moe = cuda_lib
+    c = _inputs("tiny_bwd")
+    w, (W1, W3, W2) = c["w"], c["W"]
+    sh = moe.shape(**w.shape())
+    T, k, rm = w.n_tokens, w.k, moe.rows_max(sh)
+    ids = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    gates = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    moe.moe_route_topk(c["lg"].to(DEV), ids, gates, sh)
+    b = moe.alloc_schedule_outputs(sh)
+    st = b["dev_status"]
+    moe.moe_schedule(ids, b["phi"], b["offsets"], b["counts"], b["route_row"], b["ws"], st, sh)
+    xg = torch.empty((rm, w.H), dtype=torch.bfloat16, device=DEV)
+    moe.moe_dispatch(c["x"].to(DEV), b["phi"], b["offsets"], xg, st, sh)
+    h = torch.empty((rm, w.I), dtype=torch.bfloat16, device=DEV)
+    ab = torch.empty((rm, 2 * w.I), dtype=torch.bfloat16, device=DEV)
+    y = torch.empty((rm, w.H), dtype=torch.float32, device=DEV)
+    moe.moe_expert_ffn_train(xg, W1, W3, W2, b["offsets"], None, h, ab, y, st, sh)
+    dys = torch.empty((rm, w.H), dtype=torch.bfloat16, device=DEV)
+    gate_row = torch.empty(rm, dtype=torch.float32, device=DEV)
+    moe.moe_reverse_combine(c["dout"].to(DEV), b["phi"], b["offsets"], b["route_row"], gates, dys,
+                            gate_row, st, sh)
+    outs = []
+    for counts in (b["counts"], None):
+        dab = torch.empty((rm, 2 * w.I), dtype=torch.bfloat16, device=DEV)
+        hg = torch.empty((rm, w.I), dtype=torch.bfloat16, device=DEV)
+        part = torch.empty((rm, w.I // 128), dtype=torch.float32, device=DEV)
+        dxg = torch.empty((rm, w.H), dtype=torch.float32, device=DEV)
+        moe.moe_expert_ffn_dgrad(dys, gate_row, ab, h, W1, W3, W2, b["offsets"], counts, dab, hg,
+                                 part, dxg, st, sh)
+        dW1 = torch.empty((w.E, w.H, w.I), dtype=torch.float32, device=DEV)
+        dW3, dW2 = torch.empty_like(dW1), torch.empty((w.E, w.I, w.H), dtype=torch.float32,
+                                                      device=DEV)
+        moe.moe_expert_ffn_wgrad(xg, dys, dab, hg, b["offsets"], counts, dW1, dW3, dW2, st, sh)
+        outs.append((dab, hg, part, dxg, dW1, dW3, dW2))
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rows = int(b["offsets"][-1].item())
+    real = torch.from_numpy(np.nonzero(b["phi"][:rows, 0].cpu().numpy() >= 0)[0]).to(DEV)
+    for a, b_ in zip(outs[0][:4], outs[1][:4]):
+        assert torch.equal(a[real], b_[real])
+    for a, b_ in zip(outs[0][4:], outs[1][4:]):
+        assert torch.equal(a, b_)
+
+
 def test_layer_backward_no_tokens(cuda_lib):
     moe = cuda_lib
     w = inputs.Workload("empty", 8, P=2, N=0, E=4, k=2, H=256, I=256)
