@@ -691,9 +691,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 }  // namespace
 
-// Per-device counter the scheduler threads of the persistent GEMMs take tile
-// ids from; zeroed on the stream before every launch.
-__device__ int g_tile_counter[1];
+// Tile counters the scheduler threads of the persistent GEMMs take tile ids
+// from. Each launch takes the next slot of the pool (round robin) and zeroes
+// it on its stream first, so GEMMs running at the same time on different
+// streams never share a counter: a slot comes round again only 256 launches
+// later, far more kernels than a device runs at once.
+constexpr int kTileCounterSlots = 256;
+__device__ int g_tile_counter[kTileCounterSlots];
 
 // ---------------------------------------------------------------- host side
 namespace {
@@ -730,6 +734,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
 cudaError_t tile_counter_for_current_device(int** out) {
   static std::mutex mu;
   static int* ptrs[64] = {nullptr};
+  static uint32_t next[64] = {0};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -740,7 +745,7 @@ cudaError_t tile_counter_for_current_device(int** out) {
     if ((e = cudaGetSymbolAddress(&ptr, g_tile_counter)) != cudaSuccess) return e;
     ptrs[dev] = static_cast<int*>(ptr);
   }
-  *out = ptrs[dev];
+  *out = ptrs[dev] + (next[dev]++ % kTileCounterSlots);
   return cudaSuccess;
 }
 

@@ -64,9 +64,8 @@ cudaError_t launch_combine(const float* y, const int32_t* route_row, const float
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
               uint32_t box_outer, bool fp32 = false);
 
-// Device address of the tile counter of the persistent GEMMs on the current
-// device (looked up once per device). One counter per device: the FFN
-// launches of one device must not run concurrently.
+// A tile counter for one launch of a persistent GEMM on the current device:
+// the next slot of a per-device pool (the caller zeroes it on its stream).
 cudaError_t tile_counter_for_current_device(int** out);
 
 // ---------------------------------------------------------------- backward

@@ -177,10 +177,9 @@ moe_status_t moe_dispatch(const uint16_t* x, const int32_t* phi, const int32_t* 
  * padding rows are skipped and their h/y rows are left unwritten; rows that
  * carry routes are always written. Each output element is computed by one
  * CTA (pair) with a fixed K order: the result is bitwise deterministic.
- * The GEMM kernels take their tiles from a tile counter inside the library
- * (one per device, zeroed on `stream` before each GEMM): FFN calls
- * (moe_expert_ffn, moe_expert_ffn_gather, the layer entries) must not
- * overlap on the GPU -- serialise calls made on different streams.
+ * The GEMM kernels take their tiles from a tile counter inside the library:
+ * each GEMM launch takes the next of 256 per-device slots and zeroes it on
+ * `stream`, so FFN calls on different streams may run at the same time.
  * offsets must be non-decreasing multiples of 128 with offsets[E] <=
  * moe_rows_max (else MOE_DEV_BAD_SCHEDULE, nothing written). */
 moe_status_t moe_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint16_t* W3,

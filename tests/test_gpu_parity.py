@@ -480,6 +480,31 @@ def test_layer_host_async_entry_matches_device_entry(cuda_lib, minibatch):
     assert int(st.item()) == 0
 
 
+def test_layer_concurrent_streams(cuda_lib):
+    """Two layer calls running at the same time on two streams (own workspaces):
+    each GEMM launch takes its own tile counter, so both outputs equal the
+    single-stream result bit for bit."""
+    moe = cuda_lib
+    w, lg, x, W = _layer_inputs("mid")
+    Wd = [t.to(DEV) for t in W]
+    lg_d, x_d = lg.to(DEV), x.to(DEV)
+    ref, _ = _layer_gpu(moe, w, lg_d, x_d, Wd)
+    sh = moe.shape(**w.shape())
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    wss = [torch.empty(moe.layer_workspace_bytes(sh), dtype=torch.uint8, device=DEV) for _ in streams]
+    sts = [torch.zeros(1, dtype=torch.int32, device=DEV) for _ in streams]
+    outs = [torch.empty_like(ref) for _ in streams]
+    torch.cuda.synchronize()
+    for _ in range(3):
+        for s_, ws_, st_, o_ in zip(streams, wss, sts, outs):
+            with torch.cuda.stream(s_):
+                moe.moe_layer_forward(lg_d, x_d, *Wd, o_, ws_, st_, sh, stream=s_)
+    torch.cuda.synchronize()
+    for st_, o_ in zip(sts, outs):
+        assert int(st_.item()) == 0
+        assert torch.equal(o_, ref)
+
+
 def test_layer_pad128_single_cta_path(cuda_lib):
     """Segments padded to 128 rows run the single-CTA (128x256 tile) FFN kernels."""
     moe = cuda_lib

@@ -75,3 +75,43 @@ def test_corrupt_schedule_is_flagged_not_faulted(cuda_lib):
     torch.cuda.synchronize()
     assert int(st.item()) & moe.DEV_BAD_SCHEDULE
     assert (out.float() == 0).all()
+
+
+def test_backward_corrupt_schedule_is_flagged_not_faulted(cuda_lib):
+    """Offsets that are not multiples of the 256-row tile (or run past rows_max)
+    make every backward GEMM refuse its work and flag MOE_DEV_BAD_SCHEDULE; the
+    reverse dispatch and router gradient skip out-of-range rows. Nothing hangs."""
+    moe = cuda_lib
+    w = inputs.WORKLOADS["tiny_bwd"]
+    sh = moe.shape(**w.shape())
+    rm = moe.rows_max(sh)
+    dev = "cuda"
+    for bad_offsets in ([0, 100] + [100] * (w.E - 1), [0] + [rm + 256] * w.E):
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        offsets = torch.tensor(bad_offsets, dtype=torch.int32, device=dev)
+        z16 = lambda *s: torch.zeros(s, dtype=torch.bfloat16, device=dev)
+        z32 = lambda *s: torch.zeros(s, dtype=torch.float32, device=dev)
+        W1, W2 = z16(w.E, w.H, w.I), z16(w.E, w.I, w.H)
+        dab, hg, part, dxg = z16(rm, 2 * w.I), z16(rm, w.I), z32(rm, w.I // 128), z32(rm, w.H)
+        moe.moe_expert_ffn_dgrad(z16(rm, w.H), z32(rm), z16(rm, 2 * w.I), z16(rm, w.I), W1, W1, W2,
+                                 offsets, None, dab, hg, part, dxg, st, sh)
+        dW1, dW3 = torch.full((w.E, w.H, w.I), 5.0, device=dev), torch.full((w.E, w.H, w.I), 5.0, device=dev)
+        dW2 = torch.full((w.E, w.I, w.H), 5.0, device=dev)
+        moe.moe_expert_ffn_wgrad(z16(rm, w.H), z16(rm, w.H), dab, hg, offsets, None, dW1, dW3, dW2,
+                                 st, sh)
+        torch.cuda.synchronize()
+        assert int(st.item()) & moe.DEV_BAD_SCHEDULE
+        assert (dW1 == 5.0).all() and (dW2 == 5.0).all()  # nothing written
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    rr = torch.full((w.n_tokens, w.k), rm + 5, dtype=torch.int32, device=dev)
+    ids = torch.zeros((w.n_tokens, w.k), dtype=torch.int32, device=dev)
+    g = torch.ones((w.n_tokens, w.k), dtype=torch.float32, device=dev)
+    dx = torch.empty((w.n_tokens, w.H), dtype=torch.bfloat16, device=dev)
+    moe.moe_reverse_dispatch(torch.zeros((rm, w.H), device=dev), rr, dx, st, sh)
+    dl = torch.full((w.n_tokens, w.E), 3.0, device=dev)
+    moe.moe_router_backward(torch.zeros((rm, w.I // 128), device=dev), rr, ids, g, dl, st, sh)
+    torch.cuda.synchronize()
+    assert int(st.item()) & moe.DEV_BAD_SCHEDULE
+    assert (dx.float() == 0).all() and (dl == 0).all()
+    # the context is still usable
+    assert int(torch.arange(10, device=dev).sum().item()) == 45
