@@ -239,10 +239,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   // tile -> (first row, m-tile, n-tile, expert, K steps); false: skip (padding only).
   // dgrads: tiles are numbered expert by expert over the row tiles, in the
-  // forward's grouped raster (DGRAD_H M-tile-major like GEMM1, DGRAD_X
-  // N-block-major like GEMM2). WGRAD: expert-major, then m, then n.
+  // forward's grouped raster (N-block-major inside chunks of RM M-tiles).
+  // WGRAD: expert-major, then m, then n.
   constexpr int RM = 8;
-  constexpr int RN = (OP == OP_DGRAD_H) ? (1 << 20) : 1;
+  constexpr int RN = 1;
   auto tile_info = [&](int tile, int& row0, int& m, int& n, int& l, int& kblocks) -> bool {
     if (C::WGRAD) {
       l = tile / tiles_per_expert;
