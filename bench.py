@@ -537,10 +537,24 @@ def schedule_rows(moe, w, sh, lg) -> int:
     return int(b["offsets"][-1].item())
 
 
+def kernel_source_hash() -> str:
+    """sha256 of the FFN kernel sources (expert_ffn.cu, sm100.cuh) with comments,
+    trailing blanks and empty lines removed: edits to comments keep a recorded
+    measurement valid, any change to the code invalidates it."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for f in ("expert_ffn.cu", "sm100.cuh"):
+        src = open(os.path.join(ROOT, "combine_top_route_counting_b200", "csrc", f)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in src.splitlines()]
+        h.update("\n".join(ln for ln in lines if ln.strip()).encode())
+    return h.hexdigest()
+
+
 def gemm1_traffic(n_routes: int):
     """DRAM bytes per GEMM1 launch from the committed ncu summary, scaled to this
     launch by routes; None when the summary is missing or the kernel changed since."""
-    import hashlib
     path = os.path.join(ROOT, "profiles", "ffn_gemm1_traffic.txt")
     if not os.path.exists(path):
         return None
@@ -549,10 +563,7 @@ def gemm1_traffic(n_routes: int):
         if ":" in ln:
             a, b = ln.split(":", 1)
             kv[a.strip()] = b.strip()
-    h = hashlib.sha256()
-    for f in ("expert_ffn.cu", "sm100.cuh"):
-        h.update(open(os.path.join(ROOT, "combine_top_route_counting_b200", "csrc", f), "rb").read())
-    if kv.get("kernel_source_sha256") != h.hexdigest():
+    if kv.get("kernel_source_sha256") != kernel_source_hash():
         return None
     try:
         return float(kv["dram_bytes_per_route"]) * n_routes

@@ -33,9 +33,9 @@
 // half and CTA 1 the W3 half). A tile never straddles two experts because
 // every segment is a multiple of the tile height; the expert of a tile comes
 // from a binary search over the segment offsets held in shared memory. Tiles
-// holding only padding rows are skipped. Tiles are visited m-major, so the
-// CTAs running at one time share an expert's weights and the A rows of a few
-// M-tiles through L2.
+// holding only padding rows are skipped. Tiles are handed out dynamically in
+// an expert-by-expert, N-block-major order, so the CTAs running at one time
+// share an expert's A rows and a few weight column blocks through L2.
 //
 // Every output element is produced by one CTA with a fixed K order (no
 // split-K, no atomics): the result is bitwise deterministic and independent
