@@ -47,19 +47,14 @@
 #include <cuda_bf16.h>
 
 #include "internal.cuh"
+#include "persistent_gemm.cuh"
 #include "sm100.cuh"
 
 namespace moe {
 namespace {
 
 using namespace sm100;
-
-constexpr int NUM_THREADS = 384;  // 12 warps: TMA, MMA, 2 idle, 8 epilogue
-constexpr int EPI_WARP0 = 4;
-constexpr int NUM_EPI_WARPS = 8;
-constexpr int TMEM_COLS = 512;    // 2 accumulators x 256 fp32 columns
-constexpr int UMMA_K = 16;
-constexpr int kRing = 4;  // tile ids in flight between the scheduler and the roles
+using namespace pg;
 
 // Tile geometry for CG CTAs per MMA (1: one SM, 2: a CTA pair on two SMs).
 // TMA_STORE (GEMM2 on CTA pairs): the fp32 epilogue stages each warp's 32x32
@@ -118,13 +113,6 @@ size_t smem_bytes_for(int E) {
 
 __device__ __forceinline__ float silu(float a) { return a / (1.0f + expf(-a)); }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat16 a = __float2bfloat16_rn(lo);
-  const __nv_bfloat16 b = __float2bfloat16_rn(hi);
-  return static_cast<uint32_t>(__bfloat16_as_ushort(a)) |
-         (static_cast<uint32_t>(__bfloat16_as_ushort(b)) << 16);
-}
-
 // MODE 0: GEMM1 + SwiGLU -> bf16 h. MODE 1: GEMM2 -> fp32 y.
 // SAVE_AB (MODE 0, training): the epilogue also keeps the pre-activations
 // a = x.W1 and b = x.W3, rounded to bf16, as ab[row] = [a | b] for the
@@ -144,7 +132,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // columns [128r, 128r+128) of B, the leader (r = 0) issues the pair MMAs and
 // each CTA drains its own 128 TMEM lanes.
 template <int MODE, int CG, bool GATHER, bool SAVE_AB>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(kNumThreads, 1)
     ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmY,
                     const FfnParams p) {
@@ -174,7 +162,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bars[C::BAR_TFULL + i]), 1);
-      mbar_init(smem_u32(&bars[C::BAR_TEMPTY + i]), NUM_EPI_WARPS * CG);
+      mbar_init(smem_u32(&bars[C::BAR_TEMPTY + i]), kNumEpiWarps * CG);
     }
     mbar_init(smem_u32(&bars[C::BAR_DRAIN]), 1);
     for (int i = 0; i < kRing; ++i) {
@@ -192,27 +180,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_desc(&tmB1);
     if (C::TMA_STORE) tma_prefetch_desc(&tmY);
   }
-  for (int l = tid; l <= E; l += NUM_THREADS) s_off[l] = __ldg(p.offsets + l);
-  __syncthreads();
-  for (int l = tid; l < E; l += NUM_THREADS) {
-    const int a = s_off[l], b = s_off[l + 1];
-    bool bad = a < 0 || b < a || (a % C::BM) || (b % C::BM) || b > p.rows_max;
-    int T = b - a;
-    if (p.counts) {
-      int t = 0;
-      for (int r = 0; r < p.P; ++r) t += __ldg(p.counts + l * p.P + r);
-      if (t < 0 || t > b - a) bad = true;
-      else T = t;
-    }
-    if (bad) *bad_flag = 1;
-    s_end[l] = a + T;
-  }
+  load_segments(p.offsets, p.counts, E, p.P, C::BM, p.rows_max, s_off, s_end, bad_flag);
   if (warp == 1) {
     if (CG == 2) {
-      tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
       tmem_relinquish_pair();
     } else {
-      tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_alloc(smem_u32(tmem_slot), kTmemCols);
       tmem_relinquish();
     }
   }
@@ -230,64 +204,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int kblocks = p.K / C::BK;
   const WaitCtx wc{abort_flag, p.dev_status, p.timeout_ns, MOE_DEV_TIMEOUT};
 
-  // Dynamic tile order: the leader's scheduler thread takes tile ids from a
-  // device-wide counter and posts them, in order, to a ring that every role
-  // of both CTAs reads. CTAs that run ahead simply take more tiles, so the
-  // tiles in flight stay a narrow window of consecutive ids and the operands
-  // they share are still in L2. (A static round-robin let slow pairs fall
-  // whole experts behind, and GEMM1 read its weights 2.5-4x from DRAM.)
-  // next_tile(): the next id of this role's sequence, -1 at the end, -2 if a
-  // wait gave up. One thread per consuming warp calls it.
-  // The slot is released with a release-ordered arrive (the read of the id
-  // must not move after it): CTA scope for the leader's own roles, cluster
-  // scope only for the follower's, whose arrive is remote.
+  // Tiles come from the tile-id ring (persistent_gemm.cuh), filled by the
+  // leader's scheduler thread from a device-wide counter.
   const uint32_t tid_empty_local = smem_u32(&bars[C::BAR_TID_EMPTY]);
-  const uint32_t tid_empty_tgt0 = (CG == 2) ? mapa_shared(tid_empty_local, 0) : tid_empty_local;
+  const TileRing tring{tile_ring, smem_u32(&bars[C::BAR_TID_FULL]), tid_empty_local,
+                       (CG == 2) ? mapa_shared(tid_empty_local, 0) : tid_empty_local, !leader};
   auto next_tile = [&](int& pos, uint32_t& ph) -> int {
-    const int j = pos % kRing;
-    if (!wait_bounded<CG == 2>(smem_u32(&bars[C::BAR_TID_FULL + j]), ph, wc)) return -2;
-    const int t = reinterpret_cast<volatile int*>(tile_ring)[j];
-    if (CG == 2 && !leader) mbar_arrive_cluster(tid_empty_tgt0 + j * 8);
-    else mbar_arrive(tid_empty_local + j * 8);
-    if (++pos % kRing == 0) ph ^= 1u;
-    return t;
+    return tring.next<CG == 2>(pos, ph, wc);
   };
   const int64_t drain_ns = p.timeout_ns < 100000000ll ? p.timeout_ns : 100000000ll;
 
   // tile -> (first row, n-tile, expert); false if the tile holds only padding.
-  // Tiles are numbered expert by expert (expert e owns tiles
-  // [S[e]/BM * tiles_n, S[e+1]/BM * tiles_n)) and, inside an expert, in a
-  // grouped raster so that tiles sharing operands run close together in time
-  // and find them in L2: chunks of up to RM M-tiles; inside a chunk, groups
-  // of RN N-blocks; inside a group, N fastest. RN = 1 (N-block-major): each
-  // weight column block's M-tiles are consecutive and the chunk's A rows stay
-  // in L2. With the dynamic tile order the tiles in flight are a narrow
-  // window of ids, and this order measured faster for both GEMMs (GEMM1 21.8
-  // vs 22.7 ms against M-tile-major; GEMM2's DRAM reads equal W2 + h).
-  constexpr int RM = 8;
-  constexpr int RN = 1;
+  // Expert by expert, N-block-major inside chunks of RM M-tiles (RN = 1): each
+  // weight column block's M-tiles run back to back and the chunk's A rows stay
+  // in L2. With the dynamic tile order the tiles in flight are a narrow window
+  // of ids, and this order measured faster for both GEMMs (GEMM1 21.8 vs
+  // 22.7 ms against M-tile-major; GEMM2's DRAM reads equal W2 + h).
   auto tile_info = [&](int tile, int& row0, int& n, int& l) -> bool {
-    const int u = tile / tiles_n;  // the tile's position in M-tile units
-    int lo = 0, hi = E - 1;        // expert: largest l with S[l]/BM <= u
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_off[mid] / C::BM <= u) lo = mid;
-      else hi = mid - 1;
-    }
-    l = lo;
-    const int m0 = s_off[l] / C::BM;
-    const int mcount = s_off[l + 1] / C::BM - m0;  // >= 1 for the expert owning u
-    const int j = tile - m0 * tiles_n;               // index inside the expert
-    const int mc = j / (RM * tiles_n);               // M chunk
-    const int rows = min(RM, mcount - mc * RM);      // M-tiles in this chunk
-    const int jj = j - mc * RM * tiles_n;
-    const int ng = jj / (rows * RN);                 // N group
-    const int gsize = min(RN, tiles_n - ng * RN);    // N-blocks in this group
-    const int rr = jj - ng * rows * RN;
-    const int m = rr / gsize;
-    n = ng * RN + (rr - m * gsize);
-    row0 = (m0 + mc * RM + m) * C::BM;
-    return row0 < s_end[l];
+    return grouped_row_tile<C::BM, 8, 1>(tile, s_off, s_end, E, tiles_n, row0, n, l);
   };
 
   if ((warp == 0 || warp == 3) && GATHER) {
@@ -501,7 +435,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sB = sA + C::A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < C::BK / UMMA_K; ++kk) {
+          for (int kk = 0; kk < C::BK / kUmmaK; ++kk) {
             // A: K-major, advance 16 bf16 = 32 bytes inside the swizzled row.
             // B: MN-major, advance 16 K-rows = two 8-row groups = 2048 bytes.
             const uint64_t a_desc = smem_desc_sw128(sA + kk * 32, 16, 1024);
@@ -530,30 +464,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ tile scheduler
-    if (lane == 0 && leader) {
-      const uint32_t ring_peer = (CG == 2) ? mapa_shared(smem_u32(tile_ring), 1) : 0u;
-      const uint32_t tfull_peer =
-          (CG == 2) ? mapa_shared(smem_u32(&bars[C::BAR_TID_FULL]), 1) : 0u;
-      uint32_t eph = 0;
-      for (int i = 0;; ++i) {
-        const int j = i % kRing;
-        if (!wait_bounded<CG == 2>(smem_u32(&bars[C::BAR_TID_EMPTY + j]), eph ^ 1u, wc)) break;
-        int t = atomicAdd(p.tile_counter, 1);
-        if (t >= num_tiles) t = -1;
-        reinterpret_cast<volatile int*>(tile_ring)[j] = t;
-        mbar_arrive(smem_u32(&bars[C::BAR_TID_FULL + j]));
-        if (CG == 2) {
-          st_shared_cluster_u32(ring_peer + j * 4, static_cast<uint32_t>(t));
-          mbar_arrive_cluster(tfull_peer + j * 8);
-        }
-        if (j == kRing - 1) eph ^= 1u;
-        if (t < 0) break;
-      }
-    }
-  } else if (warp >= EPI_WARP0) {
+    if (lane == 0 && leader) tring.schedule<CG == 2>(p.tile_counter, num_tiles, wc);
+  } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
-    const int half = (warp - EPI_WARP0) >> 2;  // which half of the tile's columns
+    const int half = (warp - kEpiWarp0) >> 2;  // which half of the tile's columns
     const uint32_t tempty0 = smem_u32(&bars[C::BAR_TEMPTY]);
     const uint32_t tempty_tgt0 = (CG == 2) ? mapa_shared(tempty0, 0) : tempty0;
     int acc = 0;
@@ -622,7 +537,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // row `lane` of this warp's 32x32 block goes to the staging slot with
         // 16-byte chunk j at position j ^ (lane & 7): the 128-byte swizzle the
         // tensor map expects, and no bank conflicts for the 16-byte writes.
-        const uint32_t stg = smem_u32(staging) + (warp - EPI_WARP0) * 4096;
+        const uint32_t stg = smem_u32(staging) + (warp - kEpiWarp0) * 4096;
         const uint64_t pol_y = l2_policy_evict_first();
         const int ycol = n * C::BN + half * 128;
         const int yrow0 = row0 + static_cast<int>(rank) * 128 + q * 32;
@@ -681,8 +596,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    if (CG == 2) tmem_dealloc_pair(tmem_base, TMEM_COLS);
-    else tmem_dealloc(tmem_base, TMEM_COLS);
+    if (CG == 2) tmem_dealloc_pair(tmem_base, kTmemCols);
+    else tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -694,32 +609,11 @@ template <int MODE, int CG, bool GATHER = false, bool SAVE_AB = false>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const CUtensorMap& yo, FfnParams p, cudaStream_t s) {
   const size_t smem = smem_bytes_for<CG, MODE>(p.E);
-  cudaError_t ce = tile_counter_for_current_device(&p.tile_counter);
-  if (ce != cudaSuccess) return ce;
-  if ((ce = cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s)) != cudaSuccess) return ce;
-  cudaError_t e = cudaFuncSetAttribute(ffn_gemm_kernel<MODE, CG, GATHER, SAVE_AB>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = tile_counter_for_current_device(&p.tile_counter);
   if (e != cudaSuccess) return e;
-  const int sms = device_sm_count();
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  cfg.gridDim = dim3(CG == 2 ? (sms / 2) * 2 : sms);
-  cfg.blockDim = dim3(NUM_THREADS);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  if (CG == 2) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-  }
-  e = cudaLaunchKernelEx(&cfg, ffn_gemm_kernel<MODE, CG, GATHER, SAVE_AB>, a, b0, b1, yo, p);
-  note_launches(1);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  if ((e = cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s)) != cudaSuccess) return e;
+  return launch_persistent(ffn_gemm_kernel<MODE, CG, GATHER, SAVE_AB>, CG, smem, s, a, b0, b1, yo,
+                           p);
 }
 
 }  // namespace

@@ -50,19 +50,14 @@
 #include <cuda_bf16.h>
 
 #include "internal.cuh"
+#include "persistent_gemm.cuh"
 #include "sm100.cuh"
 
 namespace moe {
 namespace {
 
 using namespace sm100;
-
-constexpr int NUM_THREADS = 384;  // warps: 0 TMA, 1 MMA, 2 tile scheduler, 3 idle, 4-11 epilogue
-constexpr int EPI_WARP0 = 4;
-constexpr int NUM_EPI_WARPS = 8;
-constexpr int TMEM_COLS = 512;    // 2 accumulators x 256 fp32 columns
-constexpr int UMMA_K = 16;
-constexpr int kRing = 4;          // tile ids in flight between the scheduler and the roles
+using namespace pg;
 
 enum : int { OP_DGRAD_H = 0, OP_DGRAD_X = 1, OP_WGRAD = 2 };
 
@@ -123,12 +118,6 @@ size_t bwd_smem_bytes(int E) {
          C::NUM_BARS * 8 + 16 + kRing * 4 + static_cast<size_t>(2 * E + 1) * 4;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat16 a = __float2bfloat16_rn(lo);
-  const __nv_bfloat16 b = __float2bfloat16_rn(hi);
-  return static_cast<uint32_t>(__bfloat16_as_ushort(a)) |
-         (static_cast<uint32_t>(__bfloat16_as_ushort(b)) << 16);
-}
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
@@ -139,7 +128,7 @@ __device__ __forceinline__ void st_global_v4(void* ptr, uint32_t a, uint32_t b, 
 }
 
 template <int OP>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(kNumThreads, 1)
     ffn_bwd_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmY0,
                    const __grid_constant__ CUtensorMap tmY1, const BwdParams p) {
@@ -168,7 +157,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&bars[C::BAR_TFULL + i]), 1);
-      mbar_init(smem_u32(&bars[C::BAR_TEMPTY + i]), NUM_EPI_WARPS * 2);
+      mbar_init(smem_u32(&bars[C::BAR_TEMPTY + i]), kNumEpiWarps * 2);
     }
     mbar_init(smem_u32(&bars[C::BAR_DRAIN]), 1);
     for (int i = 0; i < kRing; ++i) {
@@ -188,23 +177,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tma_prefetch_desc(&tmY1);
     }
   }
-  for (int l = tid; l <= E; l += NUM_THREADS) s_off[l] = __ldg(p.offsets + l);
-  __syncthreads();
-  for (int l = tid; l < E; l += NUM_THREADS) {
-    const int a = s_off[l], b = s_off[l + 1];
-    bool bad = a < 0 || b < a || (a % C::BM) || (b % C::BM) || b > p.rows_max;
-    int T = b - a;
-    if (p.counts) {
-      int t = 0;
-      for (int r = 0; r < p.P; ++r) t += __ldg(p.counts + l * p.P + r);
-      if (t < 0 || t > b - a) bad = true;
-      else T = t;
-    }
-    if (bad) *bad_flag = 1;
-    s_end[l] = a + T;
-  }
+  load_segments(p.offsets, p.counts, E, p.P, C::BM, p.rows_max, s_off, s_end, bad_flag);
   if (warp == 1) {
-    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish_pair();
   }
   tc_fence_before();
@@ -222,19 +197,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bad_sched ? 0 : (C::WGRAD ? E * tiles_per_expert : (s_off[E] / C::BM) * tiles_n);
   const WaitCtx wc{abort_flag, p.dev_status, p.timeout_ns, MOE_DEV_TIMEOUT};
 
-  // Tile ids come from the device-wide counter through the leader's
-  // scheduler thread and a ring both CTAs read (as in the forward kernel).
+  // Tiles come from the tile-id ring (persistent_gemm.cuh), filled by the
+  // leader's scheduler thread from a device-wide counter.
   const uint32_t tid_empty_local = smem_u32(&bars[C::BAR_TID_EMPTY]);
-  const uint32_t tid_empty_tgt0 = mapa_shared(tid_empty_local, 0);
-  auto next_tile = [&](int& pos, uint32_t& ph) -> int {
-    const int j = pos % kRing;
-    if (!wait_bounded<true>(smem_u32(&bars[C::BAR_TID_FULL + j]), ph, wc)) return -2;
-    const int t = reinterpret_cast<volatile int*>(tile_ring)[j];
-    if (!leader) mbar_arrive_cluster(tid_empty_tgt0 + j * 8);
-    else mbar_arrive(tid_empty_local + j * 8);
-    if (++pos % kRing == 0) ph ^= 1u;
-    return t;
-  };
+  const TileRing tring{tile_ring, smem_u32(&bars[C::BAR_TID_FULL]), tid_empty_local,
+                       mapa_shared(tid_empty_local, 0), !leader};
+  auto next_tile = [&](int& pos, uint32_t& ph) -> int { return tring.next<true>(pos, ph, wc); };
   const int64_t drain_ns = p.timeout_ns < 100000000ll ? p.timeout_ns : 100000000ll;
 
   // tile -> (first row, m-tile, n-tile, expert, K steps); false: skip (padding only).
@@ -253,29 +221,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       kblocks = (s_end[l] - s_off[l] + C::BK - 1) / C::BK;
       return true;
     }
-    const int u = tile / tiles_n;
-    int lo = 0, hi = E - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_off[mid] / C::BM <= u) lo = mid;
-      else hi = mid - 1;
-    }
-    l = lo;
-    const int m0 = s_off[l] / C::BM;
-    const int mcount = s_off[l + 1] / C::BM - m0;
-    const int j = tile - m0 * tiles_n;
-    const int mc = j / (RM * tiles_n);
-    const int rows = min(RM, mcount - mc * RM);
-    const int jj = j - mc * RM * tiles_n;
-    const int ng = jj / (rows * RN);
-    const int gsize = min(RN, tiles_n - ng * RN);
-    const int rr = jj - ng * rows * RN;
-    const int mm = rr / gsize;
-    n = ng * RN + (rr - mm * gsize);
     m = 0;
-    row0 = (m0 + mc * RM + mm) * C::BM;
     kblocks = p.K / C::BK;
-    return row0 < s_end[l];
+    return grouped_row_tile<C::BM, RM, RN>(tile, s_off, s_end, E, tiles_n, row0, n, l);
   };
 
   if (warp == 0) {
@@ -367,7 +315,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sB = sA + C::A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < C::BK / UMMA_K; ++kk) {
+          for (int kk = 0; kk < C::BK / kUmmaK; ++kk) {
             uint64_t a_desc, b_desc;
             if (C::WGRAD) {  // MN-major: 16 K-rows = two 8-row groups = 2048 bytes
               a_desc = smem_desc_sw128(sA + kk * 2048, C::ATOM_BYTES, 1024);
@@ -394,29 +342,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ tile scheduler
-    if (lane == 0 && leader) {
-      const uint32_t ring_peer = mapa_shared(smem_u32(tile_ring), 1);
-      const uint32_t tfull_peer = mapa_shared(smem_u32(&bars[C::BAR_TID_FULL]), 1);
-      uint32_t eph = 0;
-      for (int i = 0;; ++i) {
-        const int j = i % kRing;
-        if (!wait_bounded<true>(smem_u32(&bars[C::BAR_TID_EMPTY + j]), eph ^ 1u, wc)) break;
-        int t = atomicAdd(p.tile_counter, 1);
-        if (t >= num_tiles) t = -1;
-        reinterpret_cast<volatile int*>(tile_ring)[j] = t;
-        mbar_arrive(smem_u32(&bars[C::BAR_TID_FULL + j]));
-        st_shared_cluster_u32(ring_peer + j * 4, static_cast<uint32_t>(t));
-        mbar_arrive_cluster(tfull_peer + j * 8);
-        if (j == kRing - 1) eph ^= 1u;
-        if (t < 0) break;
-      }
-    }
-  } else if (warp >= EPI_WARP0) {
+    if (lane == 0 && leader) tring.schedule<true>(p.tile_counter, num_tiles, wc);
+  } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                    // TMEM lane quarter of this warp
-    const int half = (warp - EPI_WARP0) >> 2;  // which 128 of the tile's 256 columns
+    const int half = (warp - kEpiWarp0) >> 2;  // which 128 of the tile's 256 columns
     const uint32_t tempty_tgt0 = mapa_shared(smem_u32(&bars[C::BAR_TEMPTY]), 0);
-    const uint32_t stg = smem_u32(staging) + (warp - EPI_WARP0) * 4096;  // TMA_STORE only
+    const uint32_t stg = smem_u32(staging) + (warp - kEpiWarp0) * 4096;  // TMA_STORE only
     const uint64_t pol_out = l2_policy_evict_first();
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -553,7 +485,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 
@@ -564,25 +496,7 @@ cudaError_t launch_bwd(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
   cudaError_t e = tile_counter_for_current_device(&p.tile_counter);
   if (e != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s)) != cudaSuccess) return e;
-  if ((e = cudaFuncSetAttribute(ffn_bwd_kernel<OP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(smem))) != cudaSuccess)
-    return e;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  cfg.gridDim = dim3((device_sm_count() / 2) * 2);
-  cfg.blockDim = dim3(NUM_THREADS);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, ffn_bwd_kernel<OP>, a, b0, b1, y0, y1, p);
-  note_launches(1);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  return launch_persistent(ffn_bwd_kernel<OP>, 2, smem, s, a, b0, b1, y0, y1, p);
 }
 
 BwdParams base_params(const int32_t* offsets, const int32_t* counts, const moe_shape_t& sh,
