@@ -538,13 +538,14 @@ def schedule_rows(moe, w, sh, lg) -> int:
 
 
 def kernel_source_hash() -> str:
-    """sha256 of the FFN kernel sources (expert_ffn.cu, sm100.cuh) with comments,
-    trailing blanks and empty lines removed: edits to comments keep a recorded
-    measurement valid, any change to the code invalidates it."""
+    """sha256 of the FFN kernel sources (expert_ffn.cu, persistent_gemm.cuh,
+    sm100.cuh) with comments, trailing blanks and empty lines removed: edits to
+    comments keep a recorded measurement valid, any change to the code
+    invalidates it."""
     import hashlib
     import re
     h = hashlib.sha256()
-    for f in ("expert_ffn.cu", "sm100.cuh"):
+    for f in ("expert_ffn.cu", "persistent_gemm.cuh", "sm100.cuh"):
         src = open(os.path.join(ROOT, "combine_top_route_counting_b200", "csrc", f)).read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
         lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in src.splitlines()]
