@@ -510,7 +510,7 @@ def run_ours(args):
                              "peak": peaks["bf16_sus"] if "tflops" in bst[top] else peaks["hbm"],
                              "unit": "TFLOP/s" if "tflops" in bst[top] else "GB/s",
                              "frac": bst[top].get("frac_bf16", bst[top].get("frac_hbm")),
-                             "traffic": None},
+                             "traffic": wgrad13_traffic(w.n_routes) if top == "wgrad_w13" else None},
                 "dout": "bf16 N(0,1), seeded",
             }
         line["clocks"] = clk
@@ -537,15 +537,14 @@ def schedule_rows(moe, w, sh, lg) -> int:
     return int(b["offsets"][-1].item())
 
 
-def kernel_source_hash() -> str:
-    """sha256 of the FFN kernel sources (expert_ffn.cu, persistent_gemm.cuh,
-    sm100.cuh) with comments, trailing blanks and empty lines removed: edits to
-    comments keep a recorded measurement valid, any change to the code
-    invalidates it."""
+def kernel_source_hash(files=("expert_ffn.cu", "persistent_gemm.cuh", "sm100.cuh")) -> str:
+    """sha256 of kernel sources (by default the forward FFN's) with comments,
+    trailing blanks and empty lines removed: edits to comments keep a recorded
+    measurement valid, any change to the code invalidates it."""
     import hashlib
     import re
     h = hashlib.sha256()
-    for f in ("expert_ffn.cu", "persistent_gemm.cuh", "sm100.cuh"):
+    for f in files:
         src = open(os.path.join(ROOT, "combine_top_route_counting_b200", "csrc", f)).read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
         lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in src.splitlines()]
@@ -553,23 +552,36 @@ def kernel_source_hash() -> str:
     return h.hexdigest()
 
 
-def gemm1_traffic(n_routes: int):
-    """DRAM bytes per GEMM1 launch from the committed ncu summary, scaled to this
-    launch by routes; None when the summary is missing or the kernel changed since."""
-    path = os.path.join(ROOT, "profiles", "ffn_gemm1_traffic.txt")
+def _recorded_traffic(name: str, files, n_routes: int):
+    """DRAM bytes per launch from a committed ncu summary (profiles/<name>),
+    scaled to this launch by routes; None when the summary is missing or the
+    kernel sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(path):
         return None
     kv = {}
     for ln in open(path):
-        if ":" in ln:
+        if ":" in ln and not ln.startswith("#"):
             a, b = ln.split(":", 1)
             kv[a.strip()] = b.strip()
-    if kv.get("kernel_source_sha256") != kernel_source_hash():
+    if kv.get("kernel_source_sha256") != kernel_source_hash(files):
         return None
     try:
         return float(kv["dram_bytes_per_route"]) * n_routes
     except (KeyError, ValueError):
         return None
+
+
+def gemm1_traffic(n_routes: int):
+    """DRAM bytes of one GEMM1 launch (profiles/ffn_gemm1_traffic.txt)."""
+    return _recorded_traffic("ffn_gemm1_traffic.txt",
+                             ("expert_ffn.cu", "persistent_gemm.cuh", "sm100.cuh"), n_routes)
+
+
+def wgrad13_traffic(n_routes: int):
+    """DRAM bytes of one dW1|dW3 launch (profiles/ffn_wgrad13_traffic.txt)."""
+    return _recorded_traffic("ffn_wgrad13_traffic.txt",
+                             ("expert_ffn_bwd.cu", "persistent_gemm.cuh", "sm100.cuh"), n_routes)
 
 
 def main(argv=None):
