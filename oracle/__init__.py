@@ -25,6 +25,7 @@ _i64p = ctypes.POINTER(ctypes.c_int64)
 _u16p = ctypes.POINTER(ctypes.c_uint16)
 _f32p = ctypes.POINTER(ctypes.c_float)
 _f64p = ctypes.POINTER(ctypes.c_double)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
 
 
 def lib():
@@ -69,6 +70,14 @@ def lib():
         L.oracle_router_bwd.argtypes = [_f64p, _f64p, _i32p, ctypes.c_int64, ctypes.c_int32,
                                         ctypes.c_int32, _f64p]
         L.oracle_router_bwd.restype = None
+        L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_value.restype = ctypes.c_double
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_double]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_mx_quantize.argtypes = [_f64p, ctypes.c_int64, ctypes.c_int32, _u8p, _u8p]
+        L.oracle_mx_quantize.restype = None
+        L.oracle_mx_dequantize.argtypes = [_u8p, _u8p, ctypes.c_int64, ctypes.c_int32, _f64p]
+        L.oracle_mx_dequantize.restype = None
         L.oracle_combine_f32.restype = None
         L.oracle_round_bf16.argtypes = [ctypes.c_double]
         L.oracle_round_bf16.restype = ctypes.c_uint16
@@ -410,3 +419,87 @@ def wgrad_sample(logits, x_bits, dout_bits, weights, k: int, E: int, experts, hs
         t, j = np.nonzero(ids == e)
         out[e] = wgrad_expert(xb[t], db_[t], g64[t, j], W1[e], W3[e], W2[e], hs, is_, exact)
     return out
+
+
+# ---------------------------------------------------------------- MXFP8
+def e4m3_value(codes) -> np.ndarray:
+    """float64 values of E4M3 codes (NaN for S.1111.111)."""
+    c = np.asarray(codes, np.uint8)
+    return np.array([lib().oracle_e4m3_value(int(x)) for x in c.reshape(-1)]).reshape(c.shape)
+
+
+def e4m3_encode(values) -> np.ndarray:
+    """E4M3 codes of values: nearest, ties to even, magnitudes above 448 clamped."""
+    v = np.asarray(values, np.float64)
+    return np.array([lib().oracle_e4m3_encode(float(x)) for x in v.reshape(-1)],
+                    np.uint8).reshape(v.shape)
+
+
+def mx_quantize(values):
+    """MX (E4M3, blocks of 32 along the last axis): (codes [..., K], scales [..., K/32])."""
+    v = np.ascontiguousarray(np.asarray(values, np.float64))
+    K = v.shape[-1]
+    if K % 32:
+        raise ValueError("the last axis must be a multiple of 32")
+    n = v.size // K
+    q = np.zeros(v.shape, np.uint8)
+    s = np.zeros(v.shape[:-1] + (K // 32,), np.uint8)
+    if n:
+        lib().oracle_mx_quantize(_p(v, _f64p), n, K, _p(q, _u8p), _p(s, _u8p))
+    return q, s
+
+
+def mx_dequantize(q, s) -> np.ndarray:
+    qq = np.ascontiguousarray(np.asarray(q, np.uint8))
+    ss = np.ascontiguousarray(np.asarray(s, np.uint8))
+    K = qq.shape[-1]
+    n = qq.size // K
+    out = np.zeros(qq.shape, np.float64)
+    if n:
+        lib().oracle_mx_dequantize(_p(qq, _u8p), _p(ss, _u8p), n, K, _p(out, _f64p))
+    return out
+
+
+def mx_round(values, axis: int = -1) -> np.ndarray:
+    """The values an MXFP8 operand stands for: quantised in blocks of 32 along
+    `axis` (the GEMM's reduction dimension), then dequantised."""
+    v = np.moveaxis(np.asarray(values, np.float64), axis, -1)
+    q, s = mx_quantize(v)
+    return np.moveaxis(mx_dequantize(q, s), -1, axis)
+
+
+def _bits_f64(b) -> np.ndarray:
+    return (np.asarray(b, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def layer_tokens_mxfp8(logits, x_bits, weights, k: int, H: int, I: int, tokens):
+    """The layer with MXFP8 routed experts ("Mixture-of-Kittens", section 5),
+    for a set of tokens: every GEMM operand is MX-quantised along its reduction
+    dimension -- x rows along H, W1/W3 along H (per column i), h rows along I,
+    W2 along I (per column) -- and the products, SwiGLU and combine run in
+    fp64 on the values the quantised operands stand for:
+      a = mx(x).mx(W1), b = mx(x).mx(W3), h = silu(a) * b,
+      y = mx(h).mx(W2), out[t] = sum_j g_j y_j (gates: fp64 softmax of the top k).
+    Returns dict out64 [n, H], ids, gates64."""
+    ids, g32, g64 = route_topk(logits, k)
+    toks = np.asarray(list(tokens), np.int64)
+    W1, W3, W2 = weights
+    cache = {}
+
+    def expert(e):
+        if e not in cache:
+            cache[e] = (mx_round(_bits_f64(W1[e]), axis=0), mx_round(_bits_f64(W3[e]), axis=0),
+                        mx_round(_bits_f64(W2[e]), axis=0))
+        return cache[e]
+
+    xb = np.asarray(x_bits, np.uint16)
+    out = np.zeros((len(toks), H), np.float64)
+    for a_i, t in enumerate(toks):
+        xt = mx_round(_bits_f64(xb[t]))
+        for j in range(k):
+            w1, w3, w2 = expert(int(ids[t, j]))
+            a = xt @ w1
+            b = xt @ w3
+            h = a / (1.0 + np.exp(-a)) * b
+            out[a_i] += g64[t, j] * (mx_round(h) @ w2)
+    return dict(out64=out, ids=ids, gates64=g64)

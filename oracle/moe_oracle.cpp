@@ -37,6 +37,10 @@
 //  R8 SwiGLU: h = bf16_rne(silu(x.W1) * (x.W3)), y = h.W2;
 //  R9 combine: out = bf16_rne(sum_j g_j * y_j) accumulated from 0 in
 //     ascending slot order (the fp32 fixed-order form uses fmaf).
+//  MX MXFP8 routed experts ("Mixture-of-Kittens", section 5; the OCP
+//     Microscaling (MX) formats, MXFP8 with E4M3 elements): every GEMM operand
+//     quantised in blocks of 32 along its reduction dimension, one E8M0 scale
+//     per block (see the MX functions below).
 //  B1 backward ("Mixture-of-Kittens", MoK overview: one table serves the
 //     forward and backward phases; pull-reverse-combine, push-reverse-
 //     dispatch; section 5: router gradients from the inner product of the
@@ -601,3 +605,88 @@ void oracle_router_bwd(const double* dgate, const double* g, const int32_t* ids,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// MXFP8 (MX). E4M3 element: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa
+// bits; no infinities; S.1111.111 is NaN; the largest finite magnitude is
+// 448 = 1.75 * 2^8; below 2^-6 the values are subnormal with step 2^-9. The
+// code of a non-negative finite value is monotonic in the value. E8M0 scale:
+// X = 2^(code - 127). For each block of 32 consecutive values along the
+// reduction dimension:
+//   amax = max |v_i|;  e = floor(log2 amax) - 8, clamped to [-127, 127]
+//   (8: the exponent of E4M3's largest normal); an all-zero block takes -127;
+//   q_i = E4M3(v_i / 2^e): nearest, ties to even; magnitudes above 448
+//   clamp to 448 (the only finite choice: 480 would be the NaN code).
+// ---------------------------------------------------------------------------
+namespace {
+
+double e4m3_value(uint8_t c) {
+  const int E = (c >> 3) & 15, M = c & 7;
+  if (E == 15 && M == 7) return std::nan("");
+  const double mag = E == 0 ? std::ldexp(static_cast<double>(M), -9)
+                            : std::ldexp(static_cast<double>(8 + M), E - 10);
+  return (c & 0x80) ? -mag : mag;
+}
+
+uint8_t e4m3_encode(double v) {
+  const uint8_t sign = std::signbit(v) ? 0x80 : 0x00;
+  if (std::isnan(v)) return sign | 0x7F;
+  const double a = std::fabs(v);
+  if (!(a < 464.0)) return sign | 0x7E;   // 448: saturate (ties at 464 go to even 448)
+  if (a < std::ldexp(1.0, -6)) {          // subnormal: code = value / 2^-9 (0..8, 8 = 2^-6)
+    const double m = std::nearbyint(std::ldexp(a, 9));
+    return sign | static_cast<uint8_t>(m);
+  }
+  int x;
+  std::frexp(a, &x);                      // a = f * 2^x, 0.5 <= f < 1: floor(log2 a) = x - 1
+  const int e = x - 1;
+  double m = std::nearbyint(std::ldexp(a, 3 - e));  // 8..16 units of 2^(e-3)
+  int ee = e;
+  if (m == 16.0) {
+    m = 8.0;
+    ++ee;
+  }
+  int code = ((ee + 7) << 3) | (static_cast<int>(m) - 8);
+  if (code > 0x7E) code = 0x7E;
+  return sign | static_cast<uint8_t>(code);
+}
+
+}  // namespace
+
+extern "C" {
+
+double oracle_e4m3_value(uint8_t c) { return e4m3_value(c); }
+uint8_t oracle_e4m3_encode(double v) { return e4m3_encode(v); }
+
+// MX quantisation of n rows of K values (K a multiple of 32), blocks along
+// the row: q [n, K] E4M3 codes, scale [n, K/32] E8M0 codes.
+void oracle_mx_quantize(const double* v, int64_t n, int32_t K, uint8_t* q, uint8_t* scale) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < n; ++r) {
+    for (int32_t b = 0; b < K / 32; ++b) {
+      const double* blk = v + r * K + b * 32;
+      double amax = 0.0;
+      for (int i = 0; i < 32; ++i) amax = std::max(amax, std::fabs(blk[i]));
+      int e = -127;
+      if (amax > 0.0) {
+        int x;
+        std::frexp(amax, &x);
+        e = std::min(127, std::max(-127, x - 1 - 8));
+      }
+      scale[r * (K / 32) + b] = static_cast<uint8_t>(e + 127);
+      for (int i = 0; i < 32; ++i) q[r * K + b * 32 + i] = e4m3_encode(std::ldexp(blk[i], -e));
+    }
+  }
+}
+
+// The values the quantised rows stand for: q * 2^(scale - 127).
+void oracle_mx_dequantize(const uint8_t* q, const uint8_t* scale, int64_t n, int32_t K,
+                          double* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < n; ++r)
+    for (int32_t i = 0; i < K; ++i)
+      out[r * K + i] = std::ldexp(e4m3_value(q[r * K + i]), scale[r * (K / 32) + i / 32] - 127);
+}
+
+}  // extern "C"
+
