@@ -345,6 +345,31 @@ def run_ours(args):
         torch.cuda.synchronize()
         mb_row = t0e.elapsed_time(t1e)
 
+    # the MXFP8 building block: the pull dispatch with the MX quantisation fused
+    mx = None
+    if not args.no_mxfp8 and mb == 0:
+        ids_mx = torch.empty((w.n_tokens, w.k), dtype=torch.int32, device=dev)
+        gates_mx = torch.empty((w.n_tokens, w.k), dtype=torch.float32, device=dev)
+        moe.moe_route_topk(lg, ids_mx, gates_mx, sh)
+        bmx = moe.alloc_schedule_outputs(sh, device=dev)
+        moe.moe_schedule(ids_mx, bmx["phi"], bmx["offsets"], bmx["counts"], bmx["route_row"],
+                         bmx["ws"], bmx["dev_status"], sh)
+        rm = moe.rows_max(sh)
+        xq = torch.empty((rm, w.H), dtype=torch.uint8, device=dev)
+        xs = torch.empty((rm, w.H // 32), dtype=torch.uint8, device=dev)
+        for _ in range(args.warmup):
+            moe.moe_dispatch_mxfp8(x, bmx["phi"], bmx["offsets"], xq, xs, bmx["dev_status"], sh)
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        m0.record()
+        for _ in range(args.steps):
+            moe.moe_dispatch_mxfp8(x, bmx["phi"], bmx["offsets"], xq, xs, bmx["dev_status"], sh)
+        m1.record()
+        torch.cuda.synchronize()
+        if int(bmx["dev_status"].item()) != 0:
+            raise RuntimeError(f"device status {int(bmx['dev_status'].item())} in the MX dispatch")
+        mx = dict(ms=m0.elapsed_time(m1) / args.steps, rows=int(bmx["offsets"][-1].item()))
+        del xq, xs, bmx
+
     # end to end through the host-buffer entry: H2D of logits and x, the layer,
     # D2H of out; each call's input copy overlaps the previous call's compute
     # and its output copy the next call's compute (the async-output entry)
@@ -492,6 +517,13 @@ def run_ours(args):
                                      "ms_per_step": mb_row / args.steps,
                                      "value": w.n_tokens * world * args.steps / (mb_row / 1e3),
                                      "unit": "tokens/s"}
+        if mx:
+            mbytes = w.n_routes * w.H * 2 + mx["rows"] * (w.H + w.H // 32)
+            gbs = mbytes / (mx["ms"] / 1e3) / 1e9
+            line["mxfp8"] = {"dispatch_mxfp8": {"ms": mx["ms"], "bytes": mbytes, "gbs": gbs,
+                                                "frac_hbm": gbs / peaks["hbm"]},
+                             "note": "pull dispatch with the MX (E4M3, E8M0 per 32) "
+                                     "quantisation fused; block-scaled expert GEMMs not built"}
         if bwd:
             bst = stage_rooflines(bwd["stages"], backward_work(w, rows_used), peaks)
             top = max(bst, key=lambda n: bst[n]["ms"])
@@ -601,6 +633,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-mxfp8", action="store_true")
     ap.add_argument("--bwd-steps", type=int, default=10)
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-row-budget", type=float, default=3.0)

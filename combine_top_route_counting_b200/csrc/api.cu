@@ -734,6 +734,27 @@ moe_status_t moe_layer_forward_host_async(const float* logits_host, const uint16
                                        static_cast<cudaEvent_t>(out_ready)));
 }
 
+moe_status_t moe_mx_quantize_rows(const uint16_t* src, int64_t n_rows, int32_t K, uint8_t* q,
+                                  uint8_t* scale, void* stream) {
+  if (n_rows < 0 || K < 32 || K % 32 != 0) return MOE_INVALID_ARG;
+  if (n_rows > 0 && (!src || !q || !scale)) return MOE_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(q)) return MOE_INVALID_ARG;
+  return from_cuda(launch_mx_quantize_rows(src, n_rows, K, q, scale,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_dispatch_mxfp8(const uint16_t* x, const int32_t* phi, const int32_t* offsets,
+                                uint8_t* xq, uint8_t* xs, int32_t* dev_status,
+                                const moe_shape_t* shape, void* stream) {
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->H < 32 || shape->H % 32 != 0) return MOE_UNSUPPORTED_SHAPE;
+  if (!phi || !offsets || !xq || !xs || !dev_status || (shape->N > 0 && !x)) return MOE_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(phi) || !aligned16(xq)) return MOE_INVALID_ARG;
+  return from_cuda(launch_dispatch_mxfp8(x, phi, offsets, xq, xs, *shape, rows_max_of(shape),
+                                         dev_status, static_cast<cudaStream_t>(stream)));
+}
+
 int64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 moe_status_t moe_selftest_bounded_wait(int32_t* dev_status, int64_t timeout_ns, void* stream) {

@@ -104,6 +104,15 @@ cudaError_t launch_expert_ffn_wgrad(const uint16_t* xg, const uint16_t* dys, con
                                     const moe_shape_t& sh, int64_t rows_max, int32_t* dev_status,
                                     cudaStream_t s, cudaEvent_t ev_mid);
 
+// ---------------------------------------------------------------- MXFP8
+// MX quantisation (E4M3 codes, one E8M0 scale per 32 values along the row).
+cudaError_t launch_mx_quantize_rows(const uint16_t* src, int64_t n_rows, int32_t K, uint8_t* q,
+                                    uint8_t* scale, cudaStream_t s);
+// The pull dispatch with the MX quantisation fused: xq/xs rows of the gathered tokens.
+cudaError_t launch_dispatch_mxfp8(const uint16_t* x, const int32_t* phi, const int32_t* offsets,
+                                  uint8_t* xq, uint8_t* xs, const moe_shape_t& sh,
+                                  int64_t rows_max, int32_t* dev_status, cudaStream_t s);
+
 // Failure-detection self test (bounded wait on an mbarrier nothing completes).
 cudaError_t launch_selftest_wait(int32_t* dev_status, int64_t timeout_ns, cudaStream_t s);
 

@@ -1,0 +1,151 @@
+// MXFP8 quantisation of bf16 rows, alone or fused into the pull dispatch
+// ("Mixture-of-Kittens: A MoE Megakernel for GB300 NVL72", section 5: MXFP8
+// routed experts with the quantisation fused into the dispatch; the OCP
+// Microscaling formats, MXFP8 with E4M3 elements).
+//
+// For each block of 32 consecutive values of a row: amax = max |v|; the
+// shared exponent e = floor(log2 amax) - 8 (8: the exponent of E4M3's largest
+// normal, 448), clamped to [-127, 127], -127 for an all-zero block; the scale
+// is stored as the E8M0 code e + 127 and each element as E4M3(v * 2^-e),
+// nearest-even with magnitudes above 448 clamped to 448 (CUDA's saturating
+// fp32 -> E4M3 conversion). floor(log2 amax) comes straight from the bf16
+// exponent bits (subnormal inputs included), and v * 2^-e is exact, so the
+// codes depend on nothing but the inputs.
+//
+// One warp per row; lane j quantises blocks j, j+32, ...: its 64 input bytes
+// and 32 output bytes are contiguous with its neighbours', so every load and
+// store of the warp is coalesced. HBM-bound: 2 bytes read and 1 + 1/32 bytes
+// written per element.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "internal.cuh"
+
+namespace moe {
+namespace {
+
+// floor(log2 |v|) of a non-zero bf16 magnitude (sign bit clear), exactly.
+__device__ __forceinline__ int bf16_floor_log2(uint32_t mag) {
+  const int ef = static_cast<int>(mag >> 7);
+  if (ef != 0) return ef - 127;
+  return -134 + (32 - __clz(mag));  // subnormal: 2^-133 * mantissa
+}
+
+// One 32-element block: 4 x 16 bytes of bf16 in, 2 x 16 bytes of E4M3 codes
+// and one E8M0 scale code out.
+__device__ __forceinline__ void mx_block(const uint4 (&in)[4], uint4 (&out)[2], uint8_t& scale) {
+  uint32_t amax = 0;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const uint32_t w[4] = {in[v].x, in[v].y, in[v].z, in[v].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      amax = max(amax, w[i] & 0x7FFFu);
+      amax = max(amax, (w[i] >> 16) & 0x7FFFu);
+    }
+  }
+  int e = -127;
+  if (amax != 0) e = max(-127, min(127, bf16_floor_log2(amax) - 8));
+  scale = static_cast<uint8_t>(e + 127);
+  uint32_t codes[8];
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const uint32_t w[4] = {in[v].x, in[v].y, in[v].z, in[v].w};
+#pragma unroll
+    for (int i = 0; i < 4; i += 2) {
+      uint32_t packed = 0;
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {  // 4 bf16 values -> 4 code bytes
+        const uint32_t word = w[i + (h >> 1)];
+        const float f = __uint_as_float((h & 1) ? (word & 0xFFFF0000u) : (word << 16));
+        const __nv_fp8_storage_t c =
+            __nv_cvt_float_to_fp8(ldexpf(f, -e), __NV_SATFINITE, __NV_E4M3);
+        packed |= static_cast<uint32_t>(c) << (8 * h);
+      }
+      codes[v * 2 + i / 2] = packed;
+    }
+  }
+  out[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+  out[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+}
+
+// GATHER: row r of the output comes from token phi[r] of x (pad rows: zeros,
+// scale code 0); otherwise row r of src.
+template <bool GATHER>
+__global__ void __launch_bounds__(256) mx_rows_kernel(const uint4* __restrict__ src,
+                                                      const int2* __restrict__ phi,
+                                                      const int32_t* __restrict__ offsets,
+                                                      uint4* __restrict__ q, uint8_t* __restrict__ sc,
+                                                      int64_t n_rows, int K, int P, int N, int E,
+                                                      int64_t rows_max, int32_t* dev_status) {
+  int64_t rows = n_rows;
+  if (GATHER) {
+    rows = __ldg(offsets + E);
+    if (rows < 0 || rows > rows_max) {
+      if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(dev_status, MOE_DEV_BAD_SCHEDULE);
+      return;
+    }
+  }
+  const int lane = threadIdx.x & 31;
+  const int nblk = K / 32;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * 8;
+  int bad = 0;
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); row < rows;
+       row += nwarps) {
+    int64_t srow = row;
+    bool zero = false;
+    if (GATHER) {
+      const int2 e = __ldg(phi + row);
+      const bool ok = e.x >= 0 && e.x < P && e.y >= 0 && e.y < N;
+      if (!ok && (e.x >= 0 || e.y != -1)) bad = 1;  // (-1,-1) is padding
+      zero = !ok;
+      srow = ok ? static_cast<int64_t>(e.x) * N + e.y : 0;
+    }
+    const uint4* s = src + srow * (K / 8);
+    uint4* qrow = q + row * (K / 16);
+    uint8_t* srow_sc = sc + row * nblk;
+    for (int b = lane; b < nblk; b += 32) {
+      uint4 in[4];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) in[v] = zero ? make_uint4(0, 0, 0, 0) : __ldg(s + b * 4 + v);
+      uint4 out[2];
+      uint8_t scale;
+      mx_block(in, out, scale);
+      qrow[b * 2] = out[0];
+      qrow[b * 2 + 1] = out[1];
+      srow_sc[b] = scale;
+    }
+  }
+  if (bad) atomicOr(dev_status, MOE_DEV_BAD_SCHEDULE);
+}
+
+int grid_for(int64_t rows) {
+  const int64_t want = (rows + 7) / 8;
+  const int64_t cap = static_cast<int64_t>(device_sm_count()) * 8;
+  return static_cast<int>(want < cap ? want : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_mx_quantize_rows(const uint16_t* src, int64_t n_rows, int32_t K, uint8_t* q,
+                                    uint8_t* scale, cudaStream_t s) {
+  if (n_rows <= 0) return cudaSuccess;
+  mx_rows_kernel<false><<<grid_for(n_rows), 256, 0, s>>>(
+      reinterpret_cast<const uint4*>(src), nullptr, nullptr, reinterpret_cast<uint4*>(q), scale,
+      n_rows, K, 0, 0, 0, 0, nullptr);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_mxfp8(const uint16_t* x, const int32_t* phi, const int32_t* offsets,
+                                  uint8_t* xq, uint8_t* xs, const moe_shape_t& sh,
+                                  int64_t rows_max, int32_t* dev_status, cudaStream_t s) {
+  if (rows_max <= 0) return cudaSuccess;
+  mx_rows_kernel<true><<<grid_for(rows_max), 256, 0, s>>>(
+      reinterpret_cast<const uint4*>(x), reinterpret_cast<const int2*>(phi), offsets,
+      reinterpret_cast<uint4*>(xq), xs, rows_max, sh.H, sh.P, sh.N, sh.E, rows_max, dev_status);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

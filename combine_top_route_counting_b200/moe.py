@@ -86,6 +86,8 @@ _SIGS = {
     "moe_expert_ffn_wgrad": ([_vp] * 10 + [ctypes.POINTER(Shape), _vp], ctypes.c_int),
     "moe_layer_backward": ([_vp] * 10 + [ctypes.c_size_t, _vp, ctypes.POINTER(Shape), _vp,
                                          ctypes.POINTER(_vp)], ctypes.c_int),
+    "moe_mx_quantize_rows": ([_vp, ctypes.c_int64, ctypes.c_int32, _vp, _vp, _vp], ctypes.c_int),
+    "moe_dispatch_mxfp8": ([_vp] * 6 + [ctypes.POINTER(Shape), _vp], ctypes.c_int),
     "moe_launch_count": ([], ctypes.c_int64),
     "moe_selftest_bounded_wait": ([_vp, ctypes.c_int64, _vp], ctypes.c_int),
 }
@@ -393,6 +395,23 @@ def moe_layer_forward_host_async(logits_host, x_host, W1, W3, W2, out_host, ws, 
         _ptr(out_host, torch.bfloat16, "out_host", device=False), int(minibatch_tokens),
         _ptr(ws, torch.uint8, "ws"), ws.numel(), _ptr(dev_status, torch.int32, "dev_status"),
         ctypes.byref(sh), _stream(stream), ctypes.c_void_p(ev)), "moe_layer_forward_host_async")
+
+
+# ---------------------------------------------------------------- MXFP8
+def moe_mx_quantize_rows(src, q, scale, stream=None):
+    """src bf16 [n, K] -> q uint8 [n, K] E4M3 codes, scale uint8 [n, K/32] E8M0 codes."""
+    n, K = src.shape
+    _check(load().moe_mx_quantize_rows(_ptr(src, torch.bfloat16, "src"), n, K,
+                                       _ptr(q, torch.uint8, "q"), _ptr(scale, torch.uint8, "scale"),
+                                       _stream(stream)), "moe_mx_quantize_rows")
+
+
+def moe_dispatch_mxfp8(x, phi, offsets, xq, xs, dev_status, sh: Shape, stream=None):
+    _check(load().moe_dispatch_mxfp8(_ptr(x, torch.bfloat16, "x"), _ptr(phi, torch.int32, "phi"),
+                                     _ptr(offsets, torch.int32, "offsets"),
+                                     _ptr(xq, torch.uint8, "xq"), _ptr(xs, torch.uint8, "xs"),
+                                     _ptr(dev_status, torch.int32, "dev_status"), ctypes.byref(sh),
+                                     _stream(stream)), "moe_dispatch_mxfp8")
 
 
 def moe_selftest_bounded_wait(dev_status, timeout_ns: int, stream=None):

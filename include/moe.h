@@ -392,6 +392,34 @@ moe_status_t moe_layer_backward(const uint16_t* dout, const uint16_t* W1, const 
                                 int32_t* dev_status, const moe_shape_t* shape, void* stream,
                                 void* const* stage_events);
 
+/* ------------------------------------------------------------------------
+ * MXFP8 ("Mixture-of-Kittens", section 5: MXFP8 routed experts, with the
+ * quantisation fused into the dispatch; the OCP Microscaling formats, MXFP8
+ * with E4M3 elements). Building blocks of an MXFP8 expert path: the
+ * block-scaled expert GEMMs that would consume them are not part of this
+ * library yet.
+ *
+ * For every block of 32 consecutive values of a row: amax = max |v|, the
+ * shared exponent e = floor(log2 amax) - 8 clamped to [-127, 127] (-127 for
+ * an all-zero block), the scale stored as the E8M0 code e + 127 and each
+ * element as the E4M3 code of v * 2^-e (nearest, ties to even, magnitudes
+ * above 448 clamped to 448). The codes depend only on the inputs.
+ * ------------------------------------------------------------------------ */
+
+/* Rows of bf16 to MXFP8: src [n_rows, K] (K a multiple of 32) -> q uint8
+ * [n_rows, K] E4M3 codes and scale uint8 [n_rows, K/32] E8M0 codes. */
+moe_status_t moe_mx_quantize_rows(const uint16_t* src, int64_t n_rows, int32_t K, uint8_t* q,
+                                  uint8_t* scale, void* stream);
+
+/* The pull dispatch of moe_dispatch with the MXFP8 quantisation fused: row
+ * `row` of xq (uint8 [moe_rows_max, H]) and xs (uint8 [moe_rows_max, H/32])
+ * is the quantised token x[src_rank*N + src_idx], (src_rank, src_idx) =
+ * phi[row]; padding rows are zero codes with scale code 0. H % 32 == 0.
+ * Errors as moe_dispatch. */
+moe_status_t moe_dispatch_mxfp8(const uint16_t* x, const int32_t* phi, const int32_t* offsets,
+                                uint8_t* xq, uint8_t* xs, int32_t* dev_status,
+                                const moe_shape_t* shape, void* stream);
+
 /* Number of kernels this library has launched in the calling process. */
 int64_t moe_launch_count(void);
 
