@@ -8,7 +8,7 @@
 // normal, 448), clamped to [-127, 127], -127 for an all-zero block; the scale
 // is stored as the E8M0 code e + 127 and each element as E4M3(v * 2^-e),
 // nearest-even with magnitudes above 448 clamped to 448 (CUDA's saturating
-// fp32 -> E4M3 conversion). floor(log2 amax) comes straight from the bf16
+// fp32 -> E4M3 pair conversion). floor(log2 amax) comes straight from the bf16
 // exponent bits (subnormal inputs included), and v * 2^-e is exact, so the
 // codes depend on nothing but the inputs.
 //
@@ -47,6 +47,10 @@ __device__ __forceinline__ void mx_block(const uint4 (&in)[4], uint4 (&out)[2], 
   int e = -127;
   if (amax != 0) e = max(-127, min(127, bf16_floor_log2(amax) - 8));
   scale = static_cast<uint8_t>(e + 127);
+  // 2^-e as a normal fp32 (bf16 magnitudes keep e <= 119); the products are
+  // exact except when they fall far below E4M3's smallest step, where the
+  // code is a signed zero either way
+  const float inv = __int_as_float((127 - e) << 23);
   uint32_t codes[8];
 #pragma unroll
   for (int v = 0; v < 4; ++v) {
@@ -55,12 +59,12 @@ __device__ __forceinline__ void mx_block(const uint4 (&in)[4], uint4 (&out)[2], 
     for (int i = 0; i < 4; i += 2) {
       uint32_t packed = 0;
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {  // 4 bf16 values -> 4 code bytes
-        const uint32_t word = w[i + (h >> 1)];
-        const float f = __uint_as_float((h & 1) ? (word & 0xFFFF0000u) : (word << 16));
-        const __nv_fp8_storage_t c =
-            __nv_cvt_float_to_fp8(ldexpf(f, -e), __NV_SATFINITE, __NV_E4M3);
-        packed |= static_cast<uint32_t>(c) << (8 * h);
+      for (int h = 0; h < 2; ++h) {  // one bf16 pair -> two code bytes (low element first)
+        const uint32_t word = w[i + h];
+        const float2 f = make_float2(__uint_as_float(word << 16) * inv,
+                                     __uint_as_float(word & 0xFFFF0000u) * inv);
+        const __nv_fp8x2_storage_t c2 = __nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, __NV_E4M3);
+        packed |= static_cast<uint32_t>(c2) << (16 * h);
       }
       codes[v * 2 + i / 2] = packed;
     }
