@@ -125,3 +125,17 @@ def test_host_async_entry_needs_an_event(lib):
     args = [p] * 6 + [0, p, 1 << 40, p, ctypes.byref(sh), None]
     assert lib.moe_layer_forward_host_async(*args, None) == 1
     assert lib.moe_layer_forward_host_async(*args[:8], 16, p, ctypes.byref(sh), None, p) == 3
+
+
+def test_mx_entry_points_argument_errors(lib):
+    L = lib
+    p = ctypes.c_void_p(256)
+    assert L.moe_mx_quantize_rows(p, 4, 48, p, p, None) == 1       # K % 32 != 0
+    assert L.moe_mx_quantize_rows(p, -1, 64, p, p, None) == 1      # negative rows
+    assert L.moe_mx_quantize_rows(None, 4, 64, p, p, None) == 1    # null source
+    assert L.moe_mx_quantize_rows(ctypes.c_void_p(264), 4, 64, p, p, None) == 1  # misaligned
+    assert L.moe_mx_quantize_rows(None, 0, 64, None, None, None) == 0            # nothing to do
+    sh = moe.shape(1, 16, 8, 2, 48, 128)                           # H % 32 != 0
+    assert L.moe_dispatch_mxfp8(p, p, p, p, p, p, ctypes.byref(sh), None) == 2
+    sh = moe.shape(1, 16, 8, 2, 256, 128)
+    assert L.moe_dispatch_mxfp8(p, None, p, p, p, p, ctypes.byref(sh), None) == 1
