@@ -12,7 +12,6 @@ numbers). The design notes list them; no function is left unpinned.
 from __future__ import annotations
 
 import ctypes
-import os
 
 import numpy as np
 

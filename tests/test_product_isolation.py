@@ -6,7 +6,6 @@ the binding must fail loudly when the CUDA library is missing instead of
 computing anything itself.
 """
 import ast
-import ctypes
 import os
 import re
 
