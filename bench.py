@@ -270,6 +270,84 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- our arm
+def assemble_line(args, w, world, ms, stage_ms, launches, e2e, e2e_mb, mb, mb_row, mx, bwd,
+                  rows_used, peaks):
+    """The bench's JSON line (without clocks and cpu_baseline) from the measured
+    times: ms for args.steps layer steps, stage_ms {stage: ms}, and the
+    optional e2e / minibatch / MXFP8 / backward legs (None when not run)."""
+    tokens = w.n_tokens * world * args.steps
+    value = tokens / (ms / 1e3)
+    work = algorithmic_work(w, rows_used, w.n_routes)
+    stages = stage_rooflines(stage_ms, work, peaks)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": workload_desc(w), "tokens_per_step_per_gpu": w.n_tokens,
+                   "minibatch_tokens": mb or w.N, "parallelism": f"replicas x{world}",
+                   "rows_padded": rows_used,
+                   "l2": "inputs larger than L2: 33.8 GB of expert weights and 14 GB of "
+                         "fp32 expert outputs stream through HBM every step",
+                   "weights": "random-init bf16 N(0,0.02)"},
+    }
+    if stage_ms:
+        line["phi_build_us"] = stage_ms["schedule"] * 1e3
+        g1 = stages["ffn_gemm1"]
+        line["roofline"] = {
+            "kernel": "ffn_gemm_kernel<0> (GEMM1 + SwiGLU)", "bound": "tensor",
+            "achieved": g1["tflops"], "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
+            "frac": g1["tflops"] / peaks["bf16_sus"],
+            "peak_note": f"dense bf16, sustained, of {peaks['source']}",
+            "traffic": gemm1_traffic(w.n_routes),
+        }
+        line["stages"] = stages
+    line["gpu_launches"] = launches
+    if e2e:
+        line["e2e"] = {"value": w.n_tokens * world * args.e2e_steps / (e2e["ms"] / 1e3),
+                       "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
+                       "d2h_bytes_per_step": e2e["d2h"],
+                       "api": "moe_layer_forward_host_async (pinned host logits/x/out; "
+                              "the output copy completes on an event, off the compute "
+                              "stream)",
+                       "transfer_minibatch_tokens": e2e_mb or w.N, "steps": args.e2e_steps,
+                       "ms_per_step": e2e["ms"] / args.e2e_steps}
+    if mb_row is not None:
+        line["minibatch_row"] = {"minibatch_tokens": w.minibatch,
+                                 "ms_per_step": mb_row / args.steps,
+                                 "value": w.n_tokens * world * args.steps / (mb_row / 1e3),
+                                 "unit": "tokens/s"}
+    if mx:
+        mbytes = w.n_routes * w.H * 2 + mx["rows"] * (w.H + w.H // 32)
+        gbs = mbytes / (mx["ms"] / 1e3) / 1e9
+        line["mxfp8"] = {"dispatch_mxfp8": {"ms": mx["ms"], "bytes": mbytes, "gbs": gbs,
+                                            "frac_hbm": gbs / peaks["hbm"]},
+                         "note": "pull dispatch with the MX (E4M3, E8M0 per 32) "
+                                 "quantisation fused; block-scaled expert GEMMs not built"}
+    if bwd:
+        bst = stage_rooflines(bwd["stages"], backward_work(w, rows_used), peaks)
+        top = max(bst, key=lambda n: bst[n]["ms"])
+        tokens_b = w.n_tokens * world * args.bwd_steps
+        line["backward"] = {
+            "value": w.n_tokens * world / (bwd["bwd_ms"] / 1e3), "unit": "tokens/s",
+            "ms_per_step": bwd["bwd_ms"],
+            "train_step": {"value": tokens_b / (bwd["train_ms"] / 1e3), "unit": "tokens/s",
+                           "ms_per_step": bwd["train_ms"] / args.bwd_steps,
+                           "what": "moe_layer_forward_train + moe_layer_backward",
+                           "gpu_launches": bwd["launches"] // args.bwd_steps},
+            "steps": args.bwd_steps, "warmup": args.warmup,
+            "stages": bst,
+            "roofline": {"kernel": top, "bound": "tensor" if "tflops" in bst[top] else "hbm",
+                         "achieved": bst[top].get("tflops", bst[top].get("gbs")),
+                         "peak": peaks["bf16_sus"] if "tflops" in bst[top] else peaks["hbm"],
+                         "unit": "TFLOP/s" if "tflops" in bst[top] else "GB/s",
+                         "frac": bst[top].get("frac_bf16", bst[top].get("frac_hbm")),
+                         "traffic": wgrad13_traffic(w.n_routes) if top == "wgrad_w13" else None},
+            "dout": "bf16 N(0,1), seeded",
+        }
+    return line
+
+
 def run_ours(args):
     import torch
 
@@ -473,78 +551,10 @@ def run_ours(args):
         e2e["ms"] = vec[-1]
 
     if rank == 0:
-        tokens = w.n_tokens * world * args.steps
-        value = tokens / (ms / 1e3)
         peaks = load_peaks()
         rows_used = schedule_rows(moe, w, sh, lg)
-        work = algorithmic_work(w, rows_used, w.n_routes)
-        stages = stage_rooflines(stage_ms, work, peaks)
-        line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
-            "config": {"workload": workload_desc(w), "tokens_per_step_per_gpu": w.n_tokens,
-                       "minibatch_tokens": mb or w.N, "parallelism": f"replicas x{world}",
-                       "rows_padded": rows_used,
-                       "l2": "inputs larger than L2: 33.8 GB of expert weights and 14 GB of "
-                             "fp32 expert outputs stream through HBM every step",
-                       "weights": "random-init bf16 N(0,0.02)"},
-        }
-        if stage_ms:
-            line["phi_build_us"] = stage_ms["schedule"] * 1e3
-            g1 = stages["ffn_gemm1"]
-            line["roofline"] = {
-                "kernel": "ffn_gemm_kernel<0> (GEMM1 + SwiGLU)", "bound": "tensor",
-                "achieved": g1["tflops"], "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
-                "frac": g1["tflops"] / peaks["bf16_sus"],
-                "peak_note": f"dense bf16, sustained, of {peaks['source']}",
-                "traffic": gemm1_traffic(w.n_routes),
-            }
-            line["stages"] = stages
-        line["gpu_launches"] = launches
-        if e2e:
-            line["e2e"] = {"value": w.n_tokens * world * args.e2e_steps / (e2e["ms"] / 1e3),
-                           "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
-                           "d2h_bytes_per_step": e2e["d2h"],
-                           "api": "moe_layer_forward_host_async (pinned host logits/x/out; "
-                                  "the output copy completes on an event, off the compute "
-                                  "stream)",
-                           "transfer_minibatch_tokens": e2e_mb or w.N, "steps": args.e2e_steps,
-                           "ms_per_step": e2e["ms"] / args.e2e_steps}
-        if mb_row is not None:
-            line["minibatch_row"] = {"minibatch_tokens": w.minibatch,
-                                     "ms_per_step": mb_row / args.steps,
-                                     "value": w.n_tokens * world * args.steps / (mb_row / 1e3),
-                                     "unit": "tokens/s"}
-        if mx:
-            mbytes = w.n_routes * w.H * 2 + mx["rows"] * (w.H + w.H // 32)
-            gbs = mbytes / (mx["ms"] / 1e3) / 1e9
-            line["mxfp8"] = {"dispatch_mxfp8": {"ms": mx["ms"], "bytes": mbytes, "gbs": gbs,
-                                                "frac_hbm": gbs / peaks["hbm"]},
-                             "note": "pull dispatch with the MX (E4M3, E8M0 per 32) "
-                                     "quantisation fused; block-scaled expert GEMMs not built"}
-        if bwd:
-            bst = stage_rooflines(bwd["stages"], backward_work(w, rows_used), peaks)
-            top = max(bst, key=lambda n: bst[n]["ms"])
-            tokens_b = w.n_tokens * world * args.bwd_steps
-            line["backward"] = {
-                "value": w.n_tokens * world / (bwd["bwd_ms"] / 1e3), "unit": "tokens/s",
-                "ms_per_step": bwd["bwd_ms"],
-                "train_step": {"value": tokens_b / (bwd["train_ms"] / 1e3), "unit": "tokens/s",
-                               "ms_per_step": bwd["train_ms"] / args.bwd_steps,
-                               "what": "moe_layer_forward_train + moe_layer_backward",
-                               "gpu_launches": bwd["launches"] // args.bwd_steps},
-                "steps": args.bwd_steps, "warmup": args.warmup,
-                "stages": bst,
-                "roofline": {"kernel": top, "bound": "tensor" if "tflops" in bst[top] else "hbm",
-                             "achieved": bst[top].get("tflops", bst[top].get("gbs")),
-                             "peak": peaks["bf16_sus"] if "tflops" in bst[top] else peaks["hbm"],
-                             "unit": "TFLOP/s" if "tflops" in bst[top] else "GB/s",
-                             "frac": bst[top].get("frac_bf16", bst[top].get("frac_hbm")),
-                             "traffic": wgrad13_traffic(w.n_routes) if top == "wgrad_w13" else None},
-                "dout": "bf16 N(0,1), seeded",
-            }
+        line = assemble_line(args, w, world, ms, stage_ms, launches, e2e, e2e_mb, mb, mb_row, mx,
+                             bwd, rows_used, peaks)
         line["clocks"] = clk
         if world == 1 and not args.no_cpu_baseline:
             r = oracle_sample(w, lg_cpu, x_cpu, W, row_budget_s=args.cpu_budget)

@@ -78,3 +78,45 @@ def test_algorithmic_work_kimi():
     assert wk["ffn_gemm1"]["flops"] + wk["ffn_gemm2"]["flops"] == 6 * w.n_routes * w.H * w.I
     assert abs(wk["ffn_gemm1"]["flops"] + wk["ffn_gemm2"]["flops"] - 4.04e13) / 4.04e13 < 0.01
     assert wk["dispatch"]["bytes"] == w.n_routes * w.H * 2 + 492288 * w.H * 2
+
+
+def test_assembled_line_meets_the_contract():
+    """The JSON line bench.py prints, assembled from synthetic measurements of
+    every leg: the contract's keys and types, throughput arithmetic, and both
+    rooflines (so a slip in the post-processing cannot cost a GPU run's line)."""
+    import argparse
+    import json
+
+    sys.path.insert(0, ROOT)
+    import bench
+    from combine_top_route_counting_b200 import inputs, moe
+
+    args = argparse.Namespace(steps=20, warmup=3, e2e_steps=20, bwd_steps=10)
+    w = inputs.WORKLOADS["kimi"]
+    stage_ms = dict(zip(moe.STAGES, (0.065, 0.053, 2.39, 21.6, 13.4, 2.21)))
+    bwd = dict(train_ms=1232.0, bwd_ms=79.8, launches=160,
+               stages=dict(zip(moe.BWD_STAGES, (2.45, 13.25, 23.79, 2.22, 0.063, 12.68, 25.38))))
+    e2e = dict(ms=830.0, h2d=910163968, d2h=822083584, chk=0.0)
+    mx = dict(ms=1.94, rows=492544)
+    peaks = bench.load_peaks()
+    line = bench.assemble_line(args, w, 1, 794.0, stage_ms, 180, e2e, 0, 0, 1188.0, mx, bwd,
+                               492544, peaks)
+    line = json.loads(json.dumps(line))
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "roofline", "e2e", "gpu_launches"):
+        assert key in line, key
+    assert line["value"] == pytest.approx(w.n_tokens * 20 / 0.794)
+    assert line["ms_per_step"] == pytest.approx(39.7)
+    assert line["config"]["workload"].startswith("kimi")
+    r = line["roofline"]
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["achieved"] == pytest.approx(2 * w.n_routes * w.H * 2 * w.I / 21.6e-3 / 1e12)
+    assert r["frac"] == pytest.approx(r["achieved"] / r["peak"])
+    assert set(line["e2e"]) >= {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"}
+    assert line["e2e"]["value"] == pytest.approx(w.n_tokens * 20 / 0.830)
+    b = line["backward"]
+    assert b["roofline"]["kernel"] == "wgrad_w13" and b["roofline"]["bound"] == "tensor"
+    assert b["value"] == pytest.approx(w.n_tokens / 0.0798)
+    assert line["mxfp8"]["dispatch_mxfp8"]["frac_hbm"] > 0
+    assert line["phi_build_us"] == pytest.approx(53.0)
