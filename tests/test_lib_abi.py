@@ -139,3 +139,36 @@ def test_mx_entry_points_argument_errors(lib):
     assert L.moe_dispatch_mxfp8(p, p, p, p, p, p, ctypes.byref(sh), None) == 2
     sh = moe.shape(1, 16, 8, 2, 256, 128)
     assert L.moe_dispatch_mxfp8(p, None, p, p, p, p, ctypes.byref(sh), None) == 1
+
+
+def test_size_queries_hold_their_invariants_on_random_shapes(lib):
+    """Host-only size queries over random shapes (hypothesis): no crash, -1/0 for
+    unsupported shapes, and rows_max / workspace bounds where supported."""
+    from hypothesis import given, settings
+    from hypothesis import strategies as st
+
+    @settings(max_examples=300, deadline=None)
+    @given(P=st.integers(-2, 70), N=st.integers(-5, 20000), E=st.integers(-1, 1100),
+           k=st.integers(-1, 20), H=st.sampled_from([0, 128, 256, 300, 512, 7168]),
+           I=st.sampled_from([0, 64, 128, 256, 384, 2048]), pad=st.sampled_from([0, 1, 64, 128, 256, 512]))
+    def check(P, N, E, k, H, I, pad):
+        sh = moe.shape(P, N, E, k, H, I, pad)
+        rm = moe.rows_max(sh)
+        ok = 1 <= P <= 64 and N >= 0 and 1 <= E <= 1024 and 1 <= k <= min(E, 16) and 1 <= pad <= 65536
+        if not ok:
+            assert rm == -1 and moe.layer_workspace_bytes(sh) == 0
+            return
+        assert rm >= P * N * k and rm % 256 == 0
+        assert rm <= P * N * k + E * (pad - 1) + 255
+        ffn_ok = H >= 256 and H % 256 == 0 and I >= 128 and I % 128 == 0 and pad % 128 == 0
+        ws = moe.layer_workspace_bytes(sh)
+        assert (ws > 0) == ffn_ok
+        if ffn_ok:
+            assert ws >= rm * (H * 2 + I * 2 + H * 4)
+            assert moe.layer_host_workspace_bytes(sh) > ws
+            tw = moe.train_workspace_bytes(sh)
+            assert (tw > 0) == (I % 256 == 0 and pad % 256 == 0)
+            if tw:
+                assert tw > ws
+
+    check()
