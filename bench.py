@@ -536,8 +536,11 @@ def run_ours(args):
     bnames = list(bwd["stages"]) if bwd else []
     vec = ([ms] + [stage_ms[n] for n in names] + ([e2e["ms"]] if e2e else []) +
            ([mb_row] if mb_row is not None else []) +
-           ([bwd["train_ms"], bwd["bwd_ms"]] + [bwd["stages"][n] for n in bnames] if bwd else []))
+           ([bwd["train_ms"], bwd["bwd_ms"]] + [bwd["stages"][n] for n in bnames] if bwd else []) +
+           ([mx["ms"]] if mx else []))
     vec = reduce_max(vec, ready, device=dev)
+    if mx:
+        mx["ms"] = vec.pop()
     if bwd:
         nb = 2 + len(bnames)
         bvec, vec = vec[-nb:], vec[:-nb]
