@@ -60,6 +60,20 @@ moe_status_t check_bwd_shape(const moe_shape_t* s) {
   return MOE_OK;
 }
 
+// Extra limits of the MXFP8 expert FFN (block-scaled CTA-pair tiles of 256
+// rows; GEMM1 output blocks of 128 h columns, GEMM2 of 256 y columns; 128 K
+// values per pipeline stage).
+moe_status_t check_mx_shape(const moe_shape_t* s) {
+  moe_status_t st = check_ffn_shape(s);
+  if (st != MOE_OK) return st;
+  if (s->pad % 256 != 0) return MOE_UNSUPPORTED_SHAPE;
+  // scale-atom indices of the TMA loads are int32
+  const int64_t atoms_w = static_cast<int64_t>(s->E) * (s->I / 128) * (s->H / 128);
+  const int64_t atoms_x = rows_max_of(s) / 128 * (s->H / 128);
+  if (atoms_w >= (int64_t{1} << 31) || atoms_x >= (int64_t{1} << 31)) return MOE_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
 // Layout of the layer workspace (offsets in bytes, each kAlign-aligned).
 // The training layout keeps what the backward reads (ids, gates, route_row,
 // Phi, offsets, counts, xg, h and the pre-activations ab) and adds the
@@ -218,6 +232,55 @@ moe_status_t layer_body(const float* logits, const uint16_t* x, const uint16_t* 
     e = run_slice(b, x, W1, W3, W2, out, sl, sh, dev_status, s, ev_use, ab);
   }
   return from_cuda(e);
+}
+
+// The MXFP8 layer on device buffers. It uses the bf16 layer's workspace: the
+// E4M3 codes and tiled scales of the gathered tokens fill the xg region
+// (rows*H + rows*H/32 bytes of rows*H*2), those of h the h region.
+// ev (7 events, may be null) as moe_layer_forward.
+cudaError_t layer_body_mx(const float* logits, const uint16_t* x, const uint8_t* W1q,
+                          const uint8_t* W1s, const uint8_t* W3q, const uint8_t* W3s,
+                          const uint8_t* W2q, const uint8_t* W2s, uint16_t* out, void* ws,
+                          int32_t* dev_status, const moe_shape_t* sh, cudaStream_t s,
+                          void* const* ev) {
+  const LayerWs w = layer_ws(sh);
+  const LayerBufs b = layer_bufs(ws, w);
+  const int64_t rows_max = rows_max_of(sh);
+  uint8_t* xq = at<uint8_t>(ws, w.xg);
+  uint8_t* xs = xq + static_cast<size_t>(rows_max) * sh->H;
+  uint8_t* hq = at<uint8_t>(ws, w.h);
+  uint8_t* hs = hq + static_cast<size_t>(rows_max) * sh->I;
+  auto rec = [&](int i) -> cudaError_t {
+    return (ev && ev[i]) ? cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), s) : cudaSuccess;
+  };
+  cudaError_t e;
+  if ((e = rec(0)) != cudaSuccess) return e;
+  if ((e = launch_route_topk(logits, b.ids, b.gates, static_cast<int64_t>(sh->P) * sh->N, sh->E,
+                             sh->k, s)) != cudaSuccess)
+    return e;
+  if (sh->N == 0) {
+    for (int i = 1; i < 7; ++i)
+      if ((e = rec(i)) != cudaSuccess) return e;
+    return cudaSuccess;
+  }
+  if ((e = rec(1)) != cudaSuccess) return e;
+  if ((e = launch_schedule(b.ids, *sh, Slice{0, sh->N}, b.phi, b.offsets, b.counts, b.route_row,
+                           b.sched, dev_status, s)) != cudaSuccess)
+    return e;
+  if ((e = rec(2)) != cudaSuccess) return e;
+  if ((e = launch_dispatch_mxfp8(x, b.phi, b.offsets, xq, xs, *sh, rows_max, dev_status, s,
+                                 /*tiled=*/true)) != cudaSuccess)
+    return e;
+  if ((e = rec(3)) != cudaSuccess) return e;
+  cudaEvent_t mid = ev ? static_cast<cudaEvent_t>(ev[4]) : nullptr;
+  if ((e = launch_expert_ffn_mxfp8(xq, xs, W1q, W1s, W3q, W3s, W2q, W2s, b.offsets, b.counts, hq,
+                                   hs, b.y, *sh, rows_max, dev_status, s, mid)) != cudaSuccess)
+    return e;
+  if ((e = rec(5)) != cudaSuccess) return e;
+  if ((e = launch_combine(b.y, b.route_row, b.gates, out, *sh, Slice{0, sh->N}, rows_max,
+                          dev_status, s)) != cudaSuccess)
+    return e;
+  return rec(6);
 }
 
 // The backward pass on the state a training forward left in `ws`.
@@ -753,6 +816,69 @@ moe_status_t moe_dispatch_mxfp8(const uint16_t* x, const int32_t* phi, const int
   if (!aligned16(x) || !aligned16(phi) || !aligned16(xq)) return MOE_INVALID_ARG;
   return from_cuda(launch_dispatch_mxfp8(x, phi, offsets, xq, xs, *shape, rows_max_of(shape),
                                          dev_status, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_dispatch_mxfp8_tiled(const uint16_t* x, const int32_t* phi,
+                                      const int32_t* offsets, uint8_t* xq, uint8_t* xs,
+                                      int32_t* dev_status, const moe_shape_t* shape,
+                                      void* stream) {
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->H < 128 || shape->H % 128 != 0) return MOE_UNSUPPORTED_SHAPE;
+  if (!phi || !offsets || !xq || !xs || !dev_status || (shape->N > 0 && !x)) return MOE_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(phi) || !aligned16(xq)) return MOE_INVALID_ARG;
+  return from_cuda(launch_dispatch_mxfp8(x, phi, offsets, xq, xs, *shape, rows_max_of(shape),
+                                         dev_status, static_cast<cudaStream_t>(stream),
+                                         /*tiled=*/true));
+}
+
+moe_status_t moe_mx_quantize_weights(const uint16_t* W, int32_t E, int32_t K, int32_t N,
+                                     uint8_t* q, uint8_t* scale, void* stream) {
+  if (E < 0 || K < 128 || K % 128 != 0 || N < 128 || N % 128 != 0) return MOE_INVALID_ARG;
+  if (static_cast<int64_t>(E) * K * N >= (int64_t{1} << 40)) return MOE_UNSUPPORTED_SHAPE;
+  if (E > 0 && (!W || !q || !scale)) return MOE_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(q)) return MOE_INVALID_ARG;
+  return from_cuda(launch_mx_quantize_weights(W, E, K, N, q, scale,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_expert_ffn_mxfp8(const uint8_t* xq, const uint8_t* xs, const uint8_t* W1q,
+                                  const uint8_t* W1s, const uint8_t* W3q, const uint8_t* W3s,
+                                  const uint8_t* W2q, const uint8_t* W2s, const int32_t* offsets,
+                                  const int32_t* counts, uint8_t* hq, uint8_t* hs, float* y,
+                                  int32_t* dev_status, const moe_shape_t* shape, void* stream) {
+  moe_status_t st = check_mx_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!xq || !xs || !W1q || !W1s || !W3q || !W3s || !W2q || !W2s || !offsets || !hq || !hs || !y ||
+      !dev_status)
+    return MOE_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(xs) || !aligned16(W1q) || !aligned16(W1s) || !aligned16(W3q) ||
+      !aligned16(W3s) || !aligned16(W2q) || !aligned16(W2s) || !aligned32(hq) || !aligned16(hs) ||
+      !aligned32(y))
+    return MOE_INVALID_ARG;
+  return from_cuda(launch_expert_ffn_mxfp8(xq, xs, W1q, W1s, W3q, W3s, W2q, W2s, offsets, counts,
+                                           hq, hs, y, *shape, rows_max_of(shape), dev_status,
+                                           static_cast<cudaStream_t>(stream), nullptr));
+}
+
+moe_status_t moe_layer_forward_mxfp8(const float* logits, const uint16_t* x, const uint8_t* W1q,
+                                     const uint8_t* W1s, const uint8_t* W3q, const uint8_t* W3s,
+                                     const uint8_t* W2q, const uint8_t* W2s, uint16_t* out,
+                                     void* ws, size_t ws_bytes, int32_t* dev_status,
+                                     const moe_shape_t* shape, void* stream,
+                                     void* const* stage_events) {
+  moe_status_t st = check_mx_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!W1q || !W1s || !W3q || !W3s || !W2q || !W2s || !ws || !dev_status ||
+      (shape->N > 0 && (!logits || !x || !out)))
+    return MOE_INVALID_ARG;
+  if (!aligned16(logits) || !aligned16(x) || !aligned16(W1q) || !aligned16(W1s) ||
+      !aligned16(W3q) || !aligned16(W3s) || !aligned16(W2q) || !aligned16(W2s) ||
+      !aligned16(out) || !aligned32(ws))
+    return MOE_INVALID_ARG;
+  if (ws_bytes < layer_ws(shape).total) return MOE_WORKSPACE_TOO_SMALL;
+  return from_cuda(layer_body_mx(logits, x, W1q, W1s, W3q, W3s, W2q, W2s, out, ws, dev_status,
+                                 shape, static_cast<cudaStream_t>(stream), stage_events));
 }
 
 int64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

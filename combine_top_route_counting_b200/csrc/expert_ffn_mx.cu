@@ -1,0 +1,474 @@
+// MXFP8 routed experts: the grouped SwiGLU expert FFN on E4M3 operands with
+// E8M0 block scales, on the block-scaled 5th-generation tensor cores.
+//
+// "Mixture-of-Kittens: A MoE Megakernel for GB300 NVL72", section 5 (MXFP8
+// routed experts; the quantisation fused into the dispatch and into the
+// SwiGLU epilogue); the OCP Microscaling formats (E4M3 elements, one E8M0
+// scale per 32 values along the reduction dimension). For each expert l and
+// its rows [S[l], S[l+1]) of the gathered, quantised tokens:
+//   GEMM1  acc = mx(x) . [mx(W1[l]) | mx(W3[l])]          fp32 in TMEM
+//          h = silu(acc_W1) * acc_W3 (fp32), quantised to MXFP8 along I
+//          (one scale per 32 h columns) by the epilogue
+//   GEMM2  y = mx(h) . mx(W2[l])                           fp32
+// where mx(v) is the value the codes stand for: code value x 2^(scale - 127).
+//
+// Operands, all K-major (the reduction dimension contiguous):
+//   A   xq [rows, H] (GEMM1), hq [rows, I] (GEMM2): E4M3 codes
+//   B   the weights transposed once: W1t, W3t [E, I, H]; W2t [E, H, I]
+//   scales of every operand in the tiled layout of mx_tiled_offset
+//   (internal.cuh): 512-byte atoms of 128 rows x 4 blocks of 32 values.
+//
+// Design: the forward FFN's persistent warp-specialised CTA-pair kernel
+// (expert_ffn.cu) with the block-scaled MMA. 256 x 256 tiles on a CTA pair
+// (tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale, M = 256, N = 256,
+// K = 32 per instruction); a pipeline stage holds 128 K values (one 128-byte
+// swizzled row per operand row, four MMAs) and their scales: the CTA's 128 A
+// rows (one atom, 512 bytes) and all 256 B columns (two atoms; each CTA of
+// the pair needs the scales of every column its rows meet). The producer
+// loads codes and scale atoms with TMA (pair form; each CTA fetches its own
+// copy). The MMA thread moves a stage's scales into TMEM with three tcgen05.cp (32x128b,
+// replicated into the four lane quarters: 4 columns for A, 8 for B) and then
+// issues the stage's four MMAs, each naming its scale byte (0..3) of the
+// 32-bit cells. Scale slots in TMEM follow the smem stages: a slot is
+// rewritten only after the MMAs that read it completed (the stage's empty
+// barrier came first).
+// TMEM: one 256-column fp32 accumulator plus STAGES x 16 scale columns.
+// Double buffering the accumulator would need all 512 columns and leave none
+// for the scales, so the epilogue of a tile is not overlapped with the next
+// tile's MMAs.
+//
+// Every output element is produced by one CTA pair in a fixed K order (no
+// split-K, no atomics): the result is deterministic and independent of which
+// other rows share the launch. Every mbarrier wait is bounded; on a timeout
+// all roles unwind, in-flight copies and MMAs are drained with a bounded
+// wait, TMEM is freed and MOE_DEV_TIMEOUT is raised.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "internal.cuh"
+#include "persistent_gemm.cuh"
+#include "sm100.cuh"
+#include "sm100_mx.cuh"
+
+namespace moe {
+namespace {
+
+using namespace sm100;
+using namespace pg;
+
+// MODE 0: GEMM1 + SwiGLU + MX quantisation of h. MODE 1: GEMM2 -> fp32 y.
+template <int MODE>
+struct MxCfg {
+  static constexpr bool TMA_STORE = MODE == 1;
+  static constexpr int STAGING_BYTES = TMA_STORE ? 8 * 4096 : 0;  // 8 warps x 32x32 fp32
+  static constexpr int BM = 256, BN = 256;
+  static constexpr int BK = 128;                       // E4M3 values (bytes) per stage
+  static constexpr int MMA_K = 32;                     // K of one block-scaled MMA
+  static constexpr int A_BYTES = 128 * BK;             // this CTA's 128 rows
+  static constexpr int B_BYTES = 128 * BK;             // this CTA's 128 of the 256 columns
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KB
+  static constexpr int SFA_BYTES = 512;                  // 128 rows x 4 scales
+  static constexpr int SFB_BYTES = 1024;                 // 256 columns x 4 scales
+  static constexpr int SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGES = TMA_STORE ? 5 : 6;
+  static constexpr int TMEM_SF = BN;    // scale columns follow the accumulator
+  static constexpr int SF_COLS = 16;    // per stage: A at +0 (4), B at +4 (8)
+  static_assert(TMEM_SF + STAGES * SF_COLS <= kTmemCols, "TMEM budget");
+  static constexpr uint32_t IDESC = idesc_mxf8_e4m3(BM, BN, 0, 0);
+  static constexpr int BAR_FULL = 0;
+  static constexpr int BAR_EMPTY = STAGES;
+  static constexpr int BAR_TFULL = 2 * STAGES;
+  static constexpr int BAR_TEMPTY = 2 * STAGES + 1;
+  static constexpr int BAR_DRAIN = 2 * STAGES + 2;
+  static constexpr int BAR_TID_FULL = 2 * STAGES + 3;
+  static constexpr int BAR_TID_EMPTY = 2 * STAGES + 3 + kRing;
+  static constexpr int NUM_BARS = 2 * STAGES + 3 + 2 * kRing;
+  // readers of each tile id: producer, MMA issuer and 8 epilogue warps of the
+  // leader; producer and 8 epilogue warps of the follower
+  static constexpr int TID_CONSUMERS = 19;
+  static_assert(STAGE_BYTES % 1024 == 0 && A_BYTES % 1024 == 0, "swizzle atoms stay 1024-aligned");
+  static_assert(BK / MMA_K == 4, "one 32-bit TMEM scale cell per row and stage");
+};
+
+struct MxParams {
+  int* tile_counter;       // next tile to hand out (zeroed before each launch)
+  const int32_t* offsets;  // [E+1] segment starts (multiples of 256)
+  const int32_t* counts;   // [E, P] or null
+  int32_t E, P;
+  int32_t K;               // reduction length: H (GEMM1), I (GEMM2)
+  int32_t Nout;            // output row length: I (GEMM1), H (GEMM2)
+  int64_t rows_max;
+  uint8_t* hq;             // GEMM1: h codes [rows_max, I]
+  uint8_t* hs;             // GEMM1: h scales, tiled over [rows_max, I/32]
+  int32_t* dev_status;
+  int64_t timeout_ns;
+};
+
+template <int MODE>
+size_t mx_smem_bytes(int E) {
+  using C = MxCfg<MODE>;
+  return 1024 + static_cast<size_t>(C::STAGES) * (C::STAGE_BYTES + C::SF_STAGE_BYTES) +
+         C::STAGING_BYTES + C::NUM_BARS * 8 + 16 + kRing * 4 + static_cast<size_t>(2 * E + 1) * 4;
+}
+
+__device__ __forceinline__ float silu(float a) { return a / (1.0f + expf(-a)); }
+
+// floor(log2 v) of a finite positive fp32, exactly (subnormals included).
+__device__ __forceinline__ int f32_floor_log2(float v) {
+  const uint32_t bits = __float_as_uint(v);
+  const int ef = static_cast<int>(bits >> 23);
+  if (ef != 0) return ef - 127;
+  return -149 + (31 - __clz(bits & 0x7FFFFFu));  // subnormal: mantissa x 2^-149
+}
+
+// MX quantisation of 32 fp32 values (one block): E4M3 codes in element order
+// (four per word, the lowest element in the low byte) and the E8M0 scale code.
+// The same rule as the dispatch's quantisation, applied to fp32 inputs.
+__device__ __forceinline__ void mx_block_f32(const float (&v)[32], uint32_t (&codes)[8],
+                                             uint8_t& scale) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  int e = -127;
+  if (amax > 0.0f) e = max(-127, min(127, f32_floor_log2(amax) - 8));
+  scale = static_cast<uint8_t>(e + 127);
+  const float inv = __int_as_float((127 - e) << 23);  // 2^-e, a normal fp32 for e in [-127, 119]
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+        make_float2(v[4 * w] * inv, v[4 * w + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+    const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+        make_float2(v[4 * w + 2] * inv, v[4 * w + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+    codes[w] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+  }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kNumThreads, 1)
+    ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmSA,
+                  const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmSB0,
+                  const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmSB1,
+                  const __grid_constant__ CUtensorMap tmY, const MxParams p) {
+  using C = MxCfg<MODE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;  // TMA_STORE only (1024-aligned)
+  uint8_t* sf = staging + C::STAGING_BYTES;              // [STAGES] x {A atom, 2 B atoms}
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sf + C::STAGES * C::SF_STAGE_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* bad_flag = abort_flag + 1;
+  int* tile_ring = reinterpret_cast<int*>(tmem_slot + 4);
+  int32_t* s_off = reinterpret_cast<int32_t*>(tile_ring + kRing);  // [E+1]
+  int32_t* s_end = s_off + (p.E + 1);                            // [E]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int E = p.E;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  if (tid == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(smem_u32(&bars[C::BAR_FULL + i]), 1);
+      mbar_init(smem_u32(&bars[C::BAR_EMPTY + i]), 1);
+    }
+    mbar_init(smem_u32(&bars[C::BAR_TFULL]), 1);
+    mbar_init(smem_u32(&bars[C::BAR_TEMPTY]), kNumEpiWarps * 2);
+    mbar_init(smem_u32(&bars[C::BAR_DRAIN]), 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(smem_u32(&bars[C::BAR_TID_FULL + i]), 1);
+      mbar_init(smem_u32(&bars[C::BAR_TID_EMPTY + i]), C::TID_CONSUMERS);
+    }
+    *abort_flag = 0;
+    *bad_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmSA);
+    tma_prefetch_desc(&tmB0);
+    tma_prefetch_desc(&tmSB0);
+    tma_prefetch_desc(&tmB1);
+    tma_prefetch_desc(&tmSB1);
+    if (C::TMA_STORE) tma_prefetch_desc(&tmY);
+  }
+  load_segments(p.offsets, p.counts, E, p.P, C::BM, p.rows_max, s_off, s_end, bad_flag);
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer's barriers exist before anything targets them
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const bool bad_sched = *bad_flag != 0;
+  if (bad_sched && tid == 0) atomicOr(p.dev_status, MOE_DEV_BAD_SCHEDULE);
+
+  const int rows_used = bad_sched ? 0 : s_off[E];
+  // GEMM1: a tile's 256 accumulator columns are 128 h columns seen through W1 and W3
+  const int tiles_n = (MODE == 0) ? p.Nout / 128 : p.Nout / C::BN;
+  const int num_tiles = (rows_used / C::BM) * tiles_n;
+  const int kblocks = p.K / C::BK;  // stages per tile = scale atoms per 128-row block
+  const WaitCtx wc{abort_flag, p.dev_status, p.timeout_ns, MOE_DEV_TIMEOUT};
+
+  const uint32_t tid_empty_local = smem_u32(&bars[C::BAR_TID_EMPTY]);
+  const TileRing tring{tile_ring, smem_u32(&bars[C::BAR_TID_FULL]), tid_empty_local,
+                       mapa_shared(tid_empty_local, 0), !leader};
+  auto next_tile = [&](int& pos, uint32_t& ph) -> int { return tring.next<true>(pos, ph, wc); };
+  const int64_t drain_ns = p.timeout_ns < 100000000ll ? p.timeout_ns : 100000000ll;
+  // tile -> (first row, n-tile, expert); the forward FFN's grouped raster
+  auto tile_info = [&](int tile, int& row0, int& n, int& l) -> bool {
+    return grouped_row_tile<C::BM, 8, 1>(tile, s_off, s_end, E, tiles_n, row0, n, l);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint32_t full0 = smem_u32(&bars[C::BAR_FULL]);
+      const uint32_t full_tgt0 = mapa_shared(full0, 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      int tpos = 0;
+      uint32_t tph = 0;
+      while (ok) {
+        const int tile = next_tile(tpos, tph);
+        if (tile < 0) break;
+        int row0, n, l;
+        if (!tile_info(tile, row0, n, l)) continue;
+        const int arow = row0 + static_cast<int>(rank) * 128;
+        // B rows (of the transposed weights) this tile meets: GEMM1: W1t and
+        // W3t rows l*I + n*128 .. +128 (CTA 0 loads W1t's, CTA 1 W3t's);
+        // GEMM2: W2t rows l*H + n*256 .. +256 (CTA r loads 128 r .. +128)
+        const int brow = (MODE == 0) ? l * p.Nout + n * 128 : l * p.Nout + n * C::BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!wait_bounded(smem_u32(&bars[C::BAR_EMPTY + stage]), phase ^ 1u, wc)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full_tgt = full_tgt0 + stage * 8;
+          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sB = sA + C::A_BYTES;
+          const uint32_t sSA = smem_u32(sf + stage * C::SF_STAGE_BYTES);
+          const uint32_t sSB = sSA + C::SFA_BYTES;
+          const int kx = kb * C::BK;
+          if (leader) mbar_arrive_expect_tx(full0 + stage * 8, 2 * (C::STAGE_BYTES + C::SF_STAGE_BYTES));
+          tma_load_2d_pair(sA, &tmA, kx, arow, full_tgt);
+          tma_load_2d_pair(sSA, &tmSA, 0, (arow / 128) * kblocks + kb, full_tgt);
+          if (MODE == 0) {
+            tma_load_2d_pair(sB, rank == 1 ? &tmB1 : &tmB0, kx, brow, full_tgt);
+            tma_load_2d_pair(sSB, &tmSB0, 0, (brow / 128) * kblocks + kb, full_tgt);
+            tma_load_2d_pair(sSB + 512, &tmSB1, 0, (brow / 128) * kblocks + kb, full_tgt);
+          } else {
+            tma_load_2d_pair(sB, &tmB0, kx, brow + static_cast<int>(rank) * 128, full_tgt);
+            tma_load_2d_pair(sSB, &tmSB0, 0, (brow / 128) * kblocks + kb, full_tgt);
+            tma_load_2d_pair(sSB + 512, &tmSB0, 0, (brow / 128 + 1) * kblocks + kb, full_tgt);
+          }
+          ++issued;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // no load may still be landing in shared memory when the CTA exits
+      const int64_t first = issued > C::STAGES ? issued - C::STAGES : 0;
+      for (int64_t j = first; j < issued; ++j) {
+        const int st = static_cast<int>(j % C::STAGES);
+        const uint32_t par = static_cast<uint32_t>((j / C::STAGES) & 1);
+        wait_drain(smem_u32(&bars[(leader ? C::BAR_FULL : C::BAR_EMPTY) + st]), par, drain_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      int tpos = 0;
+      uint32_t tph = 0;
+      while (ok) {
+        const int tile = next_tile(tpos, tph);
+        if (tile < 0) break;
+        int row0, n, l;
+        if (!tile_info(tile, row0, n, l)) continue;
+        // the single accumulator is free once both CTAs' epilogues drained it
+        if (!wait_bounded<true>(smem_u32(&bars[C::BAR_TEMPTY]), acc_phase ^ 1u, wc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!wait_bounded(smem_u32(&bars[C::BAR_FULL + stage]), phase, wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sB = sA + C::A_BYTES;
+          const uint32_t sSA = smem_u32(sf + stage * C::SF_STAGE_BYTES);
+          const uint32_t sSB = sSA + C::SFA_BYTES;
+          const uint32_t tsf = tmem_base + static_cast<uint32_t>(C::TMEM_SF + stage * C::SF_COLS);
+          // 32 rows x 16 bytes per copy: four 8-row core matrices 128 bytes apart
+          tc_cp_pair_32x128b_x4(tsf, smem_desc_noswz(sSA, 128));
+          tc_cp_pair_32x128b_x4(tsf + 4, smem_desc_noswz(sSB, 128));
+          tc_cp_pair_32x128b_x4(tsf + 8, smem_desc_noswz(sSB + 512, 128));
+#pragma unroll
+          for (int kk = 0; kk < C::BK / C::MMA_K; ++kk) {
+            // K-major: 32 E4M3 = 32 bytes inside the 128-byte swizzled row
+            const uint64_t a_desc = smem_desc_sw128(sA + kk * 32, 16, 1024);
+            const uint64_t b_desc = smem_desc_sw128(sB + kk * 32, 16, 1024);
+            const uint32_t sel = static_cast<uint32_t>(kk);
+            const uint32_t idesc = C::IDESC | (sel << 29) | (sel << 4);
+            tc_mma_mx_pair(tmem_base, a_desc, b_desc, idesc, tsf | (sel << 30),
+                           (tsf + 4) | (sel << 30), (kb | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit_pair_mc(smem_u32(&bars[C::BAR_EMPTY + stage]), 0x3);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(smem_u32(&bars[C::BAR_TFULL]), 0x3);
+        acc_phase ^= 1u;
+      }
+      tc_commit_pair(smem_u32(&bars[C::BAR_DRAIN]));
+      wait_drain(smem_u32(&bars[C::BAR_DRAIN]), 0, p.timeout_ns);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ tile scheduler
+    if (lane == 0 && leader) tring.schedule<true>(p.tile_counter, num_tiles, wc);
+  } else if (warp >= kEpiWarp0) {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                    // TMEM lane quarter of this warp
+    const int half = (warp - kEpiWarp0) >> 2;  // which half of the tile's columns
+    const uint32_t tempty_tgt = mapa_shared(smem_u32(&bars[C::BAR_TEMPTY]), 0);
+    uint32_t acc_phase = 0;
+    int tpos = 0;
+    uint32_t tph = 0;
+    for (;;) {
+      int tile = 0;
+      if (lane == 0) tile = next_tile(tpos, tph);
+      tile = __shfl_sync(0xFFFFFFFFu, tile, 0);
+      if (tile < 0) break;
+      int row0, n, l;
+      if (!tile_info(tile, row0, n, l)) continue;
+      if (!wait_bounded(smem_u32(&bars[C::BAR_TFULL]), acc_phase, wc)) break;
+      tc_fence_after();
+      const int64_t row = row0 + static_cast<int>(rank) * 128 + q * 32 + lane;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      if (MODE == 0) {
+        // accumulator columns [0,128) = x.W1, [128,256) = x.W3 for h columns
+        // n*128 + j; this warp's 64 columns are two 32-column MX blocks of h
+        const int I = p.Nout;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t ra[32], rb[32];
+          tmem_ld_32cols(tbase + half * 64 + c * 32, ra);
+          tmem_ld_32cols(tbase + 128 + half * 64 + c * 32, rb);
+          tmem_ld_wait();
+          float hv[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) hv[i] = silu(__uint_as_float(ra[i])) * __uint_as_float(rb[i]);
+          uint32_t codes[8];
+          uint8_t scale;
+          mx_block_f32(hv, codes, scale);
+          const int col = n * 128 + half * 64 + c * 32;
+          st_global_v8(p.hq + row * I + col, codes);
+          p.hs[mx_tiled_offset(row, col / 32, I / 32)] = scale;
+        }
+      } else {
+        // row `lane` of this warp's 32x32 block goes to the staging slot with
+        // 16-byte chunk j at j ^ (lane & 7) (the tensor map's 128-byte
+        // swizzle), then one TMA store; a slot is reused once the previous
+        // store has read it
+        const uint32_t stg = smem_u32(staging) + (warp - kEpiWarp0) * 4096;
+        const uint64_t pol_y = l2_policy_evict_first();
+        const int ycol = n * C::BN + half * 128;
+        const int yrow0 = row0 + static_cast<int>(rank) * 128 + q * 32;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t rv[32];
+          tmem_ld_32cols(tbase + half * 128 + c * 32, rv);
+          tmem_ld_wait();
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(stg + lane * 128 + ((j ^ (lane & 7)) << 4), rv[4 * j], rv[4 * j + 1],
+                         rv[4 * j + 2], rv[4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d_hint(&tmY, stg, ycol + c * 32, yrow0, pol_y);
+            bulk_commit_group();
+          }
+        }
+      }
+      // the accumulator may be refilled once every lane's tcgen05.ld completed
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_relaxed_cluster(tempty_tgt);
+      acc_phase ^= 1u;
+    }
+    if (C::TMA_STORE && lane == 0) bulk_wait_all();  // stores complete before the CTA exits
+  }
+
+  __syncthreads();
+  cluster_sync();  // the peer no longer reads this CTA's smem or TMEM
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
+template <int MODE>
+cudaError_t launch_mx(const CUtensorMap& a, const CUtensorMap& sa, const CUtensorMap& b0,
+                      const CUtensorMap& sb0, const CUtensorMap& b1, const CUtensorMap& sb1,
+                      const CUtensorMap& y, MxParams p, cudaStream_t s) {
+  const size_t smem = mx_smem_bytes<MODE>(p.E);
+  cudaError_t e = tile_counter_for_current_device(&p.tile_counter);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s)) != cudaSuccess) return e;
+  return launch_persistent(ffn_mx_kernel<MODE>, 2, smem, s, a, sa, b0, sb0, b1, sb1, y, p);
+}
+
+}  // namespace
+
+cudaError_t launch_expert_ffn_mxfp8(const uint8_t* xq, const uint8_t* xs, const uint8_t* W1q,
+                                    const uint8_t* W1s, const uint8_t* W3q, const uint8_t* W3s,
+                                    const uint8_t* W2q, const uint8_t* W2s,
+                                    const int32_t* offsets, const int32_t* counts, uint8_t* hq,
+                                    uint8_t* hs, float* y, const moe_shape_t& sh,
+                                    int64_t rows_max, int32_t* dev_status, cudaStream_t s,
+                                    cudaEvent_t ev_mid) {
+  const int E = sh.E, H = sh.H, I = sh.I;
+  const uint64_t EH = static_cast<uint64_t>(E) * H, EI = static_cast<uint64_t>(E) * I;
+  const uint64_t rb = static_cast<uint64_t>(rows_max) / 128;  // 128-row blocks of the activations
+  CUtensorMap mXq, mXs, mW1, mW1s, mW3, mW3s, mHq, mHs, mW2, mW2s, mY;
+  if (!make_map_u8(&mXq, xq, H, rows_max, 128, 128) || !make_map_sf_atoms(&mXs, xs, rb * (H / 128)) ||
+      !make_map_u8(&mW1, W1q, H, EI, 128, 128) ||
+      !make_map_sf_atoms(&mW1s, W1s, EI / 128 * (H / 128)) ||
+      !make_map_u8(&mW3, W3q, H, EI, 128, 128) ||
+      !make_map_sf_atoms(&mW3s, W3s, EI / 128 * (H / 128)) ||
+      !make_map_u8(&mHq, hq, I, rows_max, 128, 128) || !make_map_sf_atoms(&mHs, hs, rb * (I / 128)) ||
+      !make_map_u8(&mW2, W2q, I, EH, 128, 128) ||
+      !make_map_sf_atoms(&mW2s, W2s, EH / 128 * (I / 128)) ||
+      !make_map(&mY, y, H, rows_max, 32, 32, true))
+    return cudaErrorInvalidValue;
+  MxParams p1{nullptr, offsets, counts, E, sh.P, H, I, rows_max, hq, hs, dev_status, kWaitTimeoutNs};
+  cudaError_t e = launch_mx<0>(mXq, mXs, mW1, mW1s, mW3, mW3s, mY, p1, s);
+  if (e != cudaSuccess) return e;
+  if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
+  MxParams p2{nullptr, offsets, counts, E, sh.P, I, H, rows_max, nullptr, nullptr, dev_status,
+              kWaitTimeoutNs};
+  return launch_mx<1>(mHq, mHs, mW2, mW2s, mW2, mW2s, mY, p2, s);
+}
+
+}  // namespace moe

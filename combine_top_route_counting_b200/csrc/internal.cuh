@@ -109,9 +109,44 @@ cudaError_t launch_expert_ffn_wgrad(const uint16_t* xg, const uint16_t* dys, con
 cudaError_t launch_mx_quantize_rows(const uint16_t* src, int64_t n_rows, int32_t K, uint8_t* q,
                                     uint8_t* scale, cudaStream_t s);
 // The pull dispatch with the MX quantisation fused: xq/xs rows of the gathered tokens.
+// tiled: the scales in the tensor-core layout (mx_tiled_offset) instead of row-major.
 cudaError_t launch_dispatch_mxfp8(const uint16_t* x, const int32_t* phi, const int32_t* offsets,
                                   uint8_t* xq, uint8_t* xs, const moe_shape_t& sh,
-                                  int64_t rows_max, int32_t* dev_status, cudaStream_t s);
+                                  int64_t rows_max, int32_t* dev_status, cudaStream_t s,
+                                  bool tiled = false);
+
+// Byte offset of the E8M0 scale of row r, 32-value block b, in the tiled
+// layout of a [R, K] code matrix (R and K multiples of 128): 512-byte atoms
+// of 128 rows x 4 blocks, K-atoms of a row block consecutive; inside an atom
+// row r at (r % 32) * 16 + ((r / 32) % 4) * 4, block b at b % 4 -- the layout
+// tcgen05.cp (32x128b, warpx4) moves into TMEM for the block-scaled MMA.
+__host__ __device__ __forceinline__ int64_t mx_tiled_offset(int64_t r, int32_t b, int32_t kblocks) {
+  return ((r >> 7) * (kblocks >> 2) + (b >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (b & 3);
+}
+
+// Expert weights to MXFP8 for the block-scaled GEMMs: W bf16 [E, K, N] ->
+// codes [E, N, K] (transposed: K-major) and tiled scales over the [E*N, K/32]
+// table. K % 128 == 0, N % 128 == 0.
+cudaError_t launch_mx_quantize_weights(const uint16_t* W, int32_t E, int32_t K, int32_t N,
+                                       uint8_t* q, uint8_t* scale, cudaStream_t s);
+
+// The grouped SwiGLU expert FFN on MXFP8 operands (block-scaled tcgen05, CTA
+// pairs): GEMM1 + SwiGLU + MX quantisation of h, then GEMM2 -> fp32 y.
+// ev_mid, if not null, is recorded between the two kernels.
+cudaError_t launch_expert_ffn_mxfp8(const uint8_t* xq, const uint8_t* xs, const uint8_t* W1q,
+                                    const uint8_t* W1s, const uint8_t* W3q, const uint8_t* W3s,
+                                    const uint8_t* W2q, const uint8_t* W2s,
+                                    const int32_t* offsets, const int32_t* counts, uint8_t* hq,
+                                    uint8_t* hs, float* y, const moe_shape_t& sh,
+                                    int64_t rows_max, int32_t* dev_status, cudaStream_t s,
+                                    cudaEvent_t ev_mid);
+
+// 2D tensor map over a [outer, inner] uint8 matrix, box [box_outer, box_inner],
+// 128-byte swizzle.
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                 uint32_t box_inner, uint32_t box_outer);
+// Tensor map whose box is one 512-byte scale atom of a tiled scale table.
+bool make_map_sf_atoms(CUtensorMap* m, const void* base, uint64_t n_atoms);
 
 // Failure-detection self test (bounded wait on an mbarrier nothing completes).
 cudaError_t launch_selftest_wait(int32_t* dev_status, int64_t timeout_ns, cudaStream_t s);

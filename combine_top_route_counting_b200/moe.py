@@ -88,6 +88,12 @@ _SIGS = {
                                          ctypes.POINTER(_vp)], ctypes.c_int),
     "moe_mx_quantize_rows": ([_vp, ctypes.c_int64, ctypes.c_int32, _vp, _vp, _vp], ctypes.c_int),
     "moe_dispatch_mxfp8": ([_vp] * 6 + [ctypes.POINTER(Shape), _vp], ctypes.c_int),
+    "moe_dispatch_mxfp8_tiled": ([_vp] * 6 + [ctypes.POINTER(Shape), _vp], ctypes.c_int),
+    "moe_mx_quantize_weights": ([_vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp],
+                                ctypes.c_int),
+    "moe_expert_ffn_mxfp8": ([_vp] * 14 + [ctypes.POINTER(Shape), _vp], ctypes.c_int),
+    "moe_layer_forward_mxfp8": ([_vp] * 10 + [ctypes.c_size_t, _vp, ctypes.POINTER(Shape), _vp,
+                                              ctypes.POINTER(_vp)], ctypes.c_int),
     "moe_launch_count": ([], ctypes.c_int64),
     "moe_selftest_bounded_wait": ([_vp, ctypes.c_int64, _vp], ctypes.c_int),
 }
@@ -412,6 +418,48 @@ def moe_dispatch_mxfp8(x, phi, offsets, xq, xs, dev_status, sh: Shape, stream=No
                                      _ptr(xq, torch.uint8, "xq"), _ptr(xs, torch.uint8, "xs"),
                                      _ptr(dev_status, torch.int32, "dev_status"), ctypes.byref(sh),
                                      _stream(stream)), "moe_dispatch_mxfp8")
+
+
+def moe_dispatch_mxfp8_tiled(x, phi, offsets, xq, xs, dev_status, sh: Shape, stream=None):
+    """moe_dispatch_mxfp8 with xs in the tiled scale layout of include/moe.h."""
+    _check(load().moe_dispatch_mxfp8_tiled(
+        _ptr(x, torch.bfloat16, "x"), _ptr(phi, torch.int32, "phi"),
+        _ptr(offsets, torch.int32, "offsets"), _ptr(xq, torch.uint8, "xq"),
+        _ptr(xs, torch.uint8, "xs"), _ptr(dev_status, torch.int32, "dev_status"),
+        ctypes.byref(sh), _stream(stream)), "moe_dispatch_mxfp8_tiled")
+
+
+def moe_mx_quantize_weights(W, q, scale, stream=None):
+    """W bf16 [E, K, N] -> q uint8 [E, N, K] (transposed E4M3 codes), scale uint8
+    [E*N*K/32] (E8M0 codes of the blocks of 32 along K, tiled layout)."""
+    E, K, N = W.shape
+    _check(load().moe_mx_quantize_weights(_ptr(W, torch.bfloat16, "W"), E, K, N,
+                                          _ptr(q, torch.uint8, "q"),
+                                          _ptr(scale, torch.uint8, "scale"), _stream(stream)),
+           "moe_mx_quantize_weights")
+
+
+def moe_expert_ffn_mxfp8(xq, xs, W1q, W1s, W3q, W3s, W2q, W2s, offsets, counts, hq, hs, y,
+                         dev_status, sh: Shape, stream=None):
+    u8 = torch.uint8
+    _check(load().moe_expert_ffn_mxfp8(
+        _ptr(xq, u8, "xq"), _ptr(xs, u8, "xs"), _ptr(W1q, u8, "W1q"), _ptr(W1s, u8, "W1s"),
+        _ptr(W3q, u8, "W3q"), _ptr(W3s, u8, "W3s"), _ptr(W2q, u8, "W2q"), _ptr(W2s, u8, "W2s"),
+        _ptr(offsets, torch.int32, "offsets"), _ptr(counts, torch.int32, "counts"),
+        _ptr(hq, u8, "hq"), _ptr(hs, u8, "hs"), _ptr(y, torch.float32, "y"),
+        _ptr(dev_status, torch.int32, "dev_status"), ctypes.byref(sh), _stream(stream)),
+        "moe_expert_ffn_mxfp8")
+
+
+def moe_layer_forward_mxfp8(logits, x, W1q, W1s, W3q, W3s, W2q, W2s, out, ws, dev_status,
+                            sh: Shape, stream=None, stage_events=None):
+    u8 = torch.uint8
+    _check(load().moe_layer_forward_mxfp8(
+        _ptr(logits, torch.float32, "logits"), _ptr(x, torch.bfloat16, "x"),
+        _ptr(W1q, u8, "W1q"), _ptr(W1s, u8, "W1s"), _ptr(W3q, u8, "W3q"), _ptr(W3s, u8, "W3s"),
+        _ptr(W2q, u8, "W2q"), _ptr(W2s, u8, "W2s"), _ptr(out, torch.bfloat16, "out"),
+        _ptr(ws, u8, "ws"), ws.numel(), _ptr(dev_status, torch.int32, "dev_status"),
+        ctypes.byref(sh), _stream(stream), _events(stage_events)), "moe_layer_forward_mxfp8")
 
 
 def moe_selftest_bounded_wait(dev_status, timeout_ns: int, stream=None):

@@ -395,9 +395,8 @@ moe_status_t moe_layer_backward(const uint16_t* dout, const uint16_t* W1, const 
 /* ------------------------------------------------------------------------
  * MXFP8 ("Mixture-of-Kittens", section 5: MXFP8 routed experts, with the
  * quantisation fused into the dispatch; the OCP Microscaling formats, MXFP8
- * with E4M3 elements). Building blocks of an MXFP8 expert path: the
- * block-scaled expert GEMMs that would consume them are not part of this
- * library yet.
+ * with E4M3 elements): quantisation of rows and of expert weights, the
+ * quantising dispatch, the block-scaled expert FFN and the MXFP8 layer.
  *
  * For every block of 32 consecutive values of a row: amax = max |v|, the
  * shared exponent e = floor(log2 amax) - 8 clamped to [-127, 127] (-127 for
@@ -419,6 +418,61 @@ moe_status_t moe_mx_quantize_rows(const uint16_t* src, int64_t n_rows, int32_t K
 moe_status_t moe_dispatch_mxfp8(const uint16_t* x, const int32_t* phi, const int32_t* offsets,
                                 uint8_t* xq, uint8_t* xs, int32_t* dev_status,
                                 const moe_shape_t* shape, void* stream);
+
+/* The TILED scale layout the block-scaled tensor cores read. For a code
+ * matrix [R, K] (R and K multiples of 128; block b covers values 32b..32b+31
+ * of a row) the scale of row r, block b is the byte at
+ *   ((r / 128) * (K / 128) + b / 4) * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + b % 4,
+ * i.e. 512-byte atoms of 128 rows x 4 blocks, the K-atoms of a 128-row block
+ * consecutive. The table has R * K / 32 bytes, as the row-major one. */
+
+/* moe_dispatch_mxfp8 with xs in the TILED layout of the [moe_rows_max, H]
+ * code matrix. H % 128 == 0 (rows_max is a multiple of 256). */
+moe_status_t moe_dispatch_mxfp8_tiled(const uint16_t* x, const int32_t* phi,
+                                      const int32_t* offsets, uint8_t* xq, uint8_t* xs,
+                                      int32_t* dev_status, const moe_shape_t* shape,
+                                      void* stream);
+
+/* Expert weights to the MXFP8 operands of the block-scaled FFN: W bf16
+ * [E, K, N] (N contiguous) -> q uint8 [E, N, K], the E4M3 codes TRANSPOSED
+ * (K contiguous), and scale uint8 [E*N*K/32], the E8M0 codes of the blocks
+ * of 32 along K (W[e, 32b..32b+31, n]) in the TILED layout of the [E*N, K]
+ * code matrix (row e*N + n). K and N multiples of 128. For W1 and W3
+ * (K = H, N = I) and W2 (K = I, N = H); done once per set of weights. */
+moe_status_t moe_mx_quantize_weights(const uint16_t* W, int32_t E, int32_t K, int32_t N,
+                                     uint8_t* q, uint8_t* scale, void* stream);
+
+/* Step 3b on MXFP8 operands ("Mixture-of-Kittens", section 5), two kernels
+ * on the block-scaled tensor cores (tcgen05.mma kind::mxf8f6f4.block_scale,
+ * fp32 accumulation in a fixed K order):
+ *   GEMM1: for row r of expert l's segment, a = mx(xq[r]) . mx(W1[l]),
+ *          b = mx(xq[r]) . mx(W3[l]) (fp32), h = silu(a) * b (fp32), written
+ *          as MXFP8 along I: hq uint8 [moe_rows_max, I] codes and hs the
+ *          TILED scales of that matrix (the dispatch's quantisation rule
+ *          applied to the fp32 h);
+ *   GEMM2: y[r] = mx(hq[r]) . mx(W2[l]), fp32 [moe_rows_max, H];
+ * mx(.) = code value x 2^(scale code - 127). xq/xs: moe_dispatch_mxfp8_tiled's
+ * outputs; W1q/W1s, W3q/W3s, W2q/W2s: moe_mx_quantize_weights of W1, W3, W2.
+ * Requires the moe_expert_ffn limits and pad % 256 == 0 (CTA-pair tiles).
+ * hq, y 32-byte aligned, every other pointer 16-byte aligned. Rows of tiles
+ * holding only padding are not written. Errors as moe_expert_ffn. */
+moe_status_t moe_expert_ffn_mxfp8(const uint8_t* xq, const uint8_t* xs, const uint8_t* W1q,
+                                  const uint8_t* W1s, const uint8_t* W3q, const uint8_t* W3s,
+                                  const uint8_t* W2q, const uint8_t* W2s, const int32_t* offsets,
+                                  const int32_t* counts, uint8_t* hq, uint8_t* hs, float* y,
+                                  int32_t* dev_status, const moe_shape_t* shape, void* stream);
+
+/* Steps 1-4 with MXFP8 routed experts: route, schedule, the quantising
+ * dispatch (TILED scales), moe_expert_ffn_mxfp8 and the fixed-order combine,
+ * on `stream`. Weights as moe_expert_ffn_mxfp8; ws of moe_layer_workspace_bytes
+ * (the codes and scales of x and h take the places of xg and h);
+ * stage_events as moe_layer_forward. Limits as moe_expert_ffn_mxfp8. */
+moe_status_t moe_layer_forward_mxfp8(const float* logits, const uint16_t* x, const uint8_t* W1q,
+                                     const uint8_t* W1s, const uint8_t* W3q, const uint8_t* W3s,
+                                     const uint8_t* W2q, const uint8_t* W2s, uint16_t* out,
+                                     void* ws, size_t ws_bytes, int32_t* dev_status,
+                                     const moe_shape_t* shape, void* stream,
+                                     void* const* stage_events);
 
 /* Number of kernels this library has launched in the calling process. */
 int64_t moe_launch_count(void);

@@ -502,3 +502,35 @@ def layer_tokens_mxfp8(logits, x_bits, weights, k: int, H: int, I: int, tokens):
             h = a / (1.0 + np.exp(-a)) * b
             out[a_i] += g64[t, j] * (mx_round(h) @ w2)
     return dict(out64=out, ids=ids, gates64=g64)
+
+
+def ffn_rows_mxfp8(xg_bits, experts, W1: dict, W3: dict, W2: dict, H: int, I: int):
+    """The SwiGLU expert FFN with MXFP8 operands ("Mixture-of-Kittens",
+    section 5) for gathered rows xg_bits [n, H] (bf16 bits) with per-row
+    experts. Every GEMM operand is MX-quantised along its reduction dimension
+    and the arithmetic runs in fp64 on the values the codes stand for:
+      a = mx(x).mx(W1), b = mx(x).mx(W3), h = silu(a) * b,
+      (hq, hs) = the MX codes and scales of h (blocks of 32 along I),
+      y = dq(hq, hs).mx(W2).
+    W1/W3/W2 map expert id -> uint16 [H, I] / [H, I] / [I, H].
+    Returns hq uint8 [n, I], hs uint8 [n, I/32] (row-major), y fp64 [n, H]."""
+    xb = np.asarray(xg_bits, np.uint16)
+    ex = np.asarray(experts, np.int64)
+    n = len(ex)
+    hq = np.zeros((n, I), np.uint8)
+    hs = np.zeros((n, I // 32), np.uint8)
+    y = np.zeros((n, H), np.float64)
+    for e in np.unique(ex):
+        rows = np.nonzero(ex == e)[0]
+        xr = mx_round(_bits_f64(xb[rows]))
+        w1 = mx_round(_bits_f64(W1[int(e)]), axis=0)
+        w3 = mx_round(_bits_f64(W3[int(e)]), axis=0)
+        w2 = mx_round(_bits_f64(W2[int(e)]), axis=0)
+        a = xr @ w1
+        b = xr @ w3
+        with np.errstate(over="ignore"):
+            h = a / (1.0 + np.exp(-a)) * b
+        q, s = mx_quantize(h)
+        hq[rows], hs[rows] = q, s
+        y[rows] = mx_dequantize(q, s) @ w2
+    return hq, hs, y

@@ -52,3 +52,25 @@ def expert_weights_host(W1, W3, W2, experts):
         for d, W in zip(out, (W1, W3, W2)):
             d[e] = bits(W[e])
     return out
+
+
+def mx_tiled_offsets(R: int, K: int) -> np.ndarray:
+    """Byte offsets [R, K/32] of the E8M0 scales of an [R, K] MXFP8 code matrix
+    in the tiled layout the block-scaled tensor cores read (include/moe.h):
+    512-byte atoms of 128 rows x 4 blocks of 32, the K-atoms of a 128-row
+    block consecutive; inside an atom row r at (r % 32) * 16 + ((r // 32) % 4) * 4
+    and block b at b % 4."""
+    if R % 128 or K % 128:
+        raise ValueError("R and K must be multiples of 128")
+    r = np.arange(R, dtype=np.int64)[:, None]
+    b = np.arange(K // 32, dtype=np.int64)[None, :]
+    return ((r // 128) * (K // 128) + b // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + b % 4
+
+
+def to_tiled(scales_rows: np.ndarray) -> np.ndarray:
+    """Row-major scales [R, K/32] -> the tiled table (flat uint8, R*K/32 bytes)."""
+    s = np.asarray(scales_rows, np.uint8)
+    R, KB = s.shape
+    out = np.zeros(R * KB, np.uint8)
+    out[mx_tiled_offsets(R, KB * 32)] = s
+    return out

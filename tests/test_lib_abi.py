@@ -141,6 +141,53 @@ def test_mx_entry_points_argument_errors(lib):
     assert L.moe_dispatch_mxfp8(p, None, p, p, p, p, ctypes.byref(sh), None) == 1
 
 
+def test_mx_ffn_entry_points_argument_errors(lib):
+    L = lib
+    p = ctypes.c_void_p(256)
+    # weight quantisation: K and N multiples of 128, non-negative E, aligned pointers
+    assert L.moe_mx_quantize_weights(p, 2, 192, 256, p, p, None) == 1     # K % 128
+    assert L.moe_mx_quantize_weights(p, 2, 256, 64, p, p, None) == 1      # N % 128
+    assert L.moe_mx_quantize_weights(p, -1, 256, 256, p, p, None) == 1
+    assert L.moe_mx_quantize_weights(None, 2, 256, 256, p, p, None) == 1
+    assert L.moe_mx_quantize_weights(ctypes.c_void_p(264), 2, 256, 256, p, p, None) == 1
+    assert L.moe_mx_quantize_weights(p, 1 << 20, 1 << 12, 1 << 12, p, p, None) == 2  # too large
+    assert L.moe_mx_quantize_weights(None, 0, 256, 256, None, None, None) == 0       # nothing to do
+    # tiled dispatch: H % 128
+    sh = moe.shape(1, 16, 8, 2, 96, 128)
+    assert L.moe_dispatch_mxfp8_tiled(p, p, p, p, p, p, ctypes.byref(sh), None) == 2
+    sh = moe.shape(1, 16, 8, 2, 256, 128)
+    assert L.moe_dispatch_mxfp8_tiled(p, None, p, p, p, p, ctypes.byref(sh), None) == 1
+    # block-scaled FFN: CTA-pair tiles need pad % 256; 32-byte aligned hq and y
+    ok = moe.shape(2, 256, 8, 2, 256, 256)
+    pad128 = moe.shape(2, 256, 8, 2, 256, 256, pad=128)
+    args = [p] * 14 + [ctypes.byref(ok), None]
+    assert L.moe_expert_ffn_mxfp8(*[p] * 14, ctypes.byref(pad128), None) == 2
+    bad_h = moe.shape(2, 256, 8, 2, 384, 256)                             # H % 256
+    assert L.moe_expert_ffn_mxfp8(*[p] * 14, ctypes.byref(bad_h), None) == 2
+    for i in range(14):
+        if i == 9:
+            continue                                                      # counts may be null
+        a = list(args)
+        a[i] = None
+        assert L.moe_expert_ffn_mxfp8(*a) == 1, i
+    a = list(args)
+    a[10] = ctypes.c_void_p(256 + 16)                                     # hq not 32-byte aligned
+    assert L.moe_expert_ffn_mxfp8(*a) == 1
+    # the layer: same limits, the bf16 layer's workspace
+    need = moe.layer_workspace_bytes(ok)
+    lay = [p] * 10 + [need - 1, p, ctypes.byref(ok), None, None]
+    assert L.moe_layer_forward_mxfp8(*lay) == 3
+    lay[10] = need
+    lay[9] = ctypes.c_void_p(256 + 16)                                    # ws not 32-byte aligned
+    assert L.moe_layer_forward_mxfp8(*lay) == 1
+    lay[9] = p
+    lay[12] = ctypes.byref(pad128)
+    assert L.moe_layer_forward_mxfp8(*lay) == 2
+    lay[12] = ctypes.byref(ok)
+    lay[2] = None                                                         # W1q
+    assert L.moe_layer_forward_mxfp8(*lay) == 1
+
+
 def test_size_queries_hold_their_invariants_on_random_shapes(lib):
     """Host-only size queries over random shapes (hypothesis): no crash, -1/0 for
     unsupported shapes, and rows_max / workspace bounds where supported."""
