@@ -87,6 +87,17 @@ def backward_work(w, rows_used: int):
     }
 
 
+def mx_layer_work(w, rows_used: int):
+    """Bytes / flops of each stage of the MXFP8 layer (real routes only): the
+    dispatch reads bf16 tokens and writes E4M3 codes + E8M0 scales; the GEMMs
+    do the bf16 layer's flops on E4M3 operands."""
+    work = algorithmic_work(w, rows_used, w.n_routes)
+    work["dispatch"] = dict(bytes=w.n_routes * w.H * 2 + rows_used * (w.H + w.H // 32))
+    for g in ("ffn_gemm1", "ffn_gemm2"):
+        work[g] = dict(flops=work[g]["flops"], fp8=True)
+    return work
+
+
 def stage_rooflines(stage_ms: dict, work: dict, peaks: dict) -> dict:
     out = {}
     for name, t in stage_ms.items():
@@ -94,6 +105,10 @@ def stage_rooflines(stage_ms: dict, work: dict, peaks: dict) -> dict:
         if "bytes" in work[name]:
             gbs = work[name]["bytes"] / (t / 1e3) / 1e9
             d.update(bytes=work[name]["bytes"], gbs=gbs, frac_hbm=gbs / peaks["hbm"])
+        elif work[name].get("fp8"):
+            # E4M3 operands: the bf16 peak x the nominal fp8/bf16 ratio (4.5 / 2.25)
+            tf = work[name]["flops"] / (t / 1e3) / 1e12
+            d.update(flops=work[name]["flops"], tflops=tf, frac_fp8=tf / (2.0 * peaks["bf16_sus"]))
         else:
             tf = work[name]["flops"] / (t / 1e3) / 1e12
             d.update(flops=work[name]["flops"], tflops=tf, frac_bf16=tf / peaks["bf16_sus"])
@@ -271,7 +286,7 @@ def run_reference(args):
 
 # ---------------------------------------------------------------- our arm
 def assemble_line(args, w, world, ms, stage_ms, launches, e2e, e2e_mb, mb, mb_row, mx, bwd,
-                  rows_used, peaks):
+                  rows_used, peaks, mxl=None):
     """The bench's JSON line (without clocks and cpu_baseline) from the measured
     times: ms for args.steps layer steps, stage_ms {stage: ms}, and the
     optional e2e / minibatch / MXFP8 / backward legs (None when not run)."""
@@ -323,7 +338,17 @@ def assemble_line(args, w, world, ms, stage_ms, launches, e2e, e2e_mb, mb, mb_ro
         line["mxfp8"] = {"dispatch_mxfp8": {"ms": mx["ms"], "bytes": mbytes, "gbs": gbs,
                                             "frac_hbm": gbs / peaks["hbm"]},
                          "note": "pull dispatch with the MX (E4M3, E8M0 per 32) "
-                                 "quantisation fused; block-scaled expert GEMMs not built"}
+                                 "quantisation fused"}
+    if mxl:
+        mst = stage_rooflines(mxl["stage_ms"], mx_layer_work(w, rows_used), peaks)
+        line["mxfp8_layer"] = {
+            "value": w.n_tokens * world * args.steps / (mxl["ms"] / 1e3), "unit": "tokens/s",
+            "ms_per_step": mxl["ms"] / args.steps, "steps": args.steps,
+            "api": "moe_layer_forward_mxfp8 (weights quantised once, outside the timed region)",
+            "stages": mst,
+            "peak_note": f"fp8 peak = 2 x dense bf16 sustained of {peaks['source']} "
+                         "(the nominal fp8/bf16 ratio)",
+        }
     if bwd:
         bst = stage_rooflines(bwd["stages"], backward_work(w, rows_used), peaks)
         top = max(bst, key=lambda n: bst[n]["ms"])
@@ -448,6 +473,35 @@ def run_ours(args):
         mx = dict(ms=m0.elapsed_time(m1) / args.steps, rows=int(bmx["offsets"][-1].item()))
         del xq, xs, bmx
 
+    # the MXFP8 layer (opt in): block-scaled expert GEMMs on weights quantised once
+    mxl = None
+    if args.mxfp8_layer and mb == 0:
+        Wq = []
+        for Wt in W:
+            E_, K_, N_ = Wt.shape
+            q = torch.empty((E_, N_, K_), dtype=torch.uint8, device=dev)
+            sc = torch.empty((E_ * N_ * K_ // 32,), dtype=torch.uint8, device=dev)
+            moe.moe_mx_quantize_weights(Wt, q, sc)
+            Wq += [q, sc]
+        evm = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.N_STAGE_EVENTS)]
+               for _ in range(args.steps)]
+        for _ in range(args.warmup):
+            moe.moe_layer_forward_mxfp8(lg, x, *Wq, out, ws, st, sh)
+        torch.cuda.synchronize()
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        m0.record()
+        for i in range(args.steps):
+            moe.moe_layer_forward_mxfp8(lg, x, *Wq, out, ws, st, sh, stage_events=evm[i])
+        m1.record()
+        torch.cuda.synchronize()
+        if int(st.item()) != 0:
+            raise RuntimeError(f"device status {int(st.item())} in the MXFP8 layer")
+        mxl = dict(ms=m0.elapsed_time(m1),
+                   stage_ms={name: statistics.mean(evm[i][s_i].elapsed_time(evm[i][s_i + 1])
+                                                   for i in range(args.steps))
+                             for s_i, name in enumerate(moe.STAGES)})
+        del Wq
+
     # end to end through the host-buffer entry: H2D of logits and x, the layer,
     # D2H of out; each call's input copy overlaps the previous call's compute
     # and its output copy the next call's compute (the async-output entry)
@@ -537,8 +591,14 @@ def run_ours(args):
     vec = ([ms] + [stage_ms[n] for n in names] + ([e2e["ms"]] if e2e else []) +
            ([mb_row] if mb_row is not None else []) +
            ([bwd["train_ms"], bwd["bwd_ms"]] + [bwd["stages"][n] for n in bnames] if bwd else []) +
-           ([mx["ms"]] if mx else []))
+           ([mx["ms"]] if mx else []) +
+           ([mxl["ms"]] + [mxl["stage_ms"][n] for n in moe.STAGES] if mxl else []))
     vec = reduce_max(vec, ready, device=dev)
+    if mxl:
+        mvals = vec[-(1 + len(moe.STAGES)):]
+        vec = vec[:-(1 + len(moe.STAGES))]
+        mxl["ms"] = mvals[0]
+        mxl["stage_ms"] = dict(zip(moe.STAGES, mvals[1:]))
     if mx:
         mx["ms"] = vec.pop()
     if bwd:
@@ -557,7 +617,7 @@ def run_ours(args):
         peaks = load_peaks()
         rows_used = schedule_rows(moe, w, sh, lg)
         line = assemble_line(args, w, world, ms, stage_ms, launches, e2e, e2e_mb, mb, mb_row, mx,
-                             bwd, rows_used, peaks)
+                             bwd, rows_used, peaks, mxl=mxl)
         line["clocks"] = clk
         if world == 1 and not args.no_cpu_baseline:
             r = oracle_sample(w, lg_cpu, x_cpu, W, row_budget_s=args.cpu_budget)
@@ -647,6 +707,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-mxfp8", action="store_true")
+    ap.add_argument("--mxfp8-layer", action="store_true",
+                    help="also time moe_layer_forward_mxfp8 (block-scaled expert GEMMs)")
     ap.add_argument("--bwd-steps", type=int, default=10)
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--ref-row-budget", type=float, default=3.0)

@@ -120,3 +120,31 @@ def test_assembled_line_meets_the_contract():
     assert b["value"] == pytest.approx(w.n_tokens / 0.0798)
     assert line["mxfp8"]["dispatch_mxfp8"]["frac_hbm"] > 0
     assert line["phi_build_us"] == pytest.approx(53.0)
+
+
+def test_assembled_line_reports_the_mxfp8_layer_leg():
+    """The opt-in MXFP8 layer leg: throughput, and the GEMMs against the fp8
+    peak (twice the measured sustained bf16 peak), the dispatch against HBM."""
+    import argparse
+
+    sys.path.insert(0, ROOT)
+    import bench
+    from combine_top_route_counting_b200 import inputs, moe
+
+    args = argparse.Namespace(steps=10, warmup=3, e2e_steps=10, bwd_steps=10)
+    w = inputs.WORKLOADS["kimi"]
+    stage_ms = dict(zip(moe.STAGES, (0.065, 0.053, 2.39, 21.6, 13.4, 2.21)))
+    mxl = dict(ms=250.0, stage_ms=dict(zip(moe.STAGES, (0.065, 0.053, 1.94, 11.0, 7.0, 2.21))))
+    peaks = bench.load_peaks()
+    line = bench.assemble_line(args, w, 1, 397.0, stage_ms, 90, None, 0, 0, None, None, None,
+                               492544, peaks, mxl=mxl)
+    m = line["mxfp8_layer"]
+    assert m["value"] == pytest.approx(w.n_tokens * 10 / 0.250)
+    assert m["ms_per_step"] == pytest.approx(25.0)
+    g1 = m["stages"]["ffn_gemm1"]
+    assert g1["tflops"] == pytest.approx(2 * w.n_routes * w.H * 2 * w.I / 11.0e-3 / 1e12)
+    assert g1["frac_fp8"] == pytest.approx(g1["tflops"] / (2 * peaks["bf16_sus"]))
+    d = m["stages"]["dispatch"]
+    assert d["bytes"] == w.n_routes * w.H * 2 + 492544 * (w.H + w.H // 32)
+    assert "mxfp8_layer" not in bench.assemble_line(args, w, 1, 397.0, stage_ms, 90, None, 0, 0,
+                                                    None, None, None, 492544, peaks)
