@@ -19,23 +19,27 @@
 //   (internal.cuh): 512-byte atoms of 128 rows x 4 blocks of 32 values.
 //
 // Design: the forward FFN's persistent warp-specialised CTA-pair kernel
-// (expert_ffn.cu) with the block-scaled MMA. 256 x 256 tiles on a CTA pair
-// (tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale, M = 256, N = 256,
-// K = 32 per instruction); a pipeline stage holds 128 K values (one 128-byte
-// swizzled row per operand row, four MMAs) and their scales: the CTA's 128 A
-// rows (one atom, 512 bytes) and all 256 B columns (two atoms; each CTA of
-// the pair needs the scales of every column its rows meet). The producer
-// loads codes and scale atoms with TMA (pair form; each CTA fetches its own
-// copy). The MMA thread moves a stage's scales into TMEM with three tcgen05.cp (32x128b,
-// replicated into the four lane quarters: 4 columns for A, 8 for B) and then
-// issues the stage's four MMAs, each naming its scale byte (0..3) of the
-// 32-bit cells. Scale slots in TMEM follow the smem stages: a slot is
-// rewritten only after the MMAs that read it completed (the stage's empty
-// barrier came first).
-// TMEM: one 256-column fp32 accumulator plus STAGES x 16 scale columns.
-// Double buffering the accumulator would need all 512 columns and leave none
-// for the scales, so the epilogue of a tile is not overlapped with the next
-// tile's MMAs.
+// (expert_ffn.cu) with the block-scaled MMA
+// (tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale, M = 256, K = 32 per
+// instruction). A pipeline stage holds 128 K values (one 128-byte swizzled
+// row per operand row, four MMAs) and their scales: one 512-byte atom for the
+// CTA's 128 A rows and one atom per 128 columns of the tile (each CTA of the
+// pair needs the scales of every column its rows meet). The producer loads
+// codes and scale atoms with TMA (pair form; each CTA fetches its own copy).
+// The MMA thread moves a stage's scales into TMEM with tcgen05.cp (32x128b,
+// replicated into the four lane quarters: 4 columns per atom) and then issues
+// the stage's four MMAs, each naming its scale byte (0..3) of the 32-bit
+// cells. Scale slots in TMEM follow the smem stages: a slot is rewritten only
+// after the MMAs that read it completed (the stage's empty barrier came
+// first). TMEM holds the accumulators and STAGES x 8 or 16 scale columns:
+//   GEMM1  256 x 256 tiles (128 h columns through W1 and W3, CTA 0 holding
+//          W1's rows and CTA 1 W3's), one 256-column accumulator: a second
+//          would leave no columns for the scales, so a tile's epilogue is not
+//          overlapped with the next tile's MMAs (it writes 1 byte per h value
+//          and costs little against a 56-stage K loop);
+//   GEMM2  256 x 128 tiles, two 128-column accumulators: the next tile's MMAs
+//          run while the epilogue streams the fp32 y tile out (the larger
+//          epilogue, against a 16-stage K loop).
 //
 // Every output element is produced by one CTA pair in a fixed K order (no
 // split-K, no atomics): the result is deterministic and independent of which
@@ -61,28 +65,30 @@ template <int MODE>
 struct MxCfg {
   static constexpr bool TMA_STORE = MODE == 1;
   static constexpr int STAGING_BYTES = TMA_STORE ? 8 * 4096 : 0;  // 8 warps x 32x32 fp32
-  static constexpr int BM = 256, BN = 256;
+  static constexpr int BM = 256;
+  static constexpr int BN = MODE == 0 ? 256 : 128;     // accumulator columns per tile
+  static constexpr int ACC = MODE == 0 ? 1 : 2;        // accumulators in TMEM
   static constexpr int BK = 128;                       // E4M3 values (bytes) per stage
   static constexpr int MMA_K = 32;                     // K of one block-scaled MMA
+  static constexpr int B_ROWS = BN / 2;                // B rows (tile columns) per CTA
   static constexpr int A_BYTES = 128 * BK;             // this CTA's 128 rows
-  static constexpr int B_BYTES = 128 * BK;             // this CTA's 128 of the 256 columns
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KB
-  static constexpr int SFA_BYTES = 512;                  // 128 rows x 4 scales
-  static constexpr int SFB_BYTES = 1024;                 // 256 columns x 4 scales
-  static constexpr int SF_STAGE_BYTES = SFA_BYTES + SFB_BYTES;
-  static constexpr int STAGES = TMA_STORE ? 5 : 6;
-  static constexpr int TMEM_SF = BN;    // scale columns follow the accumulator
-  static constexpr int SF_COLS = 16;    // per stage: A at +0 (4), B at +4 (8)
+  static constexpr int B_BYTES = B_ROWS * BK;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KB / 24 KB
+  static constexpr int SFB_ATOMS = BN / 128;             // scale atoms of the tile's columns
+  static constexpr int SF_STAGE_BYTES = 512 * (1 + SFB_ATOMS);
+  static constexpr int STAGES = MODE == 0 ? 6 : 7;
+  static constexpr int TMEM_SF = ACC * BN;              // scale columns follow the accumulators
+  static constexpr int SF_COLS = 4 * (1 + SFB_ATOMS) <= 8 ? 8 : 16;  // A at +0, B at +4
   static_assert(TMEM_SF + STAGES * SF_COLS <= kTmemCols, "TMEM budget");
   static constexpr uint32_t IDESC = idesc_mxf8_e4m3(BM, BN, 0, 0);
   static constexpr int BAR_FULL = 0;
   static constexpr int BAR_EMPTY = STAGES;
   static constexpr int BAR_TFULL = 2 * STAGES;
-  static constexpr int BAR_TEMPTY = 2 * STAGES + 1;
-  static constexpr int BAR_DRAIN = 2 * STAGES + 2;
-  static constexpr int BAR_TID_FULL = 2 * STAGES + 3;
-  static constexpr int BAR_TID_EMPTY = 2 * STAGES + 3 + kRing;
-  static constexpr int NUM_BARS = 2 * STAGES + 3 + 2 * kRing;
+  static constexpr int BAR_TEMPTY = 2 * STAGES + ACC;
+  static constexpr int BAR_DRAIN = 2 * STAGES + 2 * ACC;
+  static constexpr int BAR_TID_FULL = BAR_DRAIN + 1;
+  static constexpr int BAR_TID_EMPTY = BAR_TID_FULL + kRing;
+  static constexpr int NUM_BARS = BAR_TID_EMPTY + kRing;
   // readers of each tile id: producer, MMA issuer and 8 epilogue warps of the
   // leader; producer and 8 epilogue warps of the follower
   static constexpr int TID_CONSUMERS = 19;
@@ -173,8 +179,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       mbar_init(smem_u32(&bars[C::BAR_FULL + i]), 1);
       mbar_init(smem_u32(&bars[C::BAR_EMPTY + i]), 1);
     }
-    mbar_init(smem_u32(&bars[C::BAR_TFULL]), 1);
-    mbar_init(smem_u32(&bars[C::BAR_TEMPTY]), kNumEpiWarps * 2);
+    for (int i = 0; i < C::ACC; ++i) {
+      mbar_init(smem_u32(&bars[C::BAR_TFULL + i]), 1);
+      mbar_init(smem_u32(&bars[C::BAR_TEMPTY + i]), kNumEpiWarps * 2);
+    }
     mbar_init(smem_u32(&bars[C::BAR_DRAIN]), 1);
     for (int i = 0; i < kRing; ++i) {
       mbar_init(smem_u32(&bars[C::BAR_TID_FULL + i]), 1);
@@ -207,8 +215,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   if (bad_sched && tid == 0) atomicOr(p.dev_status, MOE_DEV_BAD_SCHEDULE);
 
   const int rows_used = bad_sched ? 0 : s_off[E];
-  // GEMM1: a tile's 256 accumulator columns are 128 h columns seen through W1 and W3
-  const int tiles_n = (MODE == 0) ? p.Nout / 128 : p.Nout / C::BN;
+  // GEMM1: a tile's 256 accumulator columns are 128 h columns seen through W1
+  // and W3; GEMM2: 128 y columns
+  const int tiles_n = p.Nout / 128;
   const int num_tiles = (rows_used / C::BM) * tiles_n;
   const int kblocks = p.K / C::BK;  // stages per tile = scale atoms per 128-row block
   const WaitCtx wc{abort_flag, p.dev_status, p.timeout_ns, MOE_DEV_TIMEOUT};
@@ -242,8 +251,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const int arow = row0 + static_cast<int>(rank) * 128;
         // B rows (of the transposed weights) this tile meets: GEMM1: W1t and
         // W3t rows l*I + n*128 .. +128 (CTA 0 loads W1t's, CTA 1 W3t's);
-        // GEMM2: W2t rows l*H + n*256 .. +256 (CTA r loads 128 r .. +128)
-        const int brow = (MODE == 0) ? l * p.Nout + n * 128 : l * p.Nout + n * C::BN;
+        // GEMM2: W2t rows l*H + n*128 .. +128 (CTA r loads 64 r .. +64).
+        // Either way one scale atom per 128 rows.
+        const int brow = l * p.Nout + n * 128;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!wait_bounded(smem_u32(&bars[C::BAR_EMPTY + stage]), phase ^ 1u, wc)) {
             ok = false;
@@ -253,7 +263,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sB = sA + C::A_BYTES;
           const uint32_t sSA = smem_u32(sf + stage * C::SF_STAGE_BYTES);
-          const uint32_t sSB = sSA + C::SFA_BYTES;
+          const uint32_t sSB = sSA + 512;
           const int kx = kb * C::BK;
           if (leader) mbar_arrive_expect_tx(full0 + stage * 8, 2 * (C::STAGE_BYTES + C::SF_STAGE_BYTES));
           tma_load_2d_pair(sA, &tmA, kx, arow, full_tgt);
@@ -263,9 +273,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             tma_load_2d_pair(sSB, &tmSB0, 0, (brow / 128) * kblocks + kb, full_tgt);
             tma_load_2d_pair(sSB + 512, &tmSB1, 0, (brow / 128) * kblocks + kb, full_tgt);
           } else {
-            tma_load_2d_pair(sB, &tmB0, kx, brow + static_cast<int>(rank) * 128, full_tgt);
+            tma_load_2d_pair(sB, &tmB0, kx, brow + static_cast<int>(rank) * C::B_ROWS, full_tgt);
             tma_load_2d_pair(sSB, &tmSB0, 0, (brow / 128) * kblocks + kb, full_tgt);
-            tma_load_2d_pair(sSB + 512, &tmSB0, 0, (brow / 128 + 1) * kblocks + kb, full_tgt);
           }
           ++issued;
           if (++stage == C::STAGES) {
@@ -287,6 +296,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
+      int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       int tpos = 0;
@@ -296,12 +306,13 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         if (tile < 0) break;
         int row0, n, l;
         if (!tile_info(tile, row0, n, l)) continue;
-        // the single accumulator is free once both CTAs' epilogues drained it
-        if (!wait_bounded<true>(smem_u32(&bars[C::BAR_TEMPTY]), acc_phase ^ 1u, wc)) {
+        // an accumulator is free once both CTAs' epilogues drained it
+        if (!wait_bounded<true>(smem_u32(&bars[C::BAR_TEMPTY + acc]), acc_phase ^ 1u, wc)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!wait_bounded(smem_u32(&bars[C::BAR_FULL + stage]), phase, wc)) {
             ok = false;
@@ -311,12 +322,15 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sB = sA + C::A_BYTES;
           const uint32_t sSA = smem_u32(sf + stage * C::SF_STAGE_BYTES);
-          const uint32_t sSB = sSA + C::SFA_BYTES;
+          const uint32_t sSB = sSA + 512;
           const uint32_t tsf = tmem_base + static_cast<uint32_t>(C::TMEM_SF + stage * C::SF_COLS);
-          // 32 rows x 16 bytes per copy: four 8-row core matrices 128 bytes apart
+          // 32 rows x 16 bytes per copy: four 8-row core matrices 128 bytes
+          // apart. A's atom -> columns +0..3; B's atoms -> +4..7 (+8..11):
+          // tile column c reads its scales at column +4 + c/32
           tc_cp_pair_32x128b_x4(tsf, smem_desc_noswz(sSA, 128));
-          tc_cp_pair_32x128b_x4(tsf + 4, smem_desc_noswz(sSB, 128));
-          tc_cp_pair_32x128b_x4(tsf + 8, smem_desc_noswz(sSB + 512, 128));
+#pragma unroll
+          for (int a = 0; a < C::SFB_ATOMS; ++a)
+            tc_cp_pair_32x128b_x4(tsf + 4 + 4 * a, smem_desc_noswz(sSB + 512 * a, 128));
 #pragma unroll
           for (int kk = 0; kk < C::BK / C::MMA_K; ++kk) {
             // K-major: 32 E4M3 = 32 bytes inside the 128-byte swizzled row
@@ -324,7 +338,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             const uint64_t b_desc = smem_desc_sw128(sB + kk * 32, 16, 1024);
             const uint32_t sel = static_cast<uint32_t>(kk);
             const uint32_t idesc = C::IDESC | (sel << 29) | (sel << 4);
-            tc_mma_mx_pair(tmem_base, a_desc, b_desc, idesc, tsf | (sel << 30),
+            tc_mma_mx_pair(d_tmem, a_desc, b_desc, idesc, tsf | (sel << 30),
                            (tsf + 4) | (sel << 30), (kb | kk) != 0 ? 1u : 0u);
           }
           tc_commit_pair_mc(smem_u32(&bars[C::BAR_EMPTY + stage]), 0x3);
@@ -334,8 +348,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           }
         }
         if (!ok) break;
-        tc_commit_pair_mc(smem_u32(&bars[C::BAR_TFULL]), 0x3);
-        acc_phase ^= 1u;
+        tc_commit_pair_mc(smem_u32(&bars[C::BAR_TFULL + acc]), 0x3);
+        if (++acc == C::ACC) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
       }
       tc_commit_pair(smem_u32(&bars[C::BAR_DRAIN]));
       wait_drain(smem_u32(&bars[C::BAR_DRAIN]), 0, p.timeout_ns);
@@ -347,7 +364,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                    // TMEM lane quarter of this warp
     const int half = (warp - kEpiWarp0) >> 2;  // which half of the tile's columns
-    const uint32_t tempty_tgt = mapa_shared(smem_u32(&bars[C::BAR_TEMPTY]), 0);
+    const uint32_t tempty_tgt0 = mapa_shared(smem_u32(&bars[C::BAR_TEMPTY]), 0);
+    int acc = 0;
     uint32_t acc_phase = 0;
     int tpos = 0;
     uint32_t tph = 0;
@@ -358,10 +376,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       if (tile < 0) break;
       int row0, n, l;
       if (!tile_info(tile, row0, n, l)) continue;
-      if (!wait_bounded(smem_u32(&bars[C::BAR_TFULL]), acc_phase, wc)) break;
+      if (!wait_bounded(smem_u32(&bars[C::BAR_TFULL + acc]), acc_phase, wc)) break;
       tc_fence_after();
       const int64_t row = row0 + static_cast<int>(rank) * 128 + q * 32 + lane;
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::BN);
       if (MODE == 0) {
         // accumulator columns [0,128) = x.W1, [128,256) = x.W3 for h columns
         // n*128 + j; this warp's 64 columns are two 32-column MX blocks of h
@@ -389,12 +408,12 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         // store has read it
         const uint32_t stg = smem_u32(staging) + (warp - kEpiWarp0) * 4096;
         const uint64_t pol_y = l2_policy_evict_first();
-        const int ycol = n * C::BN + half * 128;
+        const int ycol = n * C::BN + half * 64;  // this warp's 64 of the tile's 128 columns
         const int yrow0 = row0 + static_cast<int>(rank) * 128 + q * 32;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t rv[32];
-          tmem_ld_32cols(tbase + half * 128 + c * 32, rv);
+          tmem_ld_32cols(tbase + half * 64 + c * 32, rv);
           tmem_ld_wait();
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();
@@ -413,8 +432,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       // the accumulator may be refilled once every lane's tcgen05.ld completed
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_relaxed_cluster(tempty_tgt);
-      acc_phase ^= 1u;
+      if (lane == 0) mbar_arrive_relaxed_cluster(tempty_tgt0 + acc * 8);
+      if (++acc == C::ACC) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
     if (C::TMA_STORE && lane == 0) bulk_wait_all();  // stores complete before the CTA exits
   }
@@ -458,7 +480,7 @@ cudaError_t launch_expert_ffn_mxfp8(const uint8_t* xq, const uint8_t* xs, const 
       !make_map_u8(&mW3, W3q, H, EI, 128, 128) ||
       !make_map_sf_atoms(&mW3s, W3s, EI / 128 * (H / 128)) ||
       !make_map_u8(&mHq, hq, I, rows_max, 128, 128) || !make_map_sf_atoms(&mHs, hs, rb * (I / 128)) ||
-      !make_map_u8(&mW2, W2q, I, EH, 128, 128) ||
+      !make_map_u8(&mW2, W2q, I, EH, 128, 64) ||   // GEMM2: 64 B rows per CTA
       !make_map_sf_atoms(&mW2s, W2s, EH / 128 * (I / 128)) ||
       !make_map(&mY, y, H, rows_max, 32, 32, true))
     return cudaErrorInvalidValue;

@@ -21,11 +21,19 @@ SMEM_LIMIT = 232448              # 227 KB of dynamic shared memory per CTA
 K_RING = 4
 
 
+# per MODE: tile columns, accumulators, stages, B rows per CTA, scale atoms of B
+GEOM = {0: dict(BN=256, ACC=1, STAGES=6, B_ROWS=128, SFB=2),
+        1: dict(BN=128, ACC=2, STAGES=7, B_ROWS=64, SFB=1)}
+
+
 def _smem_bytes(mode: int, E: int) -> int:
-    stages = 5 if mode == 1 else 6
+    g = GEOM[mode]
+    stage = 128 * BK + g["B_ROWS"] * BK
+    sf_stage = 512 * (1 + g["SFB"])
     staging = 8 * 4096 if mode == 1 else 0
-    num_bars = 2 * stages + 3 + 2 * K_RING
-    return 1024 + stages * (32768 + 1536) + staging + num_bars * 8 + 16 + K_RING * 4 + (2 * E + 1) * 4
+    num_bars = 2 * g["STAGES"] + 2 * g["ACC"] + 1 + 2 * K_RING
+    return (1024 + g["STAGES"] * (stage + sf_stage) + staging + num_bars * 8 + 16 + K_RING * 4
+            + (2 * E + 1) * 4)
 
 
 def _tiles(s_off: np.ndarray, s_end: np.ndarray, E: int, tiles_n: int):
@@ -51,7 +59,7 @@ def _tiles(s_off: np.ndarray, s_end: np.ndarray, E: int, tiles_n: int):
 def _check_mode(mode: int, sh: dict, s_off, s_end, rows_max: int):
     E, H, I = sh["E"], sh["H"], sh["I"]
     K, Nout = (H, I) if mode == 0 else (I, H)
-    tiles_n = Nout // 128 if mode == 0 else Nout // 256
+    tiles_n = Nout // 128
     kb_max = K // BK - 1
     valid, row0, n, l = _tiles(s_off, s_end, E, tiles_n)
     # a tile never straddles two experts, and every (row tile, column block)
@@ -71,9 +79,9 @@ def _check_mode(mode: int, sh: dict, s_off, s_end, rows_max: int):
             assert (brow + 128 <= E * I).all()
             assert ((brow // 128) * (K // BK) + kb_max < E * I // 128 * (K // BK)).all()
         else:
-            brow = l * H + n * 256                       # W2t rows of the tile
-            assert (brow + 128 * rank + 128 <= E * H).all()
-            assert ((brow // 128 + 1) * (K // BK) + kb_max < E * H // 128 * (K // BK)).all()
+            brow = l * H + n * 128                       # W2t rows of the tile
+            assert (brow + 64 * rank + 64 <= E * H).all()
+            assert ((brow // 128) * (K // BK) + kb_max < E * H // 128 * (K // BK)).all()
     # epilogue: rows row0 .. row0 + 255 of the tile
     last_row = row0 + 255
     assert (last_row < rows_max).all()
@@ -84,8 +92,8 @@ def _check_mode(mode: int, sh: dict, s_off, s_end, rows_max: int):
         last_sc = ((last_row // 128) * (kblk // 4) + (kblk - 1) // 4) * 512 + 31 * 16 + 3 * 4 + 3
         assert (last_sc < rows_max * I // 32).all()
     else:
-        # y: 32 x 32 fp32 boxes at (n*256 + half*128 + c*32, row0 + rank*128 + q*32)
-        assert (n * 256 + 128 + 3 * 32 + 32 <= H).all()
+        # y: 32 x 32 fp32 boxes at (n*128 + half*64 + c*32, row0 + rank*128 + q*32)
+        assert (n * 128 + 64 + 32 + 32 <= H).all()
 
 
 @pytest.mark.parametrize("name", ["tiny", "tiny_bwd", "mid", "kimi", "zipf", "kimi_e16"])
@@ -105,10 +113,12 @@ def test_mx_ffn_tiles_stay_inside_their_buffers(name):
 @pytest.mark.parametrize("E", [1, 8, 384, 1024])
 def test_mx_ffn_budgets(E):
     for mode in (0, 1):
+        g = GEOM[mode]
         assert _smem_bytes(mode, E) <= SMEM_LIMIT
-    stages = 6
-    assert 256 + stages * 16 <= 512              # accumulator + scale columns in TMEM
-    assert (256 + stages * 16 - 4) % 4 == 0      # each scale copy starts on a 4-column boundary
+        sf_cols = 8 if g["SFB"] == 1 else 16
+        assert g["ACC"] * g["BN"] + g["STAGES"] * sf_cols <= 512   # accumulators + scales
+        assert 4 * (1 + g["SFB"]) <= sf_cols                        # A atom + B atoms per stage
+        assert (g["ACC"] * g["BN"]) % 4 == 0 and sf_cols % 4 == 0   # copies start on 4 columns
 
 
 @pytest.mark.parametrize("E,K,N", [(1, 128, 128), (3, 256, 384), (384, 7168, 2048), (384, 2048, 7168)])
