@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;  // TMA_STORE only (1024-aligned)
-  uint8_t* sf = staging + C::STAGING_BYTES;              // [STAGES] x {A atom, 2 B atoms}
+  uint8_t* sf = staging + C::STAGING_BYTES;              // [STAGES] x {A atom, B atoms}
   uint64_t* bars = reinterpret_cast<uint64_t*>(sf + C::STAGES * C::SF_STAGE_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
