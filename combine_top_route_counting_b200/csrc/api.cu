@@ -83,6 +83,7 @@ struct LayerWs {
   size_t ids, gates, route_row, phi, offsets, counts, sched, xg, h, y, total;
   size_t logits[2], x[2], out[2], total_host;  // moe_layer_forward_host additions
   size_t ab, dys, dab, hg, gate_row, part, total_train;  // training additions
+  size_t sh_off, sh_x, sh_h, sh_y, total_mx;  // the MXFP8 layer's shared expert
 };
 
 LayerWs layer_ws(const moe_shape_t* s) {
@@ -122,6 +123,13 @@ LayerWs layer_ws(const moe_shape_t* s) {
   w.gate_row = take(ot, rows * 4);
   w.part = take(ot, rows * (s->I / 128) * 4);
   w.total_train = ot;
+  size_t om = o;
+  const size_t tok_rows = (tokens + 255) / 256 * 256;
+  w.sh_off = take(om, 8);
+  w.sh_x = take(om, tokens % 256 ? tok_rows * s->H * 2 : 0);  // padded copy of x, ragged only
+  w.sh_h = take(om, tok_rows * s->I * 2);
+  w.sh_y = take(om, tok_rows * s->H * 4);
+  w.total_mx = om;
   return w;
 }
 
@@ -240,7 +248,8 @@ moe_status_t layer_body(const float* logits, const uint16_t* x, const uint16_t* 
 // ev (7 events, may be null) as moe_layer_forward.
 cudaError_t layer_body_mx(const float* logits, const uint16_t* x, const uint8_t* W1q,
                           const uint8_t* W1s, const uint8_t* W3q, const uint8_t* W3s,
-                          const uint8_t* W2q, const uint8_t* W2s, uint16_t* out, void* ws,
+                          const uint8_t* W2q, const uint8_t* W2s, const uint16_t* Ws1,
+                          const uint16_t* Ws3, const uint16_t* Ws2, uint16_t* out, void* ws,
                           int32_t* dev_status, const moe_shape_t* sh, cudaStream_t s,
                           void* const* ev) {
   const LayerWs w = layer_ws(sh);
@@ -272,13 +281,24 @@ cudaError_t layer_body_mx(const float* logits, const uint16_t* x, const uint8_t*
                                  /*tiled=*/true)) != cudaSuccess)
     return e;
   if ((e = rec(3)) != cudaSuccess) return e;
+  // the bf16 shared expert over every token (its time counts in stage 3, the
+  // routed GEMM1's); nothing on one GPU to overlap it with
+  float* ys = nullptr;
+  if (Ws1) {
+    ys = at<float>(ws, w.sh_y);
+    if ((e = launch_dense_ffn(x, static_cast<int64_t>(sh->P) * sh->N, Ws1, Ws3, Ws2,
+                              at<uint16_t>(ws, w.sh_x), at<uint16_t>(ws, w.sh_h), ys,
+                              at<int32_t>(ws, w.sh_off), sh->H,
+                              sh->I, dev_status, s)) != cudaSuccess)
+      return e;
+  }
   cudaEvent_t mid = ev ? static_cast<cudaEvent_t>(ev[4]) : nullptr;
   if ((e = launch_expert_ffn_mxfp8(xq, xs, W1q, W1s, W3q, W3s, W2q, W2s, b.offsets, b.counts, hq,
                                    hs, b.y, *sh, rows_max, dev_status, s, mid)) != cudaSuccess)
     return e;
   if ((e = rec(5)) != cudaSuccess) return e;
   if ((e = launch_combine(b.y, b.route_row, b.gates, out, *sh, Slice{0, sh->N}, rows_max,
-                          dev_status, s)) != cudaSuccess)
+                          dev_status, s, ys)) != cudaSuccess)
     return e;
   return rec(6);
 }
@@ -861,9 +881,15 @@ moe_status_t moe_expert_ffn_mxfp8(const uint8_t* xq, const uint8_t* xs, const ui
                                            static_cast<cudaStream_t>(stream), nullptr));
 }
 
+size_t moe_layer_mxfp8_workspace_bytes(const moe_shape_t* shape) {
+  if (check_mx_shape(shape) != MOE_OK) return 0;
+  return layer_ws(shape).total_mx;
+}
+
 moe_status_t moe_layer_forward_mxfp8(const float* logits, const uint16_t* x, const uint8_t* W1q,
                                      const uint8_t* W1s, const uint8_t* W3q, const uint8_t* W3s,
-                                     const uint8_t* W2q, const uint8_t* W2s, uint16_t* out,
+                                     const uint8_t* W2q, const uint8_t* W2s, const uint16_t* Ws1,
+                                     const uint16_t* Ws3, const uint16_t* Ws2, uint16_t* out,
                                      void* ws, size_t ws_bytes, int32_t* dev_status,
                                      const moe_shape_t* shape, void* stream,
                                      void* const* stage_events) {
@@ -872,13 +898,17 @@ moe_status_t moe_layer_forward_mxfp8(const float* logits, const uint16_t* x, con
   if (!W1q || !W1s || !W3q || !W3s || !W2q || !W2s || !ws || !dev_status ||
       (shape->N > 0 && (!logits || !x || !out)))
     return MOE_INVALID_ARG;
+  const bool shared = Ws1 || Ws3 || Ws2;
+  if (shared && !(Ws1 && Ws3 && Ws2)) return MOE_INVALID_ARG;  // all three or none
   if (!aligned16(logits) || !aligned16(x) || !aligned16(W1q) || !aligned16(W1s) ||
       !aligned16(W3q) || !aligned16(W3s) || !aligned16(W2q) || !aligned16(W2s) ||
-      !aligned16(out) || !aligned32(ws))
+      !aligned16(Ws1) || !aligned16(Ws3) || !aligned16(Ws2) || !aligned16(out) || !aligned32(ws))
     return MOE_INVALID_ARG;
-  if (ws_bytes < layer_ws(shape).total) return MOE_WORKSPACE_TOO_SMALL;
-  return from_cuda(layer_body_mx(logits, x, W1q, W1s, W3q, W3s, W2q, W2s, out, ws, dev_status,
-                                 shape, static_cast<cudaStream_t>(stream), stage_events));
+  const LayerWs w = layer_ws(shape);
+  if (ws_bytes < (shared ? w.total_mx : w.total)) return MOE_WORKSPACE_TOO_SMALL;
+  return from_cuda(layer_body_mx(logits, x, W1q, W1s, W3q, W3s, W2q, W2s, Ws1, Ws3, Ws2, out, ws,
+                                 dev_status, shape, static_cast<cudaStream_t>(stream),
+                                 stage_events));
 }
 
 int64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

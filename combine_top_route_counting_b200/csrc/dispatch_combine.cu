@@ -97,14 +97,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // K > 0: compile-time k; K == 0: runtime k (<= kMaxK). gates == null: unit
-// weights (fmaf(1, v, acc) is the rounded sum acc + v).
-template <int K>
+// weights (fmaf(1, v, acc) is the rounded sum acc + v). SHARED: the sum
+// starts from the shared expert's output row shared[t] instead of 0 (the
+// shared expert as a slot before slot 0 with gate 1).
+template <int K, bool SHARED = false>
 __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ y,
                                                       const int32_t* __restrict__ route_row,
                                                       const float* __restrict__ gates,
                                                       uint2* __restrict__ out, int N, int k, int H,
                                                       int t0, int Tm, int64_t rows_max,
-                                                      int32_t* dev_status) {
+                                                      int32_t* dev_status,
+                                                      const float4* __restrict__ shared) {
   constexpr int KM = K > 0 ? K : kMaxK;
   const int kk = K > 0 ? K : k;
   const int64_t b = blockIdx.x;  // token of the slice, peer-major
@@ -134,6 +137,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
     for (int j = 0; j < KM; ++j)
       if (j < kk && rows[j] >= 0) val[j] = __ldg(y + rows[j] * nv + v);
     float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (SHARED) acc = __ldg(shared + t * nv + v);
 #pragma unroll
     for (int j = 0; j < KM; ++j) {
       if (j < kk && rows[j] >= 0) {
@@ -185,21 +189,29 @@ cudaError_t launch_reverse_combine(const uint16_t* dout, const int32_t* phi,
 
 cudaError_t launch_combine(const float* y, const int32_t* route_row, const float* gates,
                            uint16_t* out, const moe_shape_t& sh, Slice sl, int64_t rows_max,
-                           int32_t* dev_status, cudaStream_t s) {
+                           int32_t* dev_status, cudaStream_t s, const float* shared) {
   const int64_t tokens = static_cast<int64_t>(sh.P) * sl.Tm;
   if (tokens == 0) return cudaSuccess;
   const float4* y4 = reinterpret_cast<const float4*>(y);
+  const float4* s4 = reinterpret_cast<const float4*>(shared);
   uint2* o2 = reinterpret_cast<uint2*>(out);
   const unsigned grid = static_cast<unsigned>(tokens);
-#define MOE_COMBINE(KV)                                                                       \
-  combine_kernel<KV><<<grid, 256, 0, s>>>(y4, route_row, gates, o2, sh.N, sh.k, sh.H, sl.t0, \
-                                          sl.Tm, rows_max, dev_status)
-  switch (sh.k) {
-    case 1: MOE_COMBINE(1); break;
-    case 2: MOE_COMBINE(2); break;
-    case 4: MOE_COMBINE(4); break;
-    case 8: MOE_COMBINE(8); break;
-    default: MOE_COMBINE(0); break;
+#define MOE_COMBINE(KV, SH)                                                                     \
+  combine_kernel<KV, SH><<<grid, 256, 0, s>>>(y4, route_row, gates, o2, sh.N, sh.k, sh.H, sl.t0, \
+                                              sl.Tm, rows_max, dev_status, s4)
+  if (shared) {
+    switch (sh.k) {
+      case 8: MOE_COMBINE(8, true); break;
+      default: MOE_COMBINE(0, true); break;
+    }
+  } else {
+    switch (sh.k) {
+      case 1: MOE_COMBINE(1, false); break;
+      case 2: MOE_COMBINE(2, false); break;
+      case 4: MOE_COMBINE(4, false); break;
+      case 8: MOE_COMBINE(8, false); break;
+      default: MOE_COMBINE(0, false); break;
+    }
   }
 #undef MOE_COMBINE
   note_launches(1);

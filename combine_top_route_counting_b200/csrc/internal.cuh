@@ -53,10 +53,22 @@ cudaError_t launch_expert_ffn_gather(const uint16_t* x, const int32_t* phi, cons
                                      float* y, const moe_shape_t& sh, int64_t rows_max,
                                      int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_mid);
 
-// Step 4
+// Step 4. shared (optional, fp32 [P*N rows, H]): the shared expert's output,
+// the start of each token's fixed-order sum.
 cudaError_t launch_combine(const float* y, const int32_t* route_row, const float* gates,
                            uint16_t* out, const moe_shape_t& sh, Slice sl, int64_t rows_max,
-                           int32_t* dev_status, cudaStream_t s);
+                           int32_t* dev_status, cudaStream_t s, const float* shared = nullptr);
+
+// The bf16 shared expert: the SwiGLU FFN of every token x[t] (t < n_tokens)
+// with one set of weights Ws1, Ws3 [H, I], Ws2 [I, H], run as the one segment
+// of launch_expert_ffn over round_up(n_tokens, 256) rows. hs bf16 and ys fp32
+// have that many rows. xpad ([rows, H] bf16) takes a zero-padded copy of x
+// when n_tokens is not a multiple of 256 (else x is read in place and xpad
+// may be null); off: device int32[2] scratch for the one-segment table.
+cudaError_t launch_dense_ffn(const uint16_t* x, int64_t n_tokens, const uint16_t* Ws1,
+                             const uint16_t* Ws3, const uint16_t* Ws2, uint16_t* xpad,
+                             uint16_t* hs, float* ys, int32_t* off, int32_t H, int32_t I,
+                             int32_t* dev_status, cudaStream_t s);
 
 // 2D tensor map over [outer, inner] (inner contiguous) bf16 (or fp32)
 // elements with box [box_outer, box_inner] and 128-byte swizzle; false if the

@@ -92,8 +92,9 @@ _SIGS = {
     "moe_mx_quantize_weights": ([_vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp],
                                 ctypes.c_int),
     "moe_expert_ffn_mxfp8": ([_vp] * 14 + [ctypes.POINTER(Shape), _vp], ctypes.c_int),
-    "moe_layer_forward_mxfp8": ([_vp] * 10 + [ctypes.c_size_t, _vp, ctypes.POINTER(Shape), _vp,
+    "moe_layer_forward_mxfp8": ([_vp] * 13 + [ctypes.c_size_t, _vp, ctypes.POINTER(Shape), _vp,
                                               ctypes.POINTER(_vp)], ctypes.c_int),
+    "moe_layer_mxfp8_workspace_bytes": ([ctypes.POINTER(Shape)], ctypes.c_size_t),
     "moe_launch_count": ([], ctypes.c_int64),
     "moe_selftest_bounded_wait": ([_vp, ctypes.c_int64, _vp], ctypes.c_int),
 }
@@ -167,6 +168,10 @@ def layer_workspace_bytes(sh: Shape) -> int:
 
 def layer_host_workspace_bytes(sh: Shape) -> int:
     return int(load().moe_layer_host_workspace_bytes(ctypes.byref(sh)))
+
+
+def layer_mxfp8_workspace_bytes(sh: Shape) -> int:
+    return int(load().moe_layer_mxfp8_workspace_bytes(ctypes.byref(sh)))
 
 
 def train_workspace_bytes(sh: Shape) -> int:
@@ -452,12 +457,15 @@ def moe_expert_ffn_mxfp8(xq, xs, W1q, W1s, W3q, W3s, W2q, W2s, offsets, counts, 
 
 
 def moe_layer_forward_mxfp8(logits, x, W1q, W1s, W3q, W3s, W2q, W2s, out, ws, dev_status,
-                            sh: Shape, stream=None, stage_events=None):
-    u8 = torch.uint8
+                            sh: Shape, stream=None, stage_events=None, shared=None):
+    """shared: None, or the bf16 shared expert's (Ws1 [H, I], Ws3 [H, I], Ws2 [I, H])."""
+    u8, bf = torch.uint8, torch.bfloat16
+    Ws = shared if shared is not None else (None, None, None)
     _check(load().moe_layer_forward_mxfp8(
-        _ptr(logits, torch.float32, "logits"), _ptr(x, torch.bfloat16, "x"),
+        _ptr(logits, torch.float32, "logits"), _ptr(x, bf, "x"),
         _ptr(W1q, u8, "W1q"), _ptr(W1s, u8, "W1s"), _ptr(W3q, u8, "W3q"), _ptr(W3s, u8, "W3s"),
-        _ptr(W2q, u8, "W2q"), _ptr(W2s, u8, "W2s"), _ptr(out, torch.bfloat16, "out"),
+        _ptr(W2q, u8, "W2q"), _ptr(W2s, u8, "W2s"), _ptr(Ws[0], bf, "Ws1"), _ptr(Ws[1], bf, "Ws3"),
+        _ptr(Ws[2], bf, "Ws2"), _ptr(out, bf, "out"),
         _ptr(ws, u8, "ws"), ws.numel(), _ptr(dev_status, torch.int32, "dev_status"),
         ctypes.byref(sh), _stream(stream), _events(stage_events)), "moe_layer_forward_mxfp8")
 

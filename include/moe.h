@@ -462,14 +462,29 @@ moe_status_t moe_expert_ffn_mxfp8(const uint8_t* xq, const uint8_t* xs, const ui
                                   const int32_t* counts, uint8_t* hq, uint8_t* hs, float* y,
                                   int32_t* dev_status, const moe_shape_t* shape, void* stream);
 
+/* Workspace of moe_layer_forward_mxfp8 with a shared expert: the layer's
+ * workspace plus the shared expert's h (bf16) and output (fp32) over every
+ * token (and a padded copy of x when P*N % 256 != 0). 0 if the shape is not
+ * supported. */
+size_t moe_layer_mxfp8_workspace_bytes(const moe_shape_t* shape);
+
 /* Steps 1-4 with MXFP8 routed experts: route, schedule, the quantising
  * dispatch (TILED scales), moe_expert_ffn_mxfp8 and the fixed-order combine,
- * on `stream`. Weights as moe_expert_ffn_mxfp8; ws of moe_layer_workspace_bytes
- * (the codes and scales of x and h take the places of xg and h);
- * stage_events as moe_layer_forward. Limits as moe_expert_ffn_mxfp8. */
+ * on `stream`. Routed weights as moe_expert_ffn_mxfp8.
+ * Ws1, Ws3 bf16 [H, I] and Ws2 bf16 [I, H] (all three, or all null): a bf16
+ * shared expert ("Mixture-of-Kittens", section 5) every token passes through,
+ * ys[t] = bf16(silu(x[t].Ws1) * (x[t].Ws3)).Ws2 in fp32 on the bf16 FFN's
+ * kernels; the combine then starts each token's fixed-order sum from it:
+ *   acc = ys[t]; acc = fmaf(g[t,j], y[route_row[t,j]], acc), j = 0..k-1;
+ *   out[t] = bf16_rne(acc).
+ * ws: moe_layer_workspace_bytes without a shared expert (the codes and scales
+ * of x and h take the places of xg and h), moe_layer_mxfp8_workspace_bytes
+ * with one. stage_events as moe_layer_forward (the shared expert falls
+ * between the third and fourth). Limits as moe_expert_ffn_mxfp8. */
 moe_status_t moe_layer_forward_mxfp8(const float* logits, const uint16_t* x, const uint8_t* W1q,
                                      const uint8_t* W1s, const uint8_t* W3q, const uint8_t* W3s,
-                                     const uint8_t* W2q, const uint8_t* W2s, uint16_t* out,
+                                     const uint8_t* W2q, const uint8_t* W2s, const uint16_t* Ws1,
+                                     const uint16_t* Ws3, const uint16_t* Ws2, uint16_t* out,
                                      void* ws, size_t ws_bytes, int32_t* dev_status,
                                      const moe_shape_t* shape, void* stream,
                                      void* const* stage_events);

@@ -471,7 +471,7 @@ def _bits_f64(b) -> np.ndarray:
     return (np.asarray(b, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def layer_tokens_mxfp8(logits, x_bits, weights, k: int, H: int, I: int, tokens):
+def layer_tokens_mxfp8(logits, x_bits, weights, k: int, H: int, I: int, tokens, shared=None):
     """The layer with MXFP8 routed experts ("Mixture-of-Kittens", section 5),
     for a set of tokens: every GEMM operand is MX-quantised along its reduction
     dimension -- x rows along H, W1/W3 along H (per column i), h rows along I,
@@ -479,6 +479,9 @@ def layer_tokens_mxfp8(logits, x_bits, weights, k: int, H: int, I: int, tokens):
     fp64 on the values the quantised operands stand for:
       a = mx(x).mx(W1), b = mx(x).mx(W3), h = silu(a) * b,
       y = mx(h).mx(W2), out[t] = sum_j g_j y_j (gates: fp64 softmax of the top k).
+    shared: None, or the bf16 shared expert's (Ws1 [H, I], Ws3 [H, I], Ws2
+    [I, H]) bit patterns; its output, the bf16 FFN of x[t] (ffn_rows), is
+    added to every token: out[t] += y_shared[t].
     Returns dict out64 [n, H], ids, gates64."""
     ids, g32, g64 = route_topk(logits, k)
     toks = np.asarray(list(tokens), np.int64)
@@ -501,6 +504,11 @@ def layer_tokens_mxfp8(logits, x_bits, weights, k: int, H: int, I: int, tokens):
             b = xt @ w3
             h = a / (1.0 + np.exp(-a)) * b
             out[a_i] += g64[t, j] * (mx_round(h) @ w2)
+    if shared is not None and len(toks):
+        Ws1, Ws3, Ws2 = shared
+        _, ys = ffn_rows(xb[toks], np.zeros(len(toks), np.int32), {0: Ws1}, {0: Ws3}, {0: Ws2},
+                         H, I)
+        out += ys
     return dict(out64=out, ids=ids, gates64=g64)
 
 

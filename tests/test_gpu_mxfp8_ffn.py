@@ -197,3 +197,38 @@ def test_layer_mxfp8_no_tokens(cuda_lib):
     x = torch.empty((0, w.H), dtype=torch.bfloat16, device=DEV)
     out = _layer_mx(moe, w, lg, x, Wq)
     assert out.numel() == 0
+
+
+def _shared_weights(w, seed=91):
+    g = torch.Generator().manual_seed(seed)
+    return [(torch.randn(shape, generator=g) * 0.02).to(torch.bfloat16)
+            for shape in ((w.H, w.I), (w.H, w.I), (w.I, w.H))]
+
+
+@pytest.mark.parametrize("name,n_tok", [("tiny", 256), ("mid", 48),
+                                        ("ragged", 120)])   # P*N % 256 != 0: padded copy of x
+def test_layer_mxfp8_shared_expert_vs_oracle(cuda_lib, name, n_tok):
+    moe = cuda_lib
+    w = (inputs.Workload("mx_ragged", 15, P=2, N=300, E=8, k=2, H=256, I=256)
+         if name == "ragged" else inputs.WORKLOADS[name])
+    lg, x = inputs.make_logits(w), inputs.make_x(w)
+    W = inputs.make_weights(w)
+    Ws = _shared_weights(w)
+    Wq = _mx_weights_gpu(moe, W)
+    sh = moe.shape(**w.shape())
+    ws = torch.empty(moe.layer_mxfp8_workspace_bytes(sh), dtype=torch.uint8, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = torch.empty((w.n_tokens, w.H), dtype=torch.bfloat16, device=DEV)
+    moe.moe_layer_forward_mxfp8(lg.to(DEV), x.to(DEV), *Wq, out, ws, st, sh,
+                                shared=tuple(t.to(DEV) for t in Ws))
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    toks = inputs.sample_tokens(w.n_tokens, n_tok, seed=w.wid)
+    o_ids, _, _ = oracle.route_topk(lg[toks], w.k)
+    Wh = expert_weights_host(*W, np.unique(o_ids))
+    res = oracle.layer_tokens_mxfp8(lg, bits(x), Wh, w.k, w.H, w.I, toks,
+                                    shared=tuple(bits(t) for t in Ws))
+    got = bf16_to_f64(bits(out[torch.tensor(toks, device=DEV)]))
+    err = rms_floor_err(got, res["out64"])
+    print(f"{name}: MXFP8 layer + shared expert rms-floor err {err:.3e}")
+    assert err < OUT_TOL

@@ -173,19 +173,28 @@ def test_mx_ffn_entry_points_argument_errors(lib):
     a = list(args)
     a[10] = ctypes.c_void_p(256 + 16)                                     # hq not 32-byte aligned
     assert L.moe_expert_ffn_mxfp8(*a) == 1
-    # the layer: same limits, the bf16 layer's workspace
+    # the layer: same limits; the bf16 layer's workspace without a shared
+    # expert, the larger MXFP8 one with it
     need = moe.layer_workspace_bytes(ok)
-    lay = [p] * 10 + [need - 1, p, ctypes.byref(ok), None, None]
+    need_sh = moe.layer_mxfp8_workspace_bytes(ok)
+    assert need_sh > need
+    lay = [p] * 8 + [None] * 3 + [p, p] + [need - 1, p, ctypes.byref(ok), None, None]
     assert L.moe_layer_forward_mxfp8(*lay) == 3
-    lay[10] = need
-    lay[9] = ctypes.c_void_p(256 + 16)                                    # ws not 32-byte aligned
+    lay[13] = need
+    lay[12] = ctypes.c_void_p(256 + 16)                                   # ws not 32-byte aligned
     assert L.moe_layer_forward_mxfp8(*lay) == 1
-    lay[9] = p
-    lay[12] = ctypes.byref(pad128)
+    lay[12] = p
+    lay[15] = ctypes.byref(pad128)
     assert L.moe_layer_forward_mxfp8(*lay) == 2
-    lay[12] = ctypes.byref(ok)
+    lay[15] = ctypes.byref(ok)
     lay[2] = None                                                         # W1q
     assert L.moe_layer_forward_mxfp8(*lay) == 1
+    lay[2] = p
+    lay[8] = p                                                            # Ws1 without Ws3, Ws2
+    assert L.moe_layer_forward_mxfp8(*lay) == 1
+    lay[9] = lay[10] = p                                                  # a shared expert needs
+    assert L.moe_layer_forward_mxfp8(*lay) == 3                           # the larger workspace
+    assert moe.layer_mxfp8_workspace_bytes(pad128) == 0
 
 
 def test_size_queries_hold_their_invariants_on_random_shapes(lib):

@@ -134,3 +134,46 @@ def test_ffn_rows_mxfp8_close_to_bf16_ffn():
     rel_h = np.sqrt(np.mean((h_mx - h_bf) ** 2) / np.mean(h_bf ** 2))
     assert 1e-3 < rel_h < 0.1, rel_h
     assert hs.shape == (w.n_tokens, w.I // 32)
+
+
+def _shared_case():
+    w = inputs.Workload("mx_shared", 14, P=1, N=16, E=4, k=2, H=128, I=64)
+    lg, x = inputs.make_logits(w), inputs.make_x(w)
+    W = inputs.make_weights(w)
+    g = torch.Generator().manual_seed(77)
+    Ws = [(torch.randn(shape, generator=g) * 0.02).to(torch.bfloat16)
+          for shape in ((w.H, w.I), (w.H, w.I), (w.I, w.H))]
+    return w, lg, x, W, Ws
+
+
+def test_layer_mxfp8_shared_expert_alone_is_a_dense_swiglu():
+    """With every routed W2 zero the routed experts add exact zeros, and the
+    layer is the shared expert alone: a dense bf16 SwiGLU (torch fp64 matmuls
+    on the bf16 weights, h rounded to bf16 as the FFN's operand)."""
+    w, lg, x, W, Ws = _shared_case()
+    Wr = [{e: bits(t[e]) for e in range(w.E)} for t in (W[0], W[1], torch.zeros_like(W[2]))]
+    toks = range(w.n_tokens)
+    res = oracle.layer_tokens_mxfp8(lg, bits(x), Wr, w.k, w.H, w.I, toks,
+                                    shared=tuple(bits(t) for t in Ws))
+    x64, w1, w3, w2 = (t.to(torch.float64) for t in (x, *Ws))
+    a, b = x64 @ w1, x64 @ w3
+    h = (torch.nn.functional.silu(a) * b).to(torch.bfloat16).to(torch.float64)
+    ref = (h @ w2).numpy()
+    assert np.allclose(res["out64"], ref, rtol=1e-12, atol=1e-15)
+
+
+def test_layer_mxfp8_shared_expert_adds_once_per_token_with_gate_one():
+    w, lg, x, W, Ws = _shared_case()
+    Wr = [{e: bits(t[e]) for e in range(w.E)} for t in W]
+    toks = range(w.n_tokens)
+    sb = lambda s2: (bits(Ws[0]), bits(Ws[1]), bits(s2))
+    base = oracle.layer_tokens_mxfp8(lg, bits(x), Wr, w.k, w.H, w.I, toks)["out64"]
+    zero = oracle.layer_tokens_mxfp8(lg, bits(x), Wr, w.k, w.H, w.I, toks,
+                                     shared=sb(torch.zeros_like(Ws[2])))["out64"]
+    one = oracle.layer_tokens_mxfp8(lg, bits(x), Wr, w.k, w.H, w.I, toks, shared=sb(Ws[2]))["out64"]
+    two = oracle.layer_tokens_mxfp8(lg, bits(x), Wr, w.k, w.H, w.I, toks,
+                                    shared=sb((Ws[2].float() * 2).to(torch.bfloat16)))["out64"]
+    assert np.array_equal(zero, base)                      # a zero shared expert adds nothing
+    d1, d2 = one - base, two - base
+    assert np.abs(d1).max() > 0
+    assert np.allclose(d2, 2 * d1, rtol=1e-12, atol=1e-15)  # linear in Ws2, weight 1, not gated
