@@ -479,6 +479,8 @@ def layer_tokens_mxfp8(logits, x_bits, weights, k: int, H: int, I: int, tokens, 
     fp64 on the values the quantised operands stand for:
       a = mx(x).mx(W1), b = mx(x).mx(W3), h = silu(a) * b,
       y = mx(h).mx(W2), out[t] = sum_j g_j y_j (gates: fp64 softmax of the top k).
+    h is rounded to fp32 before its quantisation: the codes and scales are
+    decided in the precision the kernels hold h in (the pages fix none).
     shared: None, or the bf16 shared expert's (Ws1 [H, I], Ws3 [H, I], Ws2
     [I, H]) bit patterns; its output, the bf16 FFN of x[t] (ffn_rows), is
     added to every token: out[t] += y_shared[t].
@@ -502,7 +504,7 @@ def layer_tokens_mxfp8(logits, x_bits, weights, k: int, H: int, I: int, tokens, 
             w1, w3, w2 = expert(int(ids[t, j]))
             a = xt @ w1
             b = xt @ w3
-            h = a / (1.0 + np.exp(-a)) * b
+            h = (a / (1.0 + np.exp(-a)) * b).astype(np.float32).astype(np.float64)
             out[a_i] += g64[t, j] * (mx_round(h) @ w2)
     if shared is not None and len(toks):
         Ws1, Ws3, Ws2 = shared
@@ -518,7 +520,8 @@ def ffn_rows_mxfp8(xg_bits, experts, W1: dict, W3: dict, W2: dict, H: int, I: in
     experts. Every GEMM operand is MX-quantised along its reduction dimension
     and the arithmetic runs in fp64 on the values the codes stand for:
       a = mx(x).mx(W1), b = mx(x).mx(W3), h = silu(a) * b,
-      (hq, hs) = the MX codes and scales of h (blocks of 32 along I),
+      (hq, hs) = the MX codes and scales of h (blocks of 32 along I), decided
+      on h rounded to fp32, the precision the kernel holds h in,
       y = dq(hq, hs).mx(W2).
     W1/W3/W2 map expert id -> uint16 [H, I] / [H, I] / [I, H].
     Returns hq uint8 [n, I], hs uint8 [n, I/32] (row-major), y fp64 [n, H]."""
@@ -537,7 +540,7 @@ def ffn_rows_mxfp8(xg_bits, experts, W1: dict, W3: dict, W2: dict, H: int, I: in
         a = xr @ w1
         b = xr @ w3
         with np.errstate(over="ignore"):
-            h = a / (1.0 + np.exp(-a)) * b
+            h = (a / (1.0 + np.exp(-a)) * b).astype(np.float32).astype(np.float64)
         q, s = mx_quantize(h)
         hq[rows], hs[rows] = q, s
         y[rows] = mx_dequantize(q, s) @ w2

@@ -128,8 +128,8 @@ def _ffn_case(moe, w, sample=None):
 @pytest.mark.parametrize("name,sample", [("tiny", None), ("tiny_bwd", None), ("mid", 300)])
 def test_ffn_mxfp8_vs_oracle(cuda_lib, name, sample):
     r = _ffn_case(cuda_lib, inputs.WORKLOADS[name], sample)
-    # h is quantised from fp32 on the GPU, from fp64 in the oracle: codes may
-    # differ where the two land on either side of a rounding point
+    # both sides quantise h from fp32, but the GPU's a and b are fp32 sums in
+    # another order: codes may differ where h lands across a rounding point
     assert (r["hq"] == r["o_hq"]).mean() >= 0.99
     assert (r["hs"] == r["o_hs"]).mean() >= 0.99
     err = rms_floor_err(r["y"], r["o_y"])
