@@ -427,7 +427,8 @@ moe_status_t moe_dispatch_mxfp8(const uint16_t* x, const int32_t* phi, const int
  * consecutive. The table has R * K / 32 bytes, as the row-major one. */
 
 /* moe_dispatch_mxfp8 with xs in the TILED layout of the [moe_rows_max, H]
- * code matrix. H % 128 == 0 (rows_max is a multiple of 256). */
+ * code matrix. H % 128 == 0 (rows_max is a multiple of 256), else
+ * MOE_UNSUPPORTED_SHAPE; other errors as moe_dispatch. */
 moe_status_t moe_dispatch_mxfp8_tiled(const uint16_t* x, const int32_t* phi,
                                       const int32_t* offsets, uint8_t* xq, uint8_t* xs,
                                       int32_t* dev_status, const moe_shape_t* shape,
@@ -437,8 +438,10 @@ moe_status_t moe_dispatch_mxfp8_tiled(const uint16_t* x, const int32_t* phi,
  * [E, K, N] (N contiguous) -> q uint8 [E, N, K], the E4M3 codes TRANSPOSED
  * (K contiguous), and scale uint8 [E*N*K/32], the E8M0 codes of the blocks
  * of 32 along K (W[e, 32b..32b+31, n]) in the TILED layout of the [E*N, K]
- * code matrix (row e*N + n). K and N multiples of 128. For W1 and W3
- * (K = H, N = I) and W2 (K = I, N = H); done once per set of weights. */
+ * code matrix (row e*N + n). For W1 and W3 (K = H, N = I) and W2 (K = I,
+ * N = H); done once per set of weights. Errors: MOE_INVALID_ARG if K or N is
+ * not a positive multiple of 128, E < 0, or a pointer is null (E > 0) or not
+ * 16-byte aligned (W, q); MOE_UNSUPPORTED_SHAPE if E*K*N >= 2^40. */
 moe_status_t moe_mx_quantize_weights(const uint16_t* W, int32_t E, int32_t K, int32_t N,
                                      uint8_t* q, uint8_t* scale, void* stream);
 
