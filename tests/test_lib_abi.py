@@ -228,3 +228,15 @@ def test_size_queries_hold_their_invariants_on_random_shapes(lib):
                 assert tw > ws
 
     check()
+
+
+@pytest.mark.parametrize("P,N", [(8, 7168), (2, 300)])
+def test_mxfp8_layer_workspace_covers_the_shared_expert(lib, P, N):
+    """The layer's workspace plus the shared expert's h (bf16) and output (fp32)
+    over round_up(P*N, 256) rows, and a padded copy of x when P*N is ragged."""
+    H, I = 7168, 2048
+    sh = moe.shape(P, N, 384, 8, H, I)
+    rows = (P * N + 255) // 256 * 256
+    extra = rows * (I * 2 + H * 4) + (rows * H * 2 if (P * N) % 256 else 0)
+    assert moe.layer_mxfp8_workspace_bytes(sh) >= moe.layer_workspace_bytes(sh) + extra
+    assert moe.layer_mxfp8_workspace_bytes(sh) < moe.layer_workspace_bytes(sh) + extra + 8 * 1024
