@@ -34,9 +34,10 @@
 // first). TMEM holds the accumulators and STAGES x 8 or 16 scale columns:
 //   GEMM1  256 x 256 tiles (128 h columns through W1 and W3, CTA 0 holding
 //          W1's rows and CTA 1 W3's), one 256-column accumulator: a second
-//          would leave no columns for the scales, so a tile's epilogue is not
-//          overlapped with the next tile's MMAs (it writes 1 byte per h value
-//          and costs little against a 56-stage K loop);
+//          would leave no columns for the scales; the epilogue releases it
+//          after its last TMEM read, so only the reads and the first of its
+//          two blocks' arithmetic stall the next tile's MMAs (it writes 1 byte
+//          per h value, against a 56-stage K loop);
 //   GEMM2  256 x 128 tiles, two 128-column accumulators: the next tile's MMAs
 //          run while the epilogue streams the fp32 y tile out (the larger
 //          epilogue, against a 16-stage K loop).
@@ -383,7 +384,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::BN);
       if (MODE == 0) {
         // accumulator columns [0,128) = x.W1, [128,256) = x.W3 for h columns
-        // n*128 + j; this warp's 64 columns are two 32-column MX blocks of h
+        // n*128 + j; this warp's 64 columns are two 32-column MX blocks of h.
+        // The single accumulator is released as soon as this warp's last
+        // TMEM reads completed, so the next tile's MMAs overlap the SwiGLU,
+        // quantisation and stores of its last block.
         const int I = p.Nout;
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
@@ -391,6 +395,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           tmem_ld_32cols(tbase + half * 64 + c * 32, ra);
           tmem_ld_32cols(tbase + 128 + half * 64 + c * 32, rb);
           tmem_ld_wait();
+          if (c == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_relaxed_cluster(tempty_tgt0 + acc * 8);
+          }
           float hv[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) hv[i] = silu(__uint_as_float(ra[i])) * __uint_as_float(rb[i]);
@@ -430,9 +439,12 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         }
       }
       // the accumulator may be refilled once every lane's tcgen05.ld completed
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_relaxed_cluster(tempty_tgt0 + acc * 8);
+      // (GEMM1 released it above)
+      if (MODE != 0) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_relaxed_cluster(tempty_tgt0 + acc * 8);
+      }
       if (++acc == C::ACC) {
         acc = 0;
         acc_phase ^= 1u;
