@@ -240,3 +240,41 @@ def test_mxfp8_layer_workspace_covers_the_shared_expert(lib, P, N):
     extra = rows * (I * 2 + H * 4) + (rows * H * 2 if (P * N) % 256 else 0)
     assert moe.layer_mxfp8_workspace_bytes(sh) >= moe.layer_workspace_bytes(sh) + extra
     assert moe.layer_mxfp8_workspace_bytes(sh) < moe.layer_workspace_bytes(sh) + extra + 8 * 1024
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """include/moe.h compiles as C99 with a C compiler, and a C program linked
+    against the library calls its host-only entry points (no GPU needed)."""
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "moe.h"
+int main(void) {
+  moe_shape_t s = {8, 7168, 384, 8, 7168, 2048, 256};
+  long long rows = (long long)moe_rows_max(&s);
+  if (rows != (8LL * 7168 * 8 + 384 * 255 + 255) / 256 * 256) return 1;
+  if (strcmp(moe_status_string(MOE_WORKSPACE_TOO_SMALL), "MOE_WORKSPACE_TOO_SMALL") != 0) return 2;
+  if (moe_layer_workspace_bytes(&s) == 0) return 3;
+  if (moe_route_topk(NULL, NULL, NULL, &s, NULL) != MOE_INVALID_ARG) return 4;
+  s.pad = 0;
+  if (moe_rows_max(&s) != -1) return 5;
+  printf("ok %lld\n", rows);
+  return 0;
+}
+''')
+    lib_dir = os.path.dirname(moe.LIB_PATH)
+    exe = tmp_path / "abi"
+    r = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-pedantic-errors",
+                        "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                        "-L", lib_dir, "-l:" + os.path.basename(moe.LIB_PATH),
+                        "-Wl,-rpath," + lib_dir], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.startswith("ok"), (r.returncode, r.stdout, r.stderr)
