@@ -238,3 +238,35 @@ def test_layer_equals_direct_per_token_definition():
     # every padded row of the tiny workload is accounted for
     s = res["sched"]
     assert s["offsets"][-1] == sum(-(-int(c.sum()) // 256) * 256 for c in s["counts"])
+
+
+def test_oracle_results_do_not_depend_on_its_thread_count():
+    """The oracle splits rows and routes over OpenMP threads but every output
+    element is computed by one thread in a fixed order: one thread and all
+    threads give bitwise-identical schedules, FFN rows and gradients (the
+    baseline is timed both ways)."""
+    w = inputs.WORKLOADS["tiny_bwd"]
+    lg, x, dout = inputs.make_logits(w), inputs.make_x(w), inputs.make_dout(w)
+    W = inputs.make_weights(w)
+    Wd = _wdicts(*W)
+    ids, _, g64 = oracle.route_topk(lg, w.k)
+    n_all = oracle.num_threads()
+
+    def run():
+        s = oracle.schedule(ids.reshape(w.P, w.N, w.k), w.P, w.N, w.k, w.E, w.pad)
+        rows = np.nonzero(s["phi"][:, 0] >= 0)[0]
+        xg = oracle.dispatch_rows(_bits(x), w.N, s["phi"], rows)
+        ex = oracle.expert_of_rows(s["offsets"], rows)
+        h, y = oracle.ffn_rows(xg, ex, *Wd, H=w.H, I=w.I)
+        dys = oracle.dispatch_rows(_bits(dout), w.N, s["phi"], rows)
+        bwd = oracle.ffn_bwd_rows(xg, dys, np.ones(len(rows)), ex, *Wd, H=w.H, I=w.I)
+        return [s["phi"], s["offsets"], s["route_row"], h, y] + [np.asarray(v) for v in bwd.values()]
+
+    try:
+        oracle.set_num_threads(1)
+        one = run()
+    finally:
+        oracle.set_num_threads(n_all)
+    many = run()
+    for a, b in zip(one, many):
+        assert np.array_equal(a, b)
