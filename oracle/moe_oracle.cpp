@@ -386,8 +386,7 @@ void oracle_ffn_rows(const uint16_t* xg, int64_t n, const int32_t* expert, int32
     }
     for (int32_t i = 0; i < I; ++i) {
       const double s = acc_a[i] / (1.0 + std::exp(-acc_a[i]));
-      // rounded to bf16 from its fp32 value: the precision the kernels hold h in
-      const uint16_t hb = double_to_bf16(static_cast<double>(static_cast<float>(s * acc_b[i])));
+      const uint16_t hb = double_to_bf16(s * acc_b[i]);
       h[a * I + i] = hb;
       hv[i] = bf16_to_double(hb);
     }
@@ -464,11 +463,8 @@ void oracle_combine_f32(const float* y, int32_t H, const int64_t* sel, const flo
 // ---------------------------------------------------------------------------
 namespace {
 
-// The rounded mode's bf16 operands are rounded from their fp32 value, the
-// precision the kernels hold them in before the bf16 rounding.
-double rnd(double v, int exact) {
-  return exact ? v : bf16_to_double(double_to_bf16(static_cast<double>(static_cast<float>(v))));
-}
+// The rounded mode rounds each bf16 operand once, from its exact value.
+double rnd(double v, int exact) { return exact ? v : bf16_to_double(double_to_bf16(v)); }
 
 // The element-wise part for one (row, column i): from a, b (unrounded), dhu
 // and g, the values the two backward GEMMs and the gate gradient consume.

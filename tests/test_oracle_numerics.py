@@ -152,16 +152,62 @@ def dense_swiglu(x, W1, W3, W2):
     return hb, (h @ W2.double()).numpy()
 
 
+def near_bf16_midpoint(v, rel=1e-12):
+    """True where v lies within fp64 summation noise of the midpoint between two
+    neighbouring bf16 values (the only place two correct fp64 evaluations of
+    the same real number may round to different bf16 values)."""
+    v = np.asarray(v, np.float64)
+    lo = bf16_bits_to_f64(bits_round_bf16(v))
+    ulp = np.abs(lo) * 2.0 ** -7
+    mid_up, mid_dn = lo + ulp / 2, lo - ulp / 2
+    return np.minimum(np.abs(v - mid_up), np.abs(v - mid_dn)) <= rel * np.abs(v)
+
+
+def _assert_h_and_y_match_dense(h, y, x, W1, W3, W2):
+    """h = bf16_rne of the exact silu(a)*b, equal to the dense fp64 path's except
+    where the exact value sits on a rounding midpoint; y = h.W2 through the
+    same h, within fp64 summation noise."""
+    hb, _ = dense_swiglu(x, W1, W3, W2)
+    a = x.double() @ W1.double()
+    s = (a * torch.sigmoid(a) * (x.double() @ W3.double())).numpy()
+    diff = h != hb
+    assert diff.sum() <= 2 and near_bf16_midpoint(s[diff]).all(), int(diff.sum())
+    y_dense = (torch.from_numpy(bf16_bits_to_f64(h)) @ W2.double()).numpy()
+    np.testing.assert_allclose(y, y_dense, rtol=1e-11, atol=1e-13)
+    rows_same = ~diff.any(axis=1)
+    y_via_hb = (torch.from_numpy(bf16_bits_to_f64(hb)) @ W2.double()).numpy()
+    np.testing.assert_allclose(y[rows_same], y_via_hb[rows_same], rtol=1e-11, atol=1e-13)
+
+
 @pytest.mark.parametrize("H,I", [(64, 32), (128, 96)])
 def test_ffn_single_expert_is_dense_swiglu(H, I):
     W1, W3, W2 = _weights(1, H, I, seed=H + I)
     x = torch.randn(40, H, generator=torch.Generator().manual_seed(9)).to(torch.bfloat16)
     h, y = oracle.ffn_rows(_bits(x), np.zeros(40, np.int32), *_wdicts(W1, W3, W2), H=H, I=I)
-    hb, yr = dense_swiglu(x, W1[0], W3[0], W2[0])
-    assert (h == hb).mean() > 0.999          # rounding flips only at fp64 noise on a tie
-    y_from_h = (torch.from_numpy(bf16_bits_to_f64(h)) @ W2[0].double()).numpy()
-    np.testing.assert_allclose(y, y_from_h, rtol=1e-11, atol=1e-13)
-    np.testing.assert_allclose(y, yr, rtol=1e-2, atol=1e-6)
+    _assert_h_and_y_match_dense(h, y, x, W1[0], W3[0], W2[0])
+
+
+def test_ffn_h_is_rounded_once_from_the_exact_value():
+    """Pairs (a, b) whose silu(a)*b lies between a bf16 rounding midpoint and the
+    fp32 value next to it: rounding the exact value once and rounding it via
+    fp32 give different bf16 values there. One token x = 1 and H = 1 make a, b
+    the weights themselves; the oracle must follow the plain definition."""
+    g = np.random.default_rng(17)
+    a = bf16_bits_to_f64(bits_round_bf16(g.uniform(-4, 4, 4_000_000)))
+    b = bf16_bits_to_f64(bits_round_bf16(g.uniform(-4, 4, 4_000_000)))
+    s = a / (1.0 + np.exp(-a)) * b
+    once = bits_round_bf16(s)
+    twice = bits_round_bf16(s.astype(np.float32).astype(np.float64))
+    pick = np.nonzero((once != twice) & ~near_bf16_midpoint(s, 1e-12))[0][:64]
+    assert len(pick) >= 4, "the search finds double-rounding cases"
+    n = len(pick)
+    x = torch.ones((1, 1), dtype=torch.bfloat16)
+    W1 = torch.from_numpy(a[pick]).reshape(1, 1, n).to(torch.bfloat16)
+    W3 = torch.from_numpy(b[pick]).reshape(1, 1, n).to(torch.bfloat16)
+    W2 = torch.zeros((1, n, 1), dtype=torch.bfloat16)
+    h, _ = oracle.ffn_rows(_bits(x), np.zeros(1, np.int32), *_wdicts(W1, W3, W2), H=1, I=n)
+    assert (h[0] == once[pick]).all()
+    assert (h[0] != twice[pick]).all()
 
 
 def test_ffn_expert_selection_and_zero_rows():
@@ -174,9 +220,7 @@ def test_ffn_expert_selection_and_zero_rows():
     assert (h[5] == 0).all() and (y[5] == 0).all(), "silu(0)*0 = 0: padding rows stay zero"
     for e in range(E):
         m = ex == e
-        hb, yr = dense_swiglu(x[torch.from_numpy(m)], W1[e], W3[e], W2[e])
-        assert (h[m] == hb).mean() > 0.999
-        np.testing.assert_allclose(y[m], yr, rtol=1e-2, atol=1e-6)
+        _assert_h_and_y_match_dense(h[m], y[m], x[torch.from_numpy(m)], W1[e], W3[e], W2[e])
 
 
 # ---------------------------------------------------------------- combine
