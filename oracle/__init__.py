@@ -268,12 +268,15 @@ def expert_of_rows(offsets: np.ndarray, rows) -> np.ndarray:
 
 
 def layer_tokens(logits, x_bits, weights, P: int, N: int, k: int, E: int, H: int, I: int,
-                 tokens, pad: int = 256):
+                 tokens, pad: int = 256, experts_per_group: int = 32):
     """The whole layer for a set of tokens: route all tokens, schedule all routes,
     then dispatch, FFN and combine only the rows the chosen tokens need.
 
     weights: (W1, W3, W2) dicts expert -> numpy uint16 arrays (only the experts
-    the chosen tokens use need to be present).
+    the chosen tokens use need to be present), or a callable that returns
+    such dicts for a list of experts; the FFN then runs over groups of
+    `experts_per_group` experts at a time, so only one group's weights are
+    held in host memory at once.
     Returns dict with ids, gates32, gates64, sched, out64 [n,H], out_bf16 [n,H],
     y rows per (token, slot) and h rows.
     """
@@ -285,7 +288,16 @@ def layer_tokens(logits, x_bits, weights, P: int, N: int, k: int, E: int, H: int
     uniq, inv = np.unique(sel_rows, return_inverse=True)
     xg = dispatch_rows(x_bits, N, sch["phi"], uniq)
     ex = expert_of_rows(sch["offsets"], uniq)
-    h, y = ffn_rows(xg, ex, *weights, H=H, I=I)
+    if callable(weights):
+        h = np.zeros((len(uniq), I), np.uint16)
+        y = np.zeros((len(uniq), H), np.float64)
+        used = np.unique(ex)
+        for g0 in range(0, len(used), experts_per_group):
+            grp = used[g0:g0 + experts_per_group]
+            m = np.isin(ex, grp)
+            h[m], y[m] = ffn_rows(xg[m], ex[m], *weights(grp.tolist()), H=H, I=I)
+    else:
+        h, y = ffn_rows(xg, ex, *weights, H=H, I=I)
     out64, outb = combine_f64(y, inv.reshape(len(toks), k), g64[toks], k)
     return dict(ids=ids, gates32=g32, gates64=g64, sched=sch, out64=out64, out_bf16=outb,
                 rows=uniq, row_index=inv.reshape(len(toks), k), xg=xg, h=h, y=y,

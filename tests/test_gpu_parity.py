@@ -119,6 +119,81 @@ def test_schedule_bad_expert_id_flags_and_drops(cuda_lib):
     assert len(np.unique(placed)) == P * N * k - 1
 
 
+def _boundary_rows(offsets, counts, n_big=3, span=256):
+    """Rows a tile-order or boundary bug would hit first: the first and last
+    `span` rows of the n_big largest segments, and every non-empty segment's
+    first row, last real row and first padding row."""
+    off = np.asarray(offsets, np.int64)
+    T = np.asarray(counts, np.int64).sum(axis=1)
+    rows = []
+    for l in np.argsort(-T, kind="stable")[:n_big]:
+        a, b = off[l], off[l] + T[l]
+        rows += list(range(a, min(a + span, b))) + list(range(max(a, b - span), b))
+    for l in np.nonzero(T > 0)[0]:
+        a, real_end, seg_end = off[l], off[l] + T[l], off[l + 1]
+        rows += [a, real_end - 1] + ([real_end] if real_end < seg_end else [])
+    return np.unique(np.asarray(rows, np.int64))
+
+
+@pytest.mark.parametrize("name", ["kimi", "zipf"])
+def test_schedule_and_dispatch_full_config(cuda_lib, name):
+    """The whole Phi, offsets, counts and route_row of the Kimi-shape and Zipf
+    layers (routing on the GPU, then the schedule on its ids) bit for bit
+    against the oracle's schedule of the oracle's own ids; the dispatch bit
+    for bit on >= 4,096 rows that include the largest segments' ends and every
+    segment's boundary rows."""
+    moe = cuda_lib
+    w = inputs.WORKLOADS[name]
+    lg = inputs.make_logits(w)
+    sh = moe.shape(**w.shape())
+    ids = torch.empty((w.n_tokens, w.k), dtype=torch.int32, device=DEV)
+    gates = torch.empty((w.n_tokens, w.k), dtype=torch.float32, device=DEV)
+    moe.moe_route_topk(lg.to(DEV), ids, gates, sh)
+    b = moe.alloc_schedule_outputs(sh)
+    b["phi"].fill_(-7)
+    moe.moe_schedule(ids, b["phi"], b["offsets"], b["counts"], b["route_row"], b["ws"],
+                     b["dev_status"], sh)
+    torch.cuda.synchronize()
+    o_ids, _, _ = oracle.route_topk(lg, w.k)
+    assert (ids.cpu().numpy() == o_ids).all()
+    s = oracle.schedule(o_ids.reshape(w.P, w.N, w.k), w.P, w.N, w.k, w.E, 256)
+    g = {k_: v.cpu().numpy() for k_, v in b.items()}
+    _assert_sched_equal(g, s)
+    assert s["reads"] == 2 * w.n_routes
+    T = s["counts"].sum(axis=1)
+    seg = np.diff(s["offsets"])
+    assert (seg % 256 == 0).all() and (seg - T < 256).all() and (seg >= T).all()
+    if name == "zipf":
+        empties = inputs.empty_experts(w)
+        assert (T[empties] == 0).all() and (seg[empties] == 0).all()
+        hot = int(np.argmax(T))
+        assert T[hot] > 0.10 * w.n_routes
+        # the hot expert's routes come from every peer and from many 2,048-route blocks
+        rr = s["route_row"]
+        in_hot = (rr >= s["offsets"][hot]) & (rr < s["offsets"][hot] + T[hot])
+        q = np.nonzero(in_hot.reshape(w.P, -1))
+        assert len(np.unique(q[0])) == w.P
+        assert len(np.unique(q[1] // 2048)) == (w.N * w.k + 2047) // 2048
+    # dispatch on sampled rows
+    x = inputs.make_x(w)
+    rm = moe.rows_max(sh)
+    xg = torch.empty((rm, w.H), dtype=torch.bfloat16, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    moe.moe_dispatch(x.to(DEV), b["phi"], b["offsets"], xg, st, sh)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rows_used = int(s["offsets"][-1])
+    pick = _boundary_rows(s["offsets"], s["counts"])
+    rng = np.random.default_rng(w.wid)
+    extra = rng.choice(rows_used, max(0, 4096 - len(pick)) + 512, replace=False)
+    pick = np.unique(np.concatenate([pick, extra]))
+    assert len(pick) >= 4096
+    got = bits(xg[torch.from_numpy(pick).to(DEV)])
+    assert (got == oracle.dispatch_rows(bits(x), w.N, s["phi"], pick)).all()
+    del xg
+    torch.cuda.empty_cache()
+
+
 # ---------------------------------------------------------------- routing
 @pytest.mark.parametrize("name", ["tiny", "mid", "kimi", "zipf"])
 def test_route_topk(cuda_lib, name):
@@ -296,6 +371,42 @@ def test_ffn_gather_equals_dispatch_then_ffn(cuda_lib, name, pad):
     assert torch.equal(h2[real], r["h"][real]) and torch.equal(y2[real], r["y"][real])
 
 
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_ffn_gather_vs_oracle(cuda_lib, name):
+    """The FFN that pulls its A rows from x through Phi, against the oracle's
+    dispatch and FFN (schedule from the oracle's own routing)."""
+    moe = cuda_lib
+    w = inputs.WORKLOADS[name]
+    lg, x = inputs.make_logits(w), inputs.make_x(w)
+    W1, W3, W2 = inputs.make_weights(w)
+    sh = moe.shape(**w.shape())
+    o_ids, _, _ = oracle.route_topk(lg, w.k)
+    s = oracle.schedule(o_ids.reshape(w.P, w.N, w.k), w.P, w.N, w.k, w.E, 256)
+    rm = moe.rows_max(sh)
+    rows = int(s["offsets"][-1])
+    phi = torch.full((rm, 2), -1, dtype=torch.int32)
+    phi[:rows] = torch.from_numpy(s["phi"])
+    offs = torch.from_numpy(s["offsets"]).to(DEV)
+    cnts = torch.from_numpy(np.ascontiguousarray(s["counts"])).to(DEV)
+    h = torch.empty((rm, w.I), dtype=torch.bfloat16, device=DEV)
+    y = torch.empty((rm, w.H), dtype=torch.float32, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    moe.moe_expert_ffn_gather(x.to(DEV), phi.to(DEV), W1.to(DEV), W3.to(DEV), W2.to(DEV), offs,
+                              cnts, h, y, st, sh)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    real = np.nonzero(s["phi"][:, 0] >= 0)[0]
+    if len(real) > 600:
+        rng = np.random.default_rng(w.wid)
+        real = np.unique(np.concatenate([real[:64], real[-64:], rng.choice(real, 400, replace=False)]))
+    ex = oracle.expert_of_rows(s["offsets"], real)
+    o_xg = oracle.dispatch_rows(bits(x), w.N, s["phi"], real)
+    o_h, o_y = oracle.ffn_rows(o_xg, ex, *expert_weights_host(W1, W3, W2, ex), H=w.H, I=w.I)
+    idx = torch.from_numpy(real).to(DEV)
+    assert (bits(h[idx]) == o_h).mean() > 0.995
+    assert rms_floor_err(y[idx].cpu().numpy(), o_y) < Y_TOL
+
+
 def test_ffn_gather_flags_corrupt_phi(cuda_lib):
     """A Phi entry outside [0,P)x[0,N) is reported and its row reads as zeros."""
     moe = cuda_lib
@@ -377,15 +488,39 @@ def _layer_gpu(moe, w, lg_d, x_d, Wd, minibatch=0, ws=None):
     return out, ws
 
 
-@pytest.mark.parametrize("name,n_tok", [("tiny", 512), ("mid", 96), ("kimi", 6), ("zipf", 6)])
+def _layer_tokens_for(w, lg, n_tok):
+    """n_tok tokens: those owning the first and last real rows of the three
+    largest expert segments and the last real row of every tenth segment,
+    then seeded random tokens."""
+    o_ids, _, _ = oracle.route_topk(lg, w.k)
+    s = oracle.schedule(o_ids.reshape(w.P, w.N, w.k), w.P, w.N, w.k, w.E, 256)
+    T = s["counts"].sum(axis=1)
+    off = s["offsets"].astype(np.int64)
+    rows = []
+    for l in np.argsort(-T, kind="stable")[:3]:
+        rows += list(range(off[l], off[l] + 8)) + list(range(off[l] + T[l] - 8, off[l] + T[l]))
+    rows += [off[l] + T[l] - 1 for l in np.nonzero(T > 0)[0][::10]]
+    phi = s["phi"][np.asarray(rows, np.int64)]
+    toks = set((phi[:, 0].astype(np.int64) * w.N + phi[:, 1]).tolist())
+    rng = np.random.default_rng(w.wid)
+    while len(toks) < n_tok:
+        toks.add(int(rng.integers(w.n_tokens)))
+    return sorted(toks)
+
+
+@pytest.mark.parametrize("name,n_tok", [("tiny", 512), ("mid", 96), ("kimi", 256), ("zipf", 256)])
 def test_layer_vs_oracle(cuda_lib, name, n_tok):
     moe = cuda_lib
     w, lg, x, W = _layer_inputs(name)
     Wd = [t.to(DEV) for t in W]
     out, ws = _layer_gpu(moe, w, lg.to(DEV), x.to(DEV), Wd)
-    toks = inputs.sample_tokens(w.n_tokens, n_tok, seed=w.wid)
+    if name in ("kimi", "zipf"):
+        toks = _layer_tokens_for(w, lg, n_tok)
+    else:
+        toks = inputs.sample_tokens(w.n_tokens, n_tok, seed=w.wid)
     o_ids, _, _ = oracle.route_topk(lg[toks], w.k)
-    Wh = expert_weights_host(*Wd, np.unique(o_ids))
+    # weights go to the host one group of experts at a time
+    Wh = lambda ex: expert_weights_host(*Wd, ex)
     res = oracle.layer_tokens(lg, bits(x), Wh, w.P, w.N, w.k, w.E, w.H, w.I, toks)
     got = bf16_to_f64(bits(out[torch.tensor(toks, device=DEV)]))
     err = rms_floor_err(got, res["out64"])
@@ -398,9 +533,11 @@ def test_layer_vs_oracle(cuda_lib, name, n_tok):
         assert counts.max() > 0.10 * ids_all.size, "a hot expert takes >10% of routes"
         s = res["sched"]
         assert (np.diff(s["offsets"])[inputs.empty_experts(w)] == 0).all()
+        top3 = np.argsort(-counts, kind="stable")[:3]
+        assert all(np.isin(top3[i], o_ids) for i in range(3)), "sampled tokens reach the hot experts"
 
 
-@pytest.mark.parametrize("name", ["tiny", "mid", "kimi"])
+@pytest.mark.parametrize("name", ["tiny", "mid", "kimi", "zipf"])
 def test_layer_bitwise_deterministic_and_slice_invariant(cuda_lib, name):
     moe = cuda_lib
     w, lg, x, W = _layer_inputs(name)
@@ -411,7 +548,10 @@ def test_layer_bitwise_deterministic_and_slice_invariant(cuda_lib, name):
     for _ in range(2):
         out1, _ = _layer_gpu(moe, w, lg_d, x_d, Wd, ws=ws)
         assert sha(out1) == h0
-    for T in ([w.minibatch] if w.minibatch else []) + [max(1, w.N // 3), 97]:
+    slices = [w.minibatch] if w.minibatch else []
+    if w.N >= 4 * 2368 // 3:
+        slices = sorted(set(slices + [2368]))
+    for T in slices + [max(1, w.N // 3), 97]:
         outT, _ = _layer_gpu(moe, w, lg_d, x_d, Wd, minibatch=T, ws=ws)
         assert sha(outT) == h0, f"transfer slice {T} changed the output"
 
@@ -503,6 +643,41 @@ def test_layer_concurrent_streams(cuda_lib):
     for st_, o_ in zip(sts, outs):
         assert int(st_.item()) == 0
         assert torch.equal(o_, ref)
+
+
+def test_ffn_launch_waiting_on_an_event_while_another_stream_queues_300(cuda_lib):
+    """A GEMM launch held back on one stream (it waits for an event recorded
+    after a spin kernel) is undisturbed by 300 FFN calls (600 GEMM launches)
+    that another stream enqueues and runs meanwhile, cycling through every
+    counter of the pool: its output equals the one computed alone."""
+    moe = cuda_lib
+    w = inputs.WORKLOADS["tiny"]
+    lg, x = inputs.make_logits(w), inputs.make_x(w)
+    W1, W3, W2 = [t.to(DEV) for t in inputs.make_weights(w)]
+    r = _stage_run(moe, w, W1, W3, W2, lg.to(DEV), x.to(DEV))
+    sh = moe.shape(**w.shape())
+    ref_h, ref_y = r["h"].clone(), r["y"].clone()
+    gate, a, b = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = torch.cuda.Event()
+    h_a, y_a = torch.zeros_like(ref_h), torch.zeros_like(ref_y)
+    h_b, y_b = torch.zeros_like(ref_h), torch.zeros_like(ref_y)
+    st_a = torch.zeros(1, dtype=torch.int32, device=DEV)
+    st_b = torch.zeros(1, dtype=torch.int32, device=DEV)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(gate):
+        torch.cuda._sleep(300_000_000)  # well over 100 ms at any SM clock
+        ev.record(gate)
+    a.wait_event(ev)
+    moe.moe_expert_ffn(r["xg"], W1, W3, W2, r["offsets"], r["counts"], h_a, y_a, st_a, sh,
+                       stream=a)
+    for _ in range(300):
+        moe.moe_expert_ffn(r["xg"], W1, W3, W2, r["offsets"], r["counts"], h_b, y_b, st_b, sh,
+                           stream=b)
+    torch.cuda.synchronize()
+    assert int(st_a.item()) == 0 and int(st_b.item()) == 0
+    real = torch.from_numpy(np.nonzero(r["phi"][:int(r["offsets"][-1].item()), 0].cpu().numpy() >= 0)[0]).to(DEV)
+    for h_, y_ in ((h_a, y_a), (h_b, y_b)):
+        assert torch.equal(h_[real], ref_h[real]) and torch.equal(y_[real], ref_y[real])
 
 
 def test_layer_pad128_single_cta_path(cuda_lib):

@@ -282,6 +282,18 @@ def test_layer_equals_direct_per_token_definition():
     # every padded row of the tiny workload is accounted for
     s = res["sched"]
     assert s["offsets"][-1] == sum(-(-int(c.sum()) // 256) * 256 for c in s["counts"])
+    # weights handed over a few experts at a time give the very same result
+    W = _wdicts(W1, W3, W2)
+    calls = []
+
+    def by_group(ex):
+        calls.append(list(ex))
+        return tuple({e: d[e] for e in ex} for d in W)
+
+    res2 = oracle.layer_tokens(lg, _bits(x), by_group, w.P, w.N, w.k, w.E, w.H, w.I, toks,
+                               experts_per_group=3)
+    assert len(calls) == 3 and sorted(sum(calls, [])) == list(range(w.E))
+    assert (res2["out64"] == res["out64"]).all() and (res2["h"] == res["h"]).all()
 
 
 def test_oracle_results_do_not_depend_on_its_thread_count():
