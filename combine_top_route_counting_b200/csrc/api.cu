@@ -8,18 +8,6 @@
 
 namespace moe {
 
-namespace {
-std::atomic<int64_t> g_launches{0};
-
-constexpr size_t kAlign = 1024;
-inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-// Buffers written with 32-byte vector stores.
-bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
-
-moe_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_CUDA_ERROR; }
-
 // Basic shape limits shared by every entry point.
 moe_status_t check_shape(const moe_shape_t* s) {
   if (!s) return MOE_INVALID_ARG;
@@ -31,6 +19,19 @@ moe_status_t check_shape(const moe_shape_t* s) {
   if (routes >= (int64_t{1} << 31) || rows >= (int64_t{1} << 31)) return MOE_UNSUPPORTED_SHAPE;
   return MOE_OK;
 }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+namespace {
+std::atomic<int64_t> g_launches{0};
+
+constexpr size_t kAlign = 1024;
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Buffers written with 32-byte vector stores.
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+
+moe_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_CUDA_ERROR; }
 
 // Extra limits of the expert FFN (tcgen05 tiles of 128 rows x 256 columns,
 // K steps of 64, TMA coordinates in int32).
@@ -80,7 +81,7 @@ moe_status_t check_mx_shape(const moe_shape_t* s) {
 // backward's buffers; dxg [rows, H] fp32 reuses y, which is dead once the
 // forward's combine has run.
 struct LayerWs {
-  size_t ids, gates, route_row, phi, offsets, counts, sched, xg, h, y, total;
+  size_t ids, gates, route_row, phi, offsets, counts, sched, ctr, xg, h, y, total;
   size_t logits[2], x[2], out[2], total_host;  // moe_layer_forward_host additions
   size_t ab, dys, dab, hg, gate_row, part, total_train;  // training additions
   size_t sh_off, sh_x, sh_h, sh_y, total_mx;  // the MXFP8 layer's shared expert
@@ -104,6 +105,7 @@ LayerWs layer_ws(const moe_shape_t* s) {
   w.offsets = take(o, (s->E + 1) * 4);
   w.counts = take(o, static_cast<size_t>(s->E) * s->P * 4);
   w.sched = take(o, schedule_ws_bytes(s->P, s->N, s->k, s->E));
+  w.ctr = take(o, 8);  // the GEMMs' tile counter, zeroed at the start of each call
   w.xg = take(o, rows * s->H * 2);
   w.h = take(o, rows * s->I * 2);
   w.y = take(o, rows * s->H * 4);
@@ -159,6 +161,7 @@ namespace {
 
 struct LayerBufs {
   int32_t *ids, *route_row, *phi, *offsets, *counts, *sched;
+  int* ctr;
   float *gates, *y;
   uint16_t *xg, *h;
 };
@@ -172,6 +175,7 @@ LayerBufs layer_bufs(void* ws, const LayerWs& w) {
   b.offsets = at<int32_t>(ws, w.offsets);
   b.counts = at<int32_t>(ws, w.counts);
   b.sched = at<int32_t>(ws, w.sched);
+  b.ctr = at<int>(ws, w.ctr);
   b.xg = at<uint16_t>(ws, w.xg);
   b.h = at<uint16_t>(ws, w.h);
   b.y = at<float>(ws, w.y);
@@ -203,7 +207,7 @@ cudaError_t run_slice(const LayerBufs& b, const uint16_t* x, const uint16_t* W1,
   if ((e = rec(3)) != cudaSuccess) return e;
   cudaEvent_t mid = (ev && ev[4]) ? static_cast<cudaEvent_t>(ev[4]) : nullptr;
   if ((e = launch_expert_ffn(b.xg, W1, W3, W2, b.offsets, b.counts, b.h, b.y, *sh, rows_max,
-                             dev_status, s, mid, ab)) != cudaSuccess)
+                             dev_status, s, mid, ab, b.ctr)) != cudaSuccess)
     return e;
   if ((e = rec(5)) != cudaSuccess) return e;
   if ((e = launch_combine(b.y, b.route_row, b.gates, out, *sh, sl, rows_max, dev_status, s)) !=
@@ -227,6 +231,7 @@ moe_status_t layer_body(const float* logits, const uint16_t* x, const uint16_t* 
   void* const* ev_use = (T == N) ? ev : nullptr;  // stage events: single-slice runs only
   cudaError_t e = (ev_use && ev_use[0]) ? cudaEventRecord(static_cast<cudaEvent_t>(ev_use[0]), s)
                                         : cudaSuccess;
+  if (e == cudaSuccess) e = cudaMemsetAsync(b.ctr, 0, 8, s);
   if (e == cudaSuccess)
     e = launch_route_topk(logits, b.ids, b.gates, static_cast<int64_t>(sh->P) * N, sh->E, sh->k, s);
   if (e != cudaSuccess) return from_cuda(e);
@@ -264,6 +269,7 @@ cudaError_t layer_body_mx(const float* logits, const uint16_t* x, const uint8_t*
   };
   cudaError_t e;
   if ((e = rec(0)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(b.ctr, 0, 8, s)) != cudaSuccess) return e;
   if ((e = launch_route_topk(logits, b.ids, b.gates, static_cast<int64_t>(sh->P) * sh->N, sh->E,
                              sh->k, s)) != cudaSuccess)
     return e;
@@ -289,12 +295,12 @@ cudaError_t layer_body_mx(const float* logits, const uint16_t* x, const uint8_t*
     if ((e = launch_dense_ffn(x, static_cast<int64_t>(sh->P) * sh->N, Ws1, Ws3, Ws2,
                               at<uint16_t>(ws, w.sh_x), at<uint16_t>(ws, w.sh_h), ys,
                               at<int32_t>(ws, w.sh_off), sh->H,
-                              sh->I, dev_status, s)) != cudaSuccess)
+                              sh->I, dev_status, s, b.ctr)) != cudaSuccess)
       return e;
   }
   cudaEvent_t mid = ev ? static_cast<cudaEvent_t>(ev[4]) : nullptr;
   if ((e = launch_expert_ffn_mxfp8(xq, xs, W1q, W1s, W3q, W3s, W2q, W2s, b.offsets, b.counts, hq,
-                                   hs, b.y, *sh, rows_max, dev_status, s, mid)) != cudaSuccess)
+                                   hs, b.y, *sh, rows_max, dev_status, s, mid, b.ctr)) != cudaSuccess)
     return e;
   if ((e = rec(5)) != cudaSuccess) return e;
   if ((e = launch_combine(b.y, b.route_row, b.gates, out, *sh, Slice{0, sh->N}, rows_max,
@@ -336,12 +342,14 @@ cudaError_t backward_body(const uint16_t* dout, const uint16_t* W1, const uint16
       if ((e = rec(i)) != cudaSuccess) return e;
     return cudaSuccess;
   }
+  if ((e = cudaMemsetAsync(b.ctr, 0, 8, s)) != cudaSuccess) return e;
   if ((e = launch_reverse_combine(dout, b.phi, b.offsets, b.route_row, b.gates, dys, gate_row, *sh,
                                   rows_max, dev_status, s)) != cudaSuccess)
     return e;
   if ((e = rec(1)) != cudaSuccess) return e;
   if ((e = launch_expert_ffn_dgrad(dys, gate_row, ab, b.h, W1, W3, W2, b.offsets, b.counts, dab, hg,
-                                   part, dxg, *sh, rows_max, dev_status, s, evt(2))) != cudaSuccess)
+                                   part, dxg, *sh, rows_max, dev_status, s, evt(2), b.ctr)) !=
+      cudaSuccess)
     return e;
   if ((e = rec(3)) != cudaSuccess) return e;
   if ((e = launch_reverse_dispatch(dxg, b.route_row, dx, *sh, rows_max, dev_status, s)) !=
@@ -355,7 +363,7 @@ cudaError_t backward_body(const uint16_t* dout, const uint16_t* W1, const uint16
   if ((e = rec(5)) != cudaSuccess) return e;
   // weight gradients last: deferred until every activation gradient is done
   if ((e = launch_expert_ffn_wgrad(b.xg, dys, dab, hg, b.offsets, b.counts, dW1, dW3, dW2, *sh,
-                                   rows_max, dev_status, s, evt(6))) != cudaSuccess)
+                                   rows_max, dev_status, s, evt(6), b.ctr)) != cudaSuccess)
     return e;
   return rec(7);
 }
@@ -916,6 +924,26 @@ int64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxe
 moe_status_t moe_selftest_bounded_wait(int32_t* dev_status, int64_t timeout_ns, void* stream) {
   if (!dev_status || timeout_ns <= 0) return MOE_INVALID_ARG;
   return from_cuda(launch_selftest_wait(dev_status, timeout_ns, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_selftest_schedule_barrier(const int32_t* ids, int32_t* phi, int32_t* offsets,
+                                           int32_t* counts, int32_t* route_row, void* ws,
+                                           size_t ws_bytes, int32_t* dev_status,
+                                           const moe_shape_t* shape, int64_t timeout_ns,
+                                           void* stream) {
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (!phi || !offsets || !counts || !dev_status || !ws || timeout_ns <= 0) return MOE_INVALID_ARG;
+  if (shape->N < 1 || !ids || !route_row) return MOE_INVALID_ARG;
+  if (!aligned16(ids) || !aligned16(phi) || !aligned16(route_row) || !aligned32(ws))
+    return MOE_INVALID_ARG;
+  if (ws_bytes < schedule_ws_bytes(shape->P, shape->N, shape->k, shape->E))
+    return MOE_WORKSPACE_TOO_SMALL;
+  const cudaError_t e = launch_schedule_barrier_selftest(
+      ids, *shape, phi, offsets, counts, route_row, static_cast<int32_t*>(ws), dev_status,
+      timeout_ns, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorInvalidConfiguration) return MOE_UNSUPPORTED_SHAPE;
+  return from_cuda(e);
 }
 
 }  // extern "C"

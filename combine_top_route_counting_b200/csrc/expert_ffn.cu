@@ -88,7 +88,7 @@ struct Cfg {
 };
 
 struct FfnParams {
-  int* tile_counter;       // next tile to hand out (zeroed before each launch)
+  int* tile_counter;       // {next tile to hand out, CTAs finished}; zero at launch
   const int2* phi;         // [rows_max] (src_rank, src_idx): GATHER only
   int32_t n_per_peer;      // N (GATHER: token row = src_rank * N + src_idx)
   const int32_t* offsets;  // [E+1]
@@ -593,6 +593,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 
   __syncthreads();
   if (CG == 2) cluster_sync();  // the peer no longer reads this CTA's smem or TMEM
+  if (tid == 0) finish_tile_counter(p.tile_counter);
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -609,9 +610,10 @@ template <int MODE, int CG, bool GATHER = false, bool SAVE_AB = false>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const CUtensorMap& yo, FfnParams p, cudaStream_t s) {
   const size_t smem = smem_bytes_for<CG, MODE>(p.E);
-  cudaError_t e = tile_counter_for_current_device(&p.tile_counter);
-  if (e != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s)) != cudaSuccess) return e;
+  if (!p.tile_counter) {  // no counter of the caller's: one from the device's pool
+    const cudaError_t e = tile_counter_for_current_device(&p.tile_counter);
+    if (e != cudaSuccess) return e;
+  }
   return launch_persistent(ffn_gemm_kernel<MODE, CG, GATHER, SAVE_AB>, CG, smem, s, a, b0, b1, yo,
                            p);
 }
@@ -622,7 +624,7 @@ cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint
                               const uint16_t* W2, const int32_t* offsets, const int32_t* counts,
                               uint16_t* h, float* y, const moe_shape_t& sh, int64_t rows_max,
                               int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_mid,
-                              uint16_t* ab) {
+                              uint16_t* ab, int* counter) {
   const int E = sh.E, H = sh.H, I = sh.I;
   CUtensorMap mA1, mW1, mW3, mA2, mW2, mY;
   const uint64_t EH = static_cast<uint64_t>(E) * H, EI = static_cast<uint64_t>(E) * I;
@@ -633,7 +635,7 @@ cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint
   // Segments that are multiples of 256 rows run on CTA pairs (256x256 tiles);
   // otherwise (pad a multiple of 128 only) on single CTAs (128x256 tiles).
   const bool pair = (sh.pad % 256) == 0;
-  FfnParams p1{nullptr, nullptr, 0, offsets, counts, E, sh.P, H, I, rows_max, h, dev_status,
+  FfnParams p1{counter, nullptr, 0, offsets, counts, E, sh.P, H, I, rows_max, h, dev_status,
                kWaitTimeoutNs, ab};
   cudaError_t e;
   if (ab)  // training: keep the pre-activations (pair tiles only)
@@ -645,7 +647,7 @@ cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint
     e = cudaEventRecord(ev_mid, s);
     if (e != cudaSuccess) return e;
   }
-  FfnParams p2{nullptr, nullptr, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status,
+  FfnParams p2{counter, nullptr, 0, offsets, counts, E, sh.P, I, H, rows_max, y, dev_status,
                kWaitTimeoutNs, nullptr};
   return pair ? launch_mode<1, 2>(mA2, mW2, mW2, mY, p2, s)
               : launch_mode<1, 1>(mA2, mW2, mW2, mY, p2, s);

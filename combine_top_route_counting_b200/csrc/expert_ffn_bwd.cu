@@ -88,7 +88,7 @@ struct BCfg {
 };
 
 struct BwdParams {
-  int* tile_counter;       // next tile to hand out (zeroed before each launch)
+  int* tile_counter;       // {next tile to hand out, CTAs finished}; zero at launch
   const int32_t* offsets;  // [E+1] segment starts
   const int32_t* counts;   // [E, P] routes per (expert, peer), or null (whole segments)
   int32_t E, P;
@@ -482,6 +482,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 
   __syncthreads();
   cluster_sync();  // the peer no longer reads this CTA's smem or TMEM
+  if (tid == 0) finish_tile_counter(p.tile_counter);
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -493,14 +494,15 @@ template <int OP>
 cudaError_t launch_bwd(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                        const CUtensorMap& y0, const CUtensorMap& y1, BwdParams p, cudaStream_t s) {
   const size_t smem = bwd_smem_bytes<OP>(p.E);
-  cudaError_t e = tile_counter_for_current_device(&p.tile_counter);
-  if (e != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s)) != cudaSuccess) return e;
+  if (!p.tile_counter) {  // no counter of the caller's: one from the device's pool
+    const cudaError_t e = tile_counter_for_current_device(&p.tile_counter);
+    if (e != cudaSuccess) return e;
+  }
   return launch_persistent(ffn_bwd_kernel<OP>, 2, smem, s, a, b0, b1, y0, y1, p);
 }
 
 BwdParams base_params(const int32_t* offsets, const int32_t* counts, const moe_shape_t& sh,
-                      int64_t rows_max, int32_t* dev_status) {
+                      int64_t rows_max, int32_t* dev_status, int* counter) {
   BwdParams p{};
   p.offsets = offsets;
   p.counts = counts;
@@ -509,6 +511,7 @@ BwdParams base_params(const int32_t* offsets, const int32_t* counts, const moe_s
   p.rows_max = rows_max;
   p.dev_status = dev_status;
   p.timeout_ns = kWaitTimeoutNs;
+  p.tile_counter = counter;
   return p;
 }
 
@@ -520,7 +523,7 @@ cudaError_t launch_expert_ffn_dgrad(const uint16_t* dys, const float* gate_row, 
                                     const int32_t* counts, uint16_t* dab, uint16_t* hg,
                                     float* part, float* dxg, const moe_shape_t& sh,
                                     int64_t rows_max, int32_t* dev_status, cudaStream_t s,
-                                    cudaEvent_t ev_mid) {
+                                    cudaEvent_t ev_mid, int* counter) {
   const int E = sh.E, H = sh.H, I = sh.I;
   const uint64_t EH = static_cast<uint64_t>(E) * H, EI = static_cast<uint64_t>(E) * I;
   CUtensorMap mDys, mW2, mDab, mW1, mW3, mDxg;
@@ -529,7 +532,7 @@ cudaError_t launch_expert_ffn_dgrad(const uint16_t* dys, const float* gate_row, 
       !make_map(&mDab, dab, 2ull * I, rows_max, 64, 128) || !make_map(&mW1, W1, I, EH, 64, 128) ||
       !make_map(&mW3, W3, I, EH, 64, 128) || !make_map(&mDxg, dxg, H, rows_max, 32, 32, true))
     return cudaErrorInvalidValue;
-  BwdParams p1 = base_params(offsets, counts, sh, rows_max, dev_status);
+  BwdParams p1 = base_params(offsets, counts, sh, rows_max, dev_status, counter);
   p1.K = H;
   p1.N = I;
   p1.ab = ab;
@@ -541,7 +544,7 @@ cudaError_t launch_expert_ffn_dgrad(const uint16_t* dys, const float* gate_row, 
   cudaError_t e = launch_bwd<OP_DGRAD_H>(mDys, mW2, mW2, mDxg, mDxg, p1, s);
   if (e != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
-  BwdParams p2 = base_params(offsets, counts, sh, rows_max, dev_status);
+  BwdParams p2 = base_params(offsets, counts, sh, rows_max, dev_status, counter);
   p2.K = 2 * I;
   p2.kswitch = I;
   p2.N = H;
@@ -552,14 +555,14 @@ cudaError_t launch_expert_ffn_wgrad(const uint16_t* xg, const uint16_t* dys, con
                                     const uint16_t* hg, const int32_t* offsets,
                                     const int32_t* counts, float* dW1, float* dW3, float* dW2,
                                     const moe_shape_t& sh, int64_t rows_max, int32_t* dev_status,
-                                    cudaStream_t s, cudaEvent_t ev_mid) {
+                                    cudaStream_t s, cudaEvent_t ev_mid, int* counter) {
   const int H = sh.H, I = sh.I;
   CUtensorMap mHg, mDys, mXg, mDab;
   // MN-major operands: 64 columns x 64 rows per box
   if (!make_map(&mHg, hg, I, rows_max, 64, 64) || !make_map(&mDys, dys, H, rows_max, 64, 64) ||
       !make_map(&mXg, xg, H, rows_max, 64, 64) || !make_map(&mDab, dab, 2ull * I, rows_max, 64, 64))
     return cudaErrorInvalidValue;
-  BwdParams p1 = base_params(offsets, counts, sh, rows_max, dev_status);
+  BwdParams p1 = base_params(offsets, counts, sh, rows_max, dev_status, counter);
   p1.M = I;
   p1.N = H;
   p1.nsplit = H;
@@ -568,7 +571,7 @@ cudaError_t launch_expert_ffn_wgrad(const uint16_t* xg, const uint16_t* dys, con
   cudaError_t e = launch_bwd<OP_WGRAD>(mHg, mDys, mDys, mHg, mHg, p1, s);
   if (e != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
-  BwdParams p2 = base_params(offsets, counts, sh, rows_max, dev_status);
+  BwdParams p2 = base_params(offsets, counts, sh, rows_max, dev_status, counter);
   p2.M = H;
   p2.N = 2 * I;
   p2.nsplit = I;

@@ -98,7 +98,7 @@ struct MxCfg {
 };
 
 struct MxParams {
-  int* tile_counter;       // next tile to hand out (zeroed before each launch)
+  int* tile_counter;       // {next tile to hand out, CTAs finished}; zero at launch
   const int32_t* offsets;  // [E+1] segment starts (multiples of 256)
   const int32_t* counts;   // [E, P] or null
   int32_t E, P;
@@ -455,6 +455,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 
   __syncthreads();
   cluster_sync();  // the peer no longer reads this CTA's smem or TMEM
+  if (tid == 0) finish_tile_counter(p.tile_counter);
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -467,9 +468,10 @@ cudaError_t launch_mx(const CUtensorMap& a, const CUtensorMap& sa, const CUtenso
                       const CUtensorMap& sb0, const CUtensorMap& b1, const CUtensorMap& sb1,
                       const CUtensorMap& y, MxParams p, cudaStream_t s) {
   const size_t smem = mx_smem_bytes<MODE>(p.E);
-  cudaError_t e = tile_counter_for_current_device(&p.tile_counter);
-  if (e != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(p.tile_counter, 0, sizeof(int), s)) != cudaSuccess) return e;
+  if (!p.tile_counter) {  // no counter of the caller's: one from the device's pool
+    const cudaError_t e = tile_counter_for_current_device(&p.tile_counter);
+    if (e != cudaSuccess) return e;
+  }
   return launch_persistent(ffn_mx_kernel<MODE>, 2, smem, s, a, sa, b0, sb0, b1, sb1, y, p);
 }
 
@@ -481,7 +483,7 @@ cudaError_t launch_expert_ffn_mxfp8(const uint8_t* xq, const uint8_t* xs, const 
                                     const int32_t* offsets, const int32_t* counts, uint8_t* hq,
                                     uint8_t* hs, float* y, const moe_shape_t& sh,
                                     int64_t rows_max, int32_t* dev_status, cudaStream_t s,
-                                    cudaEvent_t ev_mid) {
+                                    cudaEvent_t ev_mid, int* counter) {
   const int E = sh.E, H = sh.H, I = sh.I;
   const uint64_t EH = static_cast<uint64_t>(E) * H, EI = static_cast<uint64_t>(E) * I;
   const uint64_t rb = static_cast<uint64_t>(rows_max) / 128;  // 128-row blocks of the activations
@@ -496,11 +498,11 @@ cudaError_t launch_expert_ffn_mxfp8(const uint8_t* xq, const uint8_t* xs, const 
       !make_map_sf_atoms(&mW2s, W2s, EH / 128 * (I / 128)) ||
       !make_map(&mY, y, H, rows_max, 32, 32, true))
     return cudaErrorInvalidValue;
-  MxParams p1{nullptr, offsets, counts, E, sh.P, H, I, rows_max, hq, hs, dev_status, kWaitTimeoutNs};
+  MxParams p1{counter, offsets, counts, E, sh.P, H, I, rows_max, hq, hs, dev_status, kWaitTimeoutNs};
   cudaError_t e = launch_mx<0>(mXq, mXs, mW1, mW1s, mW3, mW3s, mY, p1, s);
   if (e != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
-  MxParams p2{nullptr, offsets, counts, E, sh.P, I, H, rows_max, nullptr, nullptr, dev_status,
+  MxParams p2{counter, offsets, counts, E, sh.P, I, H, rows_max, nullptr, nullptr, dev_status,
               kWaitTimeoutNs};
   return launch_mx<1>(mHq, mHs, mW2, mW2s, mW2, mW2s, mY, p2, s);
 }

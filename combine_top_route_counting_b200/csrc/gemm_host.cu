@@ -7,12 +7,13 @@
 namespace moe {
 
 // Tile counters the scheduler threads of the persistent GEMMs take tile ids
-// from. Each launch takes the next slot of the pool (round robin) and zeroes
-// it on its stream first, so GEMMs running at the same time on different
-// streams never share a counter: a slot comes round again only 256 launches
-// later, far more kernels than a device runs at once.
+// from, for launches whose caller passes none: {next tile, CTAs finished}
+// per slot, zero at load time and put back to zero by the last CTA of each
+// launch. Each launch takes the next slot (round robin); nothing is written
+// to a slot when a launch is enqueued, so a launch waiting in one stream is
+// never disturbed by launches enqueued on others.
 constexpr int kTileCounterSlots = 256;
-__device__ int g_tile_counter[kTileCounterSlots];
+__device__ int g_tile_counter[kTileCounterSlots * 2];
 
 namespace {
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -84,7 +85,7 @@ cudaError_t tile_counter_for_current_device(int** out) {
     if ((e = cudaGetSymbolAddress(&ptr, g_tile_counter)) != cudaSuccess) return e;
     ptrs[dev] = static_cast<int*>(ptr);
   }
-  *out = ptrs[dev] + (next[dev]++ % kTileCounterSlots);
+  *out = ptrs[dev] + 2 * (next[dev]++ % kTileCounterSlots);
   return cudaSuccess;
 }
 

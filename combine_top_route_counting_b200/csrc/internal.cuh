@@ -13,6 +13,12 @@ namespace moe {
 // Kernels launched by this library in this process (moe_launch_count).
 void note_launches(int64_t n);
 
+// The shape limits every entry point checks (include/moe.h): MOE_OK,
+// MOE_INVALID_ARG (null shape) or MOE_UNSUPPORTED_SHAPE.
+moe_status_t check_shape(const moe_shape_t* s);
+// Pointer on a 16-byte boundary (null passes).
+bool aligned16(const void* p);
+
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 
@@ -33,10 +39,26 @@ cudaError_t launch_schedule(const int32_t* ids, const moe_shape_t& sh, Slice sl,
                             int32_t* offsets, int32_t* counts, int32_t* route_row, int32_t* ws,
                             int32_t* dev_status, cudaStream_t s);
 
+// The schedule's one-launch kernel with a grid barrier that waits for one
+// block more than the launch has: every block gives up after timeout_ns and
+// raises MOE_DEV_TIMEOUT (failure-detection self test). cudaErrorInvalidConfiguration
+// if the shape does not take the one-launch kernel.
+cudaError_t launch_schedule_barrier_selftest(const int32_t* ids, const moe_shape_t& sh,
+                                             int32_t* phi, int32_t* offsets, int32_t* counts,
+                                             int32_t* route_row, int32_t* ws, int32_t* dev_status,
+                                             int64_t timeout_ns, cudaStream_t s);
+
 // Step 3a
 cudaError_t launch_dispatch(const uint16_t* x, const int32_t* phi, const int32_t* offsets,
                             uint16_t* xg, const moe_shape_t& sh, int64_t rows_max,
                             int32_t* dev_status, cudaStream_t s);
+
+// The persistent GEMMs below take their tiles from a tile counter: two device
+// int32 words {next tile, CTAs finished} that are zero when a launch starts
+// and that the launch's last CTA puts back to zero. `counter` is the caller's
+// (the layer entry points keep one in their workspace, zeroed once per call;
+// launches on one stream reuse it one after another), or null: a slot of the
+// device's pool (tile_counter_for_current_device).
 
 // Step 3b (two kernels; ev_mid, if not null, is recorded between them).
 // ab (training, pair tiles only): also keep the bf16 pre-activations [a | b].
@@ -44,7 +66,7 @@ cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint
                               const uint16_t* W2, const int32_t* offsets, const int32_t* counts,
                               uint16_t* h, float* y, const moe_shape_t& sh, int64_t rows_max,
                               int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_mid,
-                              uint16_t* ab = nullptr);
+                              uint16_t* ab = nullptr, int* counter = nullptr);
 
 // Steps 3a+3b fused: GEMM1 pulls its A rows from x by Phi (no xg buffer)
 cudaError_t launch_expert_ffn_gather(const uint16_t* x, const int32_t* phi, const uint16_t* W1,
@@ -68,7 +90,7 @@ cudaError_t launch_combine(const float* y, const int32_t* route_row, const float
 cudaError_t launch_dense_ffn(const uint16_t* x, int64_t n_tokens, const uint16_t* Ws1,
                              const uint16_t* Ws3, const uint16_t* Ws2, uint16_t* xpad,
                              uint16_t* hs, float* ys, int32_t* off, int32_t H, int32_t I,
-                             int32_t* dev_status, cudaStream_t s);
+                             int32_t* dev_status, cudaStream_t s, int* counter = nullptr);
 
 // 2D tensor map over [outer, inner] (inner contiguous) bf16 (or fp32)
 // elements with box [box_outer, box_inner] and 128-byte swizzle; false if the
@@ -77,7 +99,11 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, 
               uint32_t box_outer, bool fp32 = false);
 
 // A tile counter for one launch of a persistent GEMM on the current device:
-// the next slot of a per-device pool (the caller zeroes it on its stream).
+// the next slot of a per-device pool of 256 (round robin). A slot is clean
+// again as soon as the launch that used it has finished, so two launches
+// share one only if both run at the same moment while 255 other pool launches
+// were enqueued between them (or one captured graph is replayed on two
+// streams at once).
 cudaError_t tile_counter_for_current_device(int** out);
 
 // ---------------------------------------------------------------- backward
@@ -96,7 +122,7 @@ cudaError_t launch_expert_ffn_dgrad(const uint16_t* dys, const float* gate_row, 
                                     const int32_t* counts, uint16_t* dab, uint16_t* hg,
                                     float* part, float* dxg, const moe_shape_t& sh,
                                     int64_t rows_max, int32_t* dev_status, cudaStream_t s,
-                                    cudaEvent_t ev_mid);
+                                    cudaEvent_t ev_mid, int* counter = nullptr);
 
 // Push-reverse-dispatch: dx[t] = bf16(sum_j dxg[route_row[t, j]]), ascending j.
 cudaError_t launch_reverse_dispatch(const float* dxg, const int32_t* route_row, uint16_t* dx,
@@ -114,7 +140,7 @@ cudaError_t launch_expert_ffn_wgrad(const uint16_t* xg, const uint16_t* dys, con
                                     const uint16_t* hg, const int32_t* offsets,
                                     const int32_t* counts, float* dW1, float* dW3, float* dW2,
                                     const moe_shape_t& sh, int64_t rows_max, int32_t* dev_status,
-                                    cudaStream_t s, cudaEvent_t ev_mid);
+                                    cudaStream_t s, cudaEvent_t ev_mid, int* counter = nullptr);
 
 // ---------------------------------------------------------------- MXFP8
 // MX quantisation (E4M3 codes, one E8M0 scale per 32 values along the row).
@@ -151,7 +177,7 @@ cudaError_t launch_expert_ffn_mxfp8(const uint8_t* xq, const uint8_t* xs, const 
                                     const int32_t* offsets, const int32_t* counts, uint8_t* hq,
                                     uint8_t* hs, float* y, const moe_shape_t& sh,
                                     int64_t rows_max, int32_t* dev_status, cudaStream_t s,
-                                    cudaEvent_t ev_mid);
+                                    cudaEvent_t ev_mid, int* counter = nullptr);
 
 // 2D tensor map over a [outer, inner] uint8 matrix, box [box_outer, box_inner],
 // 128-byte swizzle.

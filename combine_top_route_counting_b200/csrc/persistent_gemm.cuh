@@ -147,6 +147,19 @@ __device__ __forceinline__ bool grouped_row_tile(int tile, const int32_t* s_off,
   return row0 < s_end[l];
 }
 
+// A launch's tile counter is two words: the next tile id, and the CTAs that
+// have finished. Called once per CTA (one thread, after the CTA's last use of
+// the counter): the last CTA to finish puts both words back to zero, so the
+// counter is clean for whichever launch takes it next, whenever that runs.
+__device__ __forceinline__ void finish_tile_counter(int* counter) {
+  __threadfence();  // this CTA's tile fetches come before its count
+  if (atomicAdd(counter + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+    __threadfence();  // every CTA's fetches come before the reset
+    atomicExch(counter, 0);
+    atomicExch(counter + 1, 0);
+  }
+}
+
 // Launch a persistent kernel on every SM: `cg` CTAs per cluster (1 or 2),
 // 384 threads, `smem` bytes of dynamic shared memory.
 template <class... KArgs, class... Args>

@@ -17,13 +17,17 @@
 // exclusive prefix sums of integer counts. Nothing is decided by the order of
 // atomics, so Phi is deterministic and equal to the definition.
 //
-// Kernels (one stream, no host round trip):
+// One cooperative launch runs all four stages with two grid barriers when
+// every block fits on the device at once (sched_fused_kernel, below);
+// otherwise four kernels (one stream, no host round trip):
 //   count    grid (C, P): per-block expert histogram -> ws[r][c][l]
 //   scan     per (r, l): exclusive prefix over c in place; M[l][r] -> counts
 //   offsets  one block: T[l] = sum_r M, Tp = ceil(T/pad)*pad, S = prefix(Tp)
 //   scatter  grid (C, P): per-warp bases, then place every route once; pad
 //            rows of Phi are filled with (-1,-1)
-// Route reads: each route id is read by count and by scatter (2*P*R).
+// Route reads: the four-kernel chain reads each route id in count and again
+// in scatter (2*P*R, the pages' count); the one-launch kernel keeps a block's
+// ids in registers between its phases and reads each once.
 #include "internal.cuh"
 
 namespace moe {
@@ -250,6 +254,238 @@ __global__ void __launch_bounds__(kThreads) sched_scatter_kernel(SchedParams p) 
   }
 }
 
+// ---------------------------------------------------------------- one launch
+// The same four stages in one cooperative launch (every block resident at
+// once), separated by two grid barriers:
+//   A  each block (c, r) reads its 2,048 route ids once, keeps them in
+//      registers, builds its warps' expert histograms in shared memory and
+//      writes the block histogram to ws[r][c][l];
+//   |  barrier 1
+//   B  every warp of the grid takes (peer, expert) columns in turn and
+//      replaces ws[r][.][l] by its exclusive prefix over blocks (32 blocks
+//      per warp-wide scan step); the column total is M[l][r] -> counts;
+//   |  barrier 2
+//   C  every block reads M into shared memory and computes T, Tp and S
+//      itself (block (0,0) writes offsets), derives its warps' bases from its
+//      block base, then places its routes from the registers of phase A and
+//      fills its share of padding rows.
+// Each route id is read from memory once. A barrier is a counter in ws
+// (zeroed before the launch): a block arrives with a release add and waits,
+// with an acquire load, until all blocks of the launch arrived; the wait is
+// bounded (timeout_ns), after which the block raises MOE_DEV_TIMEOUT and
+// leaves without writing anything more.
+struct FusedParams {
+  SchedParams sp;
+  uint32_t* bar;      // arrival counter, zero at launch
+  int32_t expect;     // blocks that must arrive (the grid; more only in the self test)
+  int64_t timeout_ns;
+};
+
+__device__ __forceinline__ uint64_t sched_now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Grid barrier number `gen` (1, 2, ...): true once every block of the launch
+// arrived, false (MOE_DEV_TIMEOUT raised) if the wait gave up.
+__device__ __forceinline__ bool sched_grid_barrier(const FusedParams& f, uint32_t gen) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    __threadfence();  // the block's writes (ordered before by the bar.sync above)
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(f.bar) : "memory");
+    const uint32_t target = gen * static_cast<uint32_t>(f.expect);
+    const uint64_t t0 = sched_now_ns();
+    for (;;) {
+      uint32_t v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f.bar) : "memory");
+      if (v >= target) break;
+      if (sched_now_ns() - t0 > static_cast<uint64_t>(f.timeout_ns)) {
+        atomicOr(f.sp.dev_status, MOE_DEV_TIMEOUT);
+        ok = 0;
+        break;
+      }
+      __nanosleep(64);
+    }
+    __threadfence();
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+__global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
+  const SchedParams& p = f.sp;
+  extern __shared__ int32_t smem[];
+  int32_t* wbase = smem;                 // [kWarps][E] warp counts, then warp bases
+  int32_t* s_cnt = smem + kWarps * p.E;  // [E][P] M
+  int32_t* s_off = s_cnt + p.E * p.P;    // [E+1] S
+  __shared__ int32_t s_part[kThreads];
+  const int c = blockIdx.x, r = blockIdx.y;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int R = p.Tm * p.k;
+  const int E = p.E, P = p.P;
+
+  // ---- A: count (ids read once, kept in registers)
+  int32_t* wh = wbase + w * E;
+  for (int l = lane; l < E; l += 32) wh[l] = 0;
+  __syncwarp();
+  const int q0 = c * kSchedBlockRoutes + w * kWarpRoutes;
+  int key[kSteps];
+  int bad = 0;
+#pragma unroll
+  for (int s = 0; s < kSteps; ++s) {
+    const int q = q0 + s * 32 + lane;
+    const int id = (q < R) ? __ldg(p.ids + route_index(p, r, q)) : -1;
+    const bool ok = static_cast<unsigned>(id) < static_cast<unsigned>(E);
+    if (q < R && !ok) bad = 1;
+    key[s] = ok ? id : kInvalid;
+  }
+  if (bad) atomicOr(p.dev_status, MOE_DEV_BAD_EXPERT_ID);
+#pragma unroll
+  for (int s = 0; s < kSteps; ++s) {
+    const unsigned m = __match_any_sync(kFull, key[s]);
+    if (key[s] != kInvalid && lane == __ffs(m) - 1) wh[key[s]] += __popc(m);
+    __syncwarp();
+  }
+  __syncthreads();
+  {
+    int32_t* out = p.ws + (static_cast<int64_t>(r) * p.C + c) * E;
+    for (int l = threadIdx.x; l < E; l += kThreads) {
+      int h = 0;
+#pragma unroll
+      for (int ww = 0; ww < kWarps; ++ww) h += wbase[ww * E + l];
+      out[l] = h;
+    }
+  }
+  if (!sched_grid_barrier(f, 1)) return;
+
+  // ---- B: exclusive prefix over blocks of every (peer, expert) column
+  {
+    const int nwarps = gridDim.x * gridDim.y * kWarps;
+    const int gw = (blockIdx.y * gridDim.x + blockIdx.x) * kWarps + w;
+    for (int col = gw; col < P * E; col += nwarps) {
+      const int r2 = col / E, l = col - r2 * E;
+      int32_t* base = p.ws + static_cast<int64_t>(r2) * p.C * E + l;
+      int carry = 0;
+      for (int c0 = 0; c0 < p.C; c0 += 32) {
+        const int cc = c0 + lane;
+        const int v = (cc < p.C) ? __ldcg(base + static_cast<int64_t>(cc) * E) : 0;
+        int x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(kFull, x, o);
+          if (lane >= o) x += y;
+        }
+        if (cc < p.C) base[static_cast<int64_t>(cc) * E] = carry + x - v;
+        carry += __shfl_sync(kFull, x, 31);
+      }
+      if (lane == 0) p.counts[l * P + r2] = carry;
+    }
+  }
+  if (!sched_grid_barrier(f, 2)) return;
+
+  // ---- C: offsets (every block), warp bases, placement, padding
+  for (int i = threadIdx.x; i < E * P; i += kThreads) s_cnt[i] = __ldcg(p.counts + i);
+  __syncthreads();
+  {
+    // thread t owns experts [4t, 4t + 4) (E <= 1024): padded totals, then a
+    // block-wide exclusive scan of the per-thread sums
+    const int l0 = threadIdx.x * 4;
+    int tpv[4];
+    int tsum = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int l = l0 + i;
+      tpv[i] = 0;
+      if (l < E) {
+        int T = 0;
+        for (int r2 = 0; r2 < P; ++r2) T += s_cnt[l * P + r2];
+        tpv[i] = (T + p.pad - 1) / p.pad * p.pad;
+        tsum += tpv[i];
+      }
+    }
+    int x = tsum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFull, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) s_part[w] = x;
+    __syncthreads();
+    int run = x - tsum;
+    for (int ww = 0; ww < w; ++ww) run += s_part[ww];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int l = l0 + i;
+      if (l < E) s_off[l] = run;
+      run += tpv[i];
+    }
+    if (threadIdx.x == kThreads - 1) s_off[E] = run;  // the last thread's end: the total
+  }
+  __syncthreads();
+  if (blockIdx.x == 0 && blockIdx.y == 0)
+    for (int l = threadIdx.x; l <= E; l += kThreads) p.offsets[l] = s_off[l];
+
+  // warp bases = block base (exclusive over blocks) + counts of earlier warps
+  {
+    const int32_t* blk = p.ws + (static_cast<int64_t>(r) * p.C + c) * E;
+    for (int l = threadIdx.x; l < E; l += kThreads) {
+      int run = __ldcg(blk + l);
+#pragma unroll
+      for (int ww = 0; ww < kWarps; ++ww) {
+        const int v = wbase[ww * E + l];
+        wbase[ww * E + l] = run;
+        run += v;
+      }
+    }
+  }
+  __syncthreads();
+
+  const unsigned lower = (1u << lane) - 1u;
+#pragma unroll
+  for (int s = 0; s < kSteps; ++s) {
+    const int q = q0 + s * 32 + lane;
+    const int id = key[s];
+    const bool valid = id != kInvalid;
+    const unsigned m = __match_any_sync(kFull, id);
+    int o = 0;
+    if (valid) o = wh[id] + __popc(m & lower);
+    __syncwarp();
+    if (valid && lane == __ffs(m) - 1) wh[id] += __popc(m);
+    __syncwarp();
+    if (q < R) {
+      const int64_t g = route_index(p, r, q);
+      if (valid) {
+        const int32_t* Ml = s_cnt + id * P;
+        int pos = 0;
+        for (int r2 = 0; r2 < P; ++r2) {
+          const int mm = Ml[r2];
+          pos += min(mm, o);
+          pos += (r2 < r && mm > o) ? 1 : 0;
+        }
+        const int row = s_off[id] + pos;
+        reinterpret_cast<int2*>(p.phi)[row] = make_int2(r, p.t0 + q / p.k);
+        p.route_row[g] = row;
+      } else {
+        p.route_row[g] = -1;
+      }
+    }
+  }
+
+  const int nb = gridDim.x * gridDim.y;
+  const int b = blockIdx.y * gridDim.x + blockIdx.x;
+  for (int l = b; l < E; l += nb) {
+    int T = 0;
+    for (int r2 = 0; r2 < P; ++r2) T += s_cnt[l * P + r2];
+    const int start = s_off[l] + T, end = s_off[l + 1];
+    for (int row = start + threadIdx.x; row < end; row += kThreads)
+      reinterpret_cast<int2*>(p.phi)[row] = make_int2(-1, -1);
+  }
+}
+
 inline int32_t blocks_per_peer(int32_t Tm, int32_t k) {
   const int64_t R = static_cast<int64_t>(Tm) * k;
   return static_cast<int32_t>((R + kSchedBlockRoutes - 1) / kSchedBlockRoutes);
@@ -257,15 +493,69 @@ inline int32_t blocks_per_peer(int32_t Tm, int32_t k) {
 
 }  // namespace
 
-size_t schedule_ws_bytes(int32_t P, int32_t N, int32_t k, int32_t E) {
+// [P][C][E] block counters, then the one-launch path's barrier counter on
+// its own 64-byte line.
+static int64_t counter_words(int32_t P, int32_t N, int32_t k, int32_t E) {
   const int64_t C = blocks_per_peer(N, k);
-  const int64_t words = static_cast<int64_t>(P) * (C > 0 ? C : 1) * E;
+  return static_cast<int64_t>(P) * (C > 0 ? C : 1) * E;
+}
+
+size_t schedule_ws_bytes(int32_t P, int32_t N, int32_t k, int32_t E) {
+  const int64_t words = (counter_words(P, N, k, E) + 15) / 16 * 16 + 16;
   return static_cast<size_t>(words) * sizeof(int32_t);
 }
 
-cudaError_t launch_schedule(const int32_t* ids, const moe_shape_t& sh, Slice sl, int32_t* phi,
-                            int32_t* offsets, int32_t* counts, int32_t* route_row, int32_t* ws,
-                            int32_t* dev_status, cudaStream_t s) {
+namespace {
+
+// Shared memory of the one-launch kernel: warp counts [8][E], M [E][P], S [E+1].
+size_t fused_smem_bytes(int32_t P, int32_t E) {
+  return (static_cast<size_t>(kWarps) * E + static_cast<size_t>(E) * P + E + 1) * sizeof(int32_t);
+}
+
+// Whether the one-launch kernel can run for this grid: its shared memory fits
+// and every block can be resident at once (a cooperative launch requires it).
+bool fused_fits(int32_t C, int32_t P, int32_t E) {
+  const size_t smem = fused_smem_bytes(P, E);
+  if (C <= 0 || smem > 100 * 1024) return false;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(sched_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return false;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sched_fused_kernel, kThreads, smem) !=
+      cudaSuccess)
+    return false;
+  return static_cast<int64_t>(per_sm) * device_sm_count() >= static_cast<int64_t>(C) * P;
+}
+
+cudaError_t launch_fused(const SchedParams& p, int32_t extra_expect, int64_t timeout_ns,
+                         cudaStream_t s) {
+  FusedParams f;
+  f.sp = p;
+  f.bar = reinterpret_cast<uint32_t*>(p.ws + (counter_words(p.P, p.N, p.k, p.E) + 15) / 16 * 16);
+  f.expect = p.C * p.P + extra_expect;
+  f.timeout_ns = timeout_ns;
+  cudaError_t e = cudaMemsetAsync(f.bar, 0, sizeof(uint32_t), s);
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute coop[1];
+  coop[0].id = cudaLaunchAttributeCooperative;
+  coop[0].val.cooperative = 1;
+  cudaLaunchConfig_t c = {};
+  c.gridDim = dim3(p.C, p.P);
+  c.blockDim = dim3(kThreads);
+  c.dynamicSmemBytes = fused_smem_bytes(p.P, p.E);
+  c.stream = s;
+  c.attrs = coop;
+  c.numAttrs = 1;
+  e = cudaLaunchKernelEx(&c, sched_fused_kernel, f);
+  note_launches(1);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+SchedParams make_params(const int32_t* ids, const moe_shape_t& sh, Slice sl, int32_t* phi,
+                        int32_t* offsets, int32_t* counts, int32_t* route_row, int32_t* ws,
+                        int32_t* dev_status) {
   SchedParams p;
   p.ids = ids;
   p.P = sh.P;
@@ -282,6 +572,28 @@ cudaError_t launch_schedule(const int32_t* ids, const moe_shape_t& sh, Slice sl,
   p.route_row = route_row;
   p.ws = ws;
   p.dev_status = dev_status;
+  return p;
+}
+
+}  // namespace
+
+cudaError_t launch_schedule_barrier_selftest(const int32_t* ids, const moe_shape_t& sh,
+                                             int32_t* phi, int32_t* offsets, int32_t* counts,
+                                             int32_t* route_row, int32_t* ws, int32_t* dev_status,
+                                             int64_t timeout_ns, cudaStream_t s) {
+  const SchedParams p =
+      make_params(ids, sh, Slice{0, sh.N}, phi, offsets, counts, route_row, ws, dev_status);
+  if (!fused_fits(p.C, p.P, p.E)) return cudaErrorInvalidConfiguration;
+  return launch_fused(p, /*extra_expect=*/1, timeout_ns, s);
+}
+
+cudaError_t launch_schedule(const int32_t* ids, const moe_shape_t& sh, Slice sl, int32_t* phi,
+                            int32_t* offsets, int32_t* counts, int32_t* route_row, int32_t* ws,
+                            int32_t* dev_status, cudaStream_t s) {
+  const SchedParams p = make_params(ids, sh, sl, phi, offsets, counts, route_row, ws, dev_status);
+  // one launch when every block fits on the device at once (the Kimi shape:
+  // 28 x 8 blocks); otherwise the four-kernel chain below
+  if (fused_fits(p.C, p.P, p.E)) return launch_fused(p, 0, kWaitTimeoutNs, s);
   int launched = 0;
   cudaError_t e = cudaSuccess;
   // count runs in plain stream order (after whatever wrote ids); scan, offsets

@@ -53,20 +53,13 @@ extern "C" moe_status_t moe_schedule_static_ws(const int32_t* ids, int32_t* phi,
                                                int32_t* counts, int32_t* route_row,
                                                int32_t* dev_status, const moe_shape_t* shape,
                                                void* stream) {
-  if (!shape) return MOE_INVALID_ARG;
+  // the same argument checks as moe_schedule
+  const moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
   const moe_shape_t& s = *shape;
-  if (s.P < 1 || s.P > 64 || s.N < 0 || s.E < 1 || s.E > 1024 || s.k < 1 || s.k > 16 ||
-      s.k > s.E || s.pad < 1 || s.pad > (1 << 16))
-    return MOE_UNSUPPORTED_SHAPE;
-  const int64_t routes = static_cast<int64_t>(s.P) * s.N * s.k;
-  if (routes >= (int64_t{1} << 31) ||
-      routes + static_cast<int64_t>(s.E) * (s.pad - 1) + 255 >= (int64_t{1} << 31))
-    return MOE_UNSUPPORTED_SHAPE;
   if (!phi || !offsets || !counts || !dev_status) return MOE_INVALID_ARG;
   if (s.N > 0 && (!ids || !route_row)) return MOE_INVALID_ARG;
-  const uintptr_t mis = reinterpret_cast<uintptr_t>(ids) | reinterpret_cast<uintptr_t>(phi) |
-                        reinterpret_cast<uintptr_t>(route_row);
-  if (mis & 15u) return MOE_INVALID_ARG;
+  if (!aligned16(ids) || !aligned16(phi) || !aligned16(route_row)) return MOE_INVALID_ARG;
   // the same counter layout moe_schedule uses: [P][ceil(N*k/2048)][E] int32
   if (schedule_ws_bytes(s.P, s.N, s.k, s.E) > static_cast<size_t>(kStaticSchedWords) * 4)
     return MOE_WORKSPACE_TOO_SMALL;

@@ -22,7 +22,7 @@ __global__ void one_segment_kernel(int32_t* off, int32_t rows) {
 cudaError_t launch_dense_ffn(const uint16_t* x, int64_t n_tokens, const uint16_t* Ws1,
                              const uint16_t* Ws3, const uint16_t* Ws2, uint16_t* xpad,
                              uint16_t* hs, float* ys, int32_t* off, int32_t H, int32_t I,
-                             int32_t* dev_status, cudaStream_t s) {
+                             int32_t* dev_status, cudaStream_t s, int* counter) {
   if (n_tokens <= 0) return cudaSuccess;
   const int64_t rows = (n_tokens + 255) / 256 * 256;
   const size_t row_bytes = static_cast<size_t>(H) * 2;
@@ -50,7 +50,7 @@ cudaError_t launch_dense_ffn(const uint16_t* x, int64_t n_tokens, const uint16_t
   one.I = I;
   one.pad = 256;
   return launch_expert_ffn(a, Ws1, Ws3, Ws2, off, nullptr, hs, ys, one, rows, dev_status, s,
-                           nullptr);
+                           nullptr, nullptr, counter);
 }
 
 }  // namespace moe

@@ -97,6 +97,8 @@ _SIGS = {
     "moe_layer_mxfp8_workspace_bytes": ([ctypes.POINTER(Shape)], ctypes.c_size_t),
     "moe_launch_count": ([], ctypes.c_int64),
     "moe_selftest_bounded_wait": ([_vp, ctypes.c_int64, _vp], ctypes.c_int),
+    "moe_selftest_schedule_barrier": ([_vp] * 6 + [ctypes.c_size_t, _vp, ctypes.POINTER(Shape),
+                                                   ctypes.c_int64, _vp], ctypes.c_int),
 }
 
 
@@ -474,6 +476,16 @@ def moe_selftest_bounded_wait(dev_status, timeout_ns: int, stream=None):
     _check(load().moe_selftest_bounded_wait(_ptr(dev_status, torch.int32, "dev_status"),
                                             int(timeout_ns), _stream(stream)),
            "moe_selftest_bounded_wait")
+
+
+def moe_selftest_schedule_barrier(ids, phi, offsets, counts, route_row, ws, dev_status, sh: Shape,
+                                  timeout_ns: int, stream=None):
+    _check(load().moe_selftest_schedule_barrier(
+        _ptr(ids, torch.int32, "ids"), _ptr(phi, torch.int32, "phi"),
+        _ptr(offsets, torch.int32, "offsets"), _ptr(counts, torch.int32, "counts"),
+        _ptr(route_row, torch.int32, "route_row"), _ptr(ws, torch.uint8, "ws"), ws.numel(),
+        _ptr(dev_status, torch.int32, "dev_status"), ctypes.byref(sh), int(timeout_ns),
+        _stream(stream)), "moe_selftest_schedule_barrier")
 
 
 # ---------------------------------------------------------------- buffers

@@ -149,10 +149,15 @@ moe_status_t moe_schedule(const int32_t* ids, int32_t* phi, int32_t* offsets, in
  * rejected with MOE_WORKSPACE_TOO_SMALL before anything is enqueued. The
  * first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
- * capture. All calls share the one array and it keeps the last call's
- * contents (the kernels overwrite every word they read), so calls that
- * overlap on the GPU -- e.g. on two streams at once -- race and must be
- * serialised by the caller. Allocates no device or host memory. */
+ * capture. Under lazy module loading (the CUDA default) that first call may
+ * also load the library's device code, the 4 MiB array with it; later calls
+ * allocate nothing. The address is kept for the life of the process: after a
+ * cudaDeviceReset the kept address is stale, so do not call this entry point
+ * on that device again in the same process. All calls share the one array
+ * and it keeps the last call's contents (the kernels overwrite every word
+ * they read), so calls that overlap on the GPU -- e.g. on two streams at
+ * once -- race and must be serialised by the caller. Calls no cudaMalloc,
+ * cudaFree or other allocating routine. */
 moe_status_t moe_schedule_static_ws(const int32_t* ids, int32_t* phi, int32_t* offsets,
                                     int32_t* counts, int32_t* route_row, int32_t* dev_status,
                                     const moe_shape_t* shape, void* stream);
@@ -177,9 +182,16 @@ moe_status_t moe_dispatch(const uint16_t* x, const int32_t* phi, const int32_t* 
  * padding rows are skipped and their h/y rows are left unwritten; rows that
  * carry routes are always written. Each output element is computed by one
  * CTA (pair) with a fixed K order: the result is bitwise deterministic.
- * The GEMM kernels take their tiles from a tile counter inside the library:
- * each GEMM launch takes the next of 256 per-device slots and zeroes it on
- * `stream`, so FFN calls on different streams may run at the same time.
+ * Tile counter: the GEMM kernels take their tiles from a counter of two
+ * int32 words that the last CTA of each launch puts back to zero. The GEMM
+ * entry points without a workspace (this one, moe_expert_ffn_gather,
+ * moe_expert_ffn_train, _dgrad, _wgrad, _mxfp8) take the next of 256 such
+ * counters per device, round robin; nothing is written to a counter when a
+ * launch is enqueued, so FFN calls on different streams may run at the same
+ * time. Two launches share a counter only if both run at the same moment
+ * with 255 other such launches enqueued between them, or if one captured
+ * graph holding them is replayed on two streams at once: neither is allowed.
+ * The layer entry points keep their counter in `ws` instead.
  * offsets must be non-decreasing multiples of 128 with offsets[E] <=
  * moe_rows_max (else MOE_DEV_BAD_SCHEDULE, nothing written). */
 moe_status_t moe_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint16_t* W3,
@@ -500,6 +512,20 @@ int64_t moe_launch_count(void);
  * giving up after timeout_ns nanoseconds; it then raises MOE_DEV_TIMEOUT in
  * *dev_status. The context stays usable. */
 moe_status_t moe_selftest_bounded_wait(int32_t* dev_status, int64_t timeout_ns, void* stream);
+
+/* Failure-detection self test of the schedule's one-launch kernel
+ * (moe_schedule runs it when all its blocks fit on the device at once; its
+ * two grid barriers are bounded waits): the same kernel, on the same
+ * arguments as moe_schedule, with a barrier that waits for one block more
+ * than the launch has. Every block gives up after timeout_ns nanoseconds,
+ * raises MOE_DEV_TIMEOUT in *dev_status and returns; the outputs are then
+ * incomplete and the context stays usable. MOE_UNSUPPORTED_SHAPE if the
+ * shape does not take the one-launch kernel; N >= 1. */
+moe_status_t moe_selftest_schedule_barrier(const int32_t* ids, int32_t* phi, int32_t* offsets,
+                                           int32_t* counts, int32_t* route_row, void* ws,
+                                           size_t ws_bytes, int32_t* dev_status,
+                                           const moe_shape_t* shape, int64_t timeout_ns,
+                                           void* stream);
 
 #ifdef __cplusplus
 }

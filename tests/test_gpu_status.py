@@ -22,6 +22,32 @@ def test_bounded_wait_times_out_and_context_survives(cuda_lib):
     assert int(a.sum().item()) == 45
 
 
+def test_schedule_grid_barrier_times_out_and_context_survives(cuda_lib):
+    """The schedule's one-launch kernel with a barrier expecting one block more
+    than it launched: every block gives up after 20 ms and raises
+    MOE_DEV_TIMEOUT; the next ordinary schedule on the same buffers is exact."""
+    import oracle
+    moe = cuda_lib
+    P, N, E, k = 8, 1024, 64, 4
+    ids = inputs.make_ids_uniform(P, N, E, k, seed=41)
+    sh = moe.shape(P, N, E, k)
+    b = moe.alloc_schedule_outputs(sh)
+    ids_d = ids.to("cuda")
+    moe.moe_selftest_schedule_barrier(ids_d, b["phi"], b["offsets"], b["counts"], b["route_row"],
+                                      b["ws"], b["dev_status"], sh, 20_000_000)
+    torch.cuda.synchronize()
+    assert int(b["dev_status"].item()) & moe.DEV_TIMEOUT
+    b["dev_status"].zero_()
+    moe.moe_schedule(ids_d, b["phi"], b["offsets"], b["counts"], b["route_row"], b["ws"],
+                     b["dev_status"], sh)
+    torch.cuda.synchronize()
+    assert int(b["dev_status"].item()) == 0
+    o = oracle.schedule(ids.numpy(), P, N, k, E, 256)
+    rows = int(o["offsets"][-1])
+    assert (b["phi"][:rows].cpu().numpy() == o["phi"]).all()
+    assert (b["route_row"].cpu().numpy() == o["route_row"]).all()
+
+
 def test_host_side_errors(cuda_lib):
     moe = cuda_lib
     sh = moe.shape(1, 16, 8, 2, 256, 128)
