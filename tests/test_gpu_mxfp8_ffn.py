@@ -16,10 +16,7 @@ from combine_top_route_counting_b200 import inputs
 from tests.helpers import (OUT_TOL, Y_TOL, bf16_to_f64, bits, expert_weights_host,
                            mx_tiled_offsets, rms_floor_err, sha, to_tiled)
 
-# The block-scaled GEMMs are compiled (sm_100a) but have not yet run on a
-# B200; these tests are the first thing to run there.
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skip(reason="block-scaled MXFP8 kernels not yet run on a B200")]
+pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
