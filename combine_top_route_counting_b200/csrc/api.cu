@@ -81,7 +81,7 @@ moe_status_t check_mx_shape(const moe_shape_t* s) {
 // backward's buffers; dxg [rows, H] fp32 reuses y, which is dead once the
 // forward's combine has run.
 struct LayerWs {
-  size_t ids, gates, route_row, phi, offsets, counts, sched, ctr, xg, h, y, total;
+  size_t ids, gates, route_row, phi, offsets, counts, sched, ctr, land, xg, h, y, total;
   size_t logits[2], x[2], out[2], total_host;  // moe_layer_forward_host additions
   size_t ab, dys, dab, hg, gate_row, part, total_train;  // training additions
   size_t sh_off, sh_x, sh_h, sh_y, total_mx;  // the MXFP8 layer's shared expert
@@ -106,6 +106,7 @@ LayerWs layer_ws(const moe_shape_t* s) {
   w.counts = take(o, static_cast<size_t>(s->E) * s->P * 4);
   w.sched = take(o, schedule_ws_bytes(s->P, s->N, s->k, s->E));
   w.ctr = take(o, 8);  // the GEMMs' tile counter, zeroed at the start of each call
+  w.land = take(o, (16 + rows / 128) * 4);  // fused dispatch: next block, then ready flags
   w.xg = take(o, rows * s->H * 2);
   w.h = take(o, rows * s->I * 2);
   w.y = take(o, rows * s->H * 4);
@@ -161,7 +162,7 @@ namespace {
 
 struct LayerBufs {
   int32_t *ids, *route_row, *phi, *offsets, *counts, *sched;
-  int* ctr;
+  int *ctr, *land;
   float *gates, *y;
   uint16_t *xg, *h;
 };
@@ -176,6 +177,7 @@ LayerBufs layer_bufs(void* ws, const LayerWs& w) {
   b.counts = at<int32_t>(ws, w.counts);
   b.sched = at<int32_t>(ws, w.sched);
   b.ctr = at<int>(ws, w.ctr);
+  b.land = at<int>(ws, w.land);
   b.xg = at<uint16_t>(ws, w.xg);
   b.h = at<uint16_t>(ws, w.h);
   b.y = at<float>(ws, w.y);
@@ -198,16 +200,26 @@ cudaError_t run_slice(const LayerBufs& b, const uint16_t* x, const uint16_t* W1,
   if ((e = launch_schedule(b.ids, *sh, sl, b.phi, b.offsets, b.counts, b.route_row, b.sched,
                            dev_status, s)) != cudaSuccess)
     return e;
-  // The pull dispatch runs as its own HBM-bound gather: feeding GEMM1 with row
-  // gathers instead (moe_expert_ffn_gather) measured 2.6-3x slower on B200,
-  // the gathers delivering far fewer bytes per clock than the MMAs use.
+  // With CTA-pair tiles (segments padded to 256 rows) the pull dispatch runs
+  // inside GEMM1: its spare warp lands the rows into xg block by block while
+  // the tensor cores work on the blocks already there. Otherwise the dispatch
+  // is its own HBM-bound gather before the FFN. (Feeding the MMAs straight
+  // from x by row gathers, moe_expert_ffn_gather, measured 2.6-3x slower.)
   if ((e = rec(2)) != cudaSuccess) return e;
-  if ((e = launch_dispatch(x, b.phi, b.offsets, b.xg, *sh, rows_max, dev_status, s)) != cudaSuccess)
+  const bool fused = sh->pad % 256 == 0;
+  const LandArgs land{x, b.phi, b.land, b.land + 16};
+  if (fused) {
+    if ((e = cudaMemsetAsync(b.land, 0, (16 + rows_max / 128) * sizeof(int), s)) != cudaSuccess)
+      return e;
+  } else if ((e = launch_dispatch(x, b.phi, b.offsets, b.xg, *sh, rows_max, dev_status, s)) !=
+             cudaSuccess) {
     return e;
+  }
   if ((e = rec(3)) != cudaSuccess) return e;
   cudaEvent_t mid = (ev && ev[4]) ? static_cast<cudaEvent_t>(ev[4]) : nullptr;
   if ((e = launch_expert_ffn(b.xg, W1, W3, W2, b.offsets, b.counts, b.h, b.y, *sh, rows_max,
-                             dev_status, s, mid, ab, b.ctr)) != cudaSuccess)
+                             dev_status, s, mid, ab, b.ctr, fused ? &land : nullptr)) !=
+      cudaSuccess)
     return e;
   if ((e = rec(5)) != cudaSuccess) return e;
   if ((e = launch_combine(b.y, b.route_row, b.gates, out, *sh, sl, rows_max, dev_status, s)) !=

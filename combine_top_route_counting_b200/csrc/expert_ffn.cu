@@ -57,13 +57,14 @@ using namespace sm100;
 using namespace pg;
 
 // Tile geometry for CG CTAs per MMA (1: one SM, 2: a CTA pair on two SMs).
-// TMA_STORE (GEMM2 on CTA pairs): the fp32 epilogue stages each warp's 32x32
-// block in 128-byte-swizzled shared memory and writes it with one TMA store,
-// keeping the load/store unit free; it costs one pipeline stage.
+// TMA_STORE (GEMM2 on CTA pairs): the fp32 epilogue stages each warp's 32x16
+// blocks in 64-byte-swizzled shared memory (2 KB per warp) and writes each
+// with one TMA store, keeping the load/store unit free; the 16 KB of staging
+// leave room for six pipeline stages, as GEMM1 has.
 template <int CG, int MODE>
 struct Cfg {
   static constexpr bool TMA_STORE = (CG == 2 && MODE == 1);
-  static constexpr int STAGING_BYTES = TMA_STORE ? 8 * 4096 : 0;  // 8 warps x 32x32 fp32
+  static constexpr int STAGING_BYTES = TMA_STORE ? 8 * 2048 : 0;  // 8 warps x 32x16 fp32
   static constexpr int BM = 128 * CG;      // rows per tile (each CTA holds 128)
   static constexpr int BN = 256;           // accumulator columns per tile
   static constexpr int BK = 64;            // K per stage: one 128-byte swizzle row of bf16
@@ -71,7 +72,7 @@ struct Cfg {
   static constexpr int A_BYTES = 128 * BK * 2;   // 16 KB
   static constexpr int B_ATOM_BYTES = 64 * BK * 2;  // 8 KB
   static constexpr int STAGE_BYTES = A_BYTES + B_ATOMS * B_ATOM_BYTES;  // 48 / 32 KB
-  static constexpr int STAGES = CG == 1 ? 4 : (TMA_STORE ? 5 : 6);
+  static constexpr int STAGES = CG == 1 ? 4 : 6;
   static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*B MN-major*/ 1);
   static constexpr int BAR_FULL = 0;
   static constexpr int BAR_EMPTY = STAGES;
@@ -101,8 +102,36 @@ struct FfnParams {
   int32_t* dev_status;
   int64_t timeout_ns;
   uint16_t* ab;            // SAVE_AB: bf16 pre-activations [rows_max, 2I], a | b
-  const void* x;           // GATHER: token activations bf16 [P*N, H]
+  const void* x;           // GATHER, LAND: token activations bf16 [P*N, H]
+  uint16_t* xg;            // LAND: the gathered buffer [rows_max, H] the A map reads
+  int* land_next;          // LAND: next 128-row block to land (0 at launch)
+  int* land_ready;         // LAND: [rows_max / 128] block-landed flags (0 at launch)
 };
+
+// Wait (bounded, acquire at GPU scope) until *flag != 0: the LAND producer's
+// wait for a block of gathered rows that another CTA's warp lands. Gives up
+// like wait_bounded: after timeout_ns, or once another role of the CTA gave up.
+__device__ __forceinline__ bool wait_flag_bounded(const int* flag, const WaitCtx& w) {
+  auto ready = [&]() {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    return v != 0;
+  };
+  if (ready()) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(32);
+    if (ready()) return true;
+    if ((it & 15u) == 0) {
+      if (*w.abort) return false;
+      if (globaltimer_ns() - t0 > static_cast<uint64_t>(w.timeout_ns)) {
+        *w.abort = 1;
+        atomicOr(w.dev_status, w.timeout_flag);
+        return false;
+      }
+    }
+  }
+}
 
 template <int CG, int MODE>
 size_t smem_bytes_for(int E) {
@@ -131,7 +160,17 @@ __device__ __forceinline__ float silu(float a) { return a / (1.0f + expf(-a)); }
 // CTA pair) per 256x256 tile; CTA r loads rows [128r, 128r+128) of A and
 // columns [128r, 128r+128) of B, the leader (r = 0) issues the pair MMAs and
 // each CTA drains its own 128 TMEM lanes.
-template <int MODE, int CG, bool GATHER, bool SAVE_AB>
+// LAND (MODE 0, CG 2): the pull dispatch runs inside this kernel. Warp 3 of
+// every CTA takes 128-row blocks of the expert-sorted layout in order from a
+// device counter, copies each row from x through Phi into xg (16-byte loads
+// and stores; padding rows zero-filled), and publishes the block with a
+// release store of its flag. The TMA producer waits (bounded) for the flag of
+// its CTA's 128 rows before it loads a tile's A operand, then issues a
+// cross-proxy fence, since the rows were written through the generic proxy
+// and TMA reads through the async proxy. Blocks are landed in the order the
+// tiles are handed out, so the copies run ahead of the tensor cores and the
+// HBM-bound gather overlaps the MMAs; no warp that lands rows ever waits.
+template <int MODE, int CG, bool GATHER, bool SAVE_AB, bool LAND = false>
 __global__ void __launch_bounds__(kNumThreads, 1)
     ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmY,
@@ -354,6 +393,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         if (!tile_info(tile, row0, n, l)) continue;
         const int arow = row0 + static_cast<int>(rank) * 128;
         const int yb = l * p.K;
+        if (LAND) {  // this CTA's 128 A rows must have landed
+          if (!wait_flag_bounded(p.land_ready + arow / 128, wc)) break;
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!wait_bounded(smem_u32(&bars[C::BAR_EMPTY + stage]), phase ^ 1u, wc)) {
             ok = false;
@@ -403,6 +446,48 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         wait_drain(smem_u32(&bars[(leader ? C::BAR_FULL : C::BAR_EMPTY) + st]), par, drain_ns);
       }
     }
+  } else if (warp == 3 && LAND) {
+    // ------------------------------------------------------------ pull dispatch
+    const int nblk = rows_used / 128;
+    const int chunks = p.K / 8;  // 16-byte chunks per row (H % 256 == 0: a multiple of 32)
+    const uint4* xsrc = reinterpret_cast<const uint4*>(p.x);
+    int bad = 0;
+    for (;;) {
+      int b = 0;
+      if (lane == 0) b = atomicAdd(p.land_next, 1);
+      b = __shfl_sync(0xFFFFFFFFu, b, 0);
+      if (b >= nblk || *wc.abort) break;
+#pragma unroll 1
+      for (int rr = 0; rr < 128; ++rr) {
+        const int64_t row = static_cast<int64_t>(b) * 128 + rr;
+        const int2 e = __ldg(p.phi + row);
+        const bool v = e.x >= 0 && e.x < p.P && e.y >= 0 && e.y < p.n_per_peer;
+        if (!v && (e.x >= 0 || e.y != -1)) bad = 1;  // (-1,-1) is padding
+        uint4* dst = reinterpret_cast<uint4*>(p.xg) + row * chunks;
+        const uint4* src = xsrc + (v ? (static_cast<int64_t>(e.x) * p.n_per_peer + e.y) * chunks : 0);
+        constexpr int U = 28;  // a 7,168-wide row in one round: 28 loads in flight per lane
+#pragma unroll 1
+        for (int c0 = lane; c0 < chunks; c0 += 32 * U) {
+          uint4 t[U];
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int c = c0 + 32 * u;
+            t[u] = (v && c < chunks) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int c = c0 + 32 * u;
+            if (c < chunks) dst[c] = t[u];
+          }
+        }
+      }
+      __threadfence();  // every lane's rows before the flag
+      __syncwarp();
+      if (lane == 0)
+        asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p.land_ready + b), "r"(1)
+                     : "memory");
+    }
+    if (bad) atomicOr(p.dev_status, MOE_DEV_BAD_SCHEDULE);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && leader) {
@@ -534,32 +619,32 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           if (c + 1 < 2) tmem_ld_wait();
         }
       } else if (C::TMA_STORE) {
-        // row `lane` of this warp's 32x32 block goes to the staging slot with
-        // 16-byte chunk j at position j ^ (lane & 7): the 128-byte swizzle the
-        // tensor map expects, and no bank conflicts for the 16-byte writes.
-        const uint32_t stg = smem_u32(staging) + (warp - kEpiWarp0) * 4096;
+        // row `lane` of this warp's 32x16 block goes to the staging slot with
+        // 16-byte chunk j at position j ^ ((lane >> 1) & 3): the 64-byte swizzle
+        // the tensor map expects, and no bank conflicts for the 16-byte writes.
+        const uint32_t stg = smem_u32(staging) + (warp - kEpiWarp0) * 2048;
         const uint64_t pol_y = l2_policy_evict_first();
         const int ycol = n * C::BN + half * 128;
         const int yrow0 = row0 + static_cast<int>(rank) * 128 + q * 32;
-        uint32_t rv[2][32];
-        tmem_ld_32cols(tbase + half * 128, rv[0]);
+        uint32_t rv[2][16];
+        tmem_ld_16cols(tbase + half * 128, rv[0]);
         tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c + 1 < 4) tmem_ld_32cols(tbase + half * 128 + (c + 1) * 32, rv[(c + 1) & 1]);
+        for (int c = 0; c < 8; ++c) {
+          if (c + 1 < 8) tmem_ld_16cols(tbase + half * 128 + (c + 1) * 16, rv[(c + 1) & 1]);
           if (lane == 0) bulk_wait_read_all();  // the previous store has read the slot
           __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            st_shared_v4(stg + lane * 128 + ((j ^ (lane & 7)) << 4), rv[c & 1][4 * j],
+          for (int j = 0; j < 4; ++j)
+            st_shared_v4(stg + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4), rv[c & 1][4 * j],
                          rv[c & 1][4 * j + 1], rv[c & 1][4 * j + 2], rv[c & 1][4 * j + 3]);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {  // y is streamed out and read once, by the combine
-            tma_store_2d_hint(&tmY, stg, ycol + c * 32, yrow0, pol_y);
+            tma_store_2d_hint(&tmY, stg, ycol + c * 16, yrow0, pol_y);
             bulk_commit_group();
           }
-          if (c + 1 < 4) tmem_ld_wait();
+          if (c + 1 < 8) tmem_ld_wait();
         }
       } else {
         float* yrow = reinterpret_cast<float*>(p.out) + row * p.Nout + n * C::BN + half * 128;
@@ -606,7 +691,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 
 namespace {
 
-template <int MODE, int CG, bool GATHER = false, bool SAVE_AB = false>
+template <int MODE, int CG, bool GATHER = false, bool SAVE_AB = false, bool LAND = false>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const CUtensorMap& yo, FfnParams p, cudaStream_t s) {
   const size_t smem = smem_bytes_for<CG, MODE>(p.E);
@@ -614,8 +699,8 @@ cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUten
     const cudaError_t e = tile_counter_for_current_device(&p.tile_counter);
     if (e != cudaSuccess) return e;
   }
-  return launch_persistent(ffn_gemm_kernel<MODE, CG, GATHER, SAVE_AB>, CG, smem, s, a, b0, b1, yo,
-                           p);
+  return launch_persistent(ffn_gemm_kernel<MODE, CG, GATHER, SAVE_AB, LAND>, CG, smem, s, a, b0, b1,
+                           yo, p);
 }
 
 }  // namespace
@@ -624,13 +709,13 @@ cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint
                               const uint16_t* W2, const int32_t* offsets, const int32_t* counts,
                               uint16_t* h, float* y, const moe_shape_t& sh, int64_t rows_max,
                               int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_mid,
-                              uint16_t* ab, int* counter) {
+                              uint16_t* ab, int* counter, const LandArgs* land) {
   const int E = sh.E, H = sh.H, I = sh.I;
   CUtensorMap mA1, mW1, mW3, mA2, mW2, mY;
   const uint64_t EH = static_cast<uint64_t>(E) * H, EI = static_cast<uint64_t>(E) * I;
   if (!make_map(&mA1, xg, H, rows_max, 64, 128) || !make_map(&mW1, W1, I, EH, 64, 64) ||
       !make_map(&mW3, W3, I, EH, 64, 64) || !make_map(&mA2, h, I, rows_max, 64, 128) ||
-      !make_map(&mW2, W2, H, EI, 64, 64) || !make_map(&mY, y, H, rows_max, 32, 32, true))
+      !make_map(&mW2, W2, H, EI, 64, 64) || !make_map(&mY, y, H, rows_max, 16, 32, true, true))
     return cudaErrorInvalidValue;
   // Segments that are multiples of 256 rows run on CTA pairs (256x256 tiles);
   // otherwise (pad a multiple of 128 only) on single CTAs (128x256 tiles).
@@ -638,10 +723,21 @@ cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint
   FfnParams p1{counter, nullptr, 0, offsets, counts, E, sh.P, H, I, rows_max, h, dev_status,
                kWaitTimeoutNs, ab};
   cudaError_t e;
-  if (ab)  // training: keep the pre-activations (pair tiles only)
+  if (land) {  // the pull dispatch fused into GEMM1 (pair tiles only)
+    if (!pair) return cudaErrorInvalidValue;
+    p1.phi = reinterpret_cast<const int2*>(land->phi);
+    p1.n_per_peer = sh.N;
+    p1.x = land->x;
+    p1.xg = const_cast<uint16_t*>(xg);
+    p1.land_next = land->next;
+    p1.land_ready = land->ready;
+    e = ab ? launch_mode<0, 2, false, true, true>(mA1, mW1, mW3, mA1, p1, s)
+           : launch_mode<0, 2, false, false, true>(mA1, mW1, mW3, mA1, p1, s);
+  } else if (ab) {  // training: keep the pre-activations (pair tiles only)
     e = pair ? launch_mode<0, 2, false, true>(mA1, mW1, mW3, mA1, p1, s) : cudaErrorInvalidValue;
-  else
+  } else {
     e = pair ? launch_mode<0, 2>(mA1, mW1, mW3, mA1, p1, s) : launch_mode<0, 1>(mA1, mW1, mW3, mA1, p1, s);
+  }
   if (e != cudaSuccess) return e;
   if (ev_mid) {
     e = cudaEventRecord(ev_mid, s);
@@ -663,7 +759,7 @@ cudaError_t launch_expert_ffn_gather(const uint16_t* x, const int32_t* phi, cons
   const uint64_t EH = static_cast<uint64_t>(E) * H, EI = static_cast<uint64_t>(E) * I;
   if (!make_map(&mW1, W1, I, EH, 64, 64) || !make_map(&mW3, W3, I, EH, 64, 64) ||
       !make_map(&mA2, h, I, rows_max, 64, 128) || !make_map(&mW2, W2, H, EI, 64, 64) ||
-      !make_map(&mY, y, H, rows_max, 32, 32, true))
+      !make_map(&mY, y, H, rows_max, 16, 32, true, true))
     return cudaErrorInvalidValue;
   const bool pair = (sh.pad % 256) == 0;
   // GEMM1's A rows come from x by Phi (cp.async); its A tensor map is unused

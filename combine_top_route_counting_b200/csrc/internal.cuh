@@ -60,13 +60,27 @@ cudaError_t launch_dispatch(const uint16_t* x, const int32_t* phi, const int32_t
 // launches on one stream reuse it one after another), or null: a slot of the
 // device's pool (tile_counter_for_current_device).
 
+// The pull dispatch fused into GEMM1 (steps 3a + 3b in one kernel): GEMM1's
+// spare warp lands the rows x[Phi[row]] into xg block by block while the
+// tensor cores work on blocks already landed. next (one int32) and ready
+// ([rows_max / 128] int32) are device scratch the caller zeroes before the
+// launch.
+struct LandArgs {
+  const uint16_t* x;    // token activations [P*N, H]
+  const int32_t* phi;   // [rows_max, 2]
+  int* next;
+  int* ready;
+};
+
 // Step 3b (two kernels; ev_mid, if not null, is recorded between them).
 // ab (training, pair tiles only): also keep the bf16 pre-activations [a | b].
+// land (pair tiles only): GEMM1 also performs the dispatch into xg.
 cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint16_t* W3,
                               const uint16_t* W2, const int32_t* offsets, const int32_t* counts,
                               uint16_t* h, float* y, const moe_shape_t& sh, int64_t rows_max,
                               int32_t* dev_status, cudaStream_t s, cudaEvent_t ev_mid,
-                              uint16_t* ab = nullptr, int* counter = nullptr);
+                              uint16_t* ab = nullptr, int* counter = nullptr,
+                              const LandArgs* land = nullptr);
 
 // Steps 3a+3b fused: GEMM1 pulls its A rows from x by Phi (no xg buffer)
 cudaError_t launch_expert_ffn_gather(const uint16_t* x, const int32_t* phi, const uint16_t* W1,
@@ -93,10 +107,11 @@ cudaError_t launch_dense_ffn(const uint16_t* x, int64_t n_tokens, const uint16_t
                              int32_t* dev_status, cudaStream_t s, int* counter = nullptr);
 
 // 2D tensor map over [outer, inner] (inner contiguous) bf16 (or fp32)
-// elements with box [box_outer, box_inner] and 128-byte swizzle; false if the
-// driver entry point is missing or rejects the arguments.
+// elements with box [box_outer, box_inner] and 128-byte swizzle (64-byte with
+// swizzle64); false if the driver entry point is missing or rejects the
+// arguments.
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-              uint32_t box_outer, bool fp32 = false);
+              uint32_t box_outer, bool fp32 = false, bool swizzle64 = false);
 
 // A tile counter for one launch of a persistent GEMM on the current device:
 // the next slot of a per-device pool of 256 (round robin). A slot is clean

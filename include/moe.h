@@ -98,7 +98,8 @@ int64_t moe_rows_max(const moe_shape_t* shape);
 size_t moe_schedule_workspace_bytes(const moe_shape_t* shape);
 
 /* Bytes of scratch `ws` that moe_layer_forward needs (ids, gates, Phi,
- * offsets, counts, route_row, the schedule's scratch, xg, h and y). */
+ * offsets, counts, route_row, the schedule's scratch, the GEMMs' tile counter
+ * and landing flags, xg, h and y). */
 size_t moe_layer_workspace_bytes(const moe_shape_t* shape);
 
 /* Bytes of scratch for moe_layer_forward_host: the above plus device copies
@@ -228,6 +229,13 @@ moe_status_t moe_combine(const float* y, const int32_t* route_row, const float* 
                          void* stream);
 
 /* Steps 1-4 in one call, all enqueued on `stream` with no host round trip.
+ * When pad % 256 == 0 (CTA-pair tiles) the pull dispatch runs inside the
+ * FFN's first GEMM ("Mixture-of-Kittens" notes section 2, tokens landing in
+ * the buffers the experts read; "Beyond Peak TFLOPs" section 3, one kernel
+ * overlapping data movement with the MMAs): a spare warp of every CTA copies
+ * 128-row blocks of x into the gathered buffer through Phi while the tensor
+ * cores work on blocks already landed; the result is bit for bit that of
+ * moe_dispatch + moe_expert_ffn.
  * minibatch_tokens: transfer slice T in tokens per peer (MoK notes section 3);
  * 0 or >= N = one slice. Slice s covers tokens [s*T, (s+1)*T) of every peer and
  * runs schedule -> dispatch -> FFN -> combine on them; routing runs once over

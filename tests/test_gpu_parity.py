@@ -556,6 +556,20 @@ def test_layer_bitwise_deterministic_and_slice_invariant(cuda_lib, name):
         assert sha(outT) == h0, f"transfer slice {T} changed the output"
 
 
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_layer_equals_its_stage_entries(cuda_lib, name):
+    """The layer (whose GEMM1 lands the dispatch itself when segments are padded
+    to 256 rows) gives bit for bit the output of the separate entry points:
+    moe_route_topk, moe_schedule, moe_dispatch, moe_expert_ffn, moe_combine."""
+    moe = cuda_lib
+    w, lg, x, W = _layer_inputs(name)
+    Wd = [t.to(DEV) for t in W]
+    out, _ = _layer_gpu(moe, w, lg.to(DEV), x.to(DEV), Wd)
+    r = _stage_run(moe, w, *Wd, lg.to(DEV), x.to(DEV))
+    assert int(r["dev_status"].item()) == 0
+    assert torch.equal(out, r["out"])
+
+
 @pytest.mark.parametrize("minibatch", [0, 1000, 4096, 2368])
 def test_layer_host_entry_matches_device_entry(cuda_lib, minibatch):
     """Host buffers in and out, transfers overlapped with compute slice by slice
