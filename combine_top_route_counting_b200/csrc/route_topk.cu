@@ -151,6 +151,175 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
   }
 }
 
+// Eight lanes per token, four tokens per warp (E a multiple of 4, E <= 512):
+// the same selection with a quarter of the shuffle work per token. Lane g of
+// a token's group loads float4 chunks g, g+8, g+16, ... of its logit row
+// (NV = ceil(E/32) chunks; the group's eight 16-byte loads of one step are
+// one 128-byte segment), and keeps its two largest values. tau = the k-th
+// largest of the group's 16 kept values under (value desc, position asc) --
+// at least k logits of the token are >= tau, so every chosen expert is among
+// them. The logits >= tau are compacted to shared memory and ranked exactly
+// under (value desc, id asc); more than 32 of them (heavy ties, -inf) fall
+// back to k rounds of group-wide argmax. Gates as above, summed in slot order.
+template <int NV>
+__global__ void __launch_bounds__(256, 2) route_topk_g8_kernel(const float* __restrict__ logits,
+                                                            int32_t* __restrict__ ids,
+                                                            float* __restrict__ gates,
+                                                            int64_t n_tokens, int E, int k) {
+  __shared__ float s_cv[32][kCand];
+  __shared__ int s_ci[32][kCand];
+  __shared__ float s_sv[32][kMaxK];
+  __shared__ int s_si[32][kMaxK];
+  const int lane = threadIdx.x & 31, g = lane & 7, tb = threadIdx.x >> 3;  // token in block
+  const int gbase = lane & 24;
+  const unsigned gm = 0xFFu << gbase;  // this token's eight lanes
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * 32 + tb;
+  if (t >= n_tokens) return;  // the whole group leaves together
+  const float4* row = reinterpret_cast<const float4*>(logits + t * E);
+  const int nv4 = E >> 2;
+
+  float v[NV][4];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int cidx = g + 8 * i;
+    if (cidx < nv4) {
+      const float4 q = __ldg(row + cidx);
+      v[i][0] = q.x;
+      v[i][1] = q.y;
+      v[i][2] = q.z;
+      v[i][3] = q.w;
+    } else {
+      v[i][0] = v[i][1] = v[i][2] = v[i][3] = -INFINITY;
+    }
+  }
+  // the lane's two largest values (as a multiset)
+  float m1 = -INFINITY, m2 = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < NV; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      m2 = fmaxf(m2, fminf(m1, v[i][j]));
+      m1 = fmaxf(m1, v[i][j]);
+    }
+  // tau: the value of rank k-1 among the group's 16 kept values, ordered by
+  // (value desc, position asc) with position 2h (m1) and 2h+1 (m2) of lane h
+  int ra = 0, rb = 0;
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    const float oa = __shfl_sync(gm, m1, gbase | h);
+    const float ob = __shfl_sync(gm, m2, gbase | h);
+    ra += (oa > m1 || (oa == m1 && h < g)) ? 1 : 0;
+    ra += (ob > m1 || (ob == m1 && h < g)) ? 1 : 0;  // 2h+1 < 2g  <=>  h < g
+    rb += (oa > m2 || (oa == m2 && h <= g)) ? 1 : 0;  // 2h < 2g+1 <=> h <= g
+    rb += (ob > m2 || (ob == m2 && h < g)) ? 1 : 0;
+  }
+  const unsigned own = __ballot_sync(gm, ra == k - 1 || rb == k - 1) >> gbase;
+  const float tau = __shfl_sync(gm, ra == k - 1 ? m1 : m2, gbase | (__ffs(own) - 1));
+
+  // compact the logits >= tau
+  int c = 0;
+#pragma unroll
+  for (int i = 0; i < NV; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) c += (v[i][j] >= tau && (g + 8 * i) < nv4) ? 1 : 0;
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) {
+    const int y = __shfl_up_sync(gm, incl, o, 8);
+    if (g >= o) incl += y;
+  }
+  const int total = __shfl_sync(gm, incl, gbase | 7);
+
+  if (total <= kCand) {
+    int pos = incl - c;
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (v[i][j] >= tau && (g + 8 * i) < nv4) {
+          s_cv[tb][pos] = v[i][j];
+          s_ci[tb][pos] = 4 * (g + 8 * i) + j;
+          ++pos;
+        }
+      }
+    __syncwarp(gm);
+    for (int a = g; a < total; a += 8) {
+      const float cv = s_cv[tb][a];
+      const int ci = s_ci[tb][a];
+      int rank = 0;
+      for (int b = 0; b < total; ++b) rank += better(s_cv[tb][b], s_ci[tb][b], cv, ci) ? 1 : 0;
+      if (rank < k) {
+        s_sv[tb][rank] = cv;
+        s_si[tb][rank] = ci;
+      }
+    }
+  } else {
+    // fallback: k rounds of group argmax over every logit of the token
+    uint64_t taken = 0;
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+      if (g + 8 * i >= nv4) taken |= 0xFull << (4 * i);
+    for (int r = 0; r < k; ++r) {
+      float bv = -INFINITY;
+      int bid = INT_MAX;
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int e = 4 * (g + 8 * i) + j;
+          if (!((taken >> (4 * i + j)) & 1ull) && better(v[i][j], e, bv, bid)) {
+            bv = v[i][j];
+            bid = e;
+          }
+        }
+#pragma unroll
+      for (int off = 4; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(gm, bv, off, 8);
+        const int oid = __shfl_xor_sync(gm, bid, off, 8);
+        if (better(ov, oid, bv, bid)) {
+          bv = ov;
+          bid = oid;
+        }
+      }
+      if (bid != INT_MAX && ((bid >> 2) & 7) == g) {
+        const int i = (bid >> 2) >> 3;
+        taken |= 1ull << (4 * i + (bid & 3));
+      }
+      if (g == 0) {
+        s_sv[tb][r] = bv;
+        s_si[tb][r] = bid;
+      }
+    }
+  }
+  __syncwarp(gm);
+
+  // gates: softmax over the chosen logits, summed in slot order (lane g holds
+  // slots g and g + 8)
+  const float l0 = s_sv[tb][0];
+  const float e0 = g < k ? expf(s_sv[tb][g] - l0) : 0.0f;
+  const float e1 = g + 8 < k ? expf(s_sv[tb][g + 8] - l0) : 0.0f;
+  float den = 0.0f;
+  for (int j = 0; j < k; ++j) den += __shfl_sync(gm, j < 8 ? e0 : e1, gbase | (j & 7));
+  if (g < k) {
+    ids[t * k + g] = s_si[tb][g];
+    gates[t * k + g] = e0 / den;
+  }
+  if (g + 8 < k) {
+    ids[t * k + g + 8] = s_si[tb][g + 8];
+    gates[t * k + g + 8] = e1 / den;
+  }
+}
+
+template <int NV>
+cudaError_t launch_g8(const float* logits, int32_t* ids, float* gates, int64_t n, int E, int k,
+                      cudaStream_t s) {
+  const int64_t blocks = (n + 31) / 32;
+  route_topk_g8_kernel<NV><<<static_cast<unsigned>(blocks), 256, 0, s>>>(logits, ids, gates, n, E,
+                                                                         k);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
 template <int VPL>
 cudaError_t launch_vpl(const float* logits, int32_t* ids, float* gates, int64_t n, int E, int k,
                        cudaStream_t s) {
@@ -165,6 +334,14 @@ cudaError_t launch_vpl(const float* logits, int32_t* ids, float* gates, int64_t 
 cudaError_t launch_route_topk(const float* logits, int32_t* ids, float* gates, int64_t n_tokens,
                               int32_t E, int32_t k, cudaStream_t s) {
   if (n_tokens == 0) return cudaSuccess;
+  if (E % 4 == 0 && E <= 512) {
+    if (E <= 32) return launch_g8<1>(logits, ids, gates, n_tokens, E, k, s);
+    if (E <= 64) return launch_g8<2>(logits, ids, gates, n_tokens, E, k, s);
+    if (E <= 128) return launch_g8<4>(logits, ids, gates, n_tokens, E, k, s);
+    if (E <= 256) return launch_g8<8>(logits, ids, gates, n_tokens, E, k, s);
+    if (E <= 384) return launch_g8<12>(logits, ids, gates, n_tokens, E, k, s);
+    return launch_g8<16>(logits, ids, gates, n_tokens, E, k, s);
+  }
   if (E <= 32) return launch_vpl<1>(logits, ids, gates, n_tokens, E, k, s);
   if (E <= 64) return launch_vpl<2>(logits, ids, gates, n_tokens, E, k, s);
   if (E <= 128) return launch_vpl<4>(logits, ids, gates, n_tokens, E, k, s);
