@@ -98,10 +98,23 @@ def mx_layer_work(w, rows_used: int):
     return work
 
 
-def stage_rooflines(stage_ms: dict, work: dict, peaks: dict) -> dict:
+def dispatch_fused(w) -> bool:
+    """Whether the layer runs the pull dispatch inside GEMM1 (the library does
+    so when expert segments are padded to multiples of 256 rows)."""
+    return w.pad % 256 == 0
+
+
+def stage_rooflines(stage_ms: dict, work: dict, peaks: dict, fused_dispatch: bool = False) -> dict:
     out = {}
     for name, t in stage_ms.items():
         d = {"ms": t}
+        if fused_dispatch and name == "dispatch":
+            # only the zeroing of the landing flags is left between the events
+            d.update(bytes=work[name]["bytes"], fused_into="ffn_gemm1")
+            out[name] = d
+            continue
+        if fused_dispatch and name == "ffn_gemm1":
+            d["includes"] = "the pull dispatch (its gather runs on a spare warp inside the kernel)"
         if "bytes" in work[name]:
             gbs = work[name]["bytes"] / (t / 1e3) / 1e9
             d.update(bytes=work[name]["bytes"], gbs=gbs, frac_hbm=gbs / peaks["hbm"])
@@ -115,6 +128,116 @@ def stage_rooflines(stage_ms: dict, work: dict, peaks: dict) -> dict:
             d.update(flops=work[name]["flops"], tflops=tf, frac_bf16=tf / peaks["bf16_sus"],
                      frac_bf16_burst=tf / peaks["bf16"])
         out[name] = d
+    return out
+
+
+# ---------------------------------------------------------------- the other workloads
+def _flush_l2(buf):
+    """Write a buffer larger than L2 (126 MB) so the next launch starts cold."""
+    buf.fill_(1)
+
+
+def time_configs(moe, dev, W_kimi, x_kimi, ws_big, st, steps: int, warmup: int, peaks: dict):
+    """The other workloads, timed in the same run on the same device:
+    sched: Phi build (ids -> Phi) on the scheduler workload, CUDA events around
+    each call, L2 flushed before each; zipf: the adversarial layer on the Kimi
+    shape (the Kimi weights and activations, Zipf routing), stage rooflines;
+    mid: the mid layer, stage rooflines; tiny: one layer call's latency. mid and
+    tiny fit in L2, so each timed call follows an L2 flush and is timed alone."""
+    import torch
+
+    from combine_top_route_counting_b200 import inputs
+    out = {}
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn, n, per_call_events=None):
+        """Per-call device times (ms) of n calls, each after an L2 flush."""
+        ts = []
+        for i in range(n):
+            _flush_l2(flush)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn(per_call_events[i] if per_call_events else None)
+            e1.record()
+            ts.append((e0, e1))
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in ts]
+
+    # Phi build on the scheduler workload: P=8 x 7,168 tokens, E=384, top-8 ids
+    w = inputs.WORKLOADS["sched"]
+    sh = moe.shape(**w.shape())
+    ids = inputs.make_sched_ids(w).to(dev)
+    b = moe.alloc_schedule_outputs(sh, device=dev)
+    sched = lambda _ev: moe.moe_schedule(ids, b["phi"], b["offsets"], b["counts"], b["route_row"],
+                                          b["ws"], b["dev_status"], sh)
+    for _ in range(warmup):
+        sched(None)
+    n = max(steps, 20)
+    t = timed(sched, n)
+    torch.cuda.synchronize()
+    if int(b["dev_status"].item()) != 0:
+        raise RuntimeError("device status in the scheduler workload")
+    out["sched"] = {"workload": workload_desc(w), "phi_build_us_median": 1e3 * statistics.median(t),
+                    "phi_build_us_min": 1e3 * min(t), "calls": n,
+                    "what": "moe_schedule: count, scan, offsets, scatter (4 kernels) on "
+                            "uniform ids; L2 flushed before each call"}
+    del b, ids
+
+    def layer_leg(name, W, x, ws, n_calls, flush_each):
+        w = inputs.WORKLOADS[name]
+        sh = moe.shape(**w.shape())
+        lg = inputs.make_logits(w).to(dev)
+        o = torch.empty((w.n_tokens, w.H), dtype=torch.bfloat16, device=dev)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.N_STAGE_EVENTS)]
+              for _ in range(n_calls)]
+        for row in ev:
+            for e in row:
+                e.record()  # creates the event (torch creates events lazily)
+        call = lambda e: moe.moe_layer_forward(lg, x, *W, o, ws, st, sh, stage_events=e)
+        for _ in range(warmup):
+            call(None)
+        torch.cuda.synchronize()
+        if flush_each:
+            t = timed(call, n_calls, ev)
+            ms = statistics.median(t)
+        else:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for i in range(n_calls):
+                call(ev[i])
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / n_calls
+        if int(st.item()) != 0:
+            raise RuntimeError(f"device status in the {name} layer")
+        stage_ms = {nm: statistics.median(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(n_calls))
+                    for j, nm in enumerate(moe.STAGES)}
+        rows = schedule_rows(moe, w, sh, lg)
+        d = {"workload": workload_desc(w), "value": w.n_tokens / (ms / 1e3), "unit": "tokens/s",
+             "ms_per_step": ms, "phi_build_us": 1e3 * stage_ms["schedule"], "rows_padded": rows,
+             "stages": stage_rooflines(stage_ms, algorithmic_work(w, rows, w.n_routes), peaks,
+                                       dispatch_fused(w))}
+        return d
+
+    # the adversarial layer: Kimi shapes with Zipf routing (hot and empty experts)
+    z = layer_leg("zipf", W_kimi, x_kimi, ws_big, steps, False)
+    z["note"] = ("the Kimi workload's weights and activations with Zipf(1.2) routing and 8 "
+                 "experts never chosen; inputs larger than L2")
+    out["zipf"] = z
+    for name in ("mid", "tiny"):
+        w = inputs.WORKLOADS[name]
+        sh = moe.shape(**w.shape())
+        W = inputs.make_weights(w, device=dev)
+        x = inputs.make_x(w, device=dev)
+        ws = torch.empty(moe.layer_workspace_bytes(sh), dtype=torch.uint8, device=dev)
+        d = layer_leg(name, W, x, ws, max(steps, 20), True)
+        d["note"] = "median of single calls, each after an L2 flush (the workload fits in L2)"
+        if name == "tiny":
+            d["latency_us"] = d["ms_per_step"] * 1e3
+        out[name] = d
+        del W, x, ws
+    del flush
+    torch.cuda.empty_cache()
     return out
 
 
@@ -205,25 +328,27 @@ def init_dist(world: int, local_rank: int, backend: str = "nccl"):
 
 
 # ---------------------------------------------------------------- CPU oracle sample
-def oracle_sample(w, lg, x_cpu, W_dev, row_budget_s: float, n_comb: int = 256,
+def oracle_sample(w, lg, x_cpu, W_dev, n_experts: int, n_comb: int = 256,
                   threads: int | None = None):
     """Time the CPU oracle on a bounded sample of the workload and scale it to
-    tokens/s: route + schedule over the whole batch, dispatch + FFN of R rows
-    of one expert (R grown until the budget), combine of n_comb tokens.
+    tokens/s: route + schedule over the whole batch; dispatch + FFN of every
+    row of n_experts experts, taken at evenly spaced ranks of the expert
+    sizes; combine of n_comb tokens. tokens/s = 1 / (t_route_schedule / tokens
+    + k * t_row + t_combine_per_token), each term measured.
     threads: run the oracle on that many host threads (default: all cores)."""
     import oracle
 
     all_cores = oracle.num_threads()
     if threads is None:
-        return _oracle_sample(oracle, w, lg, x_cpu, W_dev, row_budget_s, n_comb, all_cores)
+        return _oracle_sample(oracle, w, lg, x_cpu, W_dev, n_experts, n_comb, all_cores)
     oracle.set_num_threads(threads)
     try:
-        return _oracle_sample(oracle, w, lg, x_cpu, W_dev, row_budget_s, n_comb, threads)
+        return _oracle_sample(oracle, w, lg, x_cpu, W_dev, n_experts, n_comb, threads)
     finally:
         oracle.set_num_threads(all_cores)
 
 
-def _oracle_sample(oracle, w, lg, x_cpu, W_dev, row_budget_s, n_comb, cores):
+def _oracle_sample(oracle, w, lg, x_cpu, W_dev, n_experts, n_comb, cores):
     import numpy as np
     import torch
 
@@ -232,21 +357,19 @@ def _oracle_sample(oracle, w, lg, x_cpu, W_dev, row_budget_s, n_comb, cores):
     s = oracle.schedule(ids.reshape(w.P, w.N, w.k), w.P, w.N, w.k, w.E, w.pad)
     t_rs = time.perf_counter() - t0
     counts = s["counts"].sum(1)
-    e = int(np.argmax(counts))
-    seg = np.arange(s["offsets"][e], s["offsets"][e] + counts[e])
+    order = np.argsort(-counts, kind="stable")
+    used = order[counts[order] > 0]
+    n_experts = min(n_experts, len(used))
+    pick = used[np.linspace(0, len(used) - 1, n_experts).round().astype(int)]
+    rows = np.concatenate([np.arange(s["offsets"][e], s["offsets"][e] + counts[e]) for e in pick])
+    ex = oracle.expert_of_rows(s["offsets"], rows)
     to_bits = lambda t: t.contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
-    Wh = tuple({e: to_bits(W[e])} for W in W_dev)
+    Wh = tuple({int(e): to_bits(W[int(e)]) for e in pick} for W in W_dev)
     xb = to_bits(x_cpu)
-    R, t_ffn = 2, 0.0
-    while True:
-        rows = seg[:R]
-        t1 = time.perf_counter()
-        xg = oracle.dispatch_rows(xb, w.N, s["phi"], rows)
-        _, y = oracle.ffn_rows(xg, np.full(len(rows), e, np.int32), *Wh, H=w.H, I=w.I)
-        t_ffn = time.perf_counter() - t1
-        if t_ffn > row_budget_s / 3 or R >= len(seg):
-            break
-        R = min(len(seg), R * 3)
+    t1 = time.perf_counter()
+    xg = oracle.dispatch_rows(xb, w.N, s["phi"], rows)
+    _, y = oracle.ffn_rows(xg, ex, *Wh, H=w.H, I=w.I)
+    t_ffn = time.perf_counter() - t1
     t_row = t_ffn / len(rows)
     n_comb = min(n_comb, w.n_tokens)
     sel = np.random.default_rng(0).integers(0, len(rows), size=(n_comb, w.k))
@@ -254,9 +377,10 @@ def _oracle_sample(oracle, w, lg, x_cpu, W_dev, row_budget_s, n_comb, cores):
     oracle.combine_f64(y, sel, g64[:n_comb], w.k)
     t_comb = (time.perf_counter() - t2) / n_comb
     per_token = t_rs / w.n_tokens + w.k * t_row + t_comb
-    sample = (f"route+schedule over all {w.n_tokens} tokens ({t_rs:.2f} s); dispatch+FFN of "
-              f"{len(rows)} rows of expert {e} ({t_ffn:.2f} s); combine of {n_comb} tokens; "
-              f"tokens/s = 1/(t_route_sched/{w.n_tokens} + {w.k}*t_row + t_combine)")
+    sample = (f"route+schedule over all {w.n_tokens} tokens ({t_rs:.2f} s); dispatch+FFN of all "
+              f"{len(rows)} rows of {n_experts} experts at evenly spaced size ranks ({t_ffn:.2f} s); "
+              f"combine of {n_comb} tokens; tokens/s = 1/(t_route_sched/{w.n_tokens} + "
+              f"{w.k}*t_row + t_combine), extrapolated from the sample")
     return dict(value=1.0 / per_token, cores=cores, sample=sample,
                 seconds=t_rs + t_ffn + t_comb * n_comb)
 
@@ -276,19 +400,24 @@ def run_reference(args):
     vals, secs = [], []
     last = None
     for i in range(args.warmup + args.steps):
-        r = oracle_sample(w, lg, x, W, row_budget_s=args.ref_row_budget, n_comb=64)
+        r = oracle_sample(w, lg, x, W, n_experts=1, n_comb=64)
         if i >= args.warmup:
             vals.append(r["value"])
             secs.append(r["seconds"])
         last = r
     value = statistics.median(vals)
+    step_s = statistics.median(secs)
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1000.0 * w.n_tokens / value, "higher_is_better": True,
+        "ms_per_step": 1000.0 * step_s, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_desc(w), "note": "CPU oracle (plain C++/OpenMP, fp64) "
-                   "on a bounded per-step sample scaled to tokens/s"},
+        "config": {"workload": workload_desc(w),
+                   "note": "CPU oracle (plain C++/OpenMP, fp64). Each step is a bounded sample "
+                           "of the workload (route + schedule of every token, dispatch + FFN of "
+                           "one expert's rows, combine of 64 tokens); ms_per_step is the "
+                           "sample's measured time and value the throughput it extrapolates to",
+                   "tokens_per_step_equivalent": value * step_s},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": last["cores"],
                          "kind": "oracle", "sample": last["sample"]},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -307,7 +436,7 @@ def assemble_line(args, w, world, ms, stage_ms, launches, e2e, e2e_mb, mb, mb_ro
     tokens = w.n_tokens * world * args.steps
     value = tokens / (ms / 1e3)
     work = algorithmic_work(w, rows_used, w.n_routes)
-    stages = stage_rooflines(stage_ms, work, peaks)
+    stages = stage_rooflines(stage_ms, work, peaks, dispatch_fused(w))
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
@@ -325,10 +454,12 @@ def assemble_line(args, w, world, ms, stage_ms, launches, e2e, e2e_mb, mb, mb_ro
         g1 = stages["ffn_gemm1"]
         line["roofline"] = {
             "kernel": "ffn_gemm_kernel<0> (GEMM1 + SwiGLU)", "bound": "tensor",
-            "achieved": g1["tflops"], "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
-            "frac": g1["tflops"] / peaks["bf16_sus"],
-            "peak_note": f"dense bf16, sustained, of {peaks['source']}",
-            "peak_burst": peaks["bf16"], "frac_burst": g1["tflops"] / peaks["bf16"],
+            "achieved": g1["tflops"], "peak": peaks["bf16"], "unit": "TFLOP/s",
+            "frac": g1["tflops"] / peaks["bf16"],
+            "peak_note": f"dense bf16, burst, of {peaks['source']} (the conservative figure; "
+                         "the kernel runs inside a ~1 s loop under the power cap, where the "
+                         "sustained figure also applies)",
+            "peak_sustained": peaks["bf16_sus"], "frac_sustained": g1["tflops"] / peaks["bf16_sus"],
             "traffic": gemm1_traffic(w.n_routes),
         }
         line["stages"] = stages
@@ -500,6 +631,9 @@ def run_ours(args):
             Wq += [q, sc]
         evm = [[torch.cuda.Event(enable_timing=True) for _ in range(moe.N_STAGE_EVENTS)]
                for _ in range(args.steps)]
+        for row in evm:
+            for e in row:
+                e.record()  # creates the event
         for _ in range(args.warmup):
             moe.moe_layer_forward_mxfp8(lg, x, *Wq, out, ws, st, sh)
         torch.cuda.synchronize()
@@ -516,6 +650,12 @@ def run_ours(args):
                                                    for i in range(args.steps))
                              for s_i, name in enumerate(moe.STAGES)})
         del Wq
+
+    # the other workloads (Phi on the scheduler workload, the Zipf, mid and
+    # tiny layers), same device, same run
+    cfgs = None
+    if not args.no_configs and mb == 0 and w.name == "kimi":
+        cfgs = time_configs(moe, dev, W, x, ws, st, args.steps, args.warmup, load_peaks())
 
     # end to end through the host-buffer entry: H2D of logits and x, the layer,
     # D2H of out; each call's input copy overlaps the previous call's compute
@@ -634,12 +774,15 @@ def run_ours(args):
         line = assemble_line(args, w, world, ms, stage_ms, launches, e2e, e2e_mb, mb, mb_row, mx,
                              bwd, rows_used, peaks, mxl=mxl)
         line["clocks"] = clk
+        if cfgs:
+            line["configs"] = cfgs
         if world == 1 and not args.no_cpu_baseline:
-            r = oracle_sample(w, lg_cpu, x_cpu, W, row_budget_s=args.cpu_budget)
+            r = oracle_sample(w, lg_cpu, x_cpu, W, n_experts=args.cpu_experts)
             line["cpu_baseline"] = {"value": r["value"], "unit": "tokens/s", "cores": r["cores"],
-                                    "kind": "oracle", "sample": r["sample"]}
+                                    "kind": "oracle", "sample": r["sample"],
+                                    "seconds": r["seconds"]}
             if w.name in ("tiny", "mid"):  # the small configs also on one host core
-                r1 = oracle_sample(w, lg_cpu, x_cpu, W, row_budget_s=args.cpu_budget, threads=1)
+                r1 = oracle_sample(w, lg_cpu, x_cpu, W, n_experts=args.cpu_experts, threads=1)
                 line["cpu_baseline"]["one_core"] = {"value": r1["value"], "unit": "tokens/s",
                                                     "cores": 1, "sample": r1["sample"]}
         print(json.dumps(line), flush=True)
@@ -726,11 +869,13 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-mxfp8", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads (scheduler, zipf, mid, tiny)")
     ap.add_argument("--mxfp8-layer", action="store_true",
                     help="also time moe_layer_forward_mxfp8 (block-scaled expert GEMMs)")
     ap.add_argument("--bwd-steps", type=int, default=10)
-    ap.add_argument("--cpu-budget", type=float, default=20.0)
-    ap.add_argument("--ref-row-budget", type=float, default=3.0)
+    ap.add_argument("--cpu-experts", type=int, default=8,
+                    help="experts whose rows the CPU baseline runs through the oracle's FFN")
     args = ap.parse_args(argv)
     if args.e2e_steps <= 0:
         args.e2e_steps = args.steps
