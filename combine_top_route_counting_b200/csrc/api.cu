@@ -81,7 +81,7 @@ moe_status_t check_mx_shape(const moe_shape_t* s) {
 // backward's buffers; dxg [rows, H] fp32 reuses y, which is dead once the
 // forward's combine has run.
 struct LayerWs {
-  size_t ids, gates, route_row, phi, offsets, counts, sched, ctr, land, xg, h, y, total;
+  size_t ids, gates, route_row, phi, offsets, counts, sched, ctr, xg, h, y, total;
   size_t logits[2], x[2], out[2], total_host;  // moe_layer_forward_host additions
   size_t ab, dys, dab, hg, gate_row, part, total_train;  // training additions
   size_t sh_off, sh_x, sh_h, sh_y, total_mx;  // the MXFP8 layer's shared expert
@@ -105,8 +105,9 @@ LayerWs layer_ws(const moe_shape_t* s) {
   w.offsets = take(o, (s->E + 1) * 4);
   w.counts = take(o, static_cast<size_t>(s->E) * s->P * 4);
   w.sched = take(o, schedule_ws_bytes(s->P, s->N, s->k, s->E));
-  w.ctr = take(o, 8);  // the GEMMs' tile counter, zeroed at the start of each call
-  w.land = take(o, (16 + rows / 128) * 4);  // fused dispatch: next block, then ready flags
+  // the GEMMs' tile counter (words 0-1), the fused dispatch's next block
+  // (word 16) and ready flags (words 32..), zeroed at the start of each call
+  w.ctr = take(o, (32 + rows / 128) * 4);
   w.xg = take(o, rows * s->H * 2);
   w.h = take(o, rows * s->I * 2);
   w.y = take(o, rows * s->H * 4);
@@ -177,19 +178,29 @@ LayerBufs layer_bufs(void* ws, const LayerWs& w) {
   b.counts = at<int32_t>(ws, w.counts);
   b.sched = at<int32_t>(ws, w.sched);
   b.ctr = at<int>(ws, w.ctr);
-  b.land = at<int>(ws, w.land);
+  b.land = b.ctr + 16;
   b.xg = at<uint16_t>(ws, w.xg);
   b.h = at<uint16_t>(ws, w.h);
   b.y = at<float>(ws, w.y);
   return b;
 }
 
+// The scratch words a layer call's kernels expect at zero when it starts: the
+// tile counter and landing words, and the schedule's barrier. The routing
+// kernel zeroes them (first slice); later slices zero what they reuse.
+ZeroSpec call_zeroes(const LayerBufs& b, const moe_shape_t* sh) {
+  return ZeroSpec{b.ctr, static_cast<int32_t>(32 + rows_max_of(sh) / 128),
+                  schedule_barrier_word(b.sched, *sh), 1};
+}
+
 // Schedule -> dispatch -> FFN -> combine for one token slice (steps 2-4).
 // ev (7 events, may be null) marks the stage boundaries 1..6.
 // ab (training, whole batch only): GEMM1 also keeps the pre-activations.
+// first: the call's first slice, whose scratch words the routing kernel
+// zeroed (later slices zero the landing words and the barrier themselves).
 cudaError_t run_slice(const LayerBufs& b, const uint16_t* x, const uint16_t* W1, const uint16_t* W3,
                       const uint16_t* W2, uint16_t* out, Slice sl, const moe_shape_t* sh,
-                      int32_t* dev_status, cudaStream_t s, void* const* ev,
+                      int32_t* dev_status, cudaStream_t s, void* const* ev, bool first,
                       uint16_t* ab = nullptr) {
   const int64_t rows_max = rows_max_of(sh);
   auto rec = [&](int i) -> cudaError_t {
@@ -198,7 +209,7 @@ cudaError_t run_slice(const LayerBufs& b, const uint16_t* x, const uint16_t* W1,
   cudaError_t e;
   if ((e = rec(1)) != cudaSuccess) return e;
   if ((e = launch_schedule(b.ids, *sh, sl, b.phi, b.offsets, b.counts, b.route_row, b.sched,
-                           dev_status, s)) != cudaSuccess)
+                           dev_status, s, first)) != cudaSuccess)
     return e;
   // With CTA-pair tiles (segments padded to 256 rows) the pull dispatch runs
   // inside GEMM1: its spare warp lands the rows into xg block by block while
@@ -209,7 +220,8 @@ cudaError_t run_slice(const LayerBufs& b, const uint16_t* x, const uint16_t* W1,
   const bool fused = sh->pad % 256 == 0;
   const LandArgs land{x, b.phi, b.land, b.land + 16};
   if (fused) {
-    if ((e = cudaMemsetAsync(b.land, 0, (16 + rows_max / 128) * sizeof(int), s)) != cudaSuccess)
+    if (!first &&
+        (e = cudaMemsetAsync(b.land, 0, (16 + rows_max / 128) * sizeof(int), s)) != cudaSuccess)
       return e;
   } else if ((e = launch_dispatch(x, b.phi, b.offsets, b.xg, *sh, rows_max, dev_status, s)) !=
              cudaSuccess) {
@@ -243,9 +255,10 @@ moe_status_t layer_body(const float* logits, const uint16_t* x, const uint16_t* 
   void* const* ev_use = (T == N) ? ev : nullptr;  // stage events: single-slice runs only
   cudaError_t e = (ev_use && ev_use[0]) ? cudaEventRecord(static_cast<cudaEvent_t>(ev_use[0]), s)
                                         : cudaSuccess;
-  if (e == cudaSuccess) e = cudaMemsetAsync(b.ctr, 0, 8, s);
+  const ZeroSpec z = call_zeroes(b, sh);
   if (e == cudaSuccess)
-    e = launch_route_topk(logits, b.ids, b.gates, static_cast<int64_t>(sh->P) * N, sh->E, sh->k, s);
+    e = launch_route_topk(logits, b.ids, b.gates, static_cast<int64_t>(sh->P) * N, sh->E, sh->k, s,
+                          &z);
   if (e != cudaSuccess) return from_cuda(e);
   if (N == 0) {
     for (int i = 1; i < 7 && ev_use; ++i)
@@ -254,7 +267,7 @@ moe_status_t layer_body(const float* logits, const uint16_t* x, const uint16_t* 
   }
   for (int32_t t0 = 0; t0 < N && e == cudaSuccess; t0 += T) {
     const Slice sl{t0, (N - t0) < T ? (N - t0) : T};
-    e = run_slice(b, x, W1, W3, W2, out, sl, sh, dev_status, s, ev_use, ab);
+    e = run_slice(b, x, W1, W3, W2, out, sl, sh, dev_status, s, ev_use, t0 == 0, ab);
   }
   return from_cuda(e);
 }
@@ -281,9 +294,9 @@ cudaError_t layer_body_mx(const float* logits, const uint16_t* x, const uint8_t*
   };
   cudaError_t e;
   if ((e = rec(0)) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(b.ctr, 0, 8, s)) != cudaSuccess) return e;
+  const ZeroSpec z = call_zeroes(b, sh);
   if ((e = launch_route_topk(logits, b.ids, b.gates, static_cast<int64_t>(sh->P) * sh->N, sh->E,
-                             sh->k, s)) != cudaSuccess)
+                             sh->k, s, &z)) != cudaSuccess)
     return e;
   if (sh->N == 0) {
     for (int i = 1; i < 7; ++i)
@@ -292,7 +305,7 @@ cudaError_t layer_body_mx(const float* logits, const uint16_t* x, const uint8_t*
   }
   if ((e = rec(1)) != cudaSuccess) return e;
   if ((e = launch_schedule(b.ids, *sh, Slice{0, sh->N}, b.phi, b.offsets, b.counts, b.route_row,
-                           b.sched, dev_status, s)) != cudaSuccess)
+                           b.sched, dev_status, s, /*barrier_zeroed=*/true)) != cudaSuccess)
     return e;
   if ((e = rec(2)) != cudaSuccess) return e;
   if ((e = launch_dispatch_mxfp8(x, b.phi, b.offsets, xq, xs, *sh, rows_max, dev_status, s,
@@ -478,8 +491,9 @@ cudaError_t layer_host_pipeline(const float* logits_host, const uint16_t* x_host
   if ((e = cudaStreamWaitEvent(s, cr->lg, 0)) != cudaSuccess) return e;
   // the device output copy of parity b has been copied out by call i-2
   if ((e = cudaStreamWaitEvent(s, cr->out_free[b], 0)) != cudaSuccess) return e;
+  const ZeroSpec z = call_zeroes(bufs, sh);
   if ((e = launch_route_topk(logits, bufs.ids, bufs.gates, static_cast<int64_t>(tokens), sh->E,
-                             sh->k, s)) != cudaSuccess)
+                             sh->k, s, &z)) != cudaSuccess)
     return e;
   for (int32_t i = 0; i < S; ++i) {
     const int32_t t0 = i * T, tm = (N - t0) < T ? (N - t0) : T;
@@ -490,8 +504,8 @@ cudaError_t layer_host_pipeline(const float* logits_host, const uint16_t* x_host
       if ((e = cudaEventRecord(cr->ex[(i + 1) % kRing], cr->h2d)) != cudaSuccess) return e;
     }
     if ((e = cudaStreamWaitEvent(s, cr->ex[i % kRing], 0)) != cudaSuccess) return e;
-    if ((e = run_slice(bufs, x, W1, W3, W2, out, Slice{t0, tm}, sh, dev_status, s, nullptr)) !=
-        cudaSuccess)
+    if ((e = run_slice(bufs, x, W1, W3, W2, out, Slice{t0, tm}, sh, dev_status, s, nullptr,
+                       i == 0)) != cudaSuccess)
       return e;
     if ((e = cudaEventRecord(cr->ed[i % kRing], s)) != cudaSuccess) return e;
     if ((e = cudaStreamWaitEvent(cr->d2h, cr->ed[i % kRing], 0)) != cudaSuccess) return e;

@@ -28,16 +28,32 @@ struct Slice {
   int32_t t0, Tm;
 };
 
-// Step 1
+// Words of device scratch that a call's later kernels expect to find zero
+// (the GEMMs' tile counter and landing flags, the schedule's grid barrier):
+// the routing kernel, the first kernel of a layer call, zeroes them in its
+// first block, so the layer needs no memset of its own.
+struct ZeroSpec {
+  int* a;
+  int32_t na;
+  int* b;
+  int32_t nb;
+};
+
+// Step 1 (z, if not null: words to zero, as above)
 cudaError_t launch_route_topk(const float* logits, int32_t* ids, float* gates, int64_t n_tokens,
-                              int32_t E, int32_t k, cudaStream_t s);
+                              int32_t E, int32_t k, cudaStream_t s, const ZeroSpec* z = nullptr);
 
 // Step 2
 constexpr int kSchedBlockRoutes = 2048;  // routes per counting block (8 warps x 256)
 size_t schedule_ws_bytes(int32_t P, int32_t N, int32_t k, int32_t E);
+// barrier_zeroed: the grid-barrier word in ws (schedule_barrier_word) is
+// already zero (else the launch zeroes it first).
 cudaError_t launch_schedule(const int32_t* ids, const moe_shape_t& sh, Slice sl, int32_t* phi,
                             int32_t* offsets, int32_t* counts, int32_t* route_row, int32_t* ws,
-                            int32_t* dev_status, cudaStream_t s);
+                            int32_t* dev_status, cudaStream_t s, bool barrier_zeroed = false);
+// The word of the schedule's scratch that its one-launch kernel's grid
+// barrier counts on (after the [P][blocks][E] counters of the whole batch).
+int32_t* schedule_barrier_word(int32_t* ws, const moe_shape_t& sh);
 
 // The schedule's one-launch kernel with a grid barrier that waits for one
 // block more than the launch has: every block gives up after timeout_ns and

@@ -35,11 +35,20 @@ __device__ __forceinline__ bool better(float v, int id, float bv, int bid) {
   return v > bv || (v == bv && id < bid);
 }
 
+// Block 0 zeroes the scratch words the call's later kernels expect at zero.
+__device__ __forceinline__ void zero_words(const ZeroSpec& z) {
+  if (blockIdx.x != 0) return;
+  for (int i = threadIdx.x; i < z.na; i += blockDim.x) z.a[i] = 0;
+  for (int i = threadIdx.x; i < z.nb; i += blockDim.x) z.b[i] = 0;
+}
+
 template <int VPL>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits,
                                                          int32_t* __restrict__ ids,
                                                          float* __restrict__ gates,
-                                                         int64_t n_tokens, int E, int k) {
+                                                         int64_t n_tokens, int E, int k,
+                                                         ZeroSpec z) {
+  zero_words(z);
   __shared__ float s_cv[8][kCand];
   __shared__ int s_ci[8][kCand];
   __shared__ float s_sv[8][kMaxK];
@@ -165,7 +174,9 @@ template <int NV>
 __global__ void __launch_bounds__(256, 2) route_topk_g8_kernel(const float* __restrict__ logits,
                                                             int32_t* __restrict__ ids,
                                                             float* __restrict__ gates,
-                                                            int64_t n_tokens, int E, int k) {
+                                                            int64_t n_tokens, int E, int k,
+                                                            ZeroSpec z) {
+  zero_words(z);
   __shared__ float s_cv[32][kCand];
   __shared__ int s_ci[32][kCand];
   __shared__ float s_sv[32][kMaxK];
@@ -233,15 +244,19 @@ __global__ void __launch_bounds__(256, 2) route_topk_g8_kernel(const float* __re
   if (total <= kCand) {
     int pos = incl - c;
 #pragma unroll
-    for (int i = 0; i < NV; ++i)
+    for (int i = 0; i < NV; ++i) {
+      // most chunks hold no candidate: one test skips them
+      if (fmaxf(fmaxf(v[i][0], v[i][1]), fmaxf(v[i][2], v[i][3])) < tau || (g + 8 * i) >= nv4)
+        continue;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        if (v[i][j] >= tau && (g + 8 * i) < nv4) {
+        if (v[i][j] >= tau) {
           s_cv[tb][pos] = v[i][j];
           s_ci[tb][pos] = 4 * (g + 8 * i) + j;
           ++pos;
         }
       }
+    }
     __syncwarp(gm);
     for (int a = g; a < total; a += 8) {
       const float cv = s_cv[tb][a];
@@ -312,19 +327,20 @@ __global__ void __launch_bounds__(256, 2) route_topk_g8_kernel(const float* __re
 
 template <int NV>
 cudaError_t launch_g8(const float* logits, int32_t* ids, float* gates, int64_t n, int E, int k,
-                      cudaStream_t s) {
+                      cudaStream_t s, ZeroSpec z) {
   const int64_t blocks = (n + 31) / 32;
   route_topk_g8_kernel<NV><<<static_cast<unsigned>(blocks), 256, 0, s>>>(logits, ids, gates, n, E,
-                                                                         k);
+                                                                         k, z);
   note_launches(1);
   return cudaGetLastError();
 }
 
 template <int VPL>
 cudaError_t launch_vpl(const float* logits, int32_t* ids, float* gates, int64_t n, int E, int k,
-                       cudaStream_t s) {
+                       cudaStream_t s, ZeroSpec z) {
   const int64_t blocks = (n + 7) / 8;
-  route_topk_kernel<VPL><<<static_cast<unsigned>(blocks), 256, 0, s>>>(logits, ids, gates, n, E, k);
+  route_topk_kernel<VPL><<<static_cast<unsigned>(blocks), 256, 0, s>>>(logits, ids, gates, n, E, k,
+                                                                       z);
   note_launches(1);
   return cudaGetLastError();
 }
@@ -332,23 +348,30 @@ cudaError_t launch_vpl(const float* logits, int32_t* ids, float* gates, int64_t 
 }  // namespace
 
 cudaError_t launch_route_topk(const float* logits, int32_t* ids, float* gates, int64_t n_tokens,
-                              int32_t E, int32_t k, cudaStream_t s) {
-  if (n_tokens == 0) return cudaSuccess;
-  if (E % 4 == 0 && E <= 512) {
-    if (E <= 32) return launch_g8<1>(logits, ids, gates, n_tokens, E, k, s);
-    if (E <= 64) return launch_g8<2>(logits, ids, gates, n_tokens, E, k, s);
-    if (E <= 128) return launch_g8<4>(logits, ids, gates, n_tokens, E, k, s);
-    if (E <= 256) return launch_g8<8>(logits, ids, gates, n_tokens, E, k, s);
-    if (E <= 384) return launch_g8<12>(logits, ids, gates, n_tokens, E, k, s);
-    return launch_g8<16>(logits, ids, gates, n_tokens, E, k, s);
+                              int32_t E, int32_t k, cudaStream_t s, const ZeroSpec* zp) {
+  const ZeroSpec z = zp ? *zp : ZeroSpec{nullptr, 0, nullptr, 0};
+  if (n_tokens == 0) {
+    if (z.na > 0 && cudaMemsetAsync(z.a, 0, z.na * sizeof(int), s) != cudaSuccess)
+      return cudaGetLastError();
+    if (z.nb > 0 && cudaMemsetAsync(z.b, 0, z.nb * sizeof(int), s) != cudaSuccess)
+      return cudaGetLastError();
+    return cudaSuccess;
   }
-  if (E <= 32) return launch_vpl<1>(logits, ids, gates, n_tokens, E, k, s);
-  if (E <= 64) return launch_vpl<2>(logits, ids, gates, n_tokens, E, k, s);
-  if (E <= 128) return launch_vpl<4>(logits, ids, gates, n_tokens, E, k, s);
-  if (E <= 256) return launch_vpl<8>(logits, ids, gates, n_tokens, E, k, s);
-  if (E <= 384) return launch_vpl<12>(logits, ids, gates, n_tokens, E, k, s);
-  if (E <= 512) return launch_vpl<16>(logits, ids, gates, n_tokens, E, k, s);
-  return launch_vpl<32>(logits, ids, gates, n_tokens, E, k, s);
+  if (E % 4 == 0 && E <= 512) {
+    if (E <= 32) return launch_g8<1>(logits, ids, gates, n_tokens, E, k, s, z);
+    if (E <= 64) return launch_g8<2>(logits, ids, gates, n_tokens, E, k, s, z);
+    if (E <= 128) return launch_g8<4>(logits, ids, gates, n_tokens, E, k, s, z);
+    if (E <= 256) return launch_g8<8>(logits, ids, gates, n_tokens, E, k, s, z);
+    if (E <= 384) return launch_g8<12>(logits, ids, gates, n_tokens, E, k, s, z);
+    return launch_g8<16>(logits, ids, gates, n_tokens, E, k, s, z);
+  }
+  if (E <= 32) return launch_vpl<1>(logits, ids, gates, n_tokens, E, k, s, z);
+  if (E <= 64) return launch_vpl<2>(logits, ids, gates, n_tokens, E, k, s, z);
+  if (E <= 128) return launch_vpl<4>(logits, ids, gates, n_tokens, E, k, s, z);
+  if (E <= 256) return launch_vpl<8>(logits, ids, gates, n_tokens, E, k, s, z);
+  if (E <= 384) return launch_vpl<12>(logits, ids, gates, n_tokens, E, k, s, z);
+  if (E <= 512) return launch_vpl<16>(logits, ids, gates, n_tokens, E, k, s, z);
+  return launch_vpl<32>(logits, ids, gates, n_tokens, E, k, s, z);
 }
 
 // ---------------------------------------------------------------- backward

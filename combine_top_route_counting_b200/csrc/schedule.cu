@@ -320,8 +320,8 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
   const SchedParams& p = f.sp;
   extern __shared__ int32_t smem[];
   int32_t* wbase = smem;                 // [kWarps][E] warp counts, then warp bases
-  int32_t* s_cnt = smem + kWarps * p.E;  // [E][P] M
-  int32_t* s_off = s_cnt + p.E * p.P;    // [E+1] S
+  int32_t* s_mt = smem + kWarps * p.E;   // [P][E+1] M transposed: M[l][r] at r*(E+1) + l
+  int32_t* s_off = s_mt + p.P * (p.E + 1);  // [E+1] S
   __shared__ int32_t s_part[kThreads];
   const int c = blockIdx.x, r = blockIdx.y;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -388,7 +388,26 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
   if (!sched_grid_barrier(f, 2)) return;
 
   // ---- C: offsets (every block), warp bases, placement, padding
-  for (int i = threadIdx.x; i < E * P; i += kThreads) s_cnt[i] = __ldcg(p.counts + i);
+  {
+    // M into shared memory, transposed with a row stride of E+1: the
+    // placement loop below reads M[id][r] for 32 unrelated ids at once, which
+    // in the [E][P] layout would fall on P-strided banks. Eight independent
+    // loads in flight per thread.
+    const int n = E * P;
+    for (int i0 = threadIdx.x; i0 < n; i0 += 8 * kThreads) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kThreads;
+        v[u] = i < n ? __ldcg(p.counts + i) : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kThreads;
+        if (i < n) s_mt[(i % P) * (E + 1) + i / P] = v[u];
+      }
+    }
+  }
   __syncthreads();
   {
     // thread t owns experts [4t, 4t + 4) (E <= 1024): padded totals, then a
@@ -402,7 +421,7 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
       tpv[i] = 0;
       if (l < E) {
         int T = 0;
-        for (int r2 = 0; r2 < P; ++r2) T += s_cnt[l * P + r2];
+        for (int r2 = 0; r2 < P; ++r2) T += s_mt[r2 * (E + 1) + l];
         tpv[i] = (T + p.pad - 1) / p.pad * p.pad;
         tsum += tpv[i];
       }
@@ -430,10 +449,20 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
     for (int l = threadIdx.x; l <= E; l += kThreads) p.offsets[l] = s_off[l];
 
   // warp bases = block base (exclusive over blocks) + counts of earlier warps
+  // (E <= 1024: at most four experts per thread, their bases loaded at once)
   {
     const int32_t* blk = p.ws + (static_cast<int64_t>(r) * p.C + c) * E;
-    for (int l = threadIdx.x; l < E; l += kThreads) {
-      int run = __ldcg(blk + l);
+    int base[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int l = threadIdx.x + u * kThreads;
+      base[u] = l < E ? __ldcg(blk + l) : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int l = threadIdx.x + u * kThreads;
+      if (l >= E) break;
+      int run = base[u];
 #pragma unroll
       for (int ww = 0; ww < kWarps; ++ww) {
         const int v = wbase[ww * E + l];
@@ -459,10 +488,9 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
     if (q < R) {
       const int64_t g = route_index(p, r, q);
       if (valid) {
-        const int32_t* Ml = s_cnt + id * P;
         int pos = 0;
         for (int r2 = 0; r2 < P; ++r2) {
-          const int mm = Ml[r2];
+          const int mm = s_mt[r2 * (E + 1) + id];
           pos += min(mm, o);
           pos += (r2 < r && mm > o) ? 1 : 0;
         }
@@ -479,7 +507,7 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
   const int b = blockIdx.y * gridDim.x + blockIdx.x;
   for (int l = b; l < E; l += nb) {
     int T = 0;
-    for (int r2 = 0; r2 < P; ++r2) T += s_cnt[l * P + r2];
+    for (int r2 = 0; r2 < P; ++r2) T += s_mt[r2 * (E + 1) + l];
     const int start = s_off[l] + T, end = s_off[l + 1];
     for (int row = start + threadIdx.x; row < end; row += kThreads)
       reinterpret_cast<int2*>(p.phi)[row] = make_int2(-1, -1);
@@ -507,9 +535,10 @@ size_t schedule_ws_bytes(int32_t P, int32_t N, int32_t k, int32_t E) {
 
 namespace {
 
-// Shared memory of the one-launch kernel: warp counts [8][E], M [E][P], S [E+1].
+// Shared memory of the one-launch kernel: warp counts [8][E], M [P][E+1], S [E+1].
 size_t fused_smem_bytes(int32_t P, int32_t E) {
-  return (static_cast<size_t>(kWarps) * E + static_cast<size_t>(E) * P + E + 1) * sizeof(int32_t);
+  return (static_cast<size_t>(kWarps) * E + static_cast<size_t>(E + 1) * P + E + 1) *
+         sizeof(int32_t);
 }
 
 // Whether the one-launch kernel can run for this grid: its shared memory fits
@@ -529,14 +558,15 @@ bool fused_fits(int32_t C, int32_t P, int32_t E) {
 }
 
 cudaError_t launch_fused(const SchedParams& p, int32_t extra_expect, int64_t timeout_ns,
-                         cudaStream_t s) {
+                         cudaStream_t s, bool barrier_zeroed) {
   FusedParams f;
   f.sp = p;
   f.bar = reinterpret_cast<uint32_t*>(p.ws + (counter_words(p.P, p.N, p.k, p.E) + 15) / 16 * 16);
   f.expect = p.C * p.P + extra_expect;
   f.timeout_ns = timeout_ns;
-  cudaError_t e = cudaMemsetAsync(f.bar, 0, sizeof(uint32_t), s);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (!barrier_zeroed && (e = cudaMemsetAsync(f.bar, 0, sizeof(uint32_t), s)) != cudaSuccess)
+    return e;
   cudaLaunchAttribute coop[1];
   coop[0].id = cudaLaunchAttributeCooperative;
   coop[0].val.cooperative = 1;
@@ -584,16 +614,20 @@ cudaError_t launch_schedule_barrier_selftest(const int32_t* ids, const moe_shape
   const SchedParams p =
       make_params(ids, sh, Slice{0, sh.N}, phi, offsets, counts, route_row, ws, dev_status);
   if (!fused_fits(p.C, p.P, p.E)) return cudaErrorInvalidConfiguration;
-  return launch_fused(p, /*extra_expect=*/1, timeout_ns, s);
+  return launch_fused(p, /*extra_expect=*/1, timeout_ns, s, false);
+}
+
+int32_t* schedule_barrier_word(int32_t* ws, const moe_shape_t& sh) {
+  return ws + (counter_words(sh.P, sh.N, sh.k, sh.E) + 15) / 16 * 16;
 }
 
 cudaError_t launch_schedule(const int32_t* ids, const moe_shape_t& sh, Slice sl, int32_t* phi,
                             int32_t* offsets, int32_t* counts, int32_t* route_row, int32_t* ws,
-                            int32_t* dev_status, cudaStream_t s) {
+                            int32_t* dev_status, cudaStream_t s, bool barrier_zeroed) {
   const SchedParams p = make_params(ids, sh, sl, phi, offsets, counts, route_row, ws, dev_status);
   // one launch when every block fits on the device at once (the Kimi shape:
   // 28 x 8 blocks); otherwise the four-kernel chain below
-  if (fused_fits(p.C, p.P, p.E)) return launch_fused(p, 0, kWaitTimeoutNs, s);
+  if (fused_fits(p.C, p.P, p.E)) return launch_fused(p, 0, kWaitTimeoutNs, s, barrier_zeroed);
   int launched = 0;
   cudaError_t e = cudaSuccess;
   // count runs in plain stream order (after whatever wrote ids); scan, offsets
