@@ -177,10 +177,12 @@ __global__ void __launch_bounds__(256, 2) route_topk_g8_kernel(const float* __re
                                                             int64_t n_tokens, int E, int k,
                                                             ZeroSpec z) {
   zero_words(z);
-  __shared__ float s_cv[32][kCand];
-  __shared__ int s_ci[32][kCand];
-  __shared__ float s_sv[32][kMaxK];
-  __shared__ int s_si[32][kMaxK];
+  // rows padded by one word: the four tokens of a warp read the same
+  // candidate index at once, which an unpadded row stride puts in one bank
+  __shared__ float s_cv[32][kCand + 1];
+  __shared__ int s_ci[32][kCand + 1];
+  __shared__ float s_sv[32][kMaxK + 1];
+  __shared__ int s_si[32][kMaxK + 1];
   const int lane = threadIdx.x & 31, g = lane & 7, tb = threadIdx.x >> 3;  // token in block
   const int gbase = lane & 24;
   const unsigned gm = 0xFFu << gbase;  // this token's eight lanes
