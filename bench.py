@@ -619,9 +619,9 @@ def run_ours(args):
         mx = dict(ms=m0.elapsed_time(m1) / args.steps, rows=int(bmx["offsets"][-1].item()))
         del xq, xs, bmx
 
-    # the MXFP8 layer (opt in): block-scaled expert GEMMs on weights quantised once
+    # the MXFP8 layer: block-scaled expert GEMMs on weights quantised once
     mxl = None
-    if args.mxfp8_layer and mb == 0:
+    if not args.no_mxfp8_layer and mb == 0:
         Wq = []
         for Wt in W:
             E_, K_, N_ = Wt.shape
@@ -871,8 +871,8 @@ def main(argv=None):
     ap.add_argument("--no-mxfp8", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other workloads (scheduler, zipf, mid, tiny)")
-    ap.add_argument("--mxfp8-layer", action="store_true",
-                    help="also time moe_layer_forward_mxfp8 (block-scaled expert GEMMs)")
+    ap.add_argument("--no-mxfp8-layer", action="store_true",
+                    help="skip the moe_layer_forward_mxfp8 leg (block-scaled expert GEMMs)")
     ap.add_argument("--bwd-steps", type=int, default=10)
     ap.add_argument("--cpu-experts", type=int, default=8,
                     help="experts whose rows the CPU baseline runs through the oracle's FFN")
