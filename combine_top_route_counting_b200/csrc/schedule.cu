@@ -67,6 +67,19 @@ __device__ __forceinline__ int64_t route_index(const SchedParams& p, int r, int 
   return (static_cast<int64_t>(r) * p.N + p.t0) * p.k + q;
 }
 
+// The lanes of the warp whose key equals this lane's (keys in [0, 2^nbits)),
+// built from one ballot per key bit: the same mask as __match_any_sync,
+// at a fraction of its cost.
+__device__ __forceinline__ unsigned match_by_ballots(int key, int nbits) {
+  unsigned m = 0xFFFFFFFFu;
+  for (int b = 0; b < nbits; ++b) {
+    const bool bit = (key >> b) & 1;
+    const unsigned v = __ballot_sync(0xFFFFFFFFu, bit);
+    m &= bit ? v : ~v;
+  }
+  return m;
+}
+
 __global__ void __launch_bounds__(kThreads) sched_count_kernel(SchedParams p) {
   extern __shared__ int32_t hist[];
   pdl_launch_dependents();
@@ -333,7 +346,11 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
   for (int l = lane; l < E; l += 32) wh[l] = 0;
   __syncwarp();
   const int q0 = c * kSchedBlockRoutes + w * kWarpRoutes;
+  // keys: the expert id, or E for a lane without a valid route; the match
+  // masks of each step are built once here and reused by the placement
+  const int nbits = 32 - __clz(E);  // enough bits for 0..E
   int key[kSteps];
+  unsigned msk[kSteps];
   int bad = 0;
 #pragma unroll
   for (int s = 0; s < kSteps; ++s) {
@@ -341,13 +358,14 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
     const int id = (q < R) ? __ldg(p.ids + route_index(p, r, q)) : -1;
     const bool ok = static_cast<unsigned>(id) < static_cast<unsigned>(E);
     if (q < R && !ok) bad = 1;
-    key[s] = ok ? id : kInvalid;
+    key[s] = ok ? id : E;
   }
   if (bad) atomicOr(p.dev_status, MOE_DEV_BAD_EXPERT_ID);
 #pragma unroll
   for (int s = 0; s < kSteps; ++s) {
-    const unsigned m = __match_any_sync(kFull, key[s]);
-    if (key[s] != kInvalid && lane == __ffs(m) - 1) wh[key[s]] += __popc(m);
+    const unsigned m = match_by_ballots(key[s], nbits);
+    msk[s] = m;
+    if (key[s] != E && lane == __ffs(m) - 1) wh[key[s]] += __popc(m);
     __syncwarp();
   }
   __syncthreads();
@@ -366,43 +384,83 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
   {
     const int nwarps = gridDim.x * gridDim.y * kWarps;
     const int gw = (blockIdx.y * gridDim.x + blockIdx.x) * kWarps + w;
-    for (int col = gw; col < P * E; col += nwarps) {
-      const int r2 = col / E, l = col - r2 * E;
-      int32_t* base = p.ws + static_cast<int64_t>(r2) * p.C * E + l;
-      int carry = 0;
-      for (int c0 = 0; c0 < p.C; c0 += 32) {
-        const int cc = c0 + lane;
-        const int v = (cc < p.C) ? __ldcg(base + static_cast<int64_t>(cc) * E) : 0;
-        int x = v;
+    const int ncol = P * E;
+    if (p.C <= 32) {
+      // one value per lane per column: a warp's columns (up to four) are
+      // loaded in one round, then scanned
+      for (int col0 = gw; col0 < ncol; col0 += 4 * nwarps) {
+        int v[4];
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(kFull, x, o);
-          if (lane >= o) x += y;
+        for (int u = 0; u < 4; ++u) {
+          const int col = col0 + u * nwarps;
+          const int r2 = col / E, l = col - r2 * E;
+          v[u] = (col < ncol && lane < p.C)
+                     ? __ldcg(p.ws + (static_cast<int64_t>(r2) * p.C + lane) * E + l)
+                     : 0;
         }
-        if (cc < p.C) base[static_cast<int64_t>(cc) * E] = carry + x - v;
-        carry += __shfl_sync(kFull, x, 31);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int col = col0 + u * nwarps;
+          if (col >= ncol) break;
+          const int r2 = col / E, l = col - r2 * E;
+          int x = v[u];
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, x, o);
+            if (lane >= o) x += y;
+          }
+          if (lane < p.C) p.ws[(static_cast<int64_t>(r2) * p.C + lane) * E + l] = x - v[u];
+          if (lane == 31) p.counts[l * P + r2] = x;
+        }
       }
-      if (lane == 0) p.counts[l * P + r2] = carry;
+    } else {
+      for (int col = gw; col < ncol; col += nwarps) {
+        const int r2 = col / E, l = col - r2 * E;
+        int32_t* base = p.ws + static_cast<int64_t>(r2) * p.C * E + l;
+        int carry = 0;
+        for (int c0 = 0; c0 < p.C; c0 += 32) {
+          const int cc = c0 + lane;
+          const int v = (cc < p.C) ? __ldcg(base + static_cast<int64_t>(cc) * E) : 0;
+          int x = v;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, x, o);
+            if (lane >= o) x += y;
+          }
+          if (cc < p.C) base[static_cast<int64_t>(cc) * E] = carry + x - v;
+          carry += __shfl_sync(kFull, x, 31);
+        }
+        if (lane == 0) p.counts[l * P + r2] = carry;
+      }
     }
   }
   if (!sched_grid_barrier(f, 2)) return;
 
   // ---- C: offsets (every block), warp bases, placement, padding
+  // This block's bases (E <= 1024: at most four per thread) and M are loaded
+  // in one round: the bases first, then M with sixteen loads in flight per
+  // thread (one round for E * P <= 4,096 words). M goes to shared memory
+  // transposed with a row stride of E+1: the placement loop below reads
+  // M[id][r] for 32 unrelated ids at once, which in the [E][P] layout would
+  // fall on P-strided banks.
+  int base[4];
   {
-    // M into shared memory, transposed with a row stride of E+1: the
-    // placement loop below reads M[id][r] for 32 unrelated ids at once, which
-    // in the [E][P] layout would fall on P-strided banks. Eight independent
-    // loads in flight per thread.
-    const int n = E * P;
-    for (int i0 = threadIdx.x; i0 < n; i0 += 8 * kThreads) {
-      int v[8];
+    const int32_t* blk = p.ws + (static_cast<int64_t>(r) * p.C + c) * E;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 4; ++u) {
+      const int l = threadIdx.x + u * kThreads;
+      base[u] = l < E ? __ldcg(blk + l) : 0;
+    }
+    const int n = E * P;
+    for (int i0 = threadIdx.x; i0 < n; i0 += 16 * kThreads) {
+      int v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
         const int i = i0 + u * kThreads;
         v[u] = i < n ? __ldcg(p.counts + i) : 0;
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 16; ++u) {
         const int i = i0 + u * kThreads;
         if (i < n) s_mt[(i % P) * (E + 1) + i / P] = v[u];
       }
@@ -449,15 +507,7 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
     for (int l = threadIdx.x; l <= E; l += kThreads) p.offsets[l] = s_off[l];
 
   // warp bases = block base (exclusive over blocks) + counts of earlier warps
-  // (E <= 1024: at most four experts per thread, their bases loaded at once)
   {
-    const int32_t* blk = p.ws + (static_cast<int64_t>(r) * p.C + c) * E;
-    int base[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int l = threadIdx.x + u * kThreads;
-      base[u] = l < E ? __ldcg(blk + l) : 0;
-    }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int l = threadIdx.x + u * kThreads;
@@ -478,8 +528,8 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
   for (int s = 0; s < kSteps; ++s) {
     const int q = q0 + s * 32 + lane;
     const int id = key[s];
-    const bool valid = id != kInvalid;
-    const unsigned m = __match_any_sync(kFull, id);
+    const bool valid = id != E;
+    const unsigned m = msk[s];
     int o = 0;
     if (valid) o = wh[id] + __popc(m & lower);
     __syncwarp();
