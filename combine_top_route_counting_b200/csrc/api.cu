@@ -186,18 +186,19 @@ LayerBufs layer_bufs(void* ws, const LayerWs& w) {
 }
 
 // The scratch words a layer call's kernels expect at zero when it starts: the
-// tile counter and landing words, and the schedule's barrier. The routing
-// kernel zeroes them (first slice); later slices zero what they reuse.
+// tile counter and landing words, and the schedule's barrier and totals. The
+// routing kernel zeroes them (first slice); later slices zero what they reuse.
 ZeroSpec call_zeroes(const LayerBufs& b, const moe_shape_t* sh) {
   return ZeroSpec{b.ctr, static_cast<int32_t>(32 + rows_max_of(sh) / 128),
-                  schedule_barrier_word(b.sched, *sh), 1};
+                  schedule_barrier_word(b.sched, *sh), schedule_zero_words(*sh)};
 }
 
 // Schedule -> dispatch -> FFN -> combine for one token slice (steps 2-4).
 // ev (7 events, may be null) marks the stage boundaries 1..6.
 // ab (training, whole batch only): GEMM1 also keeps the pre-activations.
 // first: the call's first slice, whose scratch words the routing kernel
-// zeroed (later slices zero the landing words and the barrier themselves).
+// zeroed (later slices zero the landing words and the schedule's barrier and
+// totals themselves).
 cudaError_t run_slice(const LayerBufs& b, const uint16_t* x, const uint16_t* W1, const uint16_t* W3,
                       const uint16_t* W2, uint16_t* out, Slice sl, const moe_shape_t* sh,
                       int32_t* dev_status, cudaStream_t s, void* const* ev, bool first,

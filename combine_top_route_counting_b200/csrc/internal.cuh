@@ -46,14 +46,16 @@ cudaError_t launch_route_topk(const float* logits, int32_t* ids, float* gates, i
 // Step 2
 constexpr int kSchedBlockRoutes = 2048;  // routes per counting block (8 warps x 256)
 size_t schedule_ws_bytes(int32_t P, int32_t N, int32_t k, int32_t E);
-// barrier_zeroed: the grid-barrier word in ws (schedule_barrier_word) is
-// already zero (else the launch zeroes it first).
+// barrier_zeroed: the schedule_zero_words(sh) words of ws from
+// schedule_barrier_word on (the grid barrier and the totals its one-launch
+// kernel accumulates) are already zero (else the launch zeroes them first).
 cudaError_t launch_schedule(const int32_t* ids, const moe_shape_t& sh, Slice sl, int32_t* phi,
                             int32_t* offsets, int32_t* counts, int32_t* route_row, int32_t* ws,
                             int32_t* dev_status, cudaStream_t s, bool barrier_zeroed = false);
 // The word of the schedule's scratch that its one-launch kernel's grid
 // barrier counts on (after the [P][blocks][E] counters of the whole batch).
 int32_t* schedule_barrier_word(int32_t* ws, const moe_shape_t& sh);
+int32_t schedule_zero_words(const moe_shape_t& sh);
 
 // The schedule's one-launch kernel with a grid barrier that waits for one
 // block more than the launch has: every block gives up after timeout_ns and

@@ -12,12 +12,14 @@
 // pages spread a peer's routes over 1,024 logical threads with contiguous
 // chunks; any contiguous decomposition gives the same order, so here a block
 // owns 2,048 consecutive routes and each of its 8 warps 256 of them, consumed
-// 32 at a time. Ranks inside a 32-route step come from __match_any_sync and a
-// popcount of the lower lanes; ranks across steps, warps and blocks from
-// exclusive prefix sums of integer counts. Nothing is decided by the order of
-// atomics, so Phi is deterministic and equal to the definition.
+// 32 at a time. Ranks inside a 32-route step come from a match mask (equal
+// ids among the warp's lanes) and a popcount of the lower lanes; ranks across
+// steps, warps and blocks from exclusive prefix sums of integer counts. The
+// one-launch kernel adds the totals M with integer atomics, whose sum does not
+// depend on their order: nothing is decided by the order of atomics, so Phi is
+// deterministic and equal to the definition.
 //
-// One cooperative launch runs all four stages with two grid barriers when
+// One cooperative launch runs all four stages with one grid barrier when
 // every block fits on the device at once (sched_fused_kernel, below);
 // otherwise four kernels (one stream, no host round trip):
 //   count    grid (C, P): per-block expert histogram -> ws[r][c][l]
@@ -290,9 +292,17 @@ __global__ void __launch_bounds__(kThreads) sched_scatter_kernel(SchedParams p) 
 struct FusedParams {
   SchedParams sp;
   uint32_t* bar;      // arrival counter, zero at launch
+  int32_t* m;         // [E][P] route totals M, zero at launch (integer atomics)
   int32_t expect;     // blocks that must arrive (the grid; more only in the self test)
   int64_t timeout_ns;
 };
+
+// Row stride of the one-launch kernel's shared copy of M: P rounded up to
+// whole 16-byte vectors, made an odd number of vectors.
+__host__ __device__ __forceinline__ int m_row_stride(int P) {
+  const int v = (P + 3) / 4;
+  return 4 * (v % 2 ? v : v + 1);
+}
 
 __device__ __forceinline__ uint64_t sched_now_ns() {
   uint64_t t;
@@ -331,10 +341,12 @@ __device__ __forceinline__ bool sched_grid_barrier(const FusedParams& f, uint32_
 
 __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
   const SchedParams& p = f.sp;
-  extern __shared__ int32_t smem[];
-  int32_t* wbase = smem;                 // [kWarps][E] warp counts, then warp bases
-  int32_t* s_mt = smem + kWarps * p.E;   // [P][E+1] M transposed: M[l][r] at r*(E+1) + l
-  int32_t* s_off = s_mt + p.P * (p.E + 1);  // [E+1] S
+  extern __shared__ __align__(16) int32_t smem[];
+  const int SP = m_row_stride(p.P);
+  int32_t* s_m = smem;                   // [E][SP] M, zeros after column P
+  int32_t* wbase = s_m + p.E * SP;       // [kWarps][E] warp counts, then warp bases
+  int32_t* s_off = wbase + kWarps * p.E;  // [E+1] S
+  int32_t* s_base = s_off + p.E + 1;     // [E] routes of earlier blocks of this peer
   __shared__ int32_t s_part[kThreads];
   const int c = blockIdx.x, r = blockIdx.y;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -344,6 +356,10 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
   // ---- A: count (ids read once, kept in registers)
   int32_t* wh = wbase + w * E;
   for (int l = lane; l < E; l += 32) wh[l] = 0;
+  for (int l = threadIdx.x; l < E; l += kThreads) {
+    s_base[l] = 0;
+    for (int q = P; q < SP; ++q) s_m[l * SP + q] = 0;
+  }
   __syncwarp();
   const int q0 = c * kSchedBlockRoutes + w * kWarpRoutes;
   // keys: the expert id, or E for a lane without a valid route; the match
@@ -375,114 +391,98 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
       int h = 0;
 #pragma unroll
       for (int ww = 0; ww < kWarps; ++ww) h += wbase[ww * E + l];
+      if (h) atomicAdd(f.m + l * P + r, h);  // M[l][r]: integer sums, any order
       out[l] = h;
     }
   }
   if (!sched_grid_barrier(f, 1)) return;
 
-  // ---- B: exclusive prefix over blocks of every (peer, expert) column
+  // ---- C: M, this block's bases, offsets, warp bases, placement, padding
+  // M (E * P words) and the block's bases are loaded in one round. The base
+  // of expert l is the sum of H[r][c'][l] over the earlier blocks c' < c of
+  // this peer: rows 0..c-1 of the peer's [C][E] slab, contiguous. Thread
+  // (w, lane) takes experts lane + 32 j and rows w + 8 i (48 loads per round
+  // for E <= 384 and c <= 32) and adds its sums into s_base with shared
+  // atomics. M goes to shared memory as [E][SP] rows (m_row_stride): the
+  // placement loop below reads a route's row as 16-byte vectors, and with an
+  // odd number of vectors per row the rows of 8 unrelated ids start in
+  // distinct groups of four banks.
   {
-    const int nwarps = gridDim.x * gridDim.y * kWarps;
-    const int gw = (blockIdx.y * gridDim.x + blockIdx.x) * kWarps + w;
-    const int ncol = P * E;
-    if (p.C <= 32) {
-      // one value per lane per column: a warp's columns (up to four) are
-      // loaded in one round, then scanned
-      for (int col0 = gw; col0 < ncol; col0 += 4 * nwarps) {
-        int v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int col = col0 + u * nwarps;
-          const int r2 = col / E, l = col - r2 * E;
-          v[u] = (col < ncol && lane < p.C)
-                     ? __ldcg(p.ws + (static_cast<int64_t>(r2) * p.C + lane) * E + l)
-                     : 0;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int col = col0 + u * nwarps;
-          if (col >= ncol) break;
-          const int r2 = col / E, l = col - r2 * E;
-          int x = v[u];
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(kFull, x, o);
-            if (lane >= o) x += y;
-          }
-          if (lane < p.C) p.ws[(static_cast<int64_t>(r2) * p.C + lane) * E + l] = x - v[u];
-          if (lane == 31) p.counts[l * P + r2] = x;
-        }
-      }
-    } else {
-      for (int col = gw; col < ncol; col += nwarps) {
-        const int r2 = col / E, l = col - r2 * E;
-        int32_t* base = p.ws + static_cast<int64_t>(r2) * p.C * E + l;
-        int carry = 0;
-        for (int c0 = 0; c0 < p.C; c0 += 32) {
-          const int cc = c0 + lane;
-          const int v = (cc < p.C) ? __ldcg(base + static_cast<int64_t>(cc) * E) : 0;
-          int x = v;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(kFull, x, o);
-            if (lane >= o) x += y;
-          }
-          if (cc < p.C) base[static_cast<int64_t>(cc) * E] = carry + x - v;
-          carry += __shfl_sync(kFull, x, 31);
-        }
-        if (lane == 0) p.counts[l * P + r2] = carry;
-      }
-    }
-  }
-  if (!sched_grid_barrier(f, 2)) return;
-
-  // ---- C: offsets (every block), warp bases, placement, padding
-  // This block's bases (E <= 1024: at most four per thread) and M are loaded
-  // in one round: the bases first, then M with sixteen loads in flight per
-  // thread (one round for E * P <= 4,096 words). M goes to shared memory
-  // transposed with a row stride of E+1: the placement loop below reads
-  // M[id][r] for 32 unrelated ids at once, which in the [E][P] layout would
-  // fall on P-strided banks.
-  int base[4];
-  {
-    const int32_t* blk = p.ws + (static_cast<int64_t>(r) * p.C + c) * E;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int l = threadIdx.x + u * kThreads;
-      base[u] = l < E ? __ldcg(blk + l) : 0;
-    }
     const int n = E * P;
-    for (int i0 = threadIdx.x; i0 < n; i0 += 16 * kThreads) {
-      int v[16];
+    int mv[16];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int i = i0 + u * kThreads;
-        v[u] = i < n ? __ldcg(p.counts + i) : 0;
-      }
+    for (int u = 0; u < 16; ++u) {
+      const int i = threadIdx.x + u * kThreads;
+      mv[u] = i < n ? __ldcg(f.m + i) : 0;
+    }
+    const int32_t* hb = p.ws + static_cast<int64_t>(r) * p.C * E;
+    constexpr int kJ = 12, kI = 4;  // experts per lane, rows per warp in one round
+    for (int j0 = 0; j0 < E; j0 += 32 * kJ) {
+      for (int i0 = 0; i0 < c; i0 += kWarps * kI) {
+        int hv[kJ][kI];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int i = i0 + u * kThreads;
-        if (i < n) s_mt[(i % P) * (E + 1) + i / P] = v[u];
+        for (int jj = 0; jj < kJ; ++jj)
+#pragma unroll
+          for (int ii = 0; ii < kI; ++ii) {
+            const int l = j0 + lane + 32 * jj, cc = i0 + w + kWarps * ii;
+            hv[jj][ii] = (l < E && cc < c) ? __ldcg(hb + static_cast<int64_t>(cc) * E + l) : 0;
+          }
+#pragma unroll
+        for (int jj = 0; jj < kJ; ++jj) {
+          const int l = j0 + lane + 32 * jj;
+          int sum = 0;
+#pragma unroll
+          for (int ii = 0; ii < kI; ++ii) sum += hv[jj][ii];
+          if (sum) atomicAdd(s_base + l, sum);
+        }
       }
+    }
+    // (i / P, i % P) for i = threadIdx.x + u * kThreads, stepped without dividing
+    int q = threadIdx.x / P, rem = threadIdx.x - (threadIdx.x / P) * P;
+    const int sq = kThreads / P, sr = kThreads - (kThreads / P) * P;
+    const bool first_block = blockIdx.x == 0 && blockIdx.y == 0;
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int i = threadIdx.x + u * kThreads;
+      if (i < n) {
+        s_m[q * SP + rem] = mv[u];
+        if (first_block) p.counts[i] = mv[u];
+      }
+      q += sq;
+      rem += sr;
+      if (rem >= P) {
+        rem -= P;
+        ++q;
+      }
+    }
+    for (int i = threadIdx.x + 16 * kThreads; i < n; i += kThreads) {  // E * P > 4,096
+      const int v = __ldcg(f.m + i);
+      s_m[(i / P) * SP + i % P] = v;
+      if (first_block) p.counts[i] = v;
     }
   }
   __syncthreads();
+  // padded totals Tp[l] into s_off, one expert per thread (its M row as vectors)
+  for (int l = threadIdx.x; l < E; l += kThreads) {
+    int T = 0;
+    for (int q = 0; q < P; q += 4) {
+      const int4 v = *reinterpret_cast<const int4*>(s_m + l * SP + q);
+      T += v.x + v.y + v.z + v.w;
+    }
+    s_off[l] = (T + p.pad - 1) / p.pad * p.pad;
+  }
+  __syncthreads();
   {
-    // thread t owns experts [4t, 4t + 4) (E <= 1024): padded totals, then a
-    // block-wide exclusive scan of the per-thread sums
+    // thread t owns experts [4t, 4t + 4) (E <= 1024): a block-wide exclusive
+    // scan of the per-thread sums of Tp, written over Tp
     const int l0 = threadIdx.x * 4;
     int tpv[4];
     int tsum = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int l = l0 + i;
-      tpv[i] = 0;
-      if (l < E) {
-        int T = 0;
-        for (int r2 = 0; r2 < P; ++r2) T += s_mt[r2 * (E + 1) + l];
-        tpv[i] = (T + p.pad - 1) / p.pad * p.pad;
-        tsum += tpv[i];
-      }
+      tpv[i] = l < E ? s_off[l] : 0;
+      tsum += tpv[i];
     }
     int x = tsum;
 #pragma unroll
@@ -512,7 +512,7 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
     for (int u = 0; u < 4; ++u) {
       const int l = threadIdx.x + u * kThreads;
       if (l >= E) break;
-      int run = base[u];
+      int run = s_base[l];
 #pragma unroll
       for (int ww = 0; ww < kWarps; ++ww) {
         const int v = wbase[ww * E + l];
@@ -538,11 +538,13 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
     if (q < R) {
       const int64_t g = route_index(p, r, q);
       if (valid) {
+        // columns past P hold zeros, which add nothing (o >= 0)
         int pos = 0;
-        for (int r2 = 0; r2 < P; ++r2) {
-          const int mm = s_mt[r2 * (E + 1) + id];
-          pos += min(mm, o);
-          pos += (r2 < r && mm > o) ? 1 : 0;
+        for (int q = 0; q < P; q += 4) {
+          const int4 v = *reinterpret_cast<const int4*>(s_m + id * SP + q);
+          pos += min(v.x, o) + min(v.y, o) + min(v.z, o) + min(v.w, o);
+          pos += (q < r && v.x > o) + (q + 1 < r && v.y > o) + (q + 2 < r && v.z > o) +
+                 (q + 3 < r && v.w > o);
         }
         const int row = s_off[id] + pos;
         reinterpret_cast<int2*>(p.phi)[row] = make_int2(r, p.t0 + q / p.k);
@@ -557,7 +559,10 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
   const int b = blockIdx.y * gridDim.x + blockIdx.x;
   for (int l = b; l < E; l += nb) {
     int T = 0;
-    for (int r2 = 0; r2 < P; ++r2) T += s_mt[r2 * (E + 1) + l];
+    for (int q = 0; q < P; q += 4) {
+      const int4 v = *reinterpret_cast<const int4*>(s_m + l * SP + q);
+      T += v.x + v.y + v.z + v.w;
+    }
     const int start = s_off[l] + T, end = s_off[l + 1];
     for (int row = start + threadIdx.x; row < end; row += kThreads)
       reinterpret_cast<int2*>(p.phi)[row] = make_int2(-1, -1);
@@ -571,23 +576,29 @@ inline int32_t blocks_per_peer(int32_t Tm, int32_t k) {
 
 }  // namespace
 
-// [P][C][E] block counters, then the one-launch path's barrier counter on
-// its own 64-byte line.
+// [P][C][E] block counters; then, on a 64-byte boundary, the one-launch
+// path's barrier counter (alone on its line) and its [E][P] totals M.
 static int64_t counter_words(int32_t P, int32_t N, int32_t k, int32_t E) {
   const int64_t C = blocks_per_peer(N, k);
   return static_cast<int64_t>(P) * (C > 0 ? C : 1) * E;
 }
 
+static int64_t barrier_offset(int32_t P, int32_t N, int32_t k, int32_t E) {
+  return (counter_words(P, N, k, E) + 15) / 16 * 16;
+}
+
 size_t schedule_ws_bytes(int32_t P, int32_t N, int32_t k, int32_t E) {
-  const int64_t words = (counter_words(P, N, k, E) + 15) / 16 * 16 + 16;
+  const int64_t words = barrier_offset(P, N, k, E) + 16 + static_cast<int64_t>(E) * P;
   return static_cast<size_t>(words) * sizeof(int32_t);
 }
 
 namespace {
 
-// Shared memory of the one-launch kernel: warp counts [8][E], M [P][E+1], S [E+1].
+// Shared memory of the one-launch kernel: M [E][m_row_stride(P)], warp
+// counts [8][E], S [E+1], block bases [E].
 size_t fused_smem_bytes(int32_t P, int32_t E) {
-  return (static_cast<size_t>(kWarps) * E + static_cast<size_t>(E + 1) * P + E + 1) *
+  return (static_cast<size_t>(E) * m_row_stride(P) + static_cast<size_t>(kWarps) * E + E + 1 +
+          E) *
          sizeof(int32_t);
 }
 
@@ -611,11 +622,15 @@ cudaError_t launch_fused(const SchedParams& p, int32_t extra_expect, int64_t tim
                          cudaStream_t s, bool barrier_zeroed) {
   FusedParams f;
   f.sp = p;
-  f.bar = reinterpret_cast<uint32_t*>(p.ws + (counter_words(p.P, p.N, p.k, p.E) + 15) / 16 * 16);
+  int32_t* bar = p.ws + barrier_offset(p.P, p.N, p.k, p.E);
+  f.bar = reinterpret_cast<uint32_t*>(bar);
+  f.m = bar + 16;
   f.expect = p.C * p.P + extra_expect;
   f.timeout_ns = timeout_ns;
   cudaError_t e = cudaSuccess;
-  if (!barrier_zeroed && (e = cudaMemsetAsync(f.bar, 0, sizeof(uint32_t), s)) != cudaSuccess)
+  if (!barrier_zeroed &&
+      (e = cudaMemsetAsync(bar, 0, sizeof(int32_t) * (16 + static_cast<size_t>(p.E) * p.P), s)) !=
+          cudaSuccess)
     return e;
   cudaLaunchAttribute coop[1];
   coop[0].id = cudaLaunchAttributeCooperative;
@@ -668,8 +683,10 @@ cudaError_t launch_schedule_barrier_selftest(const int32_t* ids, const moe_shape
 }
 
 int32_t* schedule_barrier_word(int32_t* ws, const moe_shape_t& sh) {
-  return ws + (counter_words(sh.P, sh.N, sh.k, sh.E) + 15) / 16 * 16;
+  return ws + barrier_offset(sh.P, sh.N, sh.k, sh.E);
 }
+
+int32_t schedule_zero_words(const moe_shape_t& sh) { return 16 + sh.E * sh.P; }
 
 cudaError_t launch_schedule(const int32_t* ids, const moe_shape_t& sh, Slice sl, int32_t* phi,
                             int32_t* offsets, int32_t* counts, int32_t* route_row, int32_t* ws,

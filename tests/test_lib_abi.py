@@ -36,8 +36,9 @@ def test_host_only_queries(lib):
     sh = moe.shape(8, 7168, 384, 8, 7168, 2048)
     # rows_max = P*N*k + E*(pad-1) rounded up to 256
     assert moe.rows_max(sh) == (8 * 7168 * 8 + 384 * 255 + 255) // 256 * 256
-    # [P][blocks of 2048 routes][E] counters, then a 64-byte line for the grid barrier
-    assert moe.schedule_workspace_bytes(sh) == (8 * 28 * 384 + 16) * 4
+    # [P][blocks of 2048 routes][E] counters, then a 64-byte line for the grid
+    # barrier and the [E][P] totals the one-launch schedule accumulates
+    assert moe.schedule_workspace_bytes(sh) == (8 * 28 * 384 + 16 + 384 * 8) * 4
     ws = moe.layer_workspace_bytes(sh)
     rm = moe.rows_max(sh)
     assert ws >= rm * (7168 * 2 + 2048 * 2 + 7168 * 4)  # xg, h and y
