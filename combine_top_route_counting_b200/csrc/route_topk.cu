@@ -327,6 +327,227 @@ __global__ void __launch_bounds__(256, 2) route_topk_g8_kernel(const float* __re
   }
 }
 
+// Four lanes per token, eight tokens per warp (E a multiple of 16, E <= 512,
+// k <= 8). Lane g of a token's quad loads float4 chunks g, g+4, g+8, ... of
+// the logit row (NC >= E/16 chunks; the quad's four 16-byte loads of one step
+// are one 64-byte segment) and keeps each chunk's maximum, plus the four
+// largest of them (sorted). tau = the k-th largest value of the quad's 16
+// kept chunk maxima (two merge steps of sorted lists across the quad): these
+// are actual logits, so at least k logits are >= tau and every chosen expert
+// is among them. Only the chunks whose maximum reaches tau are read again
+// (from L1); their logits >= tau go to the lane's 16 candidate slots, and
+// each candidate's rank under (value desc, id asc) among the quad's
+// candidates is counted: ranks 0..k-1 are the slots. More than 16 candidates
+// in one lane (heavy ties, -inf logits) send the quad to k rounds of
+// quad-wide argmax over all its logits, round r taking the best logit that
+// comes after round r-1's in that order. Gates as above, summed in slot order.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Sorts a bitonic sequence of 8 values into descending order.
+__device__ __forceinline__ void bitonic_merge8_desc(float (&c)[8]) {
+#pragma unroll
+  for (int d = 4; d > 0; d >>= 1)
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if ((i & d) == 0) {
+        const float hi = fmaxf(c[i], c[i + d]), lo = fminf(c[i], c[i + d]);
+        c[i] = hi;
+        c[i + d] = lo;
+      }
+}
+
+constexpr int kG4Slots = 16;  // candidate slots per lane
+
+template <int NC>
+__global__ void __launch_bounds__(256) route_topk_g4_kernel(const float* __restrict__ logits,
+                                                            int32_t* __restrict__ ids,
+                                                            float* __restrict__ gates,
+                                                            int64_t n_tokens, int E, int k,
+                                                            ZeroSpec z) {
+  static_assert(NC <= 32, "one mask bit per chunk");
+  zero_words(z);
+  // token rows padded by one word: the eight quads of a warp read the same
+  // slot index at once
+  __shared__ float s_cv[64][4 * kG4Slots + 1];  // lane g's candidates at [16g, 16g + 16)
+  __shared__ int s_ci[64][4 * kG4Slots + 1];
+  __shared__ float s_sv[64][9];
+  __shared__ int s_si[64][9];
+  const int lane = threadIdx.x & 31, g = lane & 3, tb = threadIdx.x >> 2;  // token in block
+  const int gbase = lane & 28;
+  const unsigned gm = 0xFu << gbase;  // this token's four lanes
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * 64 + tb;
+  if (t >= n_tokens) return;  // the whole quad leaves together
+  const float4* row = reinterpret_cast<const float4*>(logits + t * E);
+  const int nc4 = E >> 2;
+
+  // chunk maxima and the lane's four largest of them, descending
+  float cm[NC];
+  float a[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+  constexpr int kBatch = 12;  // loads in flight per lane
+#pragma unroll
+  for (int i0 = 0; i0 < NC; i0 += kBatch) {
+    float4 q[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int c = g + 4 * (i0 + u);
+      if (i0 + u < NC)
+        q[u] = c < nc4 ? __ldg(row + c) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (i0 + u < NC) {
+        const float v = fmaxf(fmax3(q[u].x, q[u].y, q[u].z), q[u].w);
+        cm[i0 + u] = v;
+        a[3] = fmaxf(a[3], fminf(a[2], v));
+        a[2] = fmaxf(a[2], fminf(a[1], v));
+        a[1] = fmaxf(a[1], fminf(a[0], v));
+        a[0] = fmaxf(a[0], v);
+      }
+    }
+  }
+  // tau: merge with the partner lane (xor 1) into a sorted 8, then keep the
+  // top 8 of that and the other pair's sorted 8 (xor 2), sorted
+  float c8[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    c8[i] = a[i];
+    c8[7 - i] = __shfl_xor_sync(gm, a[i], 1);
+  }
+  bitonic_merge8_desc(c8);
+  float d8[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) d8[7 - i] = __shfl_xor_sync(gm, c8[i], 2);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) d8[i] = fmaxf(c8[i], d8[i]);
+  bitonic_merge8_desc(d8);
+  float tau = d8[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i)
+    if (i == k - 1) tau = d8[i];
+
+  // candidates: the logits >= tau of the chunks whose maximum reaches tau
+  unsigned pm = 0;
+#pragma unroll
+  for (int i = 0; i < NC; ++i)
+    if (g + 4 * i < nc4 && cm[i] >= tau) pm |= 1u << i;
+  int c = 0;
+  while (pm) {
+    const int i = __ffs(pm) - 1;
+    pm &= pm - 1;
+    const int ch = g + 4 * i;
+    const float4 q = __ldg(row + ch);
+    const float vv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (vv[j] >= tau) {
+        if (c < kG4Slots) {
+          s_cv[tb][kG4Slots * g + c] = vv[j];
+          s_ci[tb][kG4Slots * g + c] = 4 * ch + j;
+        }
+        ++c;
+      }
+    }
+  }
+  const bool over = (__ballot_sync(gm, c > kG4Slots) & gm) != 0;
+  __syncwarp(gm);
+
+  if (!over) {
+    // rank every candidate of the quad: lane g takes candidates g, g+4, ...
+    // of the quad's list (lane h's slots in order, then lane h+1's)
+    int cnt[4], off[5];
+    off[0] = 0;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      cnt[h] = __shfl_sync(gm, c, gbase | h);
+      off[h + 1] = off[h] + cnt[h];
+    }
+    const int total = off[4];
+    for (int ai = g; ai < total; ai += 4) {
+      const int ha = (ai >= off[1]) + (ai >= off[2]) + (ai >= off[3]);
+      const int oa = ha == 0 ? 0 : ha == 1 ? off[1] : ha == 2 ? off[2] : off[3];
+      const int sa = kG4Slots * ha + (ai - oa);
+      const float cv = s_cv[tb][sa];
+      const int ci = s_ci[tb][sa];
+      int rank = 0;
+#pragma unroll
+      for (int h = 0; h < 4; ++h)
+        for (int b = 0; b < cnt[h]; ++b)
+          rank += better(s_cv[tb][kG4Slots * h + b], s_ci[tb][kG4Slots * h + b], cv, ci) ? 1 : 0;
+      if (rank < k) {
+        s_sv[tb][rank] = cv;
+        s_si[tb][rank] = ci;
+      }
+    }
+  } else {
+    float pv = INFINITY;  // round r's pick comes after (pv, pid): none yet
+    int pid = -1;
+    for (int r = 0; r < k; ++r) {
+      float bv = -INFINITY;
+      int bid = INT_MAX;
+      for (int i = 0; i < NC; ++i) {
+        const int ch = g + 4 * i;
+        if (ch >= nc4) break;
+        const float4 q = __ldg(row + ch);
+        const float vv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int e = 4 * ch + j;
+          if (better(pv, pid, vv[j], e) && better(vv[j], e, bv, bid)) {
+            bv = vv[j];
+            bid = e;
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 2; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(gm, bv, o, 4);
+        const int oid = __shfl_xor_sync(gm, bid, o, 4);
+        if (better(ov, oid, bv, bid)) {
+          bv = ov;
+          bid = oid;
+        }
+      }
+      if (g == 0) {
+        s_sv[tb][r] = bv;
+        s_si[tb][r] = bid;
+      }
+      pv = bv;
+      pid = bid;
+    }
+  }
+  __syncwarp(gm);
+
+  // gates: softmax over the chosen logits, summed in slot order (lane g holds
+  // slots g and g + 4)
+  const float l0 = s_sv[tb][0];
+  const float e0 = g < k ? expf(s_sv[tb][g] - l0) : 0.0f;
+  const float e1 = g + 4 < k ? expf(s_sv[tb][g + 4] - l0) : 0.0f;
+  float den = 0.0f;
+  for (int j = 0; j < k; ++j) den += __shfl_sync(gm, j < 4 ? e0 : e1, gbase | (j & 3));
+  if (g < k) {
+    ids[t * k + g] = s_si[tb][g];
+    gates[t * k + g] = e0 / den;
+  }
+  if (g + 4 < k) {
+    ids[t * k + g + 4] = s_si[tb][g + 4];
+    gates[t * k + g + 4] = e1 / den;
+  }
+}
+
+template <int NC>
+cudaError_t launch_g4(const float* logits, int32_t* ids, float* gates, int64_t n, int E, int k,
+                      cudaStream_t s, ZeroSpec z) {
+  const int64_t blocks = (n + 63) / 64;
+  route_topk_g4_kernel<NC><<<static_cast<unsigned>(blocks), 256, 0, s>>>(logits, ids, gates, n, E,
+                                                                         k, z);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
 template <int NV>
 cudaError_t launch_g8(const float* logits, int32_t* ids, float* gates, int64_t n, int E, int k,
                       cudaStream_t s, ZeroSpec z) {
@@ -358,6 +579,14 @@ cudaError_t launch_route_topk(const float* logits, int32_t* ids, float* gates, i
     if (z.nb > 0 && cudaMemsetAsync(z.b, 0, z.nb * sizeof(int), s) != cudaSuccess)
       return cudaGetLastError();
     return cudaSuccess;
+  }
+  // four lanes per token for the wide rows (at E <= 128 the eight-lane
+  // kernel's twice as many blocks fill the device better)
+  if (E % 16 == 0 && E > 128 && E <= 512 && k <= 8) {
+    if (E <= 192) return launch_g4<12>(logits, ids, gates, n_tokens, E, k, s, z);
+    if (E <= 256) return launch_g4<16>(logits, ids, gates, n_tokens, E, k, s, z);
+    if (E <= 384) return launch_g4<24>(logits, ids, gates, n_tokens, E, k, s, z);
+    return launch_g4<32>(logits, ids, gates, n_tokens, E, k, s, z);
   }
   if (E % 4 == 0 && E <= 512) {
     if (E <= 32) return launch_g8<1>(logits, ids, gates, n_tokens, E, k, s, z);

@@ -254,6 +254,34 @@ def test_route_topk_heavy_ties_and_neg_inf(cuda_lib, E, k):
     assert np.all(g_[~ok] == 0)
 
 
+@pytest.mark.parametrize("E,k", [(16, 2), (48, 8), (64, 1), (128, 5), (160, 8), (256, 3),
+                                 (320, 8), (512, 8), (384, 12), (256, 16), (36, 4), (100, 8),
+                                 (388, 8), (96, 9)])
+def test_route_topk_shapes(cuda_lib, E, k):
+    """Every routing kernel variant (four lanes per token for E % 16 == 0 and
+    k <= 8, at each chunk count; eight lanes for other multiples of 4 or
+    k > 8; one warp per token otherwise) on a ragged token count: random rows,
+    rows whose winners all fall in one lane's chunks (more candidates in that
+    lane than its slots), tied rows and rows with -inf logits."""
+    moe = cuda_lib
+    g = torch.Generator().manual_seed(1000 * E + k)
+    T = 300
+    lg = torch.randn((T, E), generator=g)
+    lane0 = [c * 4 + j for c in range(0, (E + 3) // 4, 4) for j in range(4) if c * 4 + j < E]
+    lg[4::7, lane0] += 8.0                           # winners crowd the first lane of a quad
+    lg[5::7] = 0.5                                   # all tied
+    lg[6::7, ::3] = float("-inf")                    # a third of the experts unreachable
+    sh = moe.shape(1, T, E, k)
+    ids = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    gates = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    moe.moe_route_topk(lg.to(DEV), ids, gates, sh)
+    torch.cuda.synchronize()
+    o_ids, _, o_g64 = oracle.route_topk(lg, k)
+    assert (ids.cpu().numpy() == o_ids).all()
+    g_ = gates.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(g_ - o_g64) / o_g64) < 1e-6
+
+
 # ---------------------------------------------------------------- stages on small layers
 def _stage_run(moe, w, W1, W3, W2, lg, x):
     """Run every stage through its own entry point; return device tensors."""
