@@ -38,9 +38,12 @@
 //          after its last TMEM read, so only the reads and the first of its
 //          two blocks' arithmetic stall the next tile's MMAs (it writes 1 byte
 //          per h value, against a 56-stage K loop);
-//   GEMM2  256 x 128 tiles, two 128-column accumulators: the next tile's MMAs
-//          run while the epilogue streams the fp32 y tile out (the larger
-//          epilogue, against a 16-stage K loop).
+//   GEMM2  256 x 256 tiles (CTA r holding W2's columns 128 r .. +128), one
+//          256-column accumulator: each epilogue thread reads its 128
+//          accumulator values into registers and releases the accumulator
+//          before it stages and stores them, so the next tile's MMAs wait
+//          only for the TMEM reads. A block-scaled MMA of N = 128 takes as long
+//          to issue as one of N = 256, so the wider tile halves GEMM2's MMAs.
 //
 // Every output element is produced by one CTA pair in a fixed K order (no
 // split-K, no atomics): the result is deterministic and independent of which
@@ -65,19 +68,19 @@ using namespace pg;
 template <int MODE>
 struct MxCfg {
   static constexpr bool TMA_STORE = MODE == 1;
-  static constexpr int STAGING_BYTES = TMA_STORE ? 8 * 4096 : 0;  // 8 warps x 32x32 fp32
+  static constexpr int STAGING_BYTES = TMA_STORE ? 8 * 2048 : 0;  // 8 warps x 32x16 fp32
   static constexpr int BM = 256;
-  static constexpr int BN = MODE == 0 ? 256 : 128;     // accumulator columns per tile
-  static constexpr int ACC = MODE == 0 ? 1 : 2;        // accumulators in TMEM
+  static constexpr int BN = 256;                       // accumulator columns per tile
+  static constexpr int ACC = 1;                        // accumulators in TMEM
   static constexpr int BK = 128;                       // E4M3 values (bytes) per stage
   static constexpr int MMA_K = 32;                     // K of one block-scaled MMA
   static constexpr int B_ROWS = BN / 2;                // B rows (tile columns) per CTA
   static constexpr int A_BYTES = 128 * BK;             // this CTA's 128 rows
   static constexpr int B_BYTES = B_ROWS * BK;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KB / 24 KB
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KB
   static constexpr int SFB_ATOMS = BN / 128;             // scale atoms of the tile's columns
   static constexpr int SF_STAGE_BYTES = 512 * (1 + SFB_ATOMS);
-  static constexpr int STAGES = MODE == 0 ? 6 : 7;
+  static constexpr int STAGES = 6;
   static constexpr int TMEM_SF = ACC * BN;              // scale columns follow the accumulators
   static constexpr int SF_COLS = 4 * (1 + SFB_ATOMS) <= 8 ? 8 : 16;  // A at +0, B at +4
   static_assert(TMEM_SF + STAGES * SF_COLS <= kTmemCols, "TMEM budget");
@@ -217,8 +220,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 
   const int rows_used = bad_sched ? 0 : s_off[E];
   // GEMM1: a tile's 256 accumulator columns are 128 h columns seen through W1
-  // and W3; GEMM2: 128 y columns
-  const int tiles_n = p.Nout / 128;
+  // and W3; GEMM2: 256 y columns
+  const int tiles_n = p.Nout / (MODE == 0 ? 128 : C::BN);
   const int num_tiles = (rows_used / C::BM) * tiles_n;
   const int kblocks = p.K / C::BK;  // stages per tile = scale atoms per 128-row block
   const WaitCtx wc{abort_flag, p.dev_status, p.timeout_ns, MOE_DEV_TIMEOUT};
@@ -252,9 +255,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const int arow = row0 + static_cast<int>(rank) * 128;
         // B rows (of the transposed weights) this tile meets: GEMM1: W1t and
         // W3t rows l*I + n*128 .. +128 (CTA 0 loads W1t's, CTA 1 W3t's);
-        // GEMM2: W2t rows l*H + n*128 .. +128 (CTA r loads 64 r .. +64).
-        // Either way one scale atom per 128 rows.
-        const int brow = l * p.Nout + n * 128;
+        // GEMM2: W2t rows l*H + n*256 .. +256 (CTA r loads 128 r .. +128).
+        // Either way one scale atom per 128 rows, two per tile.
+        const int brow = l * p.Nout + n * (MODE == 0 ? 128 : C::BN);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!wait_bounded(smem_u32(&bars[C::BAR_EMPTY + stage]), phase ^ 1u, wc)) {
             ok = false;
@@ -276,6 +279,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           } else {
             tma_load_2d_pair(sB, &tmB0, kx, brow + static_cast<int>(rank) * C::B_ROWS, full_tgt);
             tma_load_2d_pair(sSB, &tmSB0, 0, (brow / 128) * kblocks + kb, full_tgt);
+            tma_load_2d_pair(sSB + 512, &tmSB0, 0, (brow / 128 + 1) * kblocks + kb, full_tgt);
           }
           ++issued;
           if (++stage == C::STAGES) {
@@ -411,40 +415,42 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           p.hs[mx_tiled_offset(row, col / 32, I / 32)] = scale;
         }
       } else {
-        // row `lane` of this warp's 32x32 block goes to the staging slot with
-        // 16-byte chunk j at j ^ (lane & 7) (the tensor map's 128-byte
-        // swizzle), then one TMA store; a slot is reused once the previous
-        // store has read it
-        const uint32_t stg = smem_u32(staging) + (warp - kEpiWarp0) * 4096;
+        // this warp's 128 of the tile's 256 columns, read whole into
+        // registers; the accumulator is released before the stores. Row
+        // `lane` of each 32x16 block then goes to the warp's 2 KB staging slot
+        // with 16-byte chunk j at j ^ ((lane >> 1) & 3) (the tensor map's
+        // 64-byte swizzle) and leaves with one TMA store; the slot is reused
+        // once the previous store has read it.
+        uint32_t rv[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_32cols(tbase + half * 128 + c * 32, rv[c]);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_relaxed_cluster(tempty_tgt0 + acc * 8);
+        const uint32_t stg = smem_u32(staging) + (warp - kEpiWarp0) * 2048;
         const uint64_t pol_y = l2_policy_evict_first();
-        const int ycol = n * C::BN + half * 64;  // this warp's 64 of the tile's 128 columns
+        const int ycol = n * C::BN + half * 128;
         const int yrow0 = row0 + static_cast<int>(rank) * 128 + q * 32;
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          uint32_t rv[32];
-          tmem_ld_32cols(tbase + half * 64 + c * 32, rv);
-          tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            st_shared_v4(stg + lane * 128 + ((j ^ (lane & 7)) << 4), rv[4 * j], rv[4 * j + 1],
-                         rv[4 * j + 2], rv[4 * j + 3]);
+          for (int j = 0; j < 4; ++j)
+            st_shared_v4(stg + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4),
+                         rv[c >> 1][(c & 1) * 16 + 4 * j], rv[c >> 1][(c & 1) * 16 + 4 * j + 1],
+                         rv[c >> 1][(c & 1) * 16 + 4 * j + 2], rv[c >> 1][(c & 1) * 16 + 4 * j + 3]);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) {
-            tma_store_2d_hint(&tmY, stg, ycol + c * 32, yrow0, pol_y);
+          if (lane == 0) {  // y is streamed out and read once, by the combine
+            tma_store_2d_hint(&tmY, stg, ycol + c * 16, yrow0, pol_y);
             bulk_commit_group();
           }
         }
       }
-      // the accumulator may be refilled once every lane's tcgen05.ld completed
-      // (GEMM1 released it above)
-      if (MODE != 0) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_relaxed_cluster(tempty_tgt0 + acc * 8);
-      }
+      // (both modes released the accumulator above, once every lane's
+      // tcgen05.ld had completed)
       if (++acc == C::ACC) {
         acc = 0;
         acc_phase ^= 1u;
@@ -494,9 +500,9 @@ cudaError_t launch_expert_ffn_mxfp8(const uint8_t* xq, const uint8_t* xs, const 
       !make_map_u8(&mW3, W3q, H, EI, 128, 128) ||
       !make_map_sf_atoms(&mW3s, W3s, EI / 128 * (H / 128)) ||
       !make_map_u8(&mHq, hq, I, rows_max, 128, 128) || !make_map_sf_atoms(&mHs, hs, rb * (I / 128)) ||
-      !make_map_u8(&mW2, W2q, I, EH, 128, 64) ||   // GEMM2: 64 B rows per CTA
+      !make_map_u8(&mW2, W2q, I, EH, 128, 128) ||  // GEMM2: 128 B rows per CTA
       !make_map_sf_atoms(&mW2s, W2s, EH / 128 * (I / 128)) ||
-      !make_map(&mY, y, H, rows_max, 32, 32, true))
+      !make_map(&mY, y, H, rows_max, 16, 32, true, true))
     return cudaErrorInvalidValue;
   MxParams p1{counter, offsets, counts, E, sh.P, H, I, rows_max, hq, hs, dev_status, kWaitTimeoutNs};
   cudaError_t e = launch_mx<0>(mXq, mXs, mW1, mW1s, mW3, mW3s, mY, p1, s);
