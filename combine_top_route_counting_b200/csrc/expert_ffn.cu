@@ -626,23 +626,28 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const uint64_t pol_y = l2_policy_evict_first();
         const int ycol = n * C::BN + half * 128;
         const int yrow0 = row0 + static_cast<int>(rank) * 128 + q * 32;
+        // a 32-row block wholly past the expert's routes holds only padding
+        // rows, which nothing reads: its y is not written
+        const bool keep = yrow0 < s_end[l];
         uint32_t rv[2][16];
         tmem_ld_16cols(tbase + half * 128, rv[0]);
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           if (c + 1 < 8) tmem_ld_16cols(tbase + half * 128 + (c + 1) * 16, rv[(c + 1) & 1]);
-          if (lane == 0) bulk_wait_read_all();  // the previous store has read the slot
-          __syncwarp();
+          if (keep) {
+            if (lane == 0) bulk_wait_read_all();  // the previous store has read the slot
+            __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            st_shared_v4(stg + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4), rv[c & 1][4 * j],
-                         rv[c & 1][4 * j + 1], rv[c & 1][4 * j + 2], rv[c & 1][4 * j + 3]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {  // y is streamed out and read once, by the combine
-            tma_store_2d_hint(&tmY, stg, ycol + c * 16, yrow0, pol_y);
-            bulk_commit_group();
+            for (int j = 0; j < 4; ++j)
+              st_shared_v4(stg + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4), rv[c & 1][4 * j],
+                           rv[c & 1][4 * j + 1], rv[c & 1][4 * j + 2], rv[c & 1][4 * j + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {  // y is streamed out and read once, by the combine
+              tma_store_2d_hint(&tmY, stg, ycol + c * 16, yrow0, pol_y);
+              bulk_commit_group();
+            }
           }
           if (c + 1 < 8) tmem_ld_wait();
         }

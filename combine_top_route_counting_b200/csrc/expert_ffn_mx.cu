@@ -432,8 +432,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const uint64_t pol_y = l2_policy_evict_first();
         const int ycol = n * C::BN + half * 128;
         const int yrow0 = row0 + static_cast<int>(rank) * 128 + q * 32;
+        // a 32-row block wholly past the expert's routes holds only padding
+        // rows, which nothing reads: its y is not written
+        const int nblk = yrow0 < s_end[l] ? 8 : 0;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < nblk; ++c) {
           if (lane == 0) bulk_wait_read_all();
           __syncwarp();
 #pragma unroll

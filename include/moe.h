@@ -180,8 +180,9 @@ moe_status_t moe_dispatch(const uint16_t* x, const int32_t* phi, const int32_t* 
  *   h[row] = bf16_rne( silu(xg[row].W1[l]) * (xg[row].W3[l]) ),  h: bf16 [moe_rows_max, I]
  *   y[row] = h[row].W2[l] (fp32),                                 y: fp32 [moe_rows_max, H]
  * counts (int32 [E,P], may be NULL): when given, tiles that hold only
- * padding rows are skipped and their h/y rows are left unwritten; rows that
- * carry routes are always written. Each output element is computed by one
+ * padding rows are skipped and their h/y rows are left unwritten, and y is
+ * not written for 32-row blocks past the last route of their expert; rows
+ * that carry routes are always written. Each output element is computed by one
  * CTA (pair) with a fixed K order: the result is bitwise deterministic.
  * Tile counter: the GEMM kernels take their tiles from a counter of two
  * int32 words that the last CTA of each launch puts back to zero. The GEMM
@@ -478,7 +479,8 @@ moe_status_t moe_mx_quantize_weights(const uint16_t* W, int32_t E, int32_t K, in
  * outputs; W1q/W1s, W3q/W3s, W2q/W2s: moe_mx_quantize_weights of W1, W3, W2.
  * Requires the moe_expert_ffn limits and pad % 256 == 0 (CTA-pair tiles).
  * hq, y 32-byte aligned, every other pointer 16-byte aligned. Rows of tiles
- * holding only padding are not written. Errors as moe_expert_ffn. */
+ * holding only padding are not written, nor y of 32-row blocks past the last
+ * route of their expert. Errors as moe_expert_ffn. */
 moe_status_t moe_expert_ffn_mxfp8(const uint8_t* xq, const uint8_t* xs, const uint8_t* W1q,
                                   const uint8_t* W1s, const uint8_t* W3q, const uint8_t* W3s,
                                   const uint8_t* W2q, const uint8_t* W2s, const int32_t* offsets,
