@@ -377,6 +377,37 @@ def test_ffn_no_counts_computes_padding_rows(cuda_lib):
     assert torch.equal(y2[real], r["y"][real]) and torch.equal(h2[real], r["h"][real])
 
 
+def test_ffn_counts_leave_padding_blocks_of_y_unwritten(cuda_lib):
+    """With counts, GEMM2 writes y for every row that carries a route and skips
+    the 32-row blocks wholly past their expert's last route (padding rows
+    nothing reads); the rows it writes equal the count-less run's."""
+    moe = cuda_lib
+    w = inputs.WORKLOADS["tiny"]
+    lg, x = inputs.make_logits(w), inputs.make_x(w)
+    W1, W3, W2 = [t.to(DEV) for t in inputs.make_weights(w)]
+    r = _stage_run(moe, w, W1, W3, W2, lg.to(DEV), x.to(DEV))
+    sh = moe.shape(**w.shape())
+    rows = int(r["offsets"][-1].item())
+    h2 = torch.empty_like(r["h"])
+    y2 = torch.full_like(r["y"], 7.0)
+    moe.moe_expert_ffn(r["xg"], W1, W3, W2, r["offsets"], r["counts"], h2, y2, r["dev_status"], sh)
+    torch.cuda.synchronize()
+    assert int(r["dev_status"].item()) == 0
+    phi = r["phi"][:rows, 0].cpu().numpy()
+    real = np.nonzero(phi >= 0)[0]
+    yd, y2h = r["y"].cpu(), y2.cpu()
+    assert torch.equal(y2h[real], yd[real])
+    off = r["offsets"].cpu().numpy()
+    cnt = r["counts"].cpu().numpy().sum(axis=1)
+    skipped = 0
+    for l in range(w.E):
+        end = off[l] + cnt[l]
+        for b0 in range((end + 31) // 32 * 32, off[l + 1], 32):  # blocks wholly past the routes
+            assert (y2h[b0:b0 + 32] == 7.0).all()
+            skipped += 1
+    assert skipped > 0, "the case has padding blocks past an expert's last route"
+
+
 @pytest.mark.parametrize("name,pad", [("tiny", 256), ("mid", 256), ("tiny", 128)])
 def test_ffn_gather_equals_dispatch_then_ffn(cuda_lib, name, pad):
     """The FFN that pulls its rows from x by Phi reproduces dispatch + FFN bit for bit."""
