@@ -114,7 +114,7 @@ def stage_rooflines(stage_ms: dict, work: dict, peaks: dict, fused_dispatch: boo
             out[name] = d
             continue
         if fused_dispatch and name == "ffn_gemm1":
-            d["includes"] = "the pull dispatch (its gather runs on a spare warp inside the kernel)"
+            d["includes"] = "the pull dispatch (run by a spare warp inside the kernel)"
         if "bytes" in work[name]:
             gbs = work[name]["bytes"] / (t / 1e3) / 1e9
             d.update(bytes=work[name]["bytes"], gbs=gbs, frac_hbm=gbs / peaks["hbm"])
@@ -486,7 +486,8 @@ def assemble_line(args, w, world, ms, stage_ms, launches, e2e, e2e_mb, mb, mb_ro
                          "note": "pull dispatch with the MX (E4M3, E8M0 per 32) "
                                  "quantisation fused"}
     if mxl:
-        mst = stage_rooflines(mxl["stage_ms"], mx_layer_work(w, rows_used), peaks)
+        mst = stage_rooflines(mxl["stage_ms"], mx_layer_work(w, rows_used), peaks,
+                              fused_dispatch=True)
         line["mxfp8_layer"] = {
             "value": w.n_tokens * world * args.steps / (mxl["ms"] / 1e3), "unit": "tokens/s",
             "ms_per_step": mxl["ms"] / args.steps, "steps": args.steps,

@@ -309,9 +309,10 @@ cudaError_t layer_body_mx(const float* logits, const uint16_t* x, const uint8_t*
                            b.sched, dev_status, s, /*barrier_zeroed=*/true)) != cudaSuccess)
     return e;
   if ((e = rec(2)) != cudaSuccess) return e;
-  if ((e = launch_dispatch_mxfp8(x, b.phi, b.offsets, xq, xs, *sh, rows_max, dev_status, s,
-                                 /*tiled=*/true)) != cudaSuccess)
-    return e;
+  // the quantising pull dispatch lands inside GEMM1 (its spare warp writes
+  // the codes and tiled scales of 128-row blocks as the tensor cores consume
+  // earlier ones); the landing words were zeroed by the routing kernel
+  const LandArgs land{x, b.phi, b.land, b.land + 16};
   if ((e = rec(3)) != cudaSuccess) return e;
   // the bf16 shared expert over every token (its time counts in stage 3, the
   // routed GEMM1's); nothing on one GPU to overlap it with
@@ -326,7 +327,8 @@ cudaError_t layer_body_mx(const float* logits, const uint16_t* x, const uint8_t*
   }
   cudaEvent_t mid = ev ? static_cast<cudaEvent_t>(ev[4]) : nullptr;
   if ((e = launch_expert_ffn_mxfp8(xq, xs, W1q, W1s, W3q, W3s, W2q, W2s, b.offsets, b.counts, hq,
-                                   hs, b.y, *sh, rows_max, dev_status, s, mid, b.ctr)) != cudaSuccess)
+                                   hs, b.y, *sh, rows_max, dev_status, s, mid, b.ctr, &land)) !=
+      cudaSuccess)
     return e;
   if ((e = rec(5)) != cudaSuccess) return e;
   if ((e = launch_combine(b.y, b.route_row, b.gates, out, *sh, Slice{0, sh->N}, rows_max,

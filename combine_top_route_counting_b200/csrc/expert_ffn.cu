@@ -108,31 +108,6 @@ struct FfnParams {
   int* land_ready;         // LAND: [rows_max / 128] block-landed flags (0 at launch)
 };
 
-// Wait (bounded, acquire at GPU scope) until *flag != 0: the LAND producer's
-// wait for a block of gathered rows that another CTA's warp lands. Gives up
-// like wait_bounded: after timeout_ns, or once another role of the CTA gave up.
-__device__ __forceinline__ bool wait_flag_bounded(const int* flag, const WaitCtx& w) {
-  auto ready = [&]() {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
-    return v != 0;
-  };
-  if (ready()) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    __nanosleep(32);
-    if (ready()) return true;
-    if ((it & 15u) == 0) {
-      if (*w.abort) return false;
-      if (globaltimer_ns() - t0 > static_cast<uint64_t>(w.timeout_ns)) {
-        *w.abort = 1;
-        atomicOr(w.dev_status, w.timeout_flag);
-        return false;
-      }
-    }
-  }
-}
-
 template <int CG, int MODE>
 size_t smem_bytes_for(int E) {
   using C = Cfg<CG, MODE>;

@@ -54,6 +54,7 @@
 #include <cuda_fp8.h>
 
 #include "internal.cuh"
+#include "mx_block.cuh"
 #include "persistent_gemm.cuh"
 #include "sm100.cuh"
 #include "sm100_mx.cuh"
@@ -112,6 +113,14 @@ struct MxParams {
   uint8_t* hs;             // GEMM1: h scales, tiled over [rows_max, I/32]
   int32_t* dev_status;
   int64_t timeout_ns;
+  // LAND (GEMM1): the quantising pull dispatch inside the kernel
+  const int2* phi;         // [rows_max] (src_rank, src_idx)
+  int32_t n_per_peer;      // N (token row = src_rank * N + src_idx)
+  const void* x;           // token activations bf16 [P*N, H]
+  uint8_t* xq;             // the A operand's codes [rows_max, H] the tensor map reads
+  uint8_t* xs;             // its scales, tiled over [rows_max, H/32]
+  int* land_next;          // next 128-row block to land (0 at launch)
+  int* land_ready;         // [rows_max / 128] block-landed flags (0 at launch)
 };
 
 template <int MODE>
@@ -153,7 +162,16 @@ __device__ __forceinline__ void mx_block_f32(const float (&v)[32], uint32_t (&co
   }
 }
 
-template <int MODE>
+// LAND (MODE 0): the quantising pull dispatch runs inside this kernel, as in
+// the bf16 FFN: warp 3 of every CTA takes 128-row blocks of the
+// expert-sorted layout in order from a device counter, quantises each row
+// x[Phi[row]] by the MX block rule (mx_block.cuh) into the codes and tiled
+// scales the A tensor maps read (padding rows: zero codes, scale code 0), and
+// publishes the block with a release store of its flag. The TMA producer
+// waits (bounded) for the flag of its CTA's 128 rows before it loads a tile's
+// A codes and scales, then issues a cross-proxy fence (the rows were written
+// through the generic proxy, TMA reads through the async proxy).
+template <int MODE, bool LAND = false>
 __global__ void __launch_bounds__(kNumThreads, 1)
     ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmSA,
                   const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmSB0,
@@ -258,6 +276,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         // GEMM2: W2t rows l*H + n*256 .. +256 (CTA r loads 128 r .. +128).
         // Either way one scale atom per 128 rows, two per tile.
         const int brow = l * p.Nout + n * (MODE == 0 ? 128 : C::BN);
+        if (LAND) {  // this CTA's 128 A rows must have landed
+          if (!wait_flag_bounded(p.land_ready + arow / 128, wc)) break;
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!wait_bounded(smem_u32(&bars[C::BAR_EMPTY + stage]), phase ^ 1u, wc)) {
             ok = false;
@@ -362,6 +384,60 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       tc_commit_pair(smem_u32(&bars[C::BAR_DRAIN]));
       wait_drain(smem_u32(&bars[C::BAR_DRAIN]), 0, p.timeout_ns);
     }
+  } else if (warp == 3 && LAND) {
+    // ------------------------------------------------------------ quantising pull dispatch
+    const int nblk = rows_used / 128;
+    const int kb32 = p.K / 32;  // MX blocks of a row
+    const uint4* xsrc = reinterpret_cast<const uint4*>(p.x);
+    int bad = 0;
+    for (;;) {
+      int b = 0;
+      if (lane == 0) b = atomicAdd(p.land_next, 1);
+      b = __shfl_sync(0xFFFFFFFFu, b, 0);
+      if (b >= nblk || *wc.abort) break;
+#pragma unroll 1
+      for (int rr = 0; rr < 128; ++rr) {
+        const int64_t row = static_cast<int64_t>(b) * 128 + rr;
+        const int2 e = __ldg(p.phi + row);
+        const bool v = e.x >= 0 && e.x < p.P && e.y >= 0 && e.y < p.n_per_peer;
+        if (!v && (e.x >= 0 || e.y != -1)) bad = 1;  // (-1,-1) is padding
+        const uint4* src =
+            xsrc + (v ? (static_cast<int64_t>(e.x) * p.n_per_peer + e.y) * (p.K / 8) : 0);
+        uint4* qrow = reinterpret_cast<uint4*>(p.xq) + row * (p.K / 16);
+        // lane j takes blocks j, j+32, ...: a 7,168-wide row (224 blocks) in
+        // one round of 28 16-byte loads per lane
+        constexpr int U = 7;
+#pragma unroll 1
+        for (int b0 = lane; b0 < kb32; b0 += 32 * U) {
+          uint4 in[U][4];
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int blk = b0 + 32 * u;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              in[u][c] = (v && blk < kb32) ? __ldg(src + blk * 4 + c) : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int blk = b0 + 32 * u;
+            if (blk < kb32) {
+              uint4 out[2];
+              uint8_t scale;
+              mx::mx_block(in[u], out, scale);
+              qrow[blk * 2] = out[0];
+              qrow[blk * 2 + 1] = out[1];
+              p.xs[mx_tiled_offset(row, blk, kb32)] = scale;
+            }
+          }
+        }
+      }
+      __threadfence();  // every lane's rows before the flag
+      __syncwarp();
+      if (lane == 0)
+        asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p.land_ready + b), "r"(1)
+                     : "memory");
+    }
+    if (bad) atomicOr(p.dev_status, MOE_DEV_BAD_SCHEDULE);
   } else if (warp == 2) {
     // ------------------------------------------------------------ tile scheduler
     if (lane == 0 && leader) tring.schedule<true>(p.tile_counter, num_tiles, wc);
@@ -472,7 +548,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   }
 }
 
-template <int MODE>
+template <int MODE, bool LAND = false>
 cudaError_t launch_mx(const CUtensorMap& a, const CUtensorMap& sa, const CUtensorMap& b0,
                       const CUtensorMap& sb0, const CUtensorMap& b1, const CUtensorMap& sb1,
                       const CUtensorMap& y, MxParams p, cudaStream_t s) {
@@ -481,7 +557,7 @@ cudaError_t launch_mx(const CUtensorMap& a, const CUtensorMap& sa, const CUtenso
     const cudaError_t e = tile_counter_for_current_device(&p.tile_counter);
     if (e != cudaSuccess) return e;
   }
-  return launch_persistent(ffn_mx_kernel<MODE>, 2, smem, s, a, sa, b0, sb0, b1, sb1, y, p);
+  return launch_persistent(ffn_mx_kernel<MODE, LAND>, 2, smem, s, a, sa, b0, sb0, b1, sb1, y, p);
 }
 
 }  // namespace
@@ -492,7 +568,7 @@ cudaError_t launch_expert_ffn_mxfp8(const uint8_t* xq, const uint8_t* xs, const 
                                     const int32_t* offsets, const int32_t* counts, uint8_t* hq,
                                     uint8_t* hs, float* y, const moe_shape_t& sh,
                                     int64_t rows_max, int32_t* dev_status, cudaStream_t s,
-                                    cudaEvent_t ev_mid, int* counter) {
+                                    cudaEvent_t ev_mid, int* counter, const LandArgs* land) {
   const int E = sh.E, H = sh.H, I = sh.I;
   const uint64_t EH = static_cast<uint64_t>(E) * H, EI = static_cast<uint64_t>(E) * I;
   const uint64_t rb = static_cast<uint64_t>(rows_max) / 128;  // 128-row blocks of the activations
@@ -508,7 +584,19 @@ cudaError_t launch_expert_ffn_mxfp8(const uint8_t* xq, const uint8_t* xs, const 
       !make_map(&mY, y, H, rows_max, 16, 32, true, true))
     return cudaErrorInvalidValue;
   MxParams p1{counter, offsets, counts, E, sh.P, H, I, rows_max, hq, hs, dev_status, kWaitTimeoutNs};
-  cudaError_t e = launch_mx<0>(mXq, mXs, mW1, mW1s, mW3, mW3s, mY, p1, s);
+  cudaError_t e;
+  if (land) {  // the quantising pull dispatch lands xq, xs inside GEMM1
+    p1.phi = reinterpret_cast<const int2*>(land->phi);
+    p1.n_per_peer = sh.N;
+    p1.x = land->x;
+    p1.xq = const_cast<uint8_t*>(xq);
+    p1.xs = const_cast<uint8_t*>(xs);
+    p1.land_next = land->next;
+    p1.land_ready = land->ready;
+    e = launch_mx<0, true>(mXq, mXs, mW1, mW1s, mW3, mW3s, mY, p1, s);
+  } else {
+    e = launch_mx<0>(mXq, mXs, mW1, mW1s, mW3, mW3s, mY, p1, s);
+  }
   if (e != cudaSuccess) return e;
   if (ev_mid && (e = cudaEventRecord(ev_mid, s)) != cudaSuccess) return e;
   MxParams p2{counter, offsets, counts, E, sh.P, I, H, rows_max, nullptr, nullptr, dev_status,

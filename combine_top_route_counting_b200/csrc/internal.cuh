@@ -203,14 +203,17 @@ cudaError_t launch_mx_quantize_weights(const uint16_t* W, int32_t E, int32_t K, 
 
 // The grouped SwiGLU expert FFN on MXFP8 operands (block-scaled tcgen05, CTA
 // pairs): GEMM1 + SwiGLU + MX quantisation of h, then GEMM2 -> fp32 y.
-// ev_mid, if not null, is recorded between the two kernels.
+// ev_mid, if not null, is recorded between the two kernels. land (if not
+// null): GEMM1 quantises x[Phi[row]] into xq, xs (tiled scales) itself, block
+// by block, instead of reading a dispatch's output; its flags must be zero.
 cudaError_t launch_expert_ffn_mxfp8(const uint8_t* xq, const uint8_t* xs, const uint8_t* W1q,
                                     const uint8_t* W1s, const uint8_t* W3q, const uint8_t* W3s,
                                     const uint8_t* W2q, const uint8_t* W2s,
                                     const int32_t* offsets, const int32_t* counts, uint8_t* hq,
                                     uint8_t* hs, float* y, const moe_shape_t& sh,
                                     int64_t rows_max, int32_t* dev_status, cudaStream_t s,
-                                    cudaEvent_t ev_mid, int* counter = nullptr);
+                                    cudaEvent_t ev_mid, int* counter = nullptr,
+                                    const LandArgs* land = nullptr);
 
 // 2D tensor map over a [outer, inner] uint8 matrix, box [box_outer, box_inner],
 // 128-byte swizzle.

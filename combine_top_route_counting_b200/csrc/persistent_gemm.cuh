@@ -147,6 +147,32 @@ __device__ __forceinline__ bool grouped_row_tile(int tile, const int32_t* s_off,
   return row0 < s_end[l];
 }
 
+// Wait (bounded, acquire at GPU scope) until *flag != 0: a landed-dispatch
+// producer's wait for a block of gathered rows that another CTA's warp lands.
+// Gives up like wait_bounded: after timeout_ns, or once another role of the
+// CTA gave up.
+__device__ __forceinline__ bool wait_flag_bounded(const int* flag, const sm100::WaitCtx& w) {
+  auto ready = [&]() {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    return v != 0;
+  };
+  if (ready()) return true;
+  const uint64_t t0 = sm100::globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(32);
+    if (ready()) return true;
+    if ((it & 15u) == 0) {
+      if (*w.abort) return false;
+      if (sm100::globaltimer_ns() - t0 > static_cast<uint64_t>(w.timeout_ns)) {
+        *w.abort = 1;
+        atomicOr(w.dev_status, w.timeout_flag);
+        return false;
+      }
+    }
+  }
+}
+
 // A launch's tile counter is two words: the next tile id, and the CTAs that
 // have finished. Called once per CTA (one thread, after the CTA's last use of
 // the counter): the last CTA to finish puts both words back to zero, so the

@@ -495,7 +495,10 @@ size_t moe_layer_mxfp8_workspace_bytes(const moe_shape_t* shape);
 
 /* Steps 1-4 with MXFP8 routed experts: route, schedule, the quantising
  * dispatch (TILED scales), moe_expert_ffn_mxfp8 and the fixed-order combine,
- * on `stream`. Routed weights as moe_expert_ffn_mxfp8.
+ * on `stream`; the dispatch runs inside GEMM1 (a spare warp of every CTA
+ * quantises 128-row blocks of x[Phi[row]] while the tensor cores consume
+ * earlier ones), with the results of moe_dispatch_mxfp8_tiled.
+ * Routed weights as moe_expert_ffn_mxfp8.
  * Ws1, Ws3 bf16 [H, I] and Ws2 bf16 [I, H] (all three, or all null): a bf16
  * shared expert ("Mixture-of-Kittens", section 5) every token passes through,
  * ys[t] = bf16(silu(x[t].Ws1) * (x[t].Ws3)).Ws2 in fp32 on the bf16 FFN's
