@@ -186,6 +186,38 @@ def test_layer_mxfp8_bitwise_deterministic(cuda_lib, name):
     assert sha(a) == sha(b)
 
 
+@pytest.mark.parametrize("name", ["tiny", "mid"])
+def test_layer_mxfp8_equals_its_stage_entries(cuda_lib, name):
+    """The MXFP8 layer, whose GEMM1 quantises and lands the dispatch itself,
+    gives bit for bit the output of the separate entry points: moe_route_topk,
+    moe_schedule, moe_dispatch_mxfp8_tiled, moe_expert_ffn_mxfp8, moe_combine."""
+    moe = cuda_lib
+    w = inputs.WORKLOADS[name]
+    lg, x = inputs.make_logits(w).to(DEV), inputs.make_x(w).to(DEV)
+    Wq = _mx_weights_gpu(moe, inputs.make_weights(w))
+    out = _layer_mx(moe, w, lg, x, Wq)
+    sh = moe.shape(**w.shape())
+    rm = moe.rows_max(sh)
+    ids = torch.empty((w.n_tokens, w.k), dtype=torch.int32, device=DEV)
+    gates = torch.empty((w.n_tokens, w.k), dtype=torch.float32, device=DEV)
+    moe.moe_route_topk(lg, ids, gates, sh)
+    b = moe.alloc_schedule_outputs(sh)
+    moe.moe_schedule(ids, b["phi"], b["offsets"], b["counts"], b["route_row"], b["ws"],
+                     b["dev_status"], sh)
+    xq = torch.empty((rm, w.H), dtype=torch.uint8, device=DEV)
+    xs = torch.empty((rm * w.H // 32,), dtype=torch.uint8, device=DEV)
+    moe.moe_dispatch_mxfp8_tiled(x, b["phi"], b["offsets"], xq, xs, b["dev_status"], sh)
+    hq = torch.empty((rm, w.I), dtype=torch.uint8, device=DEV)
+    hs = torch.empty((rm * w.I // 32,), dtype=torch.uint8, device=DEV)
+    y = torch.empty((rm, w.H), dtype=torch.float32, device=DEV)
+    moe.moe_expert_ffn_mxfp8(xq, xs, *Wq, b["offsets"], b["counts"], hq, hs, y, b["dev_status"], sh)
+    ref = torch.empty((w.n_tokens, w.H), dtype=torch.bfloat16, device=DEV)
+    moe.moe_combine(y, b["route_row"], gates, ref, b["dev_status"], sh)
+    torch.cuda.synchronize()
+    assert int(b["dev_status"].item()) == 0
+    assert torch.equal(out, ref)
+
+
 def test_layer_mxfp8_no_tokens(cuda_lib):
     moe = cuda_lib
     w = inputs.Workload("mx_empty", 13, P=2, N=0, E=8, k=2, H=256, I=256)
