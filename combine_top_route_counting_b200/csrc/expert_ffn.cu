@@ -145,7 +145,9 @@ __device__ __forceinline__ float silu(float a) { return a / (1.0f + expf(-a)); }
 // and TMA reads through the async proxy. Blocks are landed in the order the
 // tiles are handed out, so the copies run ahead of the tensor cores and the
 // HBM-bound gather overlaps the MMAs; no warp that lands rows ever waits.
-template <int MODE, int CG, bool GATHER, bool SAVE_AB, bool LAND = false>
+// NARROW (with LAND): rows of at most 512 values, landed several per round
+// (a separate instantiation, so the kernel for wider rows is unchanged).
+template <int MODE, int CG, bool GATHER, bool SAVE_AB, bool LAND = false, bool NARROW = false>
 __global__ void __launch_bounds__(kNumThreads, 1)
     ffn_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmY,
@@ -432,27 +434,75 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       if (lane == 0) b = atomicAdd(p.land_next, 1);
       b = __shfl_sync(0xFFFFFFFFu, b, 0);
       if (b >= nblk || *wc.abort) break;
+      constexpr int U = 28;  // 16-byte loads in flight per lane: a 7,168-wide row in one round
+      constexpr int UR = 16;  // the same for rows of at most 512 values, several per round
+      if (NARROW) {
+        // narrow rows (one or two loads per lane), whole rows per round: lane
+        // j takes chunks j, j+32, ... of the round's rows back to back
+        // (chunks is a multiple of 32), so the rows share a round instead of
+        // each costing a memory round trip
+        const int rpr = (32 * UR) / chunks;  // 8 or 16
 #pragma unroll 1
-      for (int rr = 0; rr < 128; ++rr) {
-        const int64_t row = static_cast<int64_t>(b) * 128 + rr;
-        const int2 e = __ldg(p.phi + row);
-        const bool v = e.x >= 0 && e.x < p.P && e.y >= 0 && e.y < p.n_per_peer;
-        if (!v && (e.x >= 0 || e.y != -1)) bad = 1;  // (-1,-1) is padding
-        uint4* dst = reinterpret_cast<uint4*>(p.xg) + row * chunks;
-        const uint4* src = xsrc + (v ? (static_cast<int64_t>(e.x) * p.n_per_peer + e.y) * chunks : 0);
-        constexpr int U = 28;  // a 7,168-wide row in one round: 28 loads in flight per lane
-#pragma unroll 1
-        for (int c0 = lane; c0 < chunks; c0 += 32 * U) {
-          uint4 t[U];
-#pragma unroll
-          for (int u = 0; u < U; ++u) {
-            const int c = c0 + 32 * u;
-            t[u] = (v && c < chunks) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+        for (int rr0 = 0; rr0 < 128; rr0 += rpr) {
+          // lane l < rpr looks up row rr0 + l once: the chunk offset of its
+          // token row, -1 for padding; each load below takes its row's by shuffle
+          int64_t so_l = -1;
+          if (lane < rpr && rr0 + lane < 128) {
+            const int2 e = __ldg(p.phi + static_cast<int64_t>(b) * 128 + rr0 + lane);
+            const bool v = e.x >= 0 && e.x < p.P && e.y >= 0 && e.y < p.n_per_peer;
+            if (!v && (e.x >= 0 || e.y != -1)) bad = 1;  // (-1,-1) is padding
+            if (v) so_l = (static_cast<int64_t>(e.x) * p.n_per_peer + e.y) * chunks;
           }
+          uint4 t[UR];
+          int ro = 0, c = lane;
 #pragma unroll
-          for (int u = 0; u < U; ++u) {
-            const int c = c0 + 32 * u;
-            if (c < chunks) dst[c] = t[u];
+          for (int u = 0; u < UR; ++u) {
+            const int64_t so = __shfl_sync(0xFFFFFFFFu, so_l, ro);
+            t[u] = (ro < rpr && so >= 0) ? __ldg(xsrc + so + c) : make_uint4(0, 0, 0, 0);
+            c += 32;
+            if (c >= chunks) {
+              c -= chunks;
+              ++ro;
+            }
+          }
+          ro = 0;
+          c = lane;
+#pragma unroll
+          for (int u = 0; u < UR; ++u) {
+            const int rr = rr0 + ro;
+            if (ro < rpr && rr < 128)
+              reinterpret_cast<uint4*>(p.xg)[(static_cast<int64_t>(b) * 128 + rr) * chunks + c] =
+                  t[u];
+            c += 32;
+            if (c >= chunks) {
+              c -= chunks;
+              ++ro;
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int rr = 0; rr < 128; ++rr) {
+          const int64_t row = static_cast<int64_t>(b) * 128 + rr;
+          const int2 e = __ldg(p.phi + row);
+          const bool v = e.x >= 0 && e.x < p.P && e.y >= 0 && e.y < p.n_per_peer;
+          if (!v && (e.x >= 0 || e.y != -1)) bad = 1;  // (-1,-1) is padding
+          uint4* dst = reinterpret_cast<uint4*>(p.xg) + row * chunks;
+          const uint4* src =
+              xsrc + (v ? (static_cast<int64_t>(e.x) * p.n_per_peer + e.y) * chunks : 0);
+#pragma unroll 1
+          for (int c0 = lane; c0 < chunks; c0 += 32 * U) {
+            uint4 t[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+              const int c = c0 + 32 * u;
+              t[u] = (v && c < chunks) ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+              const int c = c0 + 32 * u;
+              if (c < chunks) dst[c] = t[u];
+            }
           }
         }
       }
@@ -671,7 +721,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 
 namespace {
 
-template <int MODE, int CG, bool GATHER = false, bool SAVE_AB = false, bool LAND = false>
+template <int MODE, int CG, bool GATHER = false, bool SAVE_AB = false, bool LAND = false,
+          bool NARROW = false>
 cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const CUtensorMap& yo, FfnParams p, cudaStream_t s) {
   const size_t smem = smem_bytes_for<CG, MODE>(p.E);
@@ -679,8 +730,8 @@ cudaError_t launch_mode(const CUtensorMap& a, const CUtensorMap& b0, const CUten
     const cudaError_t e = tile_counter_for_current_device(&p.tile_counter);
     if (e != cudaSuccess) return e;
   }
-  return launch_persistent(ffn_gemm_kernel<MODE, CG, GATHER, SAVE_AB, LAND>, CG, smem, s, a, b0, b1,
-                           yo, p);
+  return launch_persistent(ffn_gemm_kernel<MODE, CG, GATHER, SAVE_AB, LAND, NARROW>, CG, smem, s,
+                           a, b0, b1, yo, p);
 }
 
 }  // namespace
@@ -711,8 +762,12 @@ cudaError_t launch_expert_ffn(const uint16_t* xg, const uint16_t* W1, const uint
     p1.xg = const_cast<uint16_t*>(xg);
     p1.land_next = land->next;
     p1.land_ready = land->ready;
-    e = ab ? launch_mode<0, 2, false, true, true>(mA1, mW1, mW3, mA1, p1, s)
-           : launch_mode<0, 2, false, false, true>(mA1, mW1, mW3, mA1, p1, s);
+    if (H <= 512)  // rows of one or two 16-byte chunks per lane: several per round
+      e = ab ? launch_mode<0, 2, false, true, true, true>(mA1, mW1, mW3, mA1, p1, s)
+             : launch_mode<0, 2, false, false, true, true>(mA1, mW1, mW3, mA1, p1, s);
+    else
+      e = ab ? launch_mode<0, 2, false, true, true>(mA1, mW1, mW3, mA1, p1, s)
+             : launch_mode<0, 2, false, false, true>(mA1, mW1, mW3, mA1, p1, s);
   } else if (ab) {  // training: keep the pre-activations (pair tiles only)
     e = pair ? launch_mode<0, 2, false, true>(mA1, mW1, mW3, mA1, p1, s) : cudaErrorInvalidValue;
   } else {

@@ -395,38 +395,84 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       if (lane == 0) b = atomicAdd(p.land_next, 1);
       b = __shfl_sync(0xFFFFFFFFu, b, 0);
       if (b >= nblk || *wc.abort) break;
+      constexpr int U = 7;  // blocks per lane in one round: a 7,168-wide row (224 blocks)
+      if (2 * kb32 <= 32 * U) {
+        // rows of at most 3,584 values, whole rows per round: lane j takes
+        // blocks j, j+32, ... of the round's rows back to back (block f of
+        // the round: row f / kb32, block f % kb32), so the rows share a round
+        // instead of each costing a memory round trip
+        const int rpr = (32 * U) / kb32;  // 2 .. 28
 #pragma unroll 1
-      for (int rr = 0; rr < 128; ++rr) {
-        const int64_t row = static_cast<int64_t>(b) * 128 + rr;
-        const int2 e = __ldg(p.phi + row);
-        const bool v = e.x >= 0 && e.x < p.P && e.y >= 0 && e.y < p.n_per_peer;
-        if (!v && (e.x >= 0 || e.y != -1)) bad = 1;  // (-1,-1) is padding
-        const uint4* src =
-            xsrc + (v ? (static_cast<int64_t>(e.x) * p.n_per_peer + e.y) * (p.K / 8) : 0);
-        uint4* qrow = reinterpret_cast<uint4*>(p.xq) + row * (p.K / 16);
-        // lane j takes blocks j, j+32, ...: a 7,168-wide row (224 blocks) in
-        // one round of 28 16-byte loads per lane
-        constexpr int U = 7;
-#pragma unroll 1
-        for (int b0 = lane; b0 < kb32; b0 += 32 * U) {
+        for (int rr0 = 0; rr0 < 128; rr0 += rpr) {
+          // lane l < rpr looks up row rr0 + l once: the 16-byte offset of its
+          // token row, -1 for padding; each block takes its row's by shuffle
+          int64_t so_l = -1;
+          if (lane < rpr && rr0 + lane < 128) {
+            const int2 e = __ldg(p.phi + static_cast<int64_t>(b) * 128 + rr0 + lane);
+            const bool v = e.x >= 0 && e.x < p.P && e.y >= 0 && e.y < p.n_per_peer;
+            if (!v && (e.x >= 0 || e.y != -1)) bad = 1;  // (-1,-1) is padding
+            if (v) so_l = (static_cast<int64_t>(e.x) * p.n_per_peer + e.y) * (p.K / 8);
+          }
           uint4 in[U][4];
 #pragma unroll
           for (int u = 0; u < U; ++u) {
-            const int blk = b0 + 32 * u;
+            const int f = lane + 32 * u;
+            const int ro = min(f / kb32, 31), blk = f - (f / kb32) * kb32;
+            const int64_t so = __shfl_sync(0xFFFFFFFFu, so_l, ro);
+            const bool ld = f < rpr * kb32 && so >= 0;
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-              in[u][c] = (v && blk < kb32) ? __ldg(src + blk * 4 + c) : make_uint4(0, 0, 0, 0);
+              in[u][c] = ld ? __ldg(xsrc + so + blk * 4 + c) : make_uint4(0, 0, 0, 0);
           }
 #pragma unroll
           for (int u = 0; u < U; ++u) {
-            const int blk = b0 + 32 * u;
-            if (blk < kb32) {
+            const int f = lane + 32 * u;
+            const int ro = f / kb32, blk = f - ro * kb32;
+            if (f < rpr * kb32 && rr0 + ro < 128) {
+              const int64_t row = static_cast<int64_t>(b) * 128 + rr0 + ro;
               uint4 out[2];
               uint8_t scale;
               mx::mx_block(in[u], out, scale);
+              uint4* qrow = reinterpret_cast<uint4*>(p.xq) + row * (p.K / 16);
               qrow[blk * 2] = out[0];
               qrow[blk * 2 + 1] = out[1];
               p.xs[mx_tiled_offset(row, blk, kb32)] = scale;
+            }
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int rr = 0; rr < 128; ++rr) {
+          const int64_t row = static_cast<int64_t>(b) * 128 + rr;
+          const int2 e = __ldg(p.phi + row);
+          const bool v = e.x >= 0 && e.x < p.P && e.y >= 0 && e.y < p.n_per_peer;
+          if (!v && (e.x >= 0 || e.y != -1)) bad = 1;  // (-1,-1) is padding
+          const uint4* src =
+              xsrc + (v ? (static_cast<int64_t>(e.x) * p.n_per_peer + e.y) * (p.K / 8) : 0);
+          uint4* qrow = reinterpret_cast<uint4*>(p.xq) + row * (p.K / 16);
+          // lane j takes blocks j, j+32, ...: a 7,168-wide row in one round of
+          // 28 16-byte loads per lane
+#pragma unroll 1
+          for (int b0 = lane; b0 < kb32; b0 += 32 * U) {
+            uint4 in[U][4];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+              const int blk = b0 + 32 * u;
+#pragma unroll
+              for (int c = 0; c < 4; ++c)
+                in[u][c] = (v && blk < kb32) ? __ldg(src + blk * 4 + c) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+              const int blk = b0 + 32 * u;
+              if (blk < kb32) {
+                uint4 out[2];
+                uint8_t scale;
+                mx::mx_block(in[u], out, scale);
+                qrow[blk * 2] = out[0];
+                qrow[blk * 2 + 1] = out[1];
+                p.xs[mx_tiled_offset(row, blk, kb32)] = scale;
+              }
             }
           }
         }
