@@ -160,8 +160,9 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
   }
 }
 
-// Eight lanes per token, four tokens per warp (E a multiple of 4, E <= 512):
-// the same selection with a quarter of the shuffle work per token. Lane g of
+// Eight lanes per token, four tokens per warp (E a multiple of 4, E <= 512;
+// used for E <= 128 or k > 8, the four-lane kernel below for the rest): the
+// same selection with a quarter of the shuffle work per token. Lane g of
 // a token's group loads float4 chunks g, g+8, g+16, ... of its logit row
 // (NV = ceil(E/32) chunks; the group's eight 16-byte loads of one step are
 // one 128-byte segment), and keeps its two largest values. tau = the k-th

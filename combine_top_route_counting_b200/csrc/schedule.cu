@@ -271,24 +271,24 @@ __global__ void __launch_bounds__(kThreads) sched_scatter_kernel(SchedParams p) 
 
 // ---------------------------------------------------------------- one launch
 // The same four stages in one cooperative launch (every block resident at
-// once), separated by two grid barriers:
-//   A  each block (c, r) reads its 2,048 route ids once, keeps them in
-//      registers, builds its warps' expert histograms in shared memory and
-//      writes the block histogram to ws[r][c][l];
-//   |  barrier 1
-//   B  every warp of the grid takes (peer, expert) columns in turn and
-//      replaces ws[r][.][l] by its exclusive prefix over blocks (32 blocks
-//      per warp-wide scan step); the column total is M[l][r] -> counts;
-//   |  barrier 2
-//   C  every block reads M into shared memory and computes T, Tp and S
-//      itself (block (0,0) writes offsets), derives its warps' bases from its
-//      block base, then places its routes from the registers of phase A and
-//      fills its share of padding rows.
-// Each route id is read from memory once. A barrier is a counter in ws
-// (zeroed before the launch): a block arrives with a release add and waits,
-// with an acquire load, until all blocks of the launch arrived; the wait is
-// bounded (timeout_ns), after which the block raises MOE_DEV_TIMEOUT and
-// leaves without writing anything more.
+// once), with one grid barrier:
+//   A  each block (c, r) reads its 2,048 route ids once and keeps them in
+//      registers; each warp builds the match masks of its 32-route steps from
+//      ballots over the id bits (kept for C) and its expert histogram in
+//      shared memory; the block writes its histogram to ws[r][c][l] and adds
+//      the nonzero entries to the totals M[l][r] with integer atomics;
+//   |  the barrier
+//   C  every block loads M and its own base, the sum of ws[r][c'][l] over
+//      the peer's earlier blocks c' < c (rows 0..c-1 of the peer's slab),
+//      computes T, Tp and S itself (block (0,0) writes offsets and counts),
+//      derives its warps' bases from its block base, then places its routes
+//      from the registers of phase A and fills its share of padding rows.
+// Each route id is read from memory once. The barrier is a counter in ws,
+// zero at launch with M (the routing kernel of a layer call zeroes them, a
+// moe_schedule call with a memset): a block arrives with a release add and
+// waits, with an acquire load, until all blocks of the launch arrived; the
+// wait is bounded (timeout_ns), after which the block raises
+// MOE_DEV_TIMEOUT and leaves without writing anything more.
 struct FusedParams {
   SchedParams sp;
   uint32_t* bar;      // arrival counter, zero at launch

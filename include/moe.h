@@ -528,7 +528,7 @@ moe_status_t moe_selftest_bounded_wait(int32_t* dev_status, int64_t timeout_ns, 
 
 /* Failure-detection self test of the schedule's one-launch kernel
  * (moe_schedule runs it when all its blocks fit on the device at once; its
- * two grid barriers are bounded waits): the same kernel, on the same
+ * grid barrier is a bounded wait): the same kernel, on the same
  * arguments as moe_schedule, with a barrier that waits for one block more
  * than the launch has. Every block gives up after timeout_ns nanoseconds,
  * raises MOE_DEV_TIMEOUT in *dev_status and returns; the outputs are then
