@@ -34,10 +34,11 @@
 // first). TMEM holds the accumulators and STAGES x 8 or 16 scale columns:
 //   GEMM1  256 x 256 tiles (128 h columns through W1 and W3, CTA 0 holding
 //          W1's rows and CTA 1 W3's), one 256-column accumulator: a second
-//          would leave no columns for the scales; the epilogue releases it
-//          after its last TMEM read, so only the reads and the first of its
-//          two blocks' arithmetic stall the next tile's MMAs (it writes 1 byte
-//          per h value, against a 56-stage K loop);
+//          would leave no columns for the scales; each epilogue thread reads
+//          both of its MX blocks (128 values) into registers and releases the
+//          accumulator before their arithmetic, so the next tile's MMAs wait
+//          only for the TMEM reads (it writes 1 byte per h value, against a
+//          56-stage K loop);
 //   GEMM2  256 x 256 tiles (CTA r holding W2's columns 128 r .. +128), one
 //          256-column accumulator: each epilogue thread reads its 128
 //          accumulator values into registers and releases the accumulator
@@ -511,24 +512,26 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       if (MODE == 0) {
         // accumulator columns [0,128) = x.W1, [128,256) = x.W3 for h columns
         // n*128 + j; this warp's 64 columns are two 32-column MX blocks of h.
-        // The single accumulator is released as soon as this warp's last
-        // TMEM reads completed, so the next tile's MMAs overlap the SwiGLU,
-        // quantisation and stores of its last block.
+        // Both blocks are read into registers first and the single
+        // accumulator is released, so the next tile's MMAs overlap the
+        // SwiGLU, quantisation and stores of both.
         const int I = p.Nout;
-#pragma unroll 1
+        uint32_t ra[2][32], rb[2][32];
+#pragma unroll
         for (int c = 0; c < 2; ++c) {
-          uint32_t ra[32], rb[32];
-          tmem_ld_32cols(tbase + half * 64 + c * 32, ra);
-          tmem_ld_32cols(tbase + 128 + half * 64 + c * 32, rb);
-          tmem_ld_wait();
-          if (c == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_relaxed_cluster(tempty_tgt0 + acc * 8);
-          }
+          tmem_ld_32cols(tbase + half * 64 + c * 32, ra[c]);
+          tmem_ld_32cols(tbase + 128 + half * 64 + c * 32, rb[c]);
+        }
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_relaxed_cluster(tempty_tgt0 + acc * 8);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
           float hv[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) hv[i] = silu(__uint_as_float(ra[i])) * __uint_as_float(rb[i]);
+          for (int i = 0; i < 32; ++i)
+            hv[i] = silu(__uint_as_float(ra[c][i])) * __uint_as_float(rb[c][i]);
           uint32_t codes[8];
           uint8_t scale;
           mx_block_f32(hv, codes, scale);
