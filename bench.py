@@ -179,8 +179,9 @@ def time_configs(moe, dev, W_kimi, x_kimi, ws_big, st, steps: int, warmup: int, 
         raise RuntimeError("device status in the scheduler workload")
     out["sched"] = {"workload": workload_desc(w), "phi_build_us_median": 1e3 * statistics.median(t),
                     "phi_build_us_min": 1e3 * min(t), "calls": n,
-                    "what": "moe_schedule: count, scan, offsets, scatter (4 kernels) on "
-                            "uniform ids; L2 flushed before each call"}
+                    "what": "moe_schedule: count, prefixes, offsets and placement in one "
+                            "cooperative launch (after a 12 KB memset of its barrier and "
+                            "totals) on uniform ids; L2 flushed before each call"}
     del b, ids
 
     def layer_leg(name, W, x, ws, n_calls, flush_each):
