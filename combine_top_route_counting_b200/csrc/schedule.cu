@@ -274,9 +274,11 @@ __global__ void __launch_bounds__(kThreads) sched_scatter_kernel(SchedParams p) 
 // once), with one grid barrier:
 //   A  each block (c, r) reads its 2,048 route ids once and keeps them in
 //      registers; each warp builds the match masks of its 32-route steps from
-//      ballots over the id bits (kept for C) and its expert histogram in
-//      shared memory; the block writes its histogram to ws[r][c][l] and adds
-//      the nonzero entries to the totals M[l][r] with integer atomics;
+//      ballots over the id bits, its expert histogram in shared memory and,
+//      from the running histogram, each route's rank among the warp's routes
+//      to its expert (kept in registers for C); the block writes its
+//      histogram to ws[r][c][l] and adds the nonzero entries to the totals
+//      M[l][r] with integer atomics;
 //   |  the barrier
 //   C  every block loads M and its own base, the sum of ws[r][c'][l] over
 //      the peer's earlier blocks c' < c (rows 0..c-1 of the peer's slab),
@@ -362,11 +364,14 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
   }
   __syncwarp();
   const int q0 = c * kSchedBlockRoutes + w * kWarpRoutes;
-  // keys: the expert id, or E for a lane without a valid route; the match
-  // masks of each step are built once here and reused by the placement
+  // keys: the expert id, or E for a lane without a valid route. pre[s]: the
+  // rank of step s's route among this warp's routes to its expert (routes of
+  // earlier steps, then of lower lanes), taken from the running histogram
+  // here so that the placement needs no running count of its own
   const int nbits = 32 - __clz(E);  // enough bits for 0..E
+  const unsigned lower = (1u << lane) - 1u;
   int key[kSteps];
-  unsigned msk[kSteps];
+  int pre[kSteps];
   int bad = 0;
 #pragma unroll
   for (int s = 0; s < kSteps; ++s) {
@@ -380,8 +385,13 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
 #pragma unroll
   for (int s = 0; s < kSteps; ++s) {
     const unsigned m = match_by_ballots(key[s], nbits);
-    msk[s] = m;
-    if (key[s] != E && lane == __ffs(m) - 1) wh[key[s]] += __popc(m);
+    const int lead = __ffs(m) - 1;  // first lane of this lane's key group
+    int before = 0;
+    if (key[s] != E && lane == lead) {
+      before = wh[key[s]];
+      wh[key[s]] = before + __popc(m);
+    }
+    pre[s] = __shfl_sync(kFull, before, lead) + __popc(m & lower);
     __syncwarp();
   }
   __syncthreads();
@@ -523,21 +533,19 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
   }
   __syncthreads();
 
-  const unsigned lower = (1u << lane) - 1u;
+  // the token of route q is q / k: one division, then stepped by 32 routes
+  int tq = (q0 + lane) / p.k, tr = (q0 + lane) - tq * p.k;
+  const int dq = 32 / p.k, dr = 32 - dq * p.k;
 #pragma unroll
   for (int s = 0; s < kSteps; ++s) {
     const int q = q0 + s * 32 + lane;
     const int id = key[s];
     const bool valid = id != E;
-    const unsigned m = msk[s];
-    int o = 0;
-    if (valid) o = wh[id] + __popc(m & lower);
-    __syncwarp();
-    if (valid && lane == __ffs(m) - 1) wh[id] += __popc(m);
-    __syncwarp();
     if (q < R) {
       const int64_t g = route_index(p, r, q);
       if (valid) {
+        // o: the route's stable rank among peer r's routes to expert id
+        const int o = wh[id] + pre[s];
         // columns past P hold zeros, which add nothing (o >= 0)
         int pos = 0;
         for (int q = 0; q < P; q += 4) {
@@ -547,11 +555,17 @@ __global__ void __launch_bounds__(kThreads) sched_fused_kernel(FusedParams f) {
                  (q + 3 < r && v.w > o);
         }
         const int row = s_off[id] + pos;
-        reinterpret_cast<int2*>(p.phi)[row] = make_int2(r, p.t0 + q / p.k);
+        reinterpret_cast<int2*>(p.phi)[row] = make_int2(r, p.t0 + tq);
         p.route_row[g] = row;
       } else {
         p.route_row[g] = -1;
       }
+    }
+    tq += dq;
+    tr += dr;
+    if (tr >= p.k) {
+      tr -= p.k;
+      ++tq;
     }
   }
 
