@@ -151,3 +151,50 @@ def test_assembled_line_reports_the_mxfp8_layer_leg():
     assert d["bytes"] == w.n_routes * w.H * 2 + 492544 * (w.H + w.H // 32)
     assert "mxfp8_layer" not in bench.assemble_line(args, w, 1, 397.0, stage_ms, 90, None, 0, 0,
                                                     None, None, None, 492544, peaks)
+
+
+def _fake_tree(root, sources):
+    csrc = root / "combine_top_route_counting_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for name, text in sources.items():
+        (csrc / name).write_text(text)
+    (root / "profiles").mkdir()
+
+
+def test_recorded_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
+    """A committed DRAM-traffic record reaches the bench line only while the
+    kernel sources hash to the value it was taken with: comments and blank
+    lines do not count, any code change does; the bytes scale by routes."""
+    sys.path.insert(0, ROOT)
+    import bench
+    files = ("a.cu", "b.cuh")
+    _fake_tree(tmp_path, {"a.cu": "int f() { return 1; }  // one\n", "b.cuh": "/* hdr */\nint g;\n"})
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h = bench.kernel_source_hash(files)
+    assert bench._recorded_traffic("t.txt", files, 10) is None  # no record
+    (tmp_path / "profiles" / "t.txt").write_text(
+        f"# comment: ignored\nkernel_source_sha256: {h}\ndram_bytes_per_route: 2.5\n")
+    assert bench._recorded_traffic("t.txt", files, 10) == 25.0
+    # comments and blank lines leave the hash and the record valid
+    (tmp_path / "combine_top_route_counting_b200" / "csrc" / "a.cu").write_text(
+        "// new comment\n\nint f() { return 1; }  // other\n")
+    assert bench.kernel_source_hash(files) == h
+    assert bench._recorded_traffic("t.txt", files, 4) == 10.0
+    # a code change invalidates it
+    (tmp_path / "combine_top_route_counting_b200" / "csrc" / "a.cu").write_text(
+        "int f() { return 2; }\n")
+    assert bench.kernel_source_hash(files) != h
+    assert bench._recorded_traffic("t.txt", files, 10) is None
+
+
+def test_committed_traffic_records_parse():
+    """The committed GEMM1 and dW1|dW3 records carry a hash and a per-route
+    byte figure in the form bench.py reads."""
+    for name in ("ffn_gemm1_traffic.txt", "ffn_wgrad13_traffic.txt"):
+        kv = {}
+        for ln in open(os.path.join(ROOT, "profiles", name)):
+            if ":" in ln and not ln.startswith("#"):
+                a, b = ln.split(":", 1)
+                kv[a.strip()] = b.strip()
+        assert len(kv["kernel_source_sha256"]) == 64
+        assert float(kv["dram_bytes_per_route"]) > 0
